@@ -1,0 +1,216 @@
+/*
+ * librmm — Reduced Matrix Multiplication (RMM) on NVIDIA B200 (sm_100a).
+ *
+ * The method (web pages on "Reduced Matrix Multiplication: Input-Adaptive
+ * Matrix-Product Reduction for LLM Inference"; gist.science summary,
+ * Resumo Técnico › Metodologia):
+ *   - "Mecanismo Central": instead of Y = A·B, compute A[:, I]·B[I, :] for a
+ *     subset I of the shared contraction dimension.
+ *   - "Estratégia de Seleção": score every contraction slice, keep the top
+ *     k = ceil(rho·K) of them, rho the user's retention ratio.
+ *   - "Escopo de Aplicação": Q·Kᵀ reduced over the head dimension, P·V
+ *     reduced over the key (token) dimension, X·W over the hidden dimension.
+ *
+ * Library defaults where the pages are silent:
+ *   - score s_k = ||A[:,k]||_2 · ||B[k,:]||_2 (RMM_SCORE_PRODUCT); the pages'
+ *     activation-only column norm ||A[:,k]||_2 is RMM_SCORE_A_ONLY;
+ *   - ties in the score go to the lower index; kept indices are ascending;
+ *   - one selection per matrix product (per batch item / attention head).
+ *
+ * Conventions for every call:
+ *   - Pointers named A, B, C, s, idx, A_S, B_St, workspace, status_word are
+ *     DEVICE pointers owned by the caller. The library never allocates.
+ *   - Matrices are row-major. "ld" is the leading dimension in elements
+ *     (distance between consecutive rows), "stride" the distance in elements
+ *     between consecutive batch items.
+ *   - bf16 data is passed as raw 16-bit words (the bits of __nv_bfloat16).
+ *   - All work is enqueued on `stream` in order; no call synchronises the
+ *     host except rmm_check.
+ *   - Argument errors are detected on the host, before any launch, and
+ *     returned as RMM_ERR_INVALID / RMM_ERR_UNSUPPORTED. A failed CUDA
+ *     runtime call returns RMM_ERR_CUDA. rmm_last_error_string() describes
+ *     the most recent failure on the calling thread.
+ *   - Errors found on the device (a non-finite score, a pipeline wait that
+ *     ran out) are OR-ed as bits into a 32-bit status word in device memory;
+ *     rmm_check() reads and clears it. No kernel traps.
+ *   - M = 0, N = 0 or batch = 0 are valid and launch nothing that writes C
+ *     (scores and selection are still produced when M = 0: all scores are 0).
+ */
+#ifndef RMM_H_
+#define RMM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RMM_OK = 0,
+  RMM_ERR_INVALID = 1,     /* bad argument (null pointer, rho outside (0,1], bad ld, small workspace) */
+  RMM_ERR_NONFINITE = 2,   /* a slice score was NaN or Inf (reported by rmm_check) */
+  RMM_ERR_CUDA = 3,        /* a CUDA runtime call failed */
+  RMM_ERR_TIMEOUT = 4,     /* a bounded pipeline wait in a kernel gave up (reported by rmm_check) */
+  RMM_ERR_UNSUPPORTED = 5  /* valid request this build does not handle (e.g. device is not sm_100) */
+} rmm_status;
+
+typedef enum { RMM_BF16 = 0, RMM_F32 = 1 } rmm_dtype;
+
+typedef enum { RMM_SCORE_PRODUCT = 0, RMM_SCORE_A_ONLY = 1 } rmm_score_mode;
+
+/* Device status-word bits (see rmm_check). */
+#define RMM_STATUS_BIT_NONFINITE 0x1u
+#define RMM_STATUS_BIT_TIMEOUT   0x2u
+
+/* ---------------------------------------------------------------- host helpers */
+
+/* k = ceil(rho·K) ("Estratégia de Seleção"), the IEEE double product rounded up.
+ * Returns -1 unless 0 < rho <= 1 and K >= 1. Never returns 0 for valid input. */
+int64_t rmm_keep_count(double rho, int64_t K);
+
+/* Contraction extent of the packed operands: k_keep rounded up to 64, the
+ * K-depth of one tensor-core pipeline stage. Padding columns hold zeros. */
+int64_t rmm_padded_keep(int64_t k_keep);
+
+/* Bytes of workspace rmm_matmul_reduced / _batched / rmm_qk_reduced /
+ * rmm_pv_reduced need for these sizes (in = input dtype). The workspace holds,
+ * each 1 KiB-aligned: the status word, scores [batch][K] f32, kept indices
+ * [batch][k_keep] i32, A_S [batch][M][k_pad] and B_St [batch][N][k_pad]. */
+size_t rmm_workspace_size(int64_t batch, int64_t M, int64_t K, int64_t N, int64_t k_keep,
+                          rmm_dtype in);
+
+/* ---------------------------------------------------------------- stage calls */
+
+/* Slice scores ("Estratégia de Seleção"; product form is the library default).
+ *   A: [batch][M][K] (ld lda, batch stride strideA), dtype `in`.
+ *   B: if b_kmajor == 0, [batch][K][N] (ld ldb), "row k of B" is B[k, :];
+ *      if b_kmajor == 1, B is given transposed as [batch][N][K] (ld ldb), so
+ *      "row k of B" is column k of that matrix (the Q·Kᵀ case, Kmat).
+ *      B is not read in RMM_SCORE_A_ONLY mode and may be NULL there.
+ *   s: [batch][K] f32 output: s_k = sqrt(sum_i A[i,k]^2) · sqrt(sum_j B[k,j]^2)
+ *      (product) or sqrt(sum_i A[i,k]^2) (a_only); sums in f32 in a fixed order,
+ *      so repeated calls give identical bits.
+ *   status_word: nullable device u32; RMM_STATUS_BIT_NONFINITE is OR-ed in when
+ *      a score is NaN/Inf (e.g. NaN inputs or f32 overflow of a sum of squares). */
+rmm_status rmm_score(const void* A, int64_t lda, int64_t strideA,
+                     const void* B, int64_t ldb, int64_t strideB, int b_kmajor,
+                     int64_t batch, int64_t M, int64_t K, int64_t N,
+                     rmm_dtype in, rmm_score_mode mode, float* s,
+                     uint32_t* status_word, cudaStream_t stream);
+
+/* Top-k selection ("Estratégia de Seleção": keep the k_keep largest scores).
+ *   s: [batch][K] f32 scores; idx: [batch][k_keep] i32 output, ascending.
+ *   Ties go to the lower index; -0.0 equals +0.0. Exact: the result depends
+ *   only on the order of the scores, never on rounding. 1 <= k_keep <= K.
+ *   A NaN score sets RMM_STATUS_BIT_NONFINITE in status_word (nullable). */
+rmm_status rmm_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,
+                      uint32_t* status_word, cudaStream_t stream);
+
+/* Pack the kept slices ("Mecanismo Central": A[:, I] and B[I, :]).
+ *   A, B as in rmm_score (B is required here); idx: [batch][k_keep] i32 indices
+ *   in [0, K) (as produced by rmm_select).
+ *   A_S:  [batch][M][k_pad] output, A_S[b][i][t] = A[b][i][idx[b][t]].
+ *   B_St: [batch][N][k_pad] output, B_St[b][j][t] = B[b][idx[b][t]][j] — the
+ *         kept rows of B stored transposed (contraction dimension contiguous),
+ *         the operand layout rmm_gemm consumes.
+ *   k_pad = rmm_padded_keep(k_keep); columns t >= k_keep are written as zero.
+ *   Copies bits exactly (no arithmetic). Indices outside [0, K) are a caller
+ *   error the kernels do not check. */
+rmm_status rmm_pack(const void* A, int64_t lda, int64_t strideA,
+                    const void* B, int64_t ldb, int64_t strideB, int b_kmajor,
+                    int64_t batch, int64_t M, int64_t K, int64_t N,
+                    const int32_t* idx, int64_t k_keep, rmm_dtype in,
+                    void* A_S, void* B_St, cudaStream_t stream);
+
+/* Reduced product on packed operands: C[b] = A_S[b] · B_St[b]ᵀ over the k_keep
+ * kept slices ("Mecanismo Central"), f32 accumulation.
+ *   A_S [batch][M][k_pad], B_St [batch][N][k_pad] as written by rmm_pack
+ *   (zero padding columns, 16-byte aligned base pointers).
+ *   in == RMM_BF16: tcgen05 tensor-core kernel (TMA, TMEM accumulators).
+ *   in == RMM_F32: CUDA-core FFMA kernel (f32 products, f32 sums).
+ *   C: [batch][M][N] with ld ldc, batch stride strideC, dtype `out`
+ *      (RMM_F32 or RMM_BF16, round-to-nearest-even).
+ *   status_word (nullable): RMM_STATUS_BIT_TIMEOUT if a pipeline wait gave up
+ *   (then C is incomplete). */
+rmm_status rmm_gemm(const void* A_S, const void* B_St, int64_t batch, int64_t M, int64_t N,
+                    int64_t k_keep, rmm_dtype in, void* C, int64_t ldc, int64_t strideC,
+                    rmm_dtype out, uint32_t* status_word, cudaStream_t stream);
+
+/* ---------------------------------------------------------------- fused calls */
+
+/* Y ≈ A·B with the top ceil(rho·K) contraction slices kept: score → select →
+ * pack → gemm, all enqueued on `stream`.
+ *   A [M][K] (ld lda), B [K][N] (ld ldb), C [M][N] (ld ldc); dtypes in/out.
+ *   idx_out: nullable device [k_keep] i32 that receives the kept indices.
+ *   workspace: device buffer of at least rmm_workspace_size(1, M, K, N, k, in)
+ *   bytes, 1 KiB-aligned; its first 4 bytes are the status word, cleared at
+ *   the start of the call. Call rmm_check(workspace, stream) to learn of
+ *   device-side errors. Workspace contents are scratch between calls. */
+rmm_status rmm_matmul_reduced(const void* A, int64_t lda, const void* B, int64_t ldb,
+                              int64_t M, int64_t K, int64_t N, double rho,
+                              rmm_dtype in, rmm_score_mode mode,
+                              void* C, int64_t ldc, rmm_dtype out, int32_t* idx_out,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Batched form: an independent selection per batch item. Layouts as in
+ * rmm_score / rmm_pack; C [batch][M][N] (ldc, strideC); idx_out nullable
+ * [batch][k_keep]. */
+rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t strideA,
+                                      const void* B, int64_t ldb, int64_t strideB, int b_kmajor,
+                                      int64_t batch, int64_t M, int64_t K, int64_t N, double rho,
+                                      rmm_dtype in, rmm_score_mode mode,
+                                      void* C, int64_t ldc, int64_t strideC, rmm_dtype out,
+                                      int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream);
+
+/* Attention scores S = Q·Kᵀ per head, reduced over the head dimension
+ * ("Escopo de Aplicação": the feature dimension of QKᵀ).
+ *   Q [bh][S_q][d], Kmat [bh][S_k][d] (contiguous); S_out [bh][S_q][S_k]
+ *   (contiguous, dtype out). One selection of ceil(rho·d) channels per head.
+ *   Workspace: rmm_workspace_size(bh, S_q, d, S_k, k, in). */
+rmm_status rmm_qk_reduced(const void* Q, const void* Kmat, int64_t bh, int64_t S_q, int64_t S_k,
+                          int64_t d, double rho, rmm_dtype in, rmm_score_mode mode,
+                          void* S_out, rmm_dtype out, int32_t* idx_out,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Attention output O = P·V per head, reduced over the keys ("Escopo de
+ * Aplicação": the token dimension of PV, which the pages mark optional).
+ *   P [bh][S_q][S_k], V [bh][S_k][d] (contiguous); O [bh][S_q][d] (contiguous,
+ *   dtype out). One selection of ceil(rho·S_k) keys per head.
+ *   Workspace: rmm_workspace_size(bh, S_q, S_k, d, k, in). */
+rmm_status rmm_pv_reduced(const void* P, const void* V, int64_t bh, int64_t S_q, int64_t S_k,
+                          int64_t d, double rho, rmm_dtype in, rmm_score_mode mode,
+                          void* O, rmm_dtype out, int32_t* idx_out,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------- diagnostics */
+
+/* Synchronises `stream`, reads the status word at `status_word` (a workspace
+ * base pointer works: the word is its first 4 bytes), clears it, and returns
+ * RMM_OK, RMM_ERR_NONFINITE or RMM_ERR_TIMEOUT (timeout wins if both). */
+rmm_status rmm_check(void* status_word, cudaStream_t stream);
+
+/* Message for the most recent failure on the calling thread ("" if none). */
+const char* rmm_last_error_string(void);
+
+/* Upper bound, in nanoseconds, on any single pipeline wait inside the
+ * tensor-core GEMM before it records RMM_STATUS_BIT_TIMEOUT and winds down
+ * (default 2e9 = 2 s; 0 restores the default). Process-wide. */
+void rmm_set_wait_limit_ns(uint64_t ns);
+
+/* Test hook, process-wide: when `on` is nonzero, the next tensor-core GEMM
+ * launches run with their TMA producer idle, so the MMA and epilogue waits run
+ * out; the kernel then records RMM_STATUS_BIT_TIMEOUT, drains, frees its
+ * tensor memory and returns. Used to test the timeout path without a fault. */
+void rmm_set_stall_producer_for_test(int on);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t rmm_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RMM_H_ */

@@ -1,0 +1,354 @@
+// The librmm C ABI: argument validation, workspace layout and the
+// score -> select -> pack -> gemm pipeline of Reduced Matrix Multiplication
+// (gist.science summary of "Reduced Matrix Multiplication: Input-Adaptive
+// Matrix-Product Reduction for LLM Inference", Resumo Técnico › Metodologia).
+// Everything is enqueued on the caller's stream; nothing here allocates or
+// synchronises, except rmm_check.
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/rmm.h"
+#include "rmm_internal.h"
+
+namespace rmm {
+
+static std::atomic<uint64_t> g_launches{0};
+static std::atomic<uint64_t> g_wait_limit_ns{0};
+static std::atomic<int> g_stall_producer{0};
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+static thread_local char g_err[512] = "";
+
+static rmm_status fail(rmm_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+static rmm_status cuda_fail(cudaError_t e, const char* what, const char* why = nullptr) {
+  return fail(RMM_ERR_CUDA, "%s: %s%s%s", what, cudaGetErrorString(e), why ? " — " : "", why ? why : "");
+}
+
+// Bind the calling thread to the stream's device (the caller's framework may
+// have made another device current).
+static rmm_status bind_device(cudaStream_t st) {
+  int dev = -1;
+  cudaError_t e = cudaStreamGetDevice(st, &dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamGetDevice");
+  int cur = -1;
+  cudaGetDevice(&cur);
+  if (cur != dev) {
+    e = cudaSetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  }
+  return RMM_OK;
+}
+
+static inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+static bool dtype_ok(rmm_dtype d) { return d == RMM_BF16 || d == RMM_F32; }
+static ElemKind kind(rmm_dtype d) { return d == RMM_BF16 ? kBF16 : kF32; }
+
+// A batch of row-major matrices (rows x cols, leading dimension ld, batch
+// stride bstride) must fit its own declared layout.
+static bool layout_ok(int64_t batch, int64_t rows, int64_t cols, int64_t ld, int64_t bstride) {
+  if (rows < 0 || cols < 0 || ld < 0 || bstride < 0) return false;
+  if (rows > 1 && ld < cols) return false;
+  if (batch > 1 && rows > 0 && bstride < (rows - 1) * ld + cols) return false;
+  return true;
+}
+
+constexpr int64_t kMaxGridBatch = 65535;
+
+struct Workspace {
+  uint32_t* status;
+  float* s;
+  int32_t* idx;
+  void* a_s;
+  void* b_st;
+  size_t bytes;
+};
+
+static Workspace carve(void* base, int64_t batch, int64_t M, int64_t K, int64_t N, int64_t k_keep, rmm_dtype in) {
+  const int64_t kp = round_up(k_keep, 64);
+  const int64_t eb = in == RMM_BF16 ? 2 : 4;
+  auto al = [](int64_t x) { return round_up(x, 1024); };
+  int64_t off = 0;
+  Workspace w;
+  const uintptr_t p = reinterpret_cast<uintptr_t>(base);
+  w.status = reinterpret_cast<uint32_t*>(p + off);
+  off += al(4);
+  w.s = reinterpret_cast<float*>(p + off);
+  off += al(batch * K * 4);
+  w.idx = reinterpret_cast<int32_t*>(p + off);
+  off += al(batch * k_keep * 4);
+  w.a_s = reinterpret_cast<void*>(p + off);
+  off += al(batch * M * kp * eb);
+  w.b_st = reinterpret_cast<void*>(p + off);
+  off += al(batch * N * kp * eb);
+  w.bytes = size_t(off);
+  return w;
+}
+
+// ---------------------------------------------------------------- stage bodies
+static rmm_status do_score(const void* A, int64_t lda, int64_t sA, const void* B, int64_t ldb, int64_t sB,
+                           int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N, rmm_dtype in,
+                           rmm_score_mode mode, float* s, uint32_t* status, cudaStream_t st) {
+  const ElemKind e = kind(in);
+  MatView a{A, lda, sA, M, K};
+  cudaError_t ce;
+  if (mode == RMM_SCORE_A_ONLY) {
+    ce = launch_colsq(a, e, batch, s, K, 2, status, st);
+    if (ce != cudaSuccess) return cuda_fail(ce, "score kernel");
+    return RMM_OK;
+  }
+  // s <- ||B[k,:]||^2, then s <- sqrt(||A[:,k]||^2) * sqrt(s)
+  if (b_kmajor) {
+    MatView bt{B, ldb, sB, N, K};
+    ce = launch_colsq(bt, e, batch, s, K, 0, status, st);
+  } else {
+    MatView bm{B, ldb, sB, K, N};
+    ce = launch_rowsq(bm, e, batch, s, K, st);
+  }
+  if (ce != cudaSuccess) return cuda_fail(ce, "score kernel (B norms)");
+  ce = launch_colsq(a, e, batch, s, K, 1, status, st);
+  if (ce != cudaSuccess) return cuda_fail(ce, "score kernel (A norms)");
+  return RMM_OK;
+}
+
+static rmm_status do_pack(const void* A, int64_t lda, int64_t sA, const void* B, int64_t ldb, int64_t sB, int b_kmajor,
+                          int64_t batch, int64_t M, int64_t K, int64_t N, const int32_t* idx, int64_t k_keep,
+                          rmm_dtype in, void* A_S, void* B_St, cudaStream_t st) {
+  const ElemKind e = kind(in);
+  const int64_t kp = round_up(k_keep, 64);
+  cudaError_t ce = launch_pack_cols(MatView{A, lda, sA, M, K}, e, batch, idx, k_keep, kp, A_S, st);
+  if (ce != cudaSuccess) return cuda_fail(ce, "pack kernel (A)");
+  if (b_kmajor)
+    ce = launch_pack_cols(MatView{B, ldb, sB, N, K}, e, batch, idx, k_keep, kp, B_St, st);
+  else
+    ce = launch_pack_rows_t(MatView{B, ldb, sB, K, N}, e, batch, idx, k_keep, kp, B_St, st);
+  if (ce != cudaSuccess) return cuda_fail(ce, "pack kernel (B)");
+  return RMM_OK;
+}
+
+static rmm_status do_gemm(const void* A_S, const void* B_St, int64_t batch, int64_t M, int64_t N, int64_t k_keep,
+                          rmm_dtype in, void* C, int64_t ldc, int64_t sC, rmm_dtype out, uint32_t* status,
+                          cudaStream_t st) {
+  GemmArgs g;
+  g.a = A_S;
+  g.b = B_St;
+  g.c = C;
+  g.batch = batch;
+  g.M = M;
+  g.N = N;
+  g.k_pad = round_up(k_keep, 64);
+  g.ldc = ldc;
+  g.strideC = sC;
+  g.out = kind(out);
+  g.status = status;
+  const uint64_t lim = g_wait_limit_ns.load();
+  g.wait_limit_ns = lim ? lim : kDefaultWaitLimitNs;
+  g.stall_producer = g_stall_producer.load();
+  cudaError_t ce;
+  const char* why = nullptr;
+  if (in == RMM_BF16)
+    ce = launch_gemm_tc(g, st, &why);
+  else
+    ce = launch_gemm_simt(g, st);
+  if (ce == cudaErrorNoKernelImageForDevice) return fail(RMM_ERR_UNSUPPORTED, "%s", why ? why : "unsupported device");
+  if (ce != cudaSuccess) return cuda_fail(ce, "gemm kernel", why);
+  return RMM_OK;
+}
+
+static rmm_status check_common(int64_t batch, int64_t M, int64_t K, int64_t N, rmm_dtype in) {
+  if (!dtype_ok(in)) return fail(RMM_ERR_INVALID, "unknown input dtype %d", int(in));
+  if (batch < 0 || M < 0 || N < 0) return fail(RMM_ERR_INVALID, "negative size");
+  if (K < 1) return fail(RMM_ERR_INVALID, "K must be >= 1 (got %lld)", (long long)K);
+  if (batch > kMaxGridBatch) return fail(RMM_ERR_UNSUPPORTED, "batch > %lld", (long long)kMaxGridBatch);
+  return RMM_OK;
+}
+
+static rmm_status check_ab(const void* A, int64_t lda, int64_t sA, const void* B, int64_t ldb, int64_t sB,
+                           int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N, bool need_b) {
+  if (batch > 0 && M > 0 && !A) return fail(RMM_ERR_INVALID, "A is NULL");
+  if (!layout_ok(batch, M, K, lda, sA)) return fail(RMM_ERR_INVALID, "A layout (lda/strideA) is too small");
+  if (need_b) {
+    if (batch > 0 && N > 0 && !B) return fail(RMM_ERR_INVALID, "B is NULL");
+    const bool ok = b_kmajor ? layout_ok(batch, N, K, ldb, sB) : layout_ok(batch, K, N, ldb, sB);
+    if (!ok) return fail(RMM_ERR_INVALID, "B layout (ldb/strideB) is too small");
+  }
+  return RMM_OK;
+}
+
+}  // namespace rmm
+
+using namespace rmm;
+
+extern "C" {
+
+int64_t rmm_keep_count(double rho, int64_t K) {
+  if (!(rho > 0.0 && rho <= 1.0) || K < 1) return -1;
+  const double k = std::ceil(rho * double(K));
+  if (k < 1.0) return 1;
+  if (k > double(K)) return K;
+  return int64_t(k);
+}
+
+int64_t rmm_padded_keep(int64_t k_keep) { return k_keep <= 0 ? 0 : round_up(k_keep, 64); }
+
+size_t rmm_workspace_size(int64_t batch, int64_t M, int64_t K, int64_t N, int64_t k_keep, rmm_dtype in) {
+  if (batch < 0 || M < 0 || K < 0 || N < 0 || k_keep < 0 || !dtype_ok(in)) return 0;
+  return carve(nullptr, batch, M, K, N, k_keep, in).bytes;
+}
+
+rmm_status rmm_score(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb, int64_t strideB,
+                     int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N, rmm_dtype in, rmm_score_mode mode,
+                     float* s, uint32_t* status_word, cudaStream_t stream) {
+  rmm_status r = check_common(batch, M, K, N, in);
+  if (r) return r;
+  if (mode != RMM_SCORE_PRODUCT && mode != RMM_SCORE_A_ONLY) return fail(RMM_ERR_INVALID, "unknown score mode");
+  r = check_ab(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, mode == RMM_SCORE_PRODUCT);
+  if (r) return r;
+  if (batch > 0 && !s) return fail(RMM_ERR_INVALID, "s is NULL");
+  if (batch == 0) return RMM_OK;
+  if ((r = bind_device(stream))) return r;
+  return do_score(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, in, mode, s, status_word, stream);
+}
+
+rmm_status rmm_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx, uint32_t* status_word,
+                      cudaStream_t stream) {
+  if (batch < 0 || K < 1) return fail(RMM_ERR_INVALID, "need batch >= 0 and K >= 1");
+  if (k_keep < 1 || k_keep > K) return fail(RMM_ERR_INVALID, "k_keep must be in [1, K]");
+  if (K > INT32_MAX) return fail(RMM_ERR_UNSUPPORTED, "K > 2^31-1");
+  if (batch > kMaxGridBatch) return fail(RMM_ERR_UNSUPPORTED, "batch > %lld", (long long)kMaxGridBatch);
+  if (batch == 0) return RMM_OK;
+  if (!s || !idx) return fail(RMM_ERR_INVALID, "s or idx is NULL");
+  rmm_status r = bind_device(stream);
+  if (r) return r;
+  cudaError_t ce = launch_select(s, batch, K, k_keep, idx, status_word, stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
+  return RMM_OK;
+}
+
+rmm_status rmm_pack(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb, int64_t strideB,
+                    int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N, const int32_t* idx, int64_t k_keep,
+                    rmm_dtype in, void* A_S, void* B_St, cudaStream_t stream) {
+  rmm_status r = check_common(batch, M, K, N, in);
+  if (r) return r;
+  if (k_keep < 1 || k_keep > K) return fail(RMM_ERR_INVALID, "k_keep must be in [1, K]");
+  r = check_ab(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, true);
+  if (r) return r;
+  if (batch == 0) return RMM_OK;
+  if (!idx) return fail(RMM_ERR_INVALID, "idx is NULL");
+  if ((M > 0 && !A_S) || (N > 0 && !B_St)) return fail(RMM_ERR_INVALID, "A_S or B_St is NULL");
+  if ((reinterpret_cast<uintptr_t>(A_S) | reinterpret_cast<uintptr_t>(B_St)) & 15u)
+    return fail(RMM_ERR_INVALID, "A_S and B_St must be 16-byte aligned");
+  if ((r = bind_device(stream))) return r;
+  return do_pack(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, idx, k_keep, in, A_S, B_St, stream);
+}
+
+rmm_status rmm_gemm(const void* A_S, const void* B_St, int64_t batch, int64_t M, int64_t N, int64_t k_keep,
+                    rmm_dtype in, void* C, int64_t ldc, int64_t strideC, rmm_dtype out, uint32_t* status_word,
+                    cudaStream_t stream) {
+  if (!dtype_ok(in) || !dtype_ok(out)) return fail(RMM_ERR_INVALID, "unknown dtype");
+  if (batch < 0 || M < 0 || N < 0) return fail(RMM_ERR_INVALID, "negative size");
+  if (k_keep < 1) return fail(RMM_ERR_INVALID, "k_keep must be >= 1");
+  if (batch > kMaxGridBatch) return fail(RMM_ERR_UNSUPPORTED, "batch > %lld", (long long)kMaxGridBatch);
+  if (!layout_ok(batch, M, N, ldc, strideC)) return fail(RMM_ERR_INVALID, "C layout (ldc/strideC) is too small");
+  if (batch == 0 || M == 0 || N == 0) return RMM_OK;
+  if (!A_S || !B_St || !C) return fail(RMM_ERR_INVALID, "A_S, B_St or C is NULL");
+  rmm_status r = bind_device(stream);
+  if (r) return r;
+  return do_gemm(A_S, B_St, batch, M, N, k_keep, in, C, ldc, strideC, out, status_word, stream);
+}
+
+rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb,
+                                      int64_t strideB, int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N,
+                                      double rho, rmm_dtype in, rmm_score_mode mode, void* C, int64_t ldc,
+                                      int64_t strideC, rmm_dtype out, int32_t* idx_out, void* workspace,
+                                      size_t workspace_bytes, cudaStream_t stream) {
+  rmm_status r = check_common(batch, M, K, N, in);
+  if (r) return r;
+  if (!dtype_ok(out)) return fail(RMM_ERR_INVALID, "unknown output dtype");
+  if (mode != RMM_SCORE_PRODUCT && mode != RMM_SCORE_A_ONLY) return fail(RMM_ERR_INVALID, "unknown score mode");
+  const int64_t k_keep = rmm_keep_count(rho, K);
+  if (k_keep < 1) return fail(RMM_ERR_INVALID, "rho must lie in (0, 1] (got %g)", rho);
+  r = check_ab(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, true);
+  if (r) return r;
+  if (!layout_ok(batch, M, N, ldc, strideC)) return fail(RMM_ERR_INVALID, "C layout (ldc/strideC) is too small");
+  if (batch > 0 && M > 0 && N > 0 && !C) return fail(RMM_ERR_INVALID, "C is NULL");
+  if (!workspace) return fail(RMM_ERR_INVALID, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(workspace) & 1023u) return fail(RMM_ERR_INVALID, "workspace must be 1 KiB aligned");
+  const Workspace w = carve(workspace, batch, M, K, N, k_keep, in);
+  if (workspace_bytes < w.bytes)
+    return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, w.bytes);
+  if ((r = bind_device(stream))) return r;
+  cudaError_t ce = cudaMemsetAsync(w.status, 0, 4, stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemsetAsync(status)");
+  if (batch == 0) return RMM_OK;
+  int32_t* idx = idx_out ? idx_out : w.idx;
+  if ((r = do_score(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, in, mode, w.s, w.status, stream)))
+    return r;
+  ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
+  if (M == 0 || N == 0) return RMM_OK;
+  if ((r = do_pack(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, idx, k_keep, in, w.a_s, w.b_st,
+                   stream)))
+    return r;
+  return do_gemm(w.a_s, w.b_st, batch, M, N, k_keep, in, C, ldc, strideC, out, w.status, stream);
+}
+
+rmm_status rmm_matmul_reduced(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t M, int64_t K, int64_t N,
+                              double rho, rmm_dtype in, rmm_score_mode mode, void* C, int64_t ldc, rmm_dtype out,
+                              int32_t* idx_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return rmm_matmul_reduced_batched(A, lda, 0, B, ldb, 0, 0, 1, M, K, N, rho, in, mode, C, ldc, 0, out, idx_out,
+                                    workspace, workspace_bytes, stream);
+}
+
+rmm_status rmm_qk_reduced(const void* Q, const void* Kmat, int64_t bh, int64_t S_q, int64_t S_k, int64_t d, double rho,
+                          rmm_dtype in, rmm_score_mode mode, void* S_out, rmm_dtype out, int32_t* idx_out,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (S_q < 0 || S_k < 0 || d < 1) return fail(RMM_ERR_INVALID, "need S_q, S_k >= 0 and d >= 1");
+  return rmm_matmul_reduced_batched(Q, d, S_q * d, Kmat, d, S_k * d, 1, bh, S_q, d, S_k, rho, in, mode, S_out, S_k,
+                                    S_q * S_k, out, idx_out, workspace, workspace_bytes, stream);
+}
+
+rmm_status rmm_pv_reduced(const void* P, const void* V, int64_t bh, int64_t S_q, int64_t S_k, int64_t d, double rho,
+                          rmm_dtype in, rmm_score_mode mode, void* O, rmm_dtype out, int32_t* idx_out, void* workspace,
+                          size_t workspace_bytes, cudaStream_t stream) {
+  if (S_q < 0 || S_k < 1 || d < 0) return fail(RMM_ERR_INVALID, "need S_q, d >= 0 and S_k >= 1");
+  return rmm_matmul_reduced_batched(P, S_k, S_q * S_k, V, d, S_k * d, 0, bh, S_q, S_k, d, rho, in, mode, O, d, S_q * d,
+                                    out, idx_out, workspace, workspace_bytes, stream);
+}
+
+rmm_status rmm_check(void* status_word, cudaStream_t stream) {
+  if (!status_word) return fail(RMM_ERR_INVALID, "status_word is NULL");
+  rmm_status r = bind_device(stream);
+  if (r) return r;
+  uint32_t w = 0;
+  cudaError_t ce = cudaMemcpyAsync(&w, status_word, 4, cudaMemcpyDeviceToHost, stream);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(stream);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(status_word, 0, 4, stream);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "rmm_check");
+  if (w & RMM_STATUS_BIT_TIMEOUT) return fail(RMM_ERR_TIMEOUT, "a pipeline wait in the GEMM ran out");
+  if (w & RMM_STATUS_BIT_NONFINITE) return fail(RMM_ERR_NONFINITE, "a slice score was NaN or Inf");
+  return RMM_OK;
+}
+
+const char* rmm_last_error_string(void) { return g_err; }
+
+void rmm_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+
+void rmm_set_stall_producer_for_test(int on) { g_stall_producer.store(on ? 1 : 0); }
+
+uint64_t rmm_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

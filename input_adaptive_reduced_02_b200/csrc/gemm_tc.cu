@@ -1,0 +1,444 @@
+// Reduced product on the B200 tensor cores ("Mecanismo Central" on the
+// gist.science summary of "Reduced Matrix Multiplication: Input-Adaptive
+// Matrix-Product Reduction for LLM Inference": C = A[:, I]·B[I, :], here on
+// the packed operands A_S [M][k_pad] and B_St [N][k_pad], both K-major).
+//
+// Persistent, warp-specialised tcgen05 kernel, one CTA per SM:
+//   warp 0      TMA producer: 128x64 A tile + BNx64 B tile per stage into a
+//               STAGES-deep shared-memory ring (128-byte swizzle, no multicast)
+//   warp 1      allocates tensor memory; one lane issues tcgen05.mma
+//               (kind::f16, bf16 x bf16 -> f32, M=128, N=BN, K=16) into one of
+//               two TMEM accumulators, and tcgen05.commit frees ring stages
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, optional bf16
+//               rounding, swizzled staging in shared memory, TMA tile store
+// The two accumulators let the epilogue of tile i overlap the mainloop of
+// tile i+1. Tiles are visited m-fastest so a column block of B is shared
+// through L2 by the CTAs working on it at the same time.
+//
+// Every mbarrier wait is bounded (rmm_set_wait_limit_ns). A role whose wait
+// runs out records RMM_STATUS_BIT_TIMEOUT, raises a shared abort flag that
+// the other roles poll, and winds down: the producer waits for its own TMA
+// loads still in flight, the MMA lane waits for its issued MMAs, the
+// epilogue waits for its TMA stores, and warp 1 frees tensor memory. No
+// thread leaves before the final CTA barrier.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "rmm_device.cuh"
+#include "rmm_internal.h"
+
+namespace rmm {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
+constexpr int kUmmaK = 16;
+constexpr int kEpiWarps = 4;
+constexpr int kTcThreads = 64 + 32 * kEpiWarps;
+
+template <int BN>
+struct TcCfg {
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t EPI_BUF = 32 * 128;  // 32 rows x 128 bytes
+  static constexpr uint32_t EPI_BYTES = kEpiWarps * 2 * EPI_BUF;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr uint32_t BAR_BYTES = 256;
+  static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
+};
+static_assert(TcCfg<256>::SMEM <= 232448, "shared memory budget");
+static_assert(TcCfg<128>::SMEM <= 232448, "shared memory budget");
+
+struct TcParams {
+  int32_t M, N, num_kb, tiles_m, tiles_n;
+  int64_t total_tiles;
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+  int stall_producer;
+  int tma_store;  // 1: TMA tile stores; 0: bounds-checked direct stores
+  int out_bf16;
+  void* c;
+  int64_t ldc, strideC;
+};
+
+__device__ __forceinline__ void decode_tile(int64_t t, const TcParams& p, int32_t& b, int32_t& mb, int32_t& nb) {
+  const int64_t per = int64_t(p.tiles_m) * p.tiles_n;
+  b = int32_t(t / per);
+  const int64_t r = t - int64_t(b) * per;
+  nb = int32_t(r / p.tiles_m);
+  mb = int32_t(r - int64_t(nb) * p.tiles_m);
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t* status) {
+  *abort_flag = 1;
+  status_or(status, RMM_TIMEOUT_BIT);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kTcThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmC, const TcParams p) {
+  using Cfg = TcCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t tc_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * Cfg::A_BYTES;
+  uint8_t* sEpi = sB + STAGES * Cfg::B_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + Cfg::EPI_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;   // [2] accumulator ready for the epilogue
+  uint64_t* tempty = tfull + 2;       // [2] accumulator drained by the epilogue
+  uint64_t* drain = tempty + 2;       // MMA completion at wind-down
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_sh = reinterpret_cast<int*>(tmem_base_sh + 1);
+  int* never_sh = abort_sh + 1;       // stays 0: waits that must not be cut short
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_sh = 0;
+    *never_sh = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (p.tma_store) tma_prefetch_desc(&tmC);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_sh, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_sh;
+  volatile int* abort_v = abort_sh;
+  const volatile int* never_v = never_sh;
+  const uint64_t limit = p.wait_limit_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    uint32_t stage = 0, phase = 0;
+    uint32_t issued = 0;         // bit s: stage s has a load issued
+    uint32_t issued_par = 0;     // bit s: parity of stage s's last issued load
+    bool ok = true;
+    for (int64_t t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
+      int32_t b, mb, nb;
+      decode_tile(t, p, b, mb, nb);
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        int w = 1;
+        if (lane == 0) w = mbar_wait_bounded(&empty[stage], phase ^ 1u, limit, abort_v);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          ok = false;
+          break;
+        }
+        if (lane == 0 && !p.stall_producer) {
+          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          tma_load_3d(sA + stage * Cfg::A_BYTES, &tmA, &full[stage], kb * BK, mb * BM, b);
+          tma_load_3d(sB + stage * Cfg::B_BYTES, &tmB, &full[stage], kb * BK, nb * BN, b);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) raise_abort(abort_v, p.status);
+    // Loads complete on their own; make sure none is still writing shared
+    // memory when the CTA exits.
+    if (lane == 0) {
+      for (int s = 0; s < STAGES; ++s)
+        if (issued & (1u << s)) mbar_wait_bounded(&full[s], (issued_par >> s) & 1u, limit, never_v);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = umma_idesc_bf16_f32(BM, BN);
+    uint32_t stage = 0, phase = 0;
+    uint32_t acc = 0, acc_phase = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
+      int w = 1;
+      if (lane == 0) w = mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, limit, abort_v);
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (!w) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        w = 1;
+        if (lane == 0) w = mbar_wait_bounded(&full[stage], phase, limit, abort_v);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_addr(sA + stage * Cfg::A_BYTES);
+          const uint32_t b0 = smem_addr(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / kUmmaK; ++kk) {
+            // advancing K by 16 elements = 32 bytes inside the swizzled row
+            umma_bf16(d_tmem, umma_desc_k_sw128(a0 + kk * 32), umma_desc_k_sw128(b0 + kk * 32), idesc,
+                      (kb | kk) != 0);
+          }
+          umma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(&tfull[acc]);
+      __syncwarp();
+      acc ^= 1u;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (!ok && lane == 0) raise_abort(abort_v, p.status);
+    // Wait for every MMA this lane issued before tensor memory is freed.
+    if (lane == 0) {
+      umma_commit(drain);
+      mbar_wait_bounded(drain, 0, limit, never_v);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    uint8_t* bufs = sEpi + (warp - 2) * 2 * Cfg::EPI_BUF;
+    uint32_t acc = 0, acc_phase = 0, nbuf = 0;
+    bool ok = true;
+    const int cols_per_chunk = p.out_bf16 ? 64 : 32;
+    const int chunks = BN / cols_per_chunk;
+    for (int64_t t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
+      int32_t b, mb, nb;
+      decode_tile(t, p, b, mb, nb);
+      int w = 1;
+      if (lane == 0) w = mbar_wait_bounded(&tfull[acc], acc_phase, limit, abort_v);
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (!w) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (uint32_t(q * 32) << 16) + acc * BN;
+      const int32_t row0 = mb * BM + q * 32;
+      for (int c = 0; c < chunks; ++c) {
+        uint32_t packed[32];
+        if (p.out_bf16) {
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(t_row + c * 64, r0);
+          tmem_ld_32x32b_x32(t_row + c * 64 + 32, r1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            packed[j] = pack_bf16x2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
+            packed[16 + j] = pack_bf16x2(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
+          }
+        } else {
+          tmem_ld_32x32b_x32(t_row + c * 32, packed);
+          tmem_ld_wait();
+        }
+        if (c == chunks - 1) {
+          // whole accumulator read: hand it back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+        const int32_t col0 = nb * BN + c * cols_per_chunk;
+        if (p.tma_store) {
+          uint8_t* buf = bufs + nbuf * Cfg::EPI_BUF;
+          if (lane == 0) tma_store_wait_read<1>();  // the store that last read `buf` is done
+          __syncwarp();
+          // row `lane` of the 32x128-byte box, 16-byte chunks in 128-byte swizzle order
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmC, buf, col0, row0, b);
+            tma_store_commit();
+          }
+          __syncwarp();
+          nbuf ^= 1u;
+        } else {
+          const int64_t row = int64_t(row0) + lane;
+          if (row < p.M) {
+            if (p.out_bf16) {
+              uint16_t* cp = static_cast<uint16_t*>(p.c) + int64_t(b) * p.strideC + row * p.ldc;
+              for (int j = 0; j < 64; ++j) {
+                const int64_t col = int64_t(col0) + j;
+                if (col < p.N) cp[col] = uint16_t(packed[j >> 1] >> ((j & 1) * 16));
+              }
+            } else {
+              float* cp = static_cast<float*>(p.c) + int64_t(b) * p.strideC + row * p.ldc;
+              for (int j = 0; j < 32; ++j) {
+                const int64_t col = int64_t(col0) + j;
+                if (col < p.N) cp[col] = __uint_as_float(packed[j]);
+              }
+            }
+          }
+        }
+      }
+      acc ^= 1u;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (!ok && lane == 0) raise_abort(abort_v, p.status);
+    if (lane == 0) tma_store_wait_all();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+bool encode_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+               uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct DevInfo {
+  int sms = 0;
+  int cc_major = 0, cc_minor = 0;
+  bool attr_done = false;
+};
+
+DevInfo& dev_info(int dev) {
+  static DevInfo info[64];
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  DevInfo& d = info[dev & 63];
+  if (!d.attr_done) {
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (d.cc_major == 10 && d.cc_minor == 0) {
+      cudaFuncSetAttribute(gemm_tc_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(TcCfg<256>::SMEM));
+      cudaFuncSetAttribute(gemm_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(TcCfg<128>::SMEM));
+    }
+    d.attr_done = true;
+  }
+  return d;
+}
+
+template <int BN>
+cudaError_t launch_bn(const GemmArgs& g, const DevInfo& di, cudaStream_t st, const char** why) {
+  const uint64_t kp = uint64_t(g.k_pad);
+  CUtensorMap tmA, tmB, tmC;
+  if (!encode_3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.a, kp, uint64_t(g.M), uint64_t(g.batch), kp * 2,
+                 kp * 2 * uint64_t(g.M), BK, BM) ||
+      !encode_3d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.b, kp, uint64_t(g.N), uint64_t(g.batch), kp * 2,
+                 kp * 2 * uint64_t(g.N), BK, BN)) {
+    *why = "cuTensorMapEncodeTiled failed for a packed operand";
+    return cudaErrorInvalidValue;
+  }
+  const uint64_t eb = g.out == kBF16 ? 2 : 4;
+  const bool c_ok = (reinterpret_cast<uintptr_t>(g.c) & 15u) == 0 && (uint64_t(g.ldc) * eb) % 16 == 0 &&
+                    (g.batch == 1 || (uint64_t(g.strideC) * eb) % 16 == 0);
+  int tma_store = 0;
+  if (c_ok) {
+    const uint64_t s2 = g.batch == 1 ? uint64_t(g.ldc) * eb * uint64_t(g.M) : uint64_t(g.strideC) * eb;
+    tma_store = encode_3d(&tmC, g.out == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                          g.c, uint64_t(g.N), uint64_t(g.M), uint64_t(g.batch), uint64_t(g.ldc) * eb,
+                          s2 == 0 ? 16 : s2, uint32_t(128 / eb), 32)
+                    ? 1
+                    : 0;
+  }
+  if (!tma_store) tmC = tmA;  // never dereferenced when tma_store == 0
+
+  TcParams p;
+  p.M = int32_t(g.M);
+  p.N = int32_t(g.N);
+  p.num_kb = int32_t(g.k_pad / BK);
+  p.tiles_m = int32_t((g.M + BM - 1) / BM);
+  p.tiles_n = int32_t((g.N + BN - 1) / BN);
+  p.total_tiles = int64_t(p.tiles_m) * p.tiles_n * g.batch;
+  p.status = g.status;
+  p.wait_limit_ns = g.wait_limit_ns;
+  p.stall_producer = g.stall_producer;
+  p.tma_store = tma_store;
+  p.out_bf16 = g.out == kBF16;
+  p.c = g.c;
+  p.ldc = g.ldc;
+  p.strideC = g.strideC;
+  const int64_t grid = std::min<int64_t>(p.total_tiles, di.sms > 0 ? di.sms : 148);
+  count_launch();
+  gemm_tc_kernel<BN><<<unsigned(grid), kTcThreads, TcCfg<BN>::SMEM, st>>>(tmA, tmB, tmC, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st, const char** why) {
+  if (g.batch == 0 || g.M == 0 || g.N == 0) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const DevInfo& di = dev_info(dev);
+  if (!(di.cc_major == 10 && di.cc_minor == 0)) {
+    *why = "the tensor-core GEMM is built for sm_100a (B200) only";
+    return cudaErrorNoKernelImageForDevice;
+  }
+  if ((reinterpret_cast<uintptr_t>(g.a) & 15u) || (reinterpret_cast<uintptr_t>(g.b) & 15u)) {
+    *why = "packed operands must be 16-byte aligned";
+    return cudaErrorInvalidValue;
+  }
+  if (g.M > INT32_MAX || g.N > INT32_MAX || g.k_pad > INT32_MAX || g.batch > INT32_MAX) {
+    *why = "a dimension exceeds 2^31-1";
+    return cudaErrorInvalidValue;
+  }
+  return g.N <= 128 ? launch_bn<128>(g, di, st, why) : launch_bn<256>(g, di, st, why);
+}
+
+}  // namespace rmm

@@ -1,0 +1,314 @@
+"""Python binding for librmm, the B200 Reduced Matrix Multiplication library.
+
+Argument marshalling only: every step of score -> select -> pack -> gemm runs in
+the library's CUDA kernels. PyTorch supplies device memory and the current
+stream. There is no fallback: if librmm.so is missing, loading fails loudly.
+
+Method (gist.science summary of "Reduced Matrix Multiplication: Input-Adaptive
+Matrix-Product Reduction for LLM Inference", Resumo Técnico › Metodologia):
+score every contraction slice k of A·B, keep the top ceil(rho·K), and compute
+A[:, I]·B[I, :]. The default score is ||A[:,k]||·||B[k,:]|| ("product"); the
+pages' activation-only column norm is mode "a_only".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmm.so")
+
+RMM_OK, RMM_ERR_INVALID, RMM_ERR_NONFINITE, RMM_ERR_CUDA, RMM_ERR_TIMEOUT, RMM_ERR_UNSUPPORTED = range(6)
+RMM_BF16, RMM_F32 = 0, 1
+SCORE_MODES = {"product": 0, "a_only": 1}
+STATUS_NAMES = {0: "RMM_OK", 1: "RMM_ERR_INVALID", 2: "RMM_ERR_NONFINITE", 3: "RMM_ERR_CUDA",
+                4: "RMM_ERR_TIMEOUT", 5: "RMM_ERR_UNSUPPORTED"}
+
+
+class RMMError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+_lib = None
+
+_vp, _i64, _f64, _i32, _u64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_double, ctypes.c_int, ctypes.c_uint64
+_SIGS = {
+    "rmm_keep_count": (_i64, [_f64, _i64]),
+    "rmm_padded_keep": (_i64, [_i64]),
+    "rmm_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64, _i64, _i32]),
+    "rmm_score": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i32, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp,
+                         _vp]),
+    "rmm_select": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "rmm_pack": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i32, _i64, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _vp,
+                        _vp]),
+    "rmm_gemm": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _i32, _vp, _i64, _i64, _i32, _vp, _vp]),
+    "rmm_matmul_reduced": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _i64, _f64, _i32, _i32, _vp, _i64, _i32, _vp,
+                                  _vp, ctypes.c_size_t, _vp]),
+    "rmm_matmul_reduced_batched": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i32, _i64, _i64, _i64, _i64, _f64,
+                                          _i32, _i32, _vp, _i64, _i64, _i32, _vp, _vp, ctypes.c_size_t, _vp]),
+    "rmm_qk_reduced": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _f64, _i32, _i32, _vp, _i32, _vp, _vp,
+                              ctypes.c_size_t, _vp]),
+    "rmm_pv_reduced": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _f64, _i32, _i32, _vp, _i32, _vp, _vp,
+                              ctypes.c_size_t, _vp]),
+    "rmm_check": (_i32, [_vp, _vp]),
+    "rmm_last_error_string": (ctypes.c_char_p, []),
+    "rmm_set_wait_limit_ns": (None, [_u64]),
+    "rmm_set_stall_producer_for_test": (None, [_i32]),
+    "rmm_launch_count": (_u64, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded librmm.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"librmm.so not found at {_LIB_PATH}; build it with "
+                              "`python -m input_adaptive_reduced_02_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _check(status: int):
+    if status != RMM_OK:
+        raise RMMError(status, lib().rmm_last_error_string().decode(errors="replace"))
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return RMM_BF16
+    if t.dtype == torch.float32:
+        return RMM_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; librmm takes bfloat16 or float32")
+
+
+def _out_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return RMM_BF16
+    if dt == torch.float32:
+        return RMM_F32
+    raise TypeError(f"unsupported output dtype {dt}")
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _mat(t: torch.Tensor, name: str):
+    """(batch, rows, cols, ld, batch_stride) of a 2-D or 3-D CUDA tensor."""
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() == 2:
+        t3 = t.unsqueeze(0)
+    elif t.dim() == 3:
+        t3 = t
+    else:
+        raise ValueError(f"{name} must be 2-D or 3-D")
+    if t3.stride(2) != 1 and t3.shape[2] > 1:
+        raise ValueError(f"{name} must be contiguous along its last dimension")
+    b, r, c = t3.shape
+    ld = t3.stride(1) if r > 1 else c
+    bs = t3.stride(0) if b > 1 else r * ld
+    return b, r, c, ld, bs
+
+
+def keep_count(rho: float, K: int) -> int:
+    k = lib().rmm_keep_count(float(rho), int(K))
+    if k < 1:
+        raise ValueError(f"rho must lie in (0, 1] and K >= 1 (rho={rho}, K={K})")
+    return int(k)
+
+
+def padded_keep(k_keep: int) -> int:
+    return int(lib().rmm_padded_keep(int(k_keep)))
+
+
+def workspace_size(batch: int, M: int, K: int, N: int, k_keep: int, dtype: torch.dtype) -> int:
+    return int(lib().rmm_workspace_size(batch, M, K, N, k_keep, _out_code(dtype)))
+
+
+class Workspace:
+    """A 1 KiB-aligned device workspace carved from one torch allocation."""
+
+    def __init__(self, nbytes: int, device):
+        self.nbytes = int(nbytes)
+        self._buf = torch.empty(self.nbytes + 1024, dtype=torch.uint8, device=device)
+        base = self._buf.data_ptr()
+        self.offset = (-base) % 1024
+        self.ptr = base + self.offset
+
+    @property
+    def status_ptr(self) -> int:
+        return self.ptr
+
+
+def _ensure_ws(ws, nbytes, device):
+    if ws is None or ws.nbytes < nbytes:
+        return Workspace(nbytes, device)
+    return ws
+
+
+def status_word(device="cuda") -> torch.Tensor:
+    """A zeroed device u32 (as int32 storage) for the stage calls' status bits."""
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def check(status, stream_tensor: torch.Tensor | None = None):
+    """Read and clear a device status word (a tensor from status_word(), or a
+    Workspace); raise RMMError on NaN/Inf scores or a pipeline timeout."""
+    if isinstance(status, Workspace):
+        ptr, dev = status.ptr, status._buf.device
+    else:
+        ptr, dev = status.data_ptr(), status.device
+    st = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    _check(lib().rmm_check(ctypes.c_void_p(ptr), st))
+
+
+# ---------------------------------------------------------------- stage calls
+def score(A: torch.Tensor, B: torch.Tensor | None, mode: str = "product", b_kmajor: bool = False,
+          out: torch.Tensor | None = None, status: torch.Tensor | None = None) -> torch.Tensor:
+    """Slice scores s [batch][K] (f32). A [b][M][K]; B [b][K][N] (or [b][N][K] with b_kmajor)."""
+    ba, M, K, lda, sA = _mat(A, "A")
+    if B is not None:
+        bb, r, c, ldb, sB = _mat(B, "B")
+        N = r if b_kmajor else c
+        if (c if b_kmajor else r) != K or bb != ba:
+            raise ValueError("A and B disagree on the contraction dimension or batch")
+    else:
+        if SCORE_MODES[mode] != 1:
+            raise ValueError("B is required in product mode")
+        N, ldb, sB = 0, 0, 0
+    if out is None:
+        out = torch.empty((ba, K) if A.dim() == 3 else (K,), dtype=torch.float32, device=A.device)
+    _check(lib().rmm_score(_ptr(A), lda, sA, _ptr(B), ldb, sB, int(b_kmajor), ba, M, K, N, _dtype(A),
+                           SCORE_MODES[mode], _ptr(out), _ptr(status), _stream(A)))
+    return out
+
+
+def select(s: torch.Tensor, k_keep: int, out: torch.Tensor | None = None,
+           status: torch.Tensor | None = None) -> torch.Tensor:
+    """Ascending int32 indices of the k_keep largest scores per row of s (ties -> lower index)."""
+    if s.dtype != torch.float32 or not s.is_cuda or not s.is_contiguous():
+        raise ValueError("s must be a contiguous float32 CUDA tensor")
+    batch, K = (1, s.shape[0]) if s.dim() == 1 else s.shape
+    if out is None:
+        out = torch.empty((k_keep,) if s.dim() == 1 else (batch, k_keep), dtype=torch.int32, device=s.device)
+    _check(lib().rmm_select(_ptr(s), batch, K, k_keep, _ptr(out), _ptr(status), _stream(s)))
+    return out
+
+
+def pack(A: torch.Tensor, B: torch.Tensor, idx: torch.Tensor, b_kmajor: bool = False, out=None):
+    """A_S [b][M][k_pad] and B_St [b][N][k_pad] (kept slices, contraction dim contiguous, zero padded).
+    `out` may supply the (A_S, B_St) pair."""
+    ba, M, K, lda, sA = _mat(A, "A")
+    bb, r, c, ldb, sB = _mat(B, "B")
+    N = r if b_kmajor else c
+    k_keep = idx.shape[-1]
+    kp = padded_keep(k_keep)
+    if out is None:
+        shp = (lambda rows: (ba, rows, kp)) if A.dim() == 3 else (lambda rows: (rows, kp))
+        A_S = torch.empty(shp(M), dtype=A.dtype, device=A.device)
+        B_St = torch.empty(shp(N), dtype=A.dtype, device=A.device)
+    else:
+        A_S, B_St = out
+        if A_S.numel() != ba * M * kp or B_St.numel() != ba * N * kp:
+            raise ValueError("pack: output buffers have the wrong size")
+    _check(lib().rmm_pack(_ptr(A), lda, sA, _ptr(B), ldb, sB, int(b_kmajor), ba, M, K, N, _ptr(idx), k_keep,
+                          _dtype(A), _ptr(A_S), _ptr(B_St), _stream(A)))
+    return A_S, B_St
+
+
+def gemm(A_S: torch.Tensor, B_St: torch.Tensor, k_keep: int, out_dtype=torch.float32,
+         out: torch.Tensor | None = None, status: torch.Tensor | None = None) -> torch.Tensor:
+    """C = A_S · B_Stᵀ over the first k_keep (of k_pad) slices."""
+    ba, M, kp, _, _ = _mat(A_S, "A_S")
+    _, N, _, _, _ = _mat(B_St, "B_St")
+    if out is None:
+        out = torch.empty((ba, M, N) if A_S.dim() == 3 else (M, N), dtype=out_dtype, device=A_S.device)
+    _, _, _, ldc, sC = _mat(out, "C")
+    _check(lib().rmm_gemm(_ptr(A_S), _ptr(B_St), ba, M, N, k_keep, _dtype(A_S), _ptr(out), ldc, sC,
+                          _out_code(out.dtype), _ptr(status), _stream(A_S)))
+    return out
+
+
+# ---------------------------------------------------------------- fused calls
+def matmul_reduced(A: torch.Tensor, B: torch.Tensor, rho: float, mode: str = "product",
+                   out_dtype=torch.float32, out: torch.Tensor | None = None, workspace: Workspace | None = None,
+                   idx_out: torch.Tensor | None = None, b_kmajor: bool = False):
+    """C ≈ A·B keeping the top ceil(rho·K) contraction slices (batched when A is 3-D).
+
+    Returns (C, workspace); the workspace can be passed back in to avoid
+    re-allocation and to read the device status with check(workspace)."""
+    ba, M, K, lda, sA = _mat(A, "A")
+    bb, r, c, ldb, sB = _mat(B, "B")
+    N = r if b_kmajor else c
+    k = keep_count(rho, K)
+    ws = _ensure_ws(workspace, workspace_size(ba, M, K, N, k, A.dtype), A.device)
+    if out is None:
+        out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
+    _, _, _, ldc, sC = _mat(out, "C")
+    _check(lib().rmm_matmul_reduced_batched(_ptr(A), lda, sA, _ptr(B), ldb, sB, int(b_kmajor), ba, M, K, N,
+                                            float(rho), _dtype(A), SCORE_MODES[mode], _ptr(out), ldc, sC,
+                                            _out_code(out.dtype), _ptr(idx_out), ctypes.c_void_p(ws.ptr),
+                                            ws.nbytes, _stream(A)))
+    return out, ws
+
+
+def qk_reduced(Q: torch.Tensor, Kmat: torch.Tensor, rho: float, mode: str = "product", out_dtype=torch.float32,
+               out: torch.Tensor | None = None, workspace: Workspace | None = None,
+               idx_out: torch.Tensor | None = None):
+    """S = Q·Kᵀ per head, reduced over head_dim. Q [bh][S_q][d], Kmat [bh][S_k][d]."""
+    bh, S_q, d = Q.shape
+    S_k = Kmat.shape[1]
+    k = keep_count(rho, d)
+    ws = _ensure_ws(workspace, workspace_size(bh, S_q, d, S_k, k, Q.dtype), Q.device)
+    if out is None:
+        out = torch.empty(bh, S_q, S_k, dtype=out_dtype, device=Q.device)
+    _check(lib().rmm_qk_reduced(_ptr(Q), _ptr(Kmat), bh, S_q, S_k, d, float(rho), _dtype(Q), SCORE_MODES[mode],
+                                _ptr(out), _out_code(out.dtype), _ptr(idx_out), ctypes.c_void_p(ws.ptr), ws.nbytes,
+                                _stream(Q)))
+    return out, ws
+
+
+def pv_reduced(P: torch.Tensor, V: torch.Tensor, rho: float, mode: str = "product", out_dtype=torch.float32,
+               out: torch.Tensor | None = None, workspace: Workspace | None = None,
+               idx_out: torch.Tensor | None = None):
+    """O = P·V per head, reduced over the keys. P [bh][S_q][S_k], V [bh][S_k][d]."""
+    bh, S_q, S_k = P.shape
+    d = V.shape[2]
+    k = keep_count(rho, S_k)
+    ws = _ensure_ws(workspace, workspace_size(bh, S_q, S_k, d, k, P.dtype), P.device)
+    if out is None:
+        out = torch.empty(bh, S_q, d, dtype=out_dtype, device=P.device)
+    _check(lib().rmm_pv_reduced(_ptr(P), _ptr(V), bh, S_q, S_k, d, float(rho), _dtype(P), SCORE_MODES[mode],
+                                _ptr(out), _out_code(out.dtype), _ptr(idx_out), ctypes.c_void_p(ws.ptr), ws.nbytes,
+                                _stream(P)))
+    return out, ws
+
+
+def set_wait_limit_ns(ns: int):
+    lib().rmm_set_wait_limit_ns(int(ns))
+
+
+def set_stall_producer_for_test(on: bool):
+    lib().rmm_set_stall_producer_for_test(int(bool(on)))
+
+
+def launch_count() -> int:
+    return int(lib().rmm_launch_count())

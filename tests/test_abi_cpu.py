@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/rmm.h declares, and its host helpers and argument
+validation behave as documented (validation runs before any CUDA call)."""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+from fractions import Fraction
+
+import pytest
+
+from input_adaptive_reduced_02_b200 import rmm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rmm.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(rmm_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    L = rmm.lib()
+    names = _declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in rmm.h but not exported"
+    assert set(names) == set(rmm._SIGS), "binding signatures out of sync with rmm.h"
+
+
+def test_keep_count_matches_exact_ceiling():
+    for K in [1, 2, 3, 7, 10, 64, 128, 256, 1000, 4096, 8192, 16384, 28672, 32768]:
+        for rho in [0.01, 0.1, 0.25, 0.3, 0.5, 0.7, 0.9, 1.0]:
+            assert rmm.keep_count(rho, K) == max(1, math.ceil(Fraction(str(rho)) * K)), (rho, K)
+    L = rmm.lib()
+    for bad in (0.0, -1.0, 1.5, float("nan"), float("inf")):
+        assert L.rmm_keep_count(bad, 10) == -1
+    assert L.rmm_keep_count(0.5, 0) == -1
+    assert L.rmm_keep_count(1e-300, 10) == 1
+
+
+def test_padded_keep_and_workspace_layout():
+    assert rmm.padded_keep(1) == 64 and rmm.padded_keep(64) == 64 and rmm.padded_keep(65) == 128
+    ws = rmm.workspace_size(1, 4096, 4096, 4096, 2048, rmm.torch.bfloat16)
+    # status + scores + indices + A_S + B_St, each 1 KiB aligned
+    expect = 1024 + 4096 * 4 + 2048 * 4 + 4096 * 2048 * 2 + 4096 * 2048 * 2
+    assert ws == expect
+    ws32 = rmm.workspace_size(2, 3, 5, 7, 3, rmm.torch.float32)
+    # A_S: 2*3*64*4 = 1536 -> 2048; B_St: 2*7*64*4 = 3584 -> 4096
+    assert ws32 == 1024 + 1024 + 1024 + 2048 + 4096
+
+
+V = ctypes.c_void_p
+
+
+def test_validation_errors_need_no_gpu():
+    L = rmm.lib()
+    null = V(0)
+    # rho outside (0, 1]
+    st = L.rmm_matmul_reduced(V(16), 8, V(16), 8, 4, 8, 8, 1.5, 0, 0, V(16), 8, 1, null, V(1024), 1 << 20, null)
+    assert st == rmm.RMM_ERR_INVALID
+    assert b"rho" in L.rmm_last_error_string()
+    # A is NULL
+    st = L.rmm_matmul_reduced(null, 8, V(16), 8, 4, 8, 8, 0.5, 0, 0, V(16), 8, 1, null, V(1024), 1 << 20, null)
+    assert st == rmm.RMM_ERR_INVALID
+    # leading dimension smaller than the row
+    st = L.rmm_score(V(16), 4, 0, V(16), 8, 0, 0, 1, 4, 8, 8, 0, 0, V(16), null, null)
+    assert st == rmm.RMM_ERR_INVALID
+    # workspace too small
+    st = L.rmm_matmul_reduced(V(16), 8, V(16), 8, 4, 8, 8, 0.5, 0, 0, V(16), 8, 1, null, V(1024), 16, null)
+    assert st == rmm.RMM_ERR_INVALID and b"workspace" in L.rmm_last_error_string()
+    # misaligned workspace
+    st = L.rmm_matmul_reduced(V(16), 8, V(16), 8, 4, 8, 8, 0.5, 0, 0, V(16), 8, 1, null, V(1040), 1 << 20, null)
+    assert st == rmm.RMM_ERR_INVALID
+    # k_keep outside [1, K]
+    assert L.rmm_select(V(16), 1, 10, 0, V(16), null, null) == rmm.RMM_ERR_INVALID
+    assert L.rmm_select(V(16), 1, 10, 11, V(16), null, null) == rmm.RMM_ERR_INVALID
+    # unknown dtype / score mode
+    assert L.rmm_score(V(16), 8, 0, V(16), 8, 0, 0, 1, 4, 8, 8, 7, 0, V(16), null, null) == rmm.RMM_ERR_INVALID
+    assert L.rmm_score(V(16), 8, 0, V(16), 8, 0, 0, 1, 4, 8, 8, 0, 9, V(16), null, null) == rmm.RMM_ERR_INVALID
+    # K = 0
+    assert L.rmm_score(V(16), 8, 0, V(16), 8, 0, 0, 1, 4, 0, 8, 0, 0, V(16), null, null) == rmm.RMM_ERR_INVALID
+    # empty batch is a no-op that needs no device
+    assert L.rmm_select(null, 0, 10, 3, null, null, null) == rmm.RMM_OK
+
+
+def test_binding_refuses_cpu_tensors():
+    A = rmm.torch.zeros(4, 8, dtype=rmm.torch.bfloat16)
+    with pytest.raises(ValueError):
+        rmm.score(A, A.t().contiguous())

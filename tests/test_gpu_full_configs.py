@@ -1,0 +1,127 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the
+benchmark times (the fused calls). Where the fp64 oracle cannot afford the
+whole product, it is applied to sub-problems whose answers the full result
+must contain exactly: a product entry depends only on its row of A and its
+column of B, and a slice score only on column k of A and row k of B.
+The integer stage (selection) is always checked on every head/matrix:
+bit-exact against the oracle's selection on the library's f32 scores, with
+the scores themselves checked against fp64."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import rmm_oracle as O
+from input_adaptive_reduced_02_b200 import inputs, rmm
+
+from _parity import check_product, check_scores, check_selection, f64
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+DEV = "cuda"
+
+
+def _rows_cols(M, N, nr, nc, seed):
+    r = np.random.default_rng(seed)
+    rows = np.sort(r.choice(M, size=min(nr, M), replace=False))
+    cols = np.sort(r.choice(N, size=min(nc, N), replace=False))
+    return rows, cols
+
+
+def _check_selection_exact(s_gpu: torch.Tensor, idx_gpu: torch.Tensor, k: int):
+    assert idx_gpu.cpu().numpy().tolist() == O.select_top(s_gpu.cpu().numpy(), k).tolist()
+
+
+def test_linear_4096_all_rhos_full_compare():
+    X, W = inputs.linear_projection(seed=0, device=DEV)
+    X64, W64 = f64(X), f64(W)
+    s_ref = O.slice_scores(X64, W64)
+    s = rmm.score(X, W)
+    check_scores(s.cpu().numpy(), s_ref)
+    ws = None
+    for rho in (0.3, 0.5, 0.7, 0.9, 1.0):
+        k = rmm.keep_count(rho, 4096)
+        idx = torch.empty(k, dtype=torch.int32, device=DEV)
+        C, ws = rmm.matmul_reduced(X, W, rho, idx_out=idx, workspace=ws)
+        rmm.check(ws)
+        _check_selection_exact(s, idx, k)
+        check_selection(idx.cpu().numpy(), s_ref, k)
+        check_product(f64(C), X64, W64, idx.cpu().numpy(), 1e-2)
+
+
+def test_qk_32x4096x128():
+    Q, Km = inputs.attention_qk(seed=0, device=DEV)
+    k = rmm.keep_count(0.5, 128)
+    idx = torch.empty(32, k, dtype=torch.int32, device=DEV)
+    S, ws = rmm.qk_reduced(Q, Km, 0.5, out_dtype=torch.float32, idx_out=idx)
+    rmm.check(ws)
+    s = rmm.score(Q, Km, b_kmajor=True)
+    for h in range(32):
+        Q64, K64 = f64(Q[h]), f64(Km[h])
+        s_ref = O.slice_scores(Q64, K64.T)
+        check_scores(s[h].cpu().numpy(), s_ref)
+        _check_selection_exact(s[h], idx[h], k)
+        check_selection(idx[h].cpu().numpy(), s_ref, k)
+        rows, cols = _rows_cols(4096, 4096, 128, 512, h)
+        check_product(f64(S[h][rows][:, cols]), Q64[rows], K64[cols].T, idx[h].cpu().numpy(), 1e-2)
+    # two heads in full
+    for h in (0, 31):
+        check_product(f64(S[h]), f64(Q[h]), f64(Km[h]).T, idx[h].cpu().numpy(), 1e-2)
+
+
+@pytest.mark.parametrize("S", [8192, 16384, 32768])
+def test_pv_long_context(S):
+    heads_checked = [0, 17]
+    P, V = inputs.attention_pv(bh=32, S=S, d=128, seed=0, device=DEV)
+    ws = None
+    s = rmm.score(P, V)
+    for rho in (0.3, 0.5, 0.7):
+        k = rmm.keep_count(rho, S)
+        idx = torch.empty(32, k, dtype=torch.int32, device=DEV)
+        Oo, ws = rmm.pv_reduced(P, V, rho, idx_out=idx, workspace=ws)
+        rmm.check(ws)
+        for h in range(32):
+            _check_selection_exact(s[h], idx[h], k)
+        for h in heads_checked:
+            rows, cols = _rows_cols(S, S, 256, 1024, h + S)
+            # scores of sampled slices against fp64
+            P_cols = f64(P[h][:, torch.as_tensor(cols, device=DEV)])
+            s_ref_cols = O.slice_scores(P_cols, f64(V[h][torch.as_tensor(cols, device=DEV)]))
+            check_scores(s[h][torch.as_tensor(cols, device=DEV)].cpu().numpy(), s_ref_cols)
+            # sampled output rows: O[r, :] = P[r, I] · V[I, :]
+            ii = idx[h].long()
+            P_rows = f64(P[h][torch.as_tensor(rows, device=DEV)][:, ii])
+            ref = P_rows @ f64(V[h][ii])
+            err = O.frobenius_rel_error(f64(Oo[h][torch.as_tensor(rows, device=DEV)]), ref)
+            assert err <= 1e-2, err
+    del P, V, ws
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("which", ["up", "down"])
+def test_mlp_70b_projections(which):
+    X, W = (inputs.mlp_up if which == "up" else inputs.mlp_down)(seed=0, device=DEV)
+    M, K = X.shape
+    N = W.shape[1]
+    s = rmm.score(X, W)
+    # all scores in fp64, column by column block to bound host memory
+    s_ref = np.concatenate([O.slice_scores(f64(X[:, c0:c0 + 4096]), f64(W[c0:c0 + 4096]))
+                            for c0 in range(0, K, 4096)])
+    check_scores(s.cpu().numpy(), s_ref)
+    ws = None
+    for rho in (0.5, 0.7, 0.9):
+        k = rmm.keep_count(rho, K)
+        idx = torch.empty(k, dtype=torch.int32, device=DEV)
+        C, ws = rmm.matmul_reduced(X, W, rho, idx_out=idx, workspace=ws)
+        rmm.check(ws)
+        _check_selection_exact(s, idx, k)
+        check_selection(idx.cpu().numpy(), s_ref, k)
+        rows, cols = _rows_cols(M, N, 128, 512, k)
+        ii = idx.long()
+        A_sub = f64(X[torch.as_tensor(rows, device=DEV)])
+        B_sub = f64(W[:, torch.as_tensor(cols, device=DEV)])
+        check_product(f64(C[torch.as_tensor(rows, device=DEV)][:, torch.as_tensor(cols, device=DEV)]),
+                      A_sub, B_sub, idx.cpu().numpy(), 1e-2)
+    del X, W, ws
+    torch.cuda.empty_cache()

@@ -1,0 +1,198 @@
+"""GPU parity: every stage of the CUDA path (through the C ABI) against the fp64
+oracle, on seeded inputs at sizes the oracle finishes in seconds that still
+span several tiles and ragged tails, plus the edge cases of the method."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import rmm_oracle as O
+from input_adaptive_reduced_02_b200 import inputs, rmm
+
+from _parity import (check_product, check_scores, check_selection, check_single, f64, product_tol)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _ab(M, K, N, dtype, seed, outlier=True):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    A = torch.randn(M, K, generator=g, device=DEV)
+    B = torch.randn(K, N, generator=g, device=DEV)
+    if outlier:
+        A *= torch.exp(torch.randn(K, generator=g, device=DEV))[None, :]
+        B *= torch.exp(torch.randn(K, generator=g, device=DEV))[:, None]
+    return A.to(dtype).contiguous(), B.to(dtype).contiguous()
+
+
+SHAPES = [
+    (300, 1000, 520),   # ragged M and N tiles, k_pad > k_keep
+    (129, 257, 257),    # one row / column past a tile, odd K (scalar score and pack paths)
+    (200, 300, 100),    # N <= 128: 128-wide tensor-core tiles
+    (1, 40, 1),         # single row / column
+    (5, 7, 3),          # K < 32
+    (257, 64, 517),     # N not a multiple of 4: direct-store epilogue
+    (384, 512, 768),    # exact tiles
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_stages_match_oracle(shape, dtype):
+    M, K, N = shape
+    A, B = _ab(M, K, N, dtype, seed=M * 7 + K)
+    A64, B64 = f64(A), f64(B)
+    for mode in ("product", "a_only"):
+        s = rmm.score(A, B, mode)
+        check_scores(s.cpu().numpy(), O.slice_scores(A64, B64, mode))
+        for rho in (0.3, 0.5, 1.0):
+            k = O.keep_count(rho, K)
+            assert rmm.keep_count(rho, K) == k
+            idx = rmm.select(s, k)
+            # integer stage: bit-exact against the oracle's selection on the same f32 scores
+            assert idx.cpu().numpy().tolist() == O.select_top(s.cpu().numpy(), k).tolist()
+            A_S, B_St = rmm.pack(A, B, idx)
+            kp = rmm.padded_keep(k)
+            ii = idx.long()
+            assert torch.equal(A_S[:, :k], A[:, ii]) and torch.equal(B_St[:, :k], B[ii, :].t())
+            assert not A_S[:, k:].any() and not B_St[:, k:].any()
+            assert A_S.shape == (M, kp) and B_St.shape == (N, kp)
+            for out_dtype in (torch.float32, torch.bfloat16):
+                C = rmm.gemm(A_S, B_St, k, out_dtype)
+                torch.cuda.synchronize()
+                check_product(f64(C), A64, B64, idx.cpu().numpy(), product_tol(dtype, out_dtype))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("rho", [0.3, 0.5, 0.7, 1.0])
+def test_fused_matmul_reduced(dtype, rho):
+    A, B = _ab(300, 1000, 520, dtype, seed=11)
+    k = rmm.keep_count(rho, 1000)
+    idx = torch.empty(k, dtype=torch.int32, device=DEV)
+    C, ws = rmm.matmul_reduced(A, B, rho, "product", torch.float32, idx_out=idx)
+    rmm.check(ws)
+    check_single(A, B, rho, "product", C, idx)
+
+
+def test_config_f32_64x256x64_end_to_end():
+    A, B = inputs.lognormal_slices_f32(64, 256, 64, seed=0, device=DEV)
+    idx = torch.empty(128, dtype=torch.int32, device=DEV)
+    C, ws = rmm.matmul_reduced(A, B, 0.5, "product", torch.float32, idx_out=idx)
+    rmm.check(ws)
+    nb, err = check_single(A, B, 0.5, "product", C, idx)
+    assert err <= 1e-5
+
+
+def test_batched_qk_small():
+    Q, Km = inputs.attention_qk(bh=3, S=300, d=128, seed=1, device=DEV)
+    Q = Q[:, :200].contiguous()  # S_q != S_k
+    k = rmm.keep_count(0.5, 128)
+    idx = torch.empty(3, k, dtype=torch.int32, device=DEV)
+    S, ws = rmm.qk_reduced(Q, Km, 0.5, out_dtype=torch.float32, idx_out=idx)
+    rmm.check(ws)
+    for h in range(3):
+        check_single(Q[h], Km[h], 0.5, "product", S[h], idx[h], b_kmajor=True)
+    S16, _ = rmm.qk_reduced(Q, Km, 0.5, out_dtype=torch.bfloat16, workspace=ws)
+    for h in range(3):
+        check_product(f64(S16[h]), f64(Q[h]), f64(Km[h]).T, idx[h].cpu().numpy(), 1e-2)
+
+
+def test_batched_pv_small():
+    P, V = inputs.attention_pv(bh=2, S=700, d=128, seed=2, device=DEV)
+    for rho in (0.3, 0.5, 0.7):
+        k = rmm.keep_count(rho, 700)
+        idx = torch.empty(2, k, dtype=torch.int32, device=DEV)
+        Oo, ws = rmm.pv_reduced(P, V, rho, idx_out=idx)
+        rmm.check(ws)
+        for h in range(2):
+            check_single(P[h], V[h], rho, "product", Oo[h], idx[h])
+
+
+def test_ties_go_to_lower_index_and_zero_slices_last():
+    # duplicated columns give exactly equal f32 scores on both sides
+    g = torch.Generator(device=DEV)
+    g.manual_seed(5)
+    base = torch.randn(70, 9, generator=g, device=DEV)
+    A = base[:, torch.arange(90, device=DEV) % 9].contiguous()  # 10 copies of each of 9 columns
+    A[:, 3::17] = 0.0                                            # some zero columns
+    B = torch.ones(90, 33, device=DEV)
+    A, B = A.to(torch.bfloat16), B.to(torch.bfloat16)
+    s = rmm.score(A, B)
+    s_ref = O.slice_scores(f64(A), f64(B))
+    check_scores(s.cpu().numpy(), s_ref)
+    for rho in (0.1, 0.35, 0.5, 0.9, 0.99):
+        k = O.keep_count(rho, 90)
+        idx = rmm.select(s, k)
+        # exact ties in both precisions: the selections must be identical
+        assert idx.cpu().numpy().tolist() == O.select_top(s_ref, k).tolist()
+
+
+def test_extreme_keep_counts():
+    A, B = _ab(100, 300, 90, torch.bfloat16, seed=21)
+    for rho in (1e-9, 1.0):
+        k = rmm.keep_count(rho, 300)
+        assert k == (1 if rho < 1 else 300)
+        idx = torch.empty(k, dtype=torch.int32, device=DEV)
+        C, ws = rmm.matmul_reduced(A, B, rho, idx_out=idx)
+        rmm.check(ws)
+        check_single(A, B, rho, "product", C, idx)
+
+
+def test_empty_rows_still_select():
+    A = torch.zeros(0, 50, dtype=torch.bfloat16, device=DEV)
+    B = torch.randn(50, 20, device=DEV).to(torch.bfloat16)
+    idx = torch.full((25,), -1, dtype=torch.int32, device=DEV)
+    C, ws = rmm.matmul_reduced(A, B, 0.5, idx_out=idx)
+    rmm.check(ws)
+    assert C.shape == (0, 20)
+    # every score is 0, so the tie rule keeps the lowest 25 indices
+    assert idx.cpu().tolist() == list(range(25))
+
+
+def test_determinism_bit_identical():
+    A, B = _ab(300, 1000, 520, torch.bfloat16, seed=31)
+    outs = []
+    for _ in range(2):
+        s = rmm.score(A, B)
+        idx = rmm.select(s, 500)
+        C, _ = rmm.matmul_reduced(A, B, 0.5)
+        outs.append((s.clone(), idx.clone(), C.clone()))
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
+
+
+def test_strided_inputs():
+    # rows of A and B taken from wider buffers (ld > cols)
+    A0, B0 = _ab(130, 600, 300, torch.bfloat16, seed=41)
+    A = A0[:, :512]
+    B = B0[:512, :264]
+    assert A.stride(0) == 600 and B.stride(0) == 300
+    idx = torch.empty(rmm.keep_count(0.5, 512), dtype=torch.int32, device=DEV)
+    C, ws = rmm.matmul_reduced(A, B, 0.5, idx_out=idx)
+    rmm.check(ws)
+    check_single(A.contiguous(), B.contiguous(), 0.5, "product", C, idx)
+
+
+def test_nonfinite_is_reported():
+    A, B = _ab(64, 128, 64, torch.bfloat16, seed=51)
+    A[3, 17] = float("nan")
+    C, ws = rmm.matmul_reduced(A, B, 0.5)
+    with pytest.raises(rmm.RMMError) as e:
+        rmm.check(ws)
+    assert e.value.status == rmm.RMM_ERR_NONFINITE
+    # the status word was cleared; a clean call reports OK
+    A[3, 17] = 0.0
+    rmm.matmul_reduced(A, B, 0.5, workspace=ws)
+    rmm.check(ws)
+
+
+def test_launch_counter_counts_kernels():
+    A, B = _ab(64, 128, 64, torch.bfloat16, seed=61)
+    n0 = rmm.launch_count()
+    rmm.matmul_reduced(A, B, 0.5)
+    torch.cuda.synchronize()
+    # score (B rows, A columns), select, pack (A, B), gemm
+    assert rmm.launch_count() - n0 == 6
