@@ -185,6 +185,35 @@ rmm_status rmm_pv_reduced(const void* P, const void* V, int64_t bh, int64_t S_q,
                           void* O, rmm_dtype out, int32_t* idx_out,
                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Allocation-free form of rmm_matmul_reduced (the paper has no counterpart:
+ * this is a deployment convenience of this library).
+ * For callers that must not allocate device memory — for example code running
+ * under another framework's memory pool or allocator hooks, a plugin that is
+ * handed only its input and output buffers, or a process whose device memory
+ * is reserved in full up front. Arguments are those of rmm_matmul_reduced
+ * minus the workspace; the scratch (status word, scores, indices, packed
+ * operands) comes from one static device array of 32 MiB that this library
+ * defines. Every device on which the call has run keeps that array until the
+ * process exits (with eager module loading, every device that loads the
+ * library does).
+ *   - Products whose rmm_workspace_size(1, M, K, N, k, in) exceeds 32 MiB
+ *     (33554432 bytes) are rejected with RMM_ERR_INVALID before any launch.
+ *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     the status word in it is cleared at the start of each call. Calls whose
+ *     work overlaps on the GPU (different streams, or other threads) race on
+ *     the array: serialise them.
+ *   - status_word: nullable device u32 that receives a copy of this call's
+ *     device status bits, in stream order; read it with rmm_check. */
+rmm_status rmm_matmul_reduced_noalloc(const void* A, int64_t lda, const void* B, int64_t ldb,
+                                      int64_t M, int64_t K, int64_t N, double rho,
+                                      rmm_dtype in, rmm_score_mode mode,
+                                      void* C, int64_t ldc, rmm_dtype out, int32_t* idx_out,
+                                      uint32_t* status_word, cudaStream_t stream);
+
 /* ---------------------------------------------------------------- diagnostics */
 
 /* Synchronises `stream`, reads the status word at `status_word` (a workspace

@@ -32,6 +32,8 @@ static rmm_status fail(rmm_status s, const char* fmt, ...) {
   return s;
 }
 
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
 static rmm_status cuda_fail(cudaError_t e, const char* what, const char* why = nullptr) {
   return fail(RMM_ERR_CUDA, "%s: %s%s%s", what, cudaGetErrorString(e), why ? " — " : "", why ? why : "");
 }

@@ -21,6 +21,8 @@ struct MatView {
 };
 
 void count_launch();
+// Sets the message rmm_last_error_string() returns on the calling thread.
+void set_last_error(const char* msg);
 
 // score.cu
 //  Column sums of squares of X (rows × cols, per batch item), combined per

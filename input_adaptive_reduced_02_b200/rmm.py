@@ -53,6 +53,8 @@ _SIGS = {
                               ctypes.c_size_t, _vp]),
     "rmm_pv_reduced": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _f64, _i32, _i32, _vp, _i32, _vp, _vp,
                               ctypes.c_size_t, _vp]),
+    "rmm_matmul_reduced_noalloc": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _i64, _f64, _i32, _i32, _vp, _i64, _i32,
+                                          _vp, _vp, _vp]),
     "rmm_check": (_i32, [_vp, _vp]),
     "rmm_last_error_string": (ctypes.c_char_p, []),
     "rmm_set_wait_limit_ns": (None, [_u64]),
@@ -312,3 +314,20 @@ def set_stall_producer_for_test(on: bool):
 
 def launch_count() -> int:
     return int(lib().rmm_launch_count())
+
+
+def matmul_reduced_noalloc(A: torch.Tensor, B: torch.Tensor, rho: float, mode: str = "product",
+                           out_dtype=torch.float32, out: torch.Tensor | None = None,
+                           idx_out: torch.Tensor | None = None, status: torch.Tensor | None = None):
+    """C ≈ A·B like matmul_reduced, but with the library's static 32 MiB device
+    scratch instead of a workspace, for callers that must not allocate device
+    memory (only C is allocated here, and only when `out` is None)."""
+    _, M, K, lda, _ = _mat(A, "A")
+    _, r, N, ldb, _ = _mat(B, "B")
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=A.device)
+    _, _, _, ldc, _ = _mat(out, "C")
+    _check(lib().rmm_matmul_reduced_noalloc(_ptr(A), lda, _ptr(B), ldb, M, K, N, float(rho), _dtype(A),
+                                            SCORE_MODES[mode], _ptr(out), ldc, _out_code(out.dtype), _ptr(idx_out),
+                                            _ptr(status), _stream(A)))
+    return out
