@@ -74,10 +74,15 @@ int64_t rmm_keep_count(double rho, int64_t K);
  * K-depth of one tensor-core pipeline stage. Padding columns hold zeros. */
 int64_t rmm_padded_keep(int64_t k_keep);
 
+/* Row pitch, in elements, of the packed N-major B operand: N rounded up to 8
+ * (so that every row starts on a 16-byte boundary). */
+int64_t rmm_packed_b_ld(int64_t N);
+
 /* Bytes of workspace rmm_matmul_reduced / _batched / rmm_qk_reduced /
  * rmm_pv_reduced need for these sizes (in = input dtype). The workspace holds,
  * each 1 KiB-aligned: the status word, scores [batch][K] f32, kept indices
- * [batch][k_keep] i32, A_S [batch][M][k_pad] and B_St [batch][N][k_pad]. */
+ * [batch][k_keep] i32, A_S [batch][M][k_pad] and the packed B operand
+ * (room for [batch][k_pad][rmm_packed_b_ld(N)]). */
 size_t rmm_workspace_size(int64_t batch, int64_t M, int64_t K, int64_t N, int64_t k_keep,
                           rmm_dtype in);
 
@@ -104,38 +109,43 @@ rmm_status rmm_score(const void* A, int64_t lda, int64_t strideA,
  *   s: [batch][K] f32 scores; idx: [batch][k_keep] i32 output, ascending.
  *   Ties go to the lower index; -0.0 equals +0.0. Exact: the result depends
  *   only on the order of the scores, never on rounding. 1 <= k_keep <= K.
- *   A NaN score sets RMM_STATUS_BIT_NONFINITE in status_word (nullable). */
+ *   A NaN score sets RMM_STATUS_BIT_NONFINITE in status_word (nullable).
+ *   K is at most 2^21 (RMM_ERR_UNSUPPORTED above; the same limit applies to
+ *   every call that selects). */
 rmm_status rmm_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,
                       uint32_t* status_word, cudaStream_t stream);
 
 /* Pack the kept slices ("Mecanismo Central": A[:, I] and B[I, :]).
  *   A, B as in rmm_score (B is required here); idx: [batch][k_keep] i32 indices
- *   in [0, K) (as produced by rmm_select).
- *   A_S:  [batch][M][k_pad] output, A_S[b][i][t] = A[b][i][idx[b][t]].
- *   B_St: [batch][N][k_pad] output, B_St[b][j][t] = B[b][idx[b][t]][j] — the
- *         kept rows of B stored transposed (contraction dimension contiguous),
- *         the operand layout rmm_gemm consumes.
- *   k_pad = rmm_padded_keep(k_keep); columns t >= k_keep are written as zero.
- *   Copies bits exactly (no arithmetic). Indices outside [0, K) are a caller
- *   error the kernels do not check. */
+ *   in [0, K) (as produced by rmm_select; 16-byte aligned for the fast path).
+ *   A_S: [batch][M][k_pad] output, A_S[b][i][t] = A[b][i][idx[b][t]]
+ *        (contraction dimension contiguous).
+ *   B_S: if b_kmajor == 0: [batch][k_pad][ldbs], ldbs = rmm_packed_b_ld(N),
+ *        B_S[b][t][j] = B[b][idx[b][t]][j] — the kept rows of B as they are;
+ *        if b_kmajor == 1: [batch][N][k_pad], B_S[b][j][t] = Kmat[b][j][idx[b][t]].
+ *   k_pad = rmm_padded_keep(k_keep); slices t >= k_keep (and columns j >= N of
+ *   the row-major form) are written as zero. Copies bits exactly (no
+ *   arithmetic). Indices outside [0, K) are a caller error the kernels do not
+ *   check. status_word (nullable) receives RMM_STATUS_BIT_TIMEOUT if a bounded
+ *   wait for a bulk copy gave up. */
 rmm_status rmm_pack(const void* A, int64_t lda, int64_t strideA,
                     const void* B, int64_t ldb, int64_t strideB, int b_kmajor,
                     int64_t batch, int64_t M, int64_t K, int64_t N,
                     const int32_t* idx, int64_t k_keep, rmm_dtype in,
-                    void* A_S, void* B_St, cudaStream_t stream);
+                    void* A_S, void* B_S, uint32_t* status_word, cudaStream_t stream);
 
-/* Reduced product on packed operands: C[b] = A_S[b] · B_St[b]ᵀ over the k_keep
+/* Reduced product on packed operands: C[b] = A_S[b] · B_S[b] over the k_keep
  * kept slices ("Mecanismo Central"), f32 accumulation.
- *   A_S [batch][M][k_pad], B_St [batch][N][k_pad] as written by rmm_pack
- *   (zero padding columns, 16-byte aligned base pointers).
+ *   A_S, B_S as written by rmm_pack with the same b_kmajor (zero padding,
+ *   16-byte aligned base pointers).
  *   in == RMM_BF16: tcgen05 tensor-core kernel (TMA, TMEM accumulators).
  *   in == RMM_F32: CUDA-core FFMA kernel (f32 products, f32 sums).
  *   C: [batch][M][N] with ld ldc, batch stride strideC, dtype `out`
  *      (RMM_F32 or RMM_BF16, round-to-nearest-even).
  *   status_word (nullable): RMM_STATUS_BIT_TIMEOUT if a pipeline wait gave up
  *   (then C is incomplete). */
-rmm_status rmm_gemm(const void* A_S, const void* B_St, int64_t batch, int64_t M, int64_t N,
-                    int64_t k_keep, rmm_dtype in, void* C, int64_t ldc, int64_t strideC,
+rmm_status rmm_gemm(const void* A_S, const void* B_S, int b_kmajor, int64_t batch, int64_t M,
+                    int64_t N, int64_t k_keep, rmm_dtype in, void* C, int64_t ldc, int64_t strideC,
                     rmm_dtype out, uint32_t* status_word, cudaStream_t stream);
 
 /* ---------------------------------------------------------------- fused calls */
@@ -234,6 +244,13 @@ void rmm_set_wait_limit_ns(uint64_t ns);
  * out; the kernel then records RMM_STATUS_BIT_TIMEOUT, drains, frees its
  * tensor memory and returns. Used to test the timeout path without a fault. */
 void rmm_set_stall_producer_for_test(int on);
+
+/* Tensor-core GEMM variant, process-wide: 2 (default) runs 2-SM MMAs on CTA
+ * pairs (256-row tiles, A and B halves in the two SMs' shared memory); 1 runs
+ * one SM per 128-row tile. Results are identical up to f32 summation order
+ * (both sum the kept slices in ascending order). Returns the previous
+ * setting; values other than 1 and 2 change nothing. */
+int rmm_set_gemm_cta_group(int cta_group);
 
 /* Number of kernels this library has launched in this process. */
 uint64_t rmm_launch_count(void);

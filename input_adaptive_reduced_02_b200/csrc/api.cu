@@ -18,6 +18,7 @@ namespace rmm {
 static std::atomic<uint64_t> g_launches{0};
 static std::atomic<uint64_t> g_wait_limit_ns{0};
 static std::atomic<int> g_stall_producer{0};
+static std::atomic<int> g_cta_group{2};
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -55,6 +56,14 @@ static rmm_status bind_device(cudaStream_t st) {
 
 static inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
+// Row pitch (elements) of the packed N-major B operand.
+static inline int64_t packed_b_ld(int64_t N) { return round_up(N, 8); }
+
+static uint64_t wait_limit() {
+  const uint64_t lim = g_wait_limit_ns.load();
+  return lim ? lim : kDefaultWaitLimitNs;
+}
+
 static bool dtype_ok(rmm_dtype d) { return d == RMM_BF16 || d == RMM_F32; }
 static ElemKind kind(rmm_dtype d) { return d == RMM_BF16 ? kBF16 : kF32; }
 
@@ -68,6 +77,9 @@ static bool layout_ok(int64_t batch, int64_t rows, int64_t cols, int64_t ld, int
 }
 
 constexpr int64_t kMaxGridBatch = 65535;
+// The select kernel's packed 16-bit histogram counters hold up to 2^16 - 1
+// keys per bin and histogram copy (32 copies): 2^21 slices per selection.
+constexpr int64_t kMaxSelectK = int64_t(1) << 21;
 
 struct Workspace {
   uint32_t* status;
@@ -94,7 +106,7 @@ static Workspace carve(void* base, int64_t batch, int64_t M, int64_t K, int64_t 
   w.a_s = reinterpret_cast<void*>(p + off);
   off += al(batch * M * kp * eb);
   w.b_st = reinterpret_cast<void*>(p + off);
-  off += al(batch * N * kp * eb);
+  off += al(batch * packed_b_ld(N) * kp * eb);
   w.bytes = size_t(off);
   return w;
 }
@@ -103,49 +115,38 @@ static Workspace carve(void* base, int64_t batch, int64_t M, int64_t K, int64_t 
 static rmm_status do_score(const void* A, int64_t lda, int64_t sA, const void* B, int64_t ldb, int64_t sB,
                            int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N, rmm_dtype in,
                            rmm_score_mode mode, float* s, uint32_t* status, cudaStream_t st) {
-  const ElemKind e = kind(in);
-  MatView a{A, lda, sA, M, K};
-  cudaError_t ce;
-  if (mode == RMM_SCORE_A_ONLY) {
-    ce = launch_colsq(a, e, batch, s, K, 2, status, st);
-    if (ce != cudaSuccess) return cuda_fail(ce, "score kernel");
-    return RMM_OK;
-  }
-  // s <- ||B[k,:]||^2, then s <- sqrt(||A[:,k]||^2) * sqrt(s)
-  if (b_kmajor) {
-    MatView bt{B, ldb, sB, N, K};
-    ce = launch_colsq(bt, e, batch, s, K, 0, status, st);
-  } else {
-    MatView bm{B, ldb, sB, K, N};
-    ce = launch_rowsq(bm, e, batch, s, K, st);
-  }
-  if (ce != cudaSuccess) return cuda_fail(ce, "score kernel (B norms)");
-  ce = launch_colsq(a, e, batch, s, K, 1, status, st);
-  if (ce != cudaSuccess) return cuda_fail(ce, "score kernel (A norms)");
+  const MatView a{A, lda, sA, M, K};
+  const int bmode = mode == RMM_SCORE_A_ONLY ? 0 : (b_kmajor ? 2 : 1);
+  const MatView b = b_kmajor ? MatView{B, ldb, sB, N, K} : MatView{B, ldb, sB, K, N};
+  const cudaError_t ce = launch_score(a, b, bmode, kind(in), batch, s, status, st);
+  if (ce != cudaSuccess) return cuda_fail(ce, "score kernel");
   return RMM_OK;
 }
 
 static rmm_status do_pack(const void* A, int64_t lda, int64_t sA, const void* B, int64_t ldb, int64_t sB, int b_kmajor,
                           int64_t batch, int64_t M, int64_t K, int64_t N, const int32_t* idx, int64_t k_keep,
-                          rmm_dtype in, void* A_S, void* B_St, cudaStream_t st) {
+                          rmm_dtype in, void* A_S, void* B_S, uint32_t* status, cudaStream_t st) {
   const ElemKind e = kind(in);
   const int64_t kp = round_up(k_keep, 64);
-  cudaError_t ce = launch_pack_cols(MatView{A, lda, sA, M, K}, e, batch, idx, k_keep, kp, A_S, st);
+  const uint64_t lim = wait_limit();
+  cudaError_t ce = launch_pack_cols(MatView{A, lda, sA, M, K}, e, batch, idx, k_keep, kp, A_S, status, lim, st);
   if (ce != cudaSuccess) return cuda_fail(ce, "pack kernel (A)");
   if (b_kmajor)
-    ce = launch_pack_cols(MatView{B, ldb, sB, N, K}, e, batch, idx, k_keep, kp, B_St, st);
+    ce = launch_pack_cols(MatView{B, ldb, sB, N, K}, e, batch, idx, k_keep, kp, B_S, status, lim, st);
   else
-    ce = launch_pack_rows_t(MatView{B, ldb, sB, K, N}, e, batch, idx, k_keep, kp, B_St, st);
+    ce = launch_pack_rows(MatView{B, ldb, sB, K, N}, e, batch, idx, k_keep, kp, B_S, packed_b_ld(N), status, lim, st);
   if (ce != cudaSuccess) return cuda_fail(ce, "pack kernel (B)");
   return RMM_OK;
 }
 
-static rmm_status do_gemm(const void* A_S, const void* B_St, int64_t batch, int64_t M, int64_t N, int64_t k_keep,
-                          rmm_dtype in, void* C, int64_t ldc, int64_t sC, rmm_dtype out, uint32_t* status,
-                          cudaStream_t st) {
+static rmm_status do_gemm(const void* A_S, const void* B_S, int b_kmajor, int64_t batch, int64_t M, int64_t N,
+                          int64_t k_keep, rmm_dtype in, void* C, int64_t ldc, int64_t sC, rmm_dtype out,
+                          uint32_t* status, cudaStream_t st) {
   GemmArgs g;
   g.a = A_S;
-  g.b = B_St;
+  g.b = B_S;
+  g.b_kmajor = b_kmajor ? 1 : 0;
+  g.ldb = packed_b_ld(N);
   g.c = C;
   g.batch = batch;
   g.M = M;
@@ -155,9 +156,9 @@ static rmm_status do_gemm(const void* A_S, const void* B_St, int64_t batch, int6
   g.strideC = sC;
   g.out = kind(out);
   g.status = status;
-  const uint64_t lim = g_wait_limit_ns.load();
-  g.wait_limit_ns = lim ? lim : kDefaultWaitLimitNs;
+  g.wait_limit_ns = wait_limit();
   g.stall_producer = g_stall_producer.load();
+  g.cta_group = g_cta_group.load();
   cudaError_t ce;
   const char* why = nullptr;
   if (in == RMM_BF16)
@@ -173,6 +174,7 @@ static rmm_status check_common(int64_t batch, int64_t M, int64_t K, int64_t N, r
   if (!dtype_ok(in)) return fail(RMM_ERR_INVALID, "unknown input dtype %d", int(in));
   if (batch < 0 || M < 0 || N < 0) return fail(RMM_ERR_INVALID, "negative size");
   if (K < 1) return fail(RMM_ERR_INVALID, "K must be >= 1 (got %lld)", (long long)K);
+  if (K > kMaxSelectK) return fail(RMM_ERR_UNSUPPORTED, "K > %lld slices per selection", (long long)kMaxSelectK);
   if (batch > kMaxGridBatch) return fail(RMM_ERR_UNSUPPORTED, "batch > %lld", (long long)kMaxGridBatch);
   return RMM_OK;
 }
@@ -228,7 +230,7 @@ rmm_status rmm_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, 
                       cudaStream_t stream) {
   if (batch < 0 || K < 1) return fail(RMM_ERR_INVALID, "need batch >= 0 and K >= 1");
   if (k_keep < 1 || k_keep > K) return fail(RMM_ERR_INVALID, "k_keep must be in [1, K]");
-  if (K > INT32_MAX) return fail(RMM_ERR_UNSUPPORTED, "K > 2^31-1");
+  if (K > kMaxSelectK) return fail(RMM_ERR_UNSUPPORTED, "K > %lld slices per selection", (long long)kMaxSelectK);
   if (batch > kMaxGridBatch) return fail(RMM_ERR_UNSUPPORTED, "batch > %lld", (long long)kMaxGridBatch);
   if (batch == 0) return RMM_OK;
   if (!s || !idx) return fail(RMM_ERR_INVALID, "s or idx is NULL");
@@ -239,9 +241,11 @@ rmm_status rmm_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, 
   return RMM_OK;
 }
 
+int64_t rmm_packed_b_ld(int64_t N) { return N < 0 ? 0 : packed_b_ld(N); }
+
 rmm_status rmm_pack(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb, int64_t strideB,
                     int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N, const int32_t* idx, int64_t k_keep,
-                    rmm_dtype in, void* A_S, void* B_St, cudaStream_t stream) {
+                    rmm_dtype in, void* A_S, void* B_S, uint32_t* status_word, cudaStream_t stream) {
   rmm_status r = check_common(batch, M, K, N, in);
   if (r) return r;
   if (k_keep < 1 || k_keep > K) return fail(RMM_ERR_INVALID, "k_keep must be in [1, K]");
@@ -249,26 +253,27 @@ rmm_status rmm_pack(const void* A, int64_t lda, int64_t strideA, const void* B, 
   if (r) return r;
   if (batch == 0) return RMM_OK;
   if (!idx) return fail(RMM_ERR_INVALID, "idx is NULL");
-  if ((M > 0 && !A_S) || (N > 0 && !B_St)) return fail(RMM_ERR_INVALID, "A_S or B_St is NULL");
-  if ((reinterpret_cast<uintptr_t>(A_S) | reinterpret_cast<uintptr_t>(B_St)) & 15u)
-    return fail(RMM_ERR_INVALID, "A_S and B_St must be 16-byte aligned");
+  if ((M > 0 && !A_S) || !B_S) return fail(RMM_ERR_INVALID, "A_S or B_S is NULL");
+  if ((reinterpret_cast<uintptr_t>(A_S) | reinterpret_cast<uintptr_t>(B_S)) & 15u)
+    return fail(RMM_ERR_INVALID, "A_S and B_S must be 16-byte aligned");
   if ((r = bind_device(stream))) return r;
-  return do_pack(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, idx, k_keep, in, A_S, B_St, stream);
+  return do_pack(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, idx, k_keep, in, A_S, B_S, status_word,
+                 stream);
 }
 
-rmm_status rmm_gemm(const void* A_S, const void* B_St, int64_t batch, int64_t M, int64_t N, int64_t k_keep,
-                    rmm_dtype in, void* C, int64_t ldc, int64_t strideC, rmm_dtype out, uint32_t* status_word,
-                    cudaStream_t stream) {
+rmm_status rmm_gemm(const void* A_S, const void* B_S, int b_kmajor, int64_t batch, int64_t M, int64_t N,
+                    int64_t k_keep, rmm_dtype in, void* C, int64_t ldc, int64_t strideC, rmm_dtype out,
+                    uint32_t* status_word, cudaStream_t stream) {
   if (!dtype_ok(in) || !dtype_ok(out)) return fail(RMM_ERR_INVALID, "unknown dtype");
   if (batch < 0 || M < 0 || N < 0) return fail(RMM_ERR_INVALID, "negative size");
   if (k_keep < 1) return fail(RMM_ERR_INVALID, "k_keep must be >= 1");
   if (batch > kMaxGridBatch) return fail(RMM_ERR_UNSUPPORTED, "batch > %lld", (long long)kMaxGridBatch);
   if (!layout_ok(batch, M, N, ldc, strideC)) return fail(RMM_ERR_INVALID, "C layout (ldc/strideC) is too small");
   if (batch == 0 || M == 0 || N == 0) return RMM_OK;
-  if (!A_S || !B_St || !C) return fail(RMM_ERR_INVALID, "A_S, B_St or C is NULL");
+  if (!A_S || !B_S || !C) return fail(RMM_ERR_INVALID, "A_S, B_S or C is NULL");
   rmm_status r = bind_device(stream);
   if (r) return r;
-  return do_gemm(A_S, B_St, batch, M, N, k_keep, in, C, ldc, strideC, out, status_word, stream);
+  return do_gemm(A_S, B_S, b_kmajor, batch, M, N, k_keep, in, C, ldc, strideC, out, status_word, stream);
 }
 
 rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb,
@@ -302,9 +307,9 @@ rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t stride
   if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
   if (M == 0 || N == 0) return RMM_OK;
   if ((r = do_pack(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, idx, k_keep, in, w.a_s, w.b_st,
-                   stream)))
+                   w.status, stream)))
     return r;
-  return do_gemm(w.a_s, w.b_st, batch, M, N, k_keep, in, C, ldc, strideC, out, w.status, stream);
+  return do_gemm(w.a_s, w.b_st, b_kmajor, batch, M, N, k_keep, in, C, ldc, strideC, out, w.status, stream);
 }
 
 rmm_status rmm_matmul_reduced(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t M, int64_t K, int64_t N,
@@ -350,6 +355,11 @@ const char* rmm_last_error_string(void) { return g_err; }
 void rmm_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
 
 void rmm_set_stall_producer_for_test(int on) { g_stall_producer.store(on ? 1 : 0); }
+
+int rmm_set_gemm_cta_group(int cta_group) {
+  if (cta_group != 1 && cta_group != 2) return g_cta_group.load();
+  return g_cta_group.exchange(cta_group);
+}
 
 uint64_t rmm_launch_count(void) { return g_launches.load(); }
 

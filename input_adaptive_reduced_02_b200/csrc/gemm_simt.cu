@@ -17,16 +17,20 @@ namespace {
 constexpr int ST = 64;   // output tile edge
 constexpr int SK = 16;   // K slice
 
+// B is K-major ([N][k_pad]) when b_kmajor, else N-major ([k_pad][ldb]).
 __global__ void __launch_bounds__(256)
-gemm_simt_kernel(const float* __restrict__ A, const float* __restrict__ Bt, void* __restrict__ C, int64_t M,
-                 int64_t N, int64_t k_pad, int64_t ldc, int64_t strideC, int out_bf16) {
+gemm_simt_kernel(const float* __restrict__ A, const float* __restrict__ Bp, int b_kmajor, int64_t ldb,
+                 void* __restrict__ C, int64_t M, int64_t N, int64_t k_pad, int64_t ldc, int64_t strideC,
+                 int out_bf16) {
   __shared__ float As[SK][ST + 4];
   __shared__ float Bs[SK][ST + 4];
   const int64_t b = blockIdx.z;
   const int64_t i0 = int64_t(blockIdx.y) * ST, j0 = int64_t(blockIdx.x) * ST;
   const float* Ab = A + b * M * k_pad;
-  const float* Bb = Bt + b * N * k_pad;
+  const float* Bb = Bp + (b_kmajor ? b * N * k_pad : b * k_pad * ldb);
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  pdl_trigger();
+  pdl_wait();
   float acc[4][4];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
@@ -39,9 +43,16 @@ gemm_simt_kernel(const float* __restrict__ A, const float* __restrict__ Bt, void
     for (int q = 0; q < 4; ++q) {
       const int e = threadIdx.x + q * 256;
       const int r = e >> 4, kk = e & 15;
-      const int64_t gi = i0 + r, gj = j0 + r;
+      const int64_t gi = i0 + r;
       As[kk][r] = gi < M ? Ab[gi * k_pad + k0 + kk] : 0.f;
-      Bs[kk][r] = gj < N ? Bb[gj * k_pad + k0 + kk] : 0.f;
+      if (b_kmajor) {
+        const int64_t gj = j0 + r;
+        Bs[kk][r] = gj < N ? Bb[gj * k_pad + k0 + kk] : 0.f;
+      } else {
+        const int kr = e >> 6, jc = e & 63;  // N fastest for coalescing
+        const int64_t gj = j0 + jc;
+        Bs[kr][jc] = gj < N ? Bb[(k0 + kr) * ldb + gj] : 0.f;
+      }
     }
     __syncthreads();
 #pragma unroll
@@ -83,10 +94,9 @@ gemm_simt_kernel(const float* __restrict__ A, const float* __restrict__ Bt, void
 cudaError_t launch_gemm_simt(const GemmArgs& g, cudaStream_t st) {
   if (g.batch == 0 || g.M == 0 || g.N == 0) return cudaSuccess;
   dim3 grid(unsigned((g.N + ST - 1) / ST), unsigned((g.M + ST - 1) / ST), unsigned(g.batch));
-  count_launch();
-  gemm_simt_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(g.a), static_cast<const float*>(g.b), g.c, g.M,
-                                         g.N, g.k_pad, g.ldc, g.strideC, g.out == kBF16);
-  return cudaGetLastError();
+  return launch_pdl(gemm_simt_kernel, grid, dim3(256), 0, st, dim3(0, 0, 0), static_cast<const float*>(g.a),
+                    static_cast<const float*>(g.b), g.b_kmajor, g.ldb, g.c, g.M, g.N, g.k_pad, g.ldc, g.strideC,
+                    int(g.out == kBF16));
 }
 
 }  // namespace rmm

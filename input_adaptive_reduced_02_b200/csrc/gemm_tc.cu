@@ -1,26 +1,33 @@
 // Reduced product on the B200 tensor cores ("Mecanismo Central" on the
 // gist.science summary of "Reduced Matrix Multiplication: Input-Adaptive
 // Matrix-Product Reduction for LLM Inference": C = A[:, I]·B[I, :], here on
-// the packed operands A_S [M][k_pad] and B_St [N][k_pad], both K-major).
+// the packed operands: A_S [M][k_pad] K-major; B either K-major B_St [N][k_pad]
+// (Q·Kᵀ, where B is given as Kmat) or N-major B_S [k_pad][N], the kept rows
+// of B as they are).
 //
-// Persistent, warp-specialised tcgen05 kernel, one CTA per SM:
-//   warp 0      TMA producer: 128x64 A tile + BNx64 B tile per stage into a
-//               STAGES-deep shared-memory ring (128-byte swizzle, no multicast)
-//   warp 1      allocates tensor memory; one lane issues tcgen05.mma
-//               (kind::f16, bf16 x bf16 -> f32, M=128, N=BN, K=16) into one of
-//               two TMEM accumulators, and tcgen05.commit frees ring stages
+// Persistent, warp-specialised tcgen05 kernel; by default CTA pairs run 2-SM
+// MMAs (cta_group::2): a pair owns a 256 x BN output tile, each CTA holds 128
+// rows of A and BN/2 columns of B in shared memory and 128 x BN accumulators in
+// its tensor memory, and the even (leader) CTA issues the MMAs for both.
+// Per CTA:
+//   warp 0      TMA producer: 128x64 A tile + (BN/CG)x64 B tile per stage into
+//               a shared-memory ring (128-byte swizzle, no multicast); both
+//               CTAs' loads complete on the leader's stage barrier
+//   warp 1      allocates tensor memory; in the leader one lane issues
+//               tcgen05.mma (kind::f16, bf16 x bf16 -> f32, K = 16) into one of
+//               two TMEM accumulators and commits ring stages back to both CTAs
 //   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, optional bf16
 //               rounding, swizzled staging in shared memory, TMA tile store
-// The two accumulators let the epilogue of tile i overlap the mainloop of
-// tile i+1. Tiles are visited m-fastest so a column block of B is shared
-// through L2 by the CTAs working on it at the same time.
+// Two accumulators let the epilogue of tile i overlap the mainloop of tile
+// i+1. Tiles are visited m-fastest so a column block of B is shared through
+// L2 by the pairs working on it at the same time.
 //
 // Every mbarrier wait is bounded (rmm_set_wait_limit_ns). A role whose wait
-// runs out records RMM_STATUS_BIT_TIMEOUT, raises a shared abort flag that
-// the other roles poll, and winds down: the producer waits for its own TMA
-// loads still in flight, the MMA lane waits for its issued MMAs, the
-// epilogue waits for its TMA stores, and warp 1 frees tensor memory. No
-// thread leaves before the final CTA barrier.
+// runs out records RMM_STATUS_BIT_TIMEOUT, raises its CTA's abort flag, and
+// winds down: the producer waits for its own TMA loads still in flight, the
+// MMA lane waits for its issued MMAs, the epilogue waits for its TMA stores,
+// and warp 1 frees tensor memory after a final CTA (and cluster) barrier. No
+// thread leaves before that barrier.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -32,26 +39,28 @@
 namespace rmm {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
+constexpr int BM = 128;  // rows of A per CTA
+constexpr int BK = 64;   // 64 bf16 = one 128-byte swizzle row
 constexpr int kUmmaK = 16;
 constexpr int kEpiWarps = 4;
 constexpr int kTcThreads = 64 + 32 * kEpiWarps;
 
-template <int BN>
+template <int BN, int CG>
 struct TcCfg {
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int BN_CTA = BN / CG;  // columns of B held by one CTA
   static constexpr uint32_t A_BYTES = BM * BK * 2;
-  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t B_BYTES = BN_CTA * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = int((192u * 1024u) / STAGE_BYTES);
   static constexpr uint32_t EPI_BUF = 32 * 128;  // 32 rows x 128 bytes
   static constexpr uint32_t EPI_BYTES = kEpiWarps * 2 * EPI_BUF;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
   static constexpr uint32_t BAR_BYTES = 256;
   static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
 };
-static_assert(TcCfg<256>::SMEM <= 232448, "shared memory budget");
-static_assert(TcCfg<128>::SMEM <= 232448, "shared memory budget");
+static_assert(TcCfg<256, 1>::SMEM <= 232448 && TcCfg<128, 1>::SMEM <= 232448, "shared memory budget");
+static_assert(TcCfg<256, 2>::SMEM <= 232448 && TcCfg<128, 2>::SMEM <= 232448, "shared memory budget");
+static_assert(TcCfg<128, 2>::STAGES * 2 + 6 <= 32, "barrier area");
 
 struct TcParams {
   int32_t M, N, num_kb, tiles_m, tiles_n;
@@ -65,6 +74,7 @@ struct TcParams {
   int64_t ldc, strideC;
 };
 
+// Tile t -> (batch item, m block of BM*CG rows, n block of BN columns), m fastest.
 __device__ __forceinline__ void decode_tile(int64_t t, const TcParams& p, int32_t& b, int32_t& mb, int32_t& nb) {
   const int64_t per = int64_t(p.tiles_m) * p.tiles_n;
   b = int32_t(t / per);
@@ -78,12 +88,13 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t* 
   status_or(status, RMM_TIMEOUT_BIT);
 }
 
-template <int BN>
+template <int BN, bool BMN, int CG>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, const TcParams p) {
-  using Cfg = TcCfg<BN>;
+  using Cfg = TcCfg<BN, CG>;
   constexpr int STAGES = Cfg::STAGES;
+  constexpr int BN_CTA = Cfg::BN_CTA;
   extern __shared__ uint8_t tc_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -92,7 +103,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + Cfg::EPI_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;   // [2] accumulator ready for the epilogue
-  uint64_t* tempty = tfull + 2;       // [2] accumulator drained by the epilogue
+  uint64_t* tempty = tfull + 2;       // [2] accumulator drained by the epilogue(s)
   uint64_t* drain = tempty + 2;       // MMA completion at wind-down
   uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(drain + 1);
   int* abort_sh = reinterpret_cast<int*>(tmem_base_sh + 1);
@@ -100,6 +111,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;  // 0 = leader
+  const int64_t pair = blockIdx.x / CG;
+  const int64_t npairs = gridDim.x / CG;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -108,7 +122,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], kEpiWarps);
+      mbar_init(&tempty[a], kEpiWarps * CG);
     }
     mbar_init(drain, 1);
     *abort_sh = 0;
@@ -121,108 +135,133 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (p.tma_store) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_base_sh, Cfg::TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc<CG>(tmem_base_sh, Cfg::TMEM_COLS);
+    tmem_relinquish<CG>();
   }
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync_all();  // the peer's barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_sh;
+  pdl_wait();  // set-up above overlaps the previous kernel's tail
   volatile int* abort_v = abort_sh;
   const volatile int* never_v = never_sh;
   const uint64_t limit = p.wait_limit_ns;
+  const uint32_t peer = rank ^ 1u;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    uint32_t stage = 0, phase = 0;
-    uint32_t issued = 0;         // bit s: stage s has a load issued
-    uint32_t issued_par = 0;     // bit s: parity of stage s's last issued load
-    bool ok = true;
-    for (int64_t t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
-      int32_t b, mb, nb;
-      decode_tile(t, p, b, mb, nb);
-      for (int kb = 0; kb < p.num_kb; ++kb) {
-        int w = 1;
-        if (lane == 0) w = mbar_wait_bounded(&empty[stage], phase ^ 1u, limit, abort_v);
-        w = __shfl_sync(0xffffffffu, w, 0);
-        if (!w) {
-          ok = false;
-          break;
-        }
-        if (lane == 0 && !p.stall_producer) {
-          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
-          tma_load_3d(sA + stage * Cfg::A_BYTES, &tmA, &full[stage], kb * BK, mb * BM, b);
-          tma_load_3d(sB + stage * Cfg::B_BYTES, &tmB, &full[stage], kb * BK, nb * BN, b);
-          issued |= 1u << stage;
-          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-        }
-        __syncwarp();
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
+    // ------------------------------------------------------------ TMA producer (one lane)
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued = 0;      // bit s: this CTA loaded stage s
+      uint32_t issued_par = 0;  // bit s: parity of that stage's last phase
+      bool ok = true;
+      for (int64_t t = pair; ok && t < p.total_tiles; t += npairs) {
+        int32_t b, mb, nb;
+        decode_tile(t, p, b, mb, nb);
+        const int32_t m_row = mb * BM * CG + int32_t(rank) * BM;
+        const int32_t n_col = nb * BN + int32_t(rank) * BN_CTA;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, limit, abort_v)) {
+            ok = false;
+            break;
+          }
+          if (!p.stall_producer) {
+            uint8_t* a_dst = sA + stage * Cfg::A_BYTES;
+            uint8_t* b_dst = sB + stage * Cfg::B_BYTES;
+            if constexpr (CG == 1) {
+              mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+              tma_load_3d(a_dst, &tmA, &full[stage], kb * BK, m_row, b);
+              if constexpr (BMN) {
+#pragma unroll
+                for (int j = 0; j < BN_CTA / 64; ++j)
+                  tma_load_3d(b_dst + j * 8192, &tmB, &full[stage], n_col + j * 64, kb * BK, b);
+              } else {
+                tma_load_3d(b_dst, &tmB, &full[stage], kb * BK, n_col, b);
+              }
+            } else {
+              // both CTAs' bytes complete on the leader's barrier; the leader arms it
+              if (rank == 0) mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES * CG);
+              const uint32_t bar = mapa_shared(smem_addr(&full[stage]), 0);
+              tma_load_3d_pair(a_dst, &tmA, bar, kb * BK, m_row, b);
+              if constexpr (BMN) {
+#pragma unroll
+                for (int j = 0; j < BN_CTA / 64; ++j)
+                  tma_load_3d_pair(b_dst + j * 8192, &tmB, bar, n_col + j * 64, kb * BK, b);
+              } else {
+                tma_load_3d_pair(b_dst, &tmB, bar, kb * BK, n_col, b);
+              }
+            }
+            issued |= 1u << stage;
+            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
-    }
-    if (!ok && lane == 0) raise_abort(abort_v, p.status);
-    // Loads complete on their own; make sure none is still writing shared
-    // memory when the CTA exits.
-    if (lane == 0) {
-      for (int s = 0; s < STAGES; ++s)
-        if (issued & (1u << s)) mbar_wait_bounded(&full[s], (issued_par >> s) & 1u, limit, never_v);
+      if (!ok) raise_abort(abort_v, p.status);
+      // Loads complete on their own; make sure none is still writing shared
+      // memory when the CTA exits. The leader waits on its stage barriers
+      // (which also count the peer's bytes); the peer's loads land on the
+      // leader's barriers, so on an abort it gives them time to land.
+      if (CG == 1 || rank == 0) {
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) mbar_wait_bounded(&full[s], (issued_par >> s) & 1u, limit, never_v);
+      } else if (!ok && issued) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000ull) __nanosleep(1000);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc = umma_idesc_bf16_f32(BM, BN);
-    uint32_t stage = 0, phase = 0;
-    uint32_t acc = 0, acc_phase = 0;
-    bool ok = true;
-    for (int64_t t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
-      int w = 1;
-      if (lane == 0) w = mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, limit, abort_v);
-      w = __shfl_sync(0xffffffffu, w, 0);
-      if (!w) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * BN;
-      for (int kb = 0; kb < p.num_kb; ++kb) {
-        w = 1;
-        if (lane == 0) w = mbar_wait_bounded(&full[stage], phase, limit, abort_v);
-        w = __shfl_sync(0xffffffffu, w, 0);
-        if (!w) {
+    // ------------------------------------------------------------ MMA issuer (one lane of the leader)
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(BM * CG, BN, BMN);
+      uint32_t stage = 0, phase = 0;
+      uint32_t acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int64_t t = pair; ok && t < p.total_tiles; t += npairs) {
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, limit, abort_v)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (lane == 0) {
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, limit, abort_v)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           const uint32_t a0 = smem_addr(sA + stage * Cfg::A_BYTES);
           const uint32_t b0 = smem_addr(sB + stage * Cfg::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / kUmmaK; ++kk) {
-            // advancing K by 16 elements = 32 bytes inside the swizzled row
-            umma_bf16(d_tmem, umma_desc_k_sw128(a0 + kk * 32), umma_desc_k_sw128(b0 + kk * 32), idesc,
-                      (kb | kk) != 0);
+            // K-major: 16 elements = 32 bytes along the swizzled row;
+            // N-major: 16 K-rows of 128 bytes
+            const uint64_t bdesc = BMN ? umma_desc_mn_sw128(b0 + kk * 2048, 8192) : umma_desc_k_sw128(b0 + kk * 32);
+            umma_bf16<CG>(d_tmem, umma_desc_k_sw128(a0 + kk * 32), bdesc, idesc, (kb | kk) != 0);
           }
-          umma_commit(&empty[stage]);
+          // this stage's smem is free in both CTAs once these MMAs are done
+          umma_commit<CG>(smem_addr(&empty[stage]));
+          if constexpr (CG == 2) umma_commit<CG>(mapa_shared(smem_addr(&empty[stage]), peer));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        __syncwarp();
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        if (!ok) break;
+        umma_commit<CG>(smem_addr(&tfull[acc]));
+        if constexpr (CG == 2) umma_commit<CG>(mapa_shared(smem_addr(&tfull[acc]), peer));
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
       }
-      if (!ok) break;
-      if (lane == 0) umma_commit(&tfull[acc]);
-      __syncwarp();
-      acc ^= 1u;
-      if (acc == 0) acc_phase ^= 1u;
-    }
-    if (!ok && lane == 0) raise_abort(abort_v, p.status);
-    // Wait for every MMA this lane issued before tensor memory is freed.
-    if (lane == 0) {
-      umma_commit(drain);
+      if (!ok) raise_abort(abort_v, p.status);
+      // Wait for every MMA this lane issued before tensor memory is freed.
+      umma_commit<CG>(smem_addr(drain));
       mbar_wait_bounded(drain, 0, limit, never_v);
     }
     __syncwarp();
@@ -234,7 +273,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     bool ok = true;
     const int cols_per_chunk = p.out_bf16 ? 64 : 32;
     const int chunks = BN / cols_per_chunk;
-    for (int64_t t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
+    for (int64_t t = pair; ok && t < p.total_tiles; t += npairs) {
       int32_t b, mb, nb;
       decode_tile(t, p, b, mb, nb);
       int w = 1;
@@ -246,7 +285,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
       tc_fence_after();
       const uint32_t t_row = tmem_base + (uint32_t(q * 32) << 16) + acc * BN;
-      const int32_t row0 = mb * BM + q * 32;
+      const int32_t row0 = mb * BM * CG + int32_t(rank) * BM + q * 32;
       for (int c = 0; c < chunks; ++c) {
         uint32_t packed[32];
         if (p.out_bf16) {
@@ -264,10 +303,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           tmem_ld_wait();
         }
         if (c == chunks - 1) {
-          // whole accumulator read: hand it back to the MMA warp
+          // whole accumulator read: hand it back to the leader's MMA lane
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[acc]);
+          if (lane == 0) {
+            if (CG == 1 || rank == 0)
+              mbar_arrive(&tempty[acc]);
+            else
+              mbar_arrive_cluster(mapa_shared(smem_addr(&tempty[acc]), 0));
+          }
         }
         const int32_t col0 = nb * BN + c * cols_per_chunk;
         if (p.tma_store) {
@@ -317,8 +361,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync_all();  // the pair is done with each other's barriers and TMEM
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  if (warp == 1) tmem_dealloc<CG>(tmem_base, Cfg::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------ host side
@@ -354,6 +399,12 @@ struct DevInfo {
   bool attr_done = false;
 };
 
+template <int BN, bool BMN, int CG>
+void set_attr() {
+  cudaFuncSetAttribute(gemm_tc_kernel<BN, BMN, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       int(TcCfg<BN, CG>::SMEM));
+}
+
 DevInfo& dev_info(int dev) {
   static DevInfo info[64];
   static std::mutex mu;
@@ -364,22 +415,36 @@ DevInfo& dev_info(int dev) {
     cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
     if (d.cc_major == 10 && d.cc_minor == 0) {
-      cudaFuncSetAttribute(gemm_tc_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(TcCfg<256>::SMEM));
-      cudaFuncSetAttribute(gemm_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(TcCfg<128>::SMEM));
+      set_attr<256, false, 1>();
+      set_attr<128, false, 1>();
+      set_attr<256, true, 1>();
+      set_attr<128, true, 1>();
+      set_attr<256, false, 2>();
+      set_attr<128, false, 2>();
+      set_attr<256, true, 2>();
+      set_attr<128, true, 2>();
     }
     d.attr_done = true;
   }
   return d;
 }
 
-template <int BN>
-cudaError_t launch_bn(const GemmArgs& g, const DevInfo& di, cudaStream_t st, const char** why) {
+template <int BN, bool BMN, int CG>
+cudaError_t launch_cfg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, const char** why) {
+  using Cfg = TcCfg<BN, CG>;
   const uint64_t kp = uint64_t(g.k_pad);
   CUtensorMap tmA, tmB, tmC;
-  if (!encode_3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.a, kp, uint64_t(g.M), uint64_t(g.batch), kp * 2,
-                 kp * 2 * uint64_t(g.M), BK, BM) ||
-      !encode_3d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.b, kp, uint64_t(g.N), uint64_t(g.batch), kp * 2,
-                 kp * 2 * uint64_t(g.N), BK, BN)) {
+  bool ok = encode_3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.a, kp, uint64_t(g.M), uint64_t(g.batch), kp * 2,
+                      kp * 2 * uint64_t(g.M), BK, BM);
+  if (BMN) {
+    const uint64_t ldb = uint64_t(g.ldb);
+    ok = ok && encode_3d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.b, uint64_t(g.N), kp, uint64_t(g.batch), ldb * 2,
+                         ldb * 2 * kp, 64, BK);
+  } else {
+    ok = ok && encode_3d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.b, kp, uint64_t(g.N), uint64_t(g.batch), kp * 2,
+                         kp * 2 * uint64_t(g.N), BK, Cfg::BN_CTA);
+  }
+  if (!ok) {
     *why = "cuTensorMapEncodeTiled failed for a packed operand";
     return cudaErrorInvalidValue;
   }
@@ -401,7 +466,7 @@ cudaError_t launch_bn(const GemmArgs& g, const DevInfo& di, cudaStream_t st, con
   p.M = int32_t(g.M);
   p.N = int32_t(g.N);
   p.num_kb = int32_t(g.k_pad / BK);
-  p.tiles_m = int32_t((g.M + BM - 1) / BM);
+  p.tiles_m = int32_t((g.M + BM * CG - 1) / (BM * CG));
   p.tiles_n = int32_t((g.N + BN - 1) / BN);
   p.total_tiles = int64_t(p.tiles_m) * p.tiles_n * g.batch;
   p.status = g.status;
@@ -412,10 +477,17 @@ cudaError_t launch_bn(const GemmArgs& g, const DevInfo& di, cudaStream_t st, con
   p.c = g.c;
   p.ldc = g.ldc;
   p.strideC = g.strideC;
-  const int64_t grid = std::min<int64_t>(p.total_tiles, di.sms > 0 ? di.sms : 148);
-  count_launch();
-  gemm_tc_kernel<BN><<<unsigned(grid), kTcThreads, TcCfg<BN>::SMEM, st>>>(tmA, tmB, tmC, p);
-  return cudaGetLastError();
+  const int64_t units = std::max<int64_t>(1, (di.sms > 0 ? di.sms : 148) / CG);
+  const int64_t grid = CG * std::min<int64_t>(p.total_tiles, units);
+  return launch_pdl(gemm_tc_kernel<BN, BMN, CG>, dim3(unsigned(grid)), dim3(kTcThreads), Cfg::SMEM, st,
+                    CG == 2 ? dim3(2, 1, 1) : dim3(0, 0, 0), tmA, tmB, tmC, p);
+}
+
+template <int CG>
+cudaError_t launch_cg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, const char** why) {
+  if (g.b_kmajor)
+    return g.N <= 128 ? launch_cfg<128, false, CG>(g, di, st, why) : launch_cfg<256, false, CG>(g, di, st, why);
+  return g.N <= 128 ? launch_cfg<128, true, CG>(g, di, st, why) : launch_cfg<256, true, CG>(g, di, st, why);
 }
 
 }  // namespace
@@ -438,7 +510,11 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st, const char** why)
     *why = "a dimension exceeds 2^31-1";
     return cudaErrorInvalidValue;
   }
-  return g.N <= 128 ? launch_bn<128>(g, di, st, why) : launch_bn<256>(g, di, st, why);
+  if (!g.b_kmajor && (uint64_t(g.ldb) * 2) % 16 != 0) {
+    *why = "the packed N-major B operand needs a row pitch that is a multiple of 8 elements";
+    return cudaErrorInvalidValue;
+  }
+  return g.cta_group == 1 ? launch_cg<1>(g, di, st, why) : launch_cg<2>(g, di, st, why);
 }
 
 }  // namespace rmm

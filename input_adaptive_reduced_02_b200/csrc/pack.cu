@@ -2,17 +2,18 @@
 // summary of "Reduced Matrix Multiplication: Input-Adaptive Matrix-Product
 // Reduction for LLM Inference": the reduced product is A[:, I]·B[I, :]).
 //
-// Both packed operands are written K-major (the kept slice index t is the
-// contiguous dimension), zero-padded to k_pad = ceil(k/64)·64, which is the
-// layout the tensor-core GEMM's TMA loads consume with 128-byte swizzle:
 //  * pack_cols: out[r][t] = X[r][idx[t]] — column compaction of a row-major
-//    matrix (A, or Kmat for Q·Kᵀ). Kept columns are spread over every 32-byte
-//    sector, so a CTA streams whole rows into shared memory with 16-byte loads
-//    and gathers from there; the packed rows leave as 16-byte stores.
-//  * pack_rows_t: out[n][t] = X[idx[t]][n] — gather of kept rows of a
-//    row-major B, transposed through a padded shared-memory tile so that both
-//    the row reads and the packed writes are whole 128-byte lines.
-// Pure bit copies; no arithmetic.
+//    matrix (A; Kmat for Q·Kᵀ). Kept columns are spread over every 32-byte
+//    sector, so whole rows are staged in shared memory by bulk-async (TMA)
+//    copies, one thread issuing all of a CTA's row copies at once; the CTA
+//    then gathers through idx and writes 16-byte vectors. Padding columns
+//    k <= t < k_pad are written as zeros. Output is K-major, the layout the
+//    tensor-core GEMM reads for A (and for B when B is given as Kmat).
+//  * pack_rows: out[t][:] = X[idx[t]][:] — the kept rows of a row-major B,
+//    copied as whole rows: bulk-async loads into shared memory, bulk-async
+//    stores back out, no register traffic. Padding rows are zeros. The GEMM
+//    reads this operand N-major.
+// Pure bit copies. Rows that are not 16-byte aligned take plain-load paths.
 #include <algorithm>
 
 #include "rmm_device.cuh"
@@ -22,14 +23,8 @@ namespace rmm {
 namespace {
 
 constexpr int kPackThreads = 256;
-
-__device__ __forceinline__ uint4 ld_stream16(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
+constexpr size_t kStageBytes = 32 * 1024;   // shared-memory rows per CTA (short rows)
+constexpr size_t kStageMax = 112 * 1024;    // one long row per CTA, two CTAs per SM
 
 template <typename T>
 union Vec16 {
@@ -37,46 +32,133 @@ union Vec16 {
   T e[16 / sizeof(T)];
 };
 
-// rows_per_cta rows of X staged in shared memory, then gathered.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_addr(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(gdst), "r"(smem_addr(smem_src)), "r"(bytes)
+               : "memory");
+}
+
+// Wait for this CTA's bulk loads; every thread polls, bounded. On a timeout the
+// status bit is set and the CTA waits once more (also bounded) so that no copy
+// is still writing shared memory when it exits.
+__device__ __forceinline__ bool wait_loads(uint64_t* bar, uint64_t limit_ns, uint32_t* status, int* never) {
+  if (mbar_wait_bounded(bar, 0, limit_ns, never)) return true;
+  if (threadIdx.x == 0) status_or(status, RMM_TIMEOUT_BIT);
+  mbar_wait_bounded(bar, 0, limit_ns, never);
+  return false;
+}
+
 template <typename T>
-__global__ void __launch_bounds__(kPackThreads)
-pack_cols_smem_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t R, int64_t C,
-                      const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
-                      int rows_per_cta, int vec_ok) {
+__device__ __forceinline__ void gather_rows(const T* srow, int nr, int64_t C, const int32_t* __restrict__ ib,
+                                            int64_t k_keep, int64_t k_pad, T* dst) {
   constexpr int V = 16 / sizeof(T);
-  extern __shared__ __align__(16) unsigned char pack_smem[];
-  T* srow = reinterpret_cast<T*>(pack_smem);
-  const int64_t b = blockIdx.y;
-  const int64_t r0 = int64_t(blockIdx.x) * rows_per_cta;
-  if (r0 >= R) return;
-  const int nr = int(min(int64_t(rows_per_cta), R - r0));
-  const T* src = X + b * bstride + r0 * ld;
-  const int32_t* ib = idx + b * k_keep;
-  T* dst = out + (b * R + r0) * k_pad;
-
-  if (vec_ok) {  // C % V == 0 and rows 16-byte aligned
-    const int64_t nvr = C / V;
-    for (int rr = 0; rr < nr; ++rr) {
-      const uint4* s4 = reinterpret_cast<const uint4*>(src + rr * ld);
-      uint4* d4 = reinterpret_cast<uint4*>(srow + rr * C);
-      for (int64_t v = threadIdx.x; v < nvr; v += kPackThreads) d4[v] = ld_stream16(s4 + v);
-    }
-  } else {
-    for (int rr = 0; rr < nr; ++rr)
-      for (int64_t c = threadIdx.x; c < C; c += kPackThreads) srow[rr * C + c] = src[rr * ld + c];
-  }
-  __syncthreads();
-
   const int64_t ng = k_pad / V;
   for (int rr = 0; rr < nr; ++rr) {
     const T* row = srow + rr * C;
     for (int64_t g = threadIdx.x; g < ng; g += kPackThreads) {
       const int64_t t0 = g * V;
       Vec16<T> v;
+      if (t0 + V <= k_keep) {
+        const int4 i0 = __ldg(reinterpret_cast<const int4*>(ib + t0));
+        if constexpr (V == 8) {
+          const int4 i1 = __ldg(reinterpret_cast<const int4*>(ib + t0 + 4));
+          v.e[0] = row[i0.x]; v.e[1] = row[i0.y]; v.e[2] = row[i0.z]; v.e[3] = row[i0.w];
+          v.e[4] = row[i1.x]; v.e[5] = row[i1.y]; v.e[6] = row[i1.z]; v.e[7] = row[i1.w];
+        } else {
+          v.e[0] = row[i0.x]; v.e[1] = row[i0.y]; v.e[2] = row[i0.z]; v.e[3] = row[i0.w];
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          const int64_t t = t0 + j;
+          v.e[j] = t < k_keep ? row[__ldg(ib + t)] : T(0);
+        }
+      }
+      reinterpret_cast<uint4*>(dst + rr * k_pad)[g] = v.u;
+    }
+  }
+}
+
+// Rows staged by bulk-async copies (rows 16-byte aligned, C·e a multiple of 16;
+// idx 16-byte aligned so that it can be read four at a time).
+template <typename T>
+__global__ void __launch_bounds__(kPackThreads)
+pack_cols_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t R, int64_t C,
+                      const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
+                      int rows_per_cta, uint32_t* status, uint64_t wait_ns) {
+  extern __shared__ __align__(128) unsigned char pack_smem[];
+  __shared__ uint64_t bar;
+  __shared__ int never;
+  T* srow = reinterpret_cast<T*>(pack_smem);
+  const int64_t b = blockIdx.y;
+  const int64_t r0 = int64_t(blockIdx.x) * rows_per_cta;
+  const int nr = int(min(int64_t(rows_per_cta), R - r0));
+  const T* src = X + b * bstride + r0 * ld;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    never = 0;
+    fence_mbar_init();
+  }
+  pdl_trigger();
+  pdl_wait();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t row_bytes = uint32_t(C * sizeof(T));
+    mbar_arrive_expect_tx(&bar, row_bytes * uint32_t(nr));
+    for (int rr = 0; rr < nr; ++rr) bulk_load(srow + rr * C, src + rr * ld, row_bytes, &bar);
+  }
+  wait_loads(&bar, wait_ns, status, &never);
+  gather_rows(srow, nr, C, idx + b * k_keep, k_keep, k_pad, out + (b * R + r0) * k_pad);
+}
+
+// Any alignment: rows staged with plain loads (eight in flight per thread).
+template <typename T>
+__global__ void __launch_bounds__(kPackThreads)
+pack_cols_plain_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t R, int64_t C,
+                       const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
+                       int rows_per_cta) {
+  constexpr int V = 16 / sizeof(T);
+  extern __shared__ __align__(128) unsigned char pack_smem[];
+  T* srow = reinterpret_cast<T*>(pack_smem);
+  const int64_t b = blockIdx.y;
+  const int64_t r0 = int64_t(blockIdx.x) * rows_per_cta;
+  const int nr = int(min(int64_t(rows_per_cta), R - r0));
+  const T* src = X + b * bstride + r0 * ld;
+  pdl_trigger();
+  pdl_wait();
+  for (int rr = 0; rr < nr; ++rr) {
+    for (int64_t c0 = threadIdx.x; c0 < C; c0 += kPackThreads * 8) {
+      T v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t c = c0 + int64_t(j) * kPackThreads;
+        v[j] = c < C ? src[rr * ld + c] : T(0);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t c = c0 + int64_t(j) * kPackThreads;
+        if (c < C) srow[rr * C + c] = v[j];
+      }
+    }
+  }
+  __syncthreads();
+  const int32_t* ib = idx + b * k_keep;
+  T* dst = out + (b * R + r0) * k_pad;
+  for (int rr = 0; rr < nr; ++rr) {
+    const T* row = srow + rr * C;
+    for (int64_t g = threadIdx.x; g < k_pad / V; g += kPackThreads) {
+      Vec16<T> v;
 #pragma unroll
       for (int j = 0; j < V; ++j) {
-        const int64_t t = t0 + j;
-        v.e[j] = t < k_keep ? row[__ldg(ib + t)] : T(0);
+        const int64_t t = g * V + j;
+        v.e[j] = t < k_keep ? row[ib[t]] : T(0);
       }
       reinterpret_cast<uint4*>(dst + rr * k_pad)[g] = v.u;
     }
@@ -91,136 +173,165 @@ pack_cols_direct_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, in
   constexpr int V = 16 / sizeof(T);
   const int64_t b = blockIdx.y;
   const int64_t r = blockIdx.x;
-  if (r >= R) return;
   const T* row = X + b * bstride + r * ld;
   const int32_t* ib = idx + b * k_keep;
   T* dst = out + (b * R + r) * k_pad;
+  pdl_trigger();
+  pdl_wait();
   for (int64_t g = threadIdx.x; g < k_pad / V; g += kPackThreads) {
     Vec16<T> v;
 #pragma unroll
     for (int j = 0; j < V; ++j) {
       const int64_t t = g * V + j;
-      v.e[j] = t < k_keep ? row[__ldg(ib + t)] : T(0);
+      v.e[j] = t < k_keep ? row[ib[t]] : T(0);
     }
     reinterpret_cast<uint4*>(dst)[g] = v.u;
   }
 }
 
-// 64 kept rows x 64 columns per CTA, transposed through shared memory.
+// Kept rows of B (N·e a multiple of 16, rows 16-byte aligned): bulk-async row
+// copies through shared memory. CTA x covers kept rows [x·rows, (x+1)·rows).
 template <typename T>
 __global__ void __launch_bounds__(kPackThreads)
-pack_rows_t_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t N,
-                   const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out, int vec_ok) {
-  constexpr int V = 16 / sizeof(T);
-  constexpr int TT = 64;      // kept rows (t) per tile
-  constexpr int TN = 64;      // columns (n) per tile
-  constexpr int P = TN + V;   // padded pitch, keeps rows 16-byte aligned
-  __shared__ __align__(16) T tile[TT][P];
-  const int64_t b = blockIdx.z;
-  const int64_t t0 = int64_t(blockIdx.x) * TT;
-  const int64_t n0 = int64_t(blockIdx.y) * TN;
-  const T* src = X + b * bstride;
-  const int32_t* ib = idx + b * k_keep;
-
-  constexpr int TPR = TN / V;           // threads per tile row
-  constexpr int RPP = kPackThreads / TPR;
-  const int cq = threadIdx.x % TPR, rq = threadIdx.x / TPR;
-  for (int tt = rq; tt < TT; tt += RPP) {
-    const int64_t t = t0 + tt;
-    const int64_t n = n0 + int64_t(cq) * V;
-    Vec16<T> v;
-    v.u = make_uint4(0u, 0u, 0u, 0u);
-    if (t < k_keep) {
-      const T* p = src + int64_t(__ldg(ib + t)) * ld + n;
-      if (vec_ok && n + V <= N) {
-        v.u = ld_stream16(p);
-      } else {
-#pragma unroll
-        for (int j = 0; j < V; ++j) v.e[j] = (n + j < N) ? p[j] : T(0);
-      }
-    }
-    *reinterpret_cast<uint4*>(&tile[tt][cq * V]) = v.u;
+pack_rows_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t N,
+                      const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
+                      int64_t ldo, int rows_per_cta, uint32_t* status, uint64_t wait_ns) {
+  extern __shared__ __align__(128) unsigned char pack_smem[];
+  __shared__ uint64_t bar;
+  __shared__ int never;
+  T* srow = reinterpret_cast<T*>(pack_smem);
+  const int64_t b = blockIdx.y;
+  const int64_t t0 = int64_t(blockIdx.x) * rows_per_cta;
+  const int nr = int(min(int64_t(rows_per_cta), k_pad - t0));
+  const int nload = int(max(int64_t(0), min(int64_t(nr), k_keep - t0)));  // kept rows in this CTA
+  const uint32_t row_bytes = uint32_t(N * sizeof(T));
+  T* dst = out + (b * k_pad + t0) * ldo;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    never = 0;
+    fence_mbar_init();
   }
+  pdl_trigger();
+  pdl_wait();
   __syncthreads();
-
-  constexpr int TPO = TT / V;           // threads per packed output row
-  constexpr int OPP = kPackThreads / TPO;
-  const int oq = threadIdx.x % TPO, orow = threadIdx.x / TPO;
-  for (int nn = orow; nn < TN; nn += OPP) {
-    const int64_t n = n0 + nn;
-    if (n >= N) break;
-    Vec16<T> v;
-#pragma unroll
-    for (int j = 0; j < V; ++j) v.e[j] = tile[oq * V + j][nn];
-    *reinterpret_cast<uint4*>(out + (b * N + n) * k_pad + t0 + oq * V) = v.u;
+  if (threadIdx.x == 0 && nload > 0) {
+    const int32_t* ib = idx + b * k_keep + t0;
+    const T* src = X + b * bstride;
+    mbar_arrive_expect_tx(&bar, row_bytes * uint32_t(nload));
+    for (int rr = 0; rr < nload; ++rr) bulk_load(srow + rr * N, src + int64_t(__ldg(ib + rr)) * ld, row_bytes, &bar);
   }
+  // padding rows (t >= k_keep) are zeros; padding columns N <= c < ldo too
+  for (int rr = nload; rr < nr; ++rr)
+    for (int64_t c = threadIdx.x; c < ldo; c += kPackThreads) dst[rr * ldo + c] = T(0);
+  if (ldo > N)
+    for (int rr = 0; rr < nload; ++rr)
+      for (int64_t c = N + threadIdx.x; c < ldo; c += kPackThreads) dst[rr * ldo + c] = T(0);
+  if (nload > 0) {
+    wait_loads(&bar, wait_ns, status, &never);
+    if (threadIdx.x == 0) {
+      for (int rr = 0; rr < nload; ++rr) bulk_store(dst + rr * ldo, srow + rr * N, row_bytes);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // smem stays live until read
+    }
+  }
+}
+
+// Kept rows of B, any alignment: plain element copies.
+template <typename T>
+__global__ void __launch_bounds__(kPackThreads)
+pack_rows_plain_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t N,
+                       const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
+                       int64_t ldo) {
+  const int64_t b = blockIdx.y;
+  const int64_t t = blockIdx.x;
+  T* dst = out + (b * k_pad + t) * ldo;
+  pdl_trigger();
+  pdl_wait();
+  if (t >= k_keep) {
+    for (int64_t c = threadIdx.x; c < ldo; c += kPackThreads) dst[c] = T(0);
+    return;
+  }
+  const T* src = X + b * bstride + int64_t(idx[b * k_keep + t]) * ld;
+  for (int64_t c = threadIdx.x; c < ldo; c += kPackThreads) dst[c] = c < N ? src[c] : T(0);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-constexpr size_t kPackSmemRowsBudget = 32 * 1024;   // several short rows per CTA
-constexpr size_t kPackSmemMax = 112 * 1024;         // one long row per CTA, 2 CTAs/SM
-
-template <typename T>
-cudaError_t launch_pack_cols_t(const MatView& X, int64_t batch, const int32_t* idx, int64_t k_keep,
-                               int64_t k_pad, void* out, cudaStream_t st) {
-  constexpr int V = 16 / sizeof(T);
-  const size_t row_bytes = size_t(X.cols) * sizeof(T);
-  const T* p = static_cast<const T*>(X.ptr);
-  T* o = static_cast<T*>(out);
-  if (row_bytes > kPackSmemMax) {
-    dim3 grid(unsigned(X.rows), unsigned(batch), 1);
-    count_launch();
-    pack_cols_direct_kernel<T><<<grid, kPackThreads, 0, st>>>(p, X.ld, X.bstride, X.rows, idx, k_keep, k_pad, o);
-    return cudaGetLastError();
-  }
-  int rows_per_cta = 1;
-  if (row_bytes <= kPackSmemRowsBudget) rows_per_cta = int(std::min<size_t>(8, kPackSmemRowsBudget / std::max<size_t>(row_bytes, 1)));
-  const size_t smem = size_t(rows_per_cta) * row_bytes;
-  const int vec_ok = aligned16(X.ptr) && X.cols % V == 0 && (X.ld * int64_t(sizeof(T))) % 16 == 0 &&
-                     (batch == 1 || (X.bstride * int64_t(sizeof(T))) % 16 == 0);
-  static bool attr_done[64] = {};
+template <typename K>
+void set_smem_attr_once(K kernel) {
+  static bool done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(pack_cols_smem_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(kPackSmemMax));
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
+  if (dev >= 0 && dev < 64 && !done[dev]) {
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kStageMax));
+    done[dev] = true;
   }
-  dim3 grid(unsigned((X.rows + rows_per_cta - 1) / rows_per_cta), unsigned(batch), 1);
-  count_launch();
-  pack_cols_smem_kernel<T><<<grid, kPackThreads, smem, st>>>(p, X.ld, X.bstride, X.rows, X.cols, idx, k_keep, k_pad,
-                                                             o, rows_per_cta, vec_ok);
-  return cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t launch_pack_rows_t_t(const MatView& X, int64_t batch, const int32_t* idx, int64_t k_keep, int64_t k_pad,
-                                 void* out, cudaStream_t st) {
-  const int vec_ok = aligned16(X.ptr) && (X.ld * int64_t(sizeof(T))) % 16 == 0 &&
-                     (batch == 1 || (X.bstride * int64_t(sizeof(T))) % 16 == 0);
-  dim3 grid(unsigned(k_pad / 64), unsigned((X.cols + 63) / 64), unsigned(batch));
-  count_launch();
-  pack_rows_t_kernel<T><<<grid, kPackThreads, 0, st>>>(static_cast<const T*>(X.ptr), X.ld, X.bstride, X.cols, idx,
-                                                        k_keep, k_pad, static_cast<T*>(out), vec_ok);
-  return cudaGetLastError();
+cudaError_t launch_pack_cols_t(const MatView& X, int64_t batch, const int32_t* idx, int64_t k_keep, int64_t k_pad,
+                               void* out, uint32_t* status, uint64_t wait_ns, cudaStream_t st) {
+  const size_t row_bytes = size_t(X.cols) * sizeof(T);
+  const T* p = static_cast<const T*>(X.ptr);
+  T* o = static_cast<T*>(out);
+  if (row_bytes > kStageMax) {
+    return launch_pdl(pack_cols_direct_kernel<T>, dim3(unsigned(X.rows), unsigned(batch)), dim3(kPackThreads), 0, st,
+                      dim3(0, 0, 0), p, X.ld, X.bstride, X.rows, idx, k_keep, k_pad, o);
+  }
+  const int rows_per_cta =
+      row_bytes <= kStageBytes ? int(std::min<size_t>(64, kStageBytes / std::max<size_t>(row_bytes, 1))) : 1;
+  const size_t smem = size_t(rows_per_cta) * row_bytes;
+  const dim3 grid(unsigned((X.rows + rows_per_cta - 1) / rows_per_cta), unsigned(batch), 1u);
+  const bool bulk = aligned16(X.ptr) && row_bytes % 16 == 0 && (X.ld * int64_t(sizeof(T))) % 16 == 0 &&
+                    (batch == 1 || (X.bstride * int64_t(sizeof(T))) % 16 == 0) && aligned16(idx) &&
+                    (batch == 1 || k_keep % 4 == 0);
+  if (bulk) {
+    set_smem_attr_once(pack_cols_bulk_kernel<T>);
+    return launch_pdl(pack_cols_bulk_kernel<T>, grid, dim3(kPackThreads), smem, st, dim3(0, 0, 0), p, X.ld, X.bstride, X.rows,
+                      X.cols, idx, k_keep, k_pad, o, rows_per_cta, status, wait_ns);
+  }
+  set_smem_attr_once(pack_cols_plain_kernel<T>);
+  return launch_pdl(pack_cols_plain_kernel<T>, grid, dim3(kPackThreads), smem, st, dim3(0, 0, 0), p, X.ld, X.bstride, X.rows,
+                    X.cols, idx, k_keep, k_pad, o, rows_per_cta);
+}
+
+template <typename T>
+cudaError_t launch_pack_rows_t(const MatView& X, int64_t batch, const int32_t* idx, int64_t k_keep, int64_t k_pad,
+                               void* out, int64_t ldo, uint32_t* status, uint64_t wait_ns, cudaStream_t st) {
+  const size_t row_bytes = size_t(X.cols) * sizeof(T);
+  const T* p = static_cast<const T*>(X.ptr);
+  T* o = static_cast<T*>(out);
+  const bool bulk = row_bytes > 0 && row_bytes % 16 == 0 && row_bytes <= kStageMax && aligned16(X.ptr) &&
+                    aligned16(out) && (X.ld * int64_t(sizeof(T))) % 16 == 0 &&
+                    (batch == 1 || (X.bstride * int64_t(sizeof(T))) % 16 == 0) && (ldo * int64_t(sizeof(T))) % 16 == 0;
+  if (bulk) {
+    const int rows_per_cta =
+        row_bytes <= kStageBytes ? int(std::min<size_t>(64, kStageBytes / row_bytes)) : 1;
+    const size_t smem = size_t(rows_per_cta) * row_bytes;
+    set_smem_attr_once(pack_rows_bulk_kernel<T>);
+    const dim3 grid(unsigned((k_pad + rows_per_cta - 1) / rows_per_cta), unsigned(batch), 1u);
+    return launch_pdl(pack_rows_bulk_kernel<T>, grid, dim3(kPackThreads), smem, st, dim3(0, 0, 0), p, X.ld, X.bstride, X.cols, idx,
+                      k_keep, k_pad, o, ldo, rows_per_cta, status, wait_ns);
+  }
+  return launch_pdl(pack_rows_plain_kernel<T>, dim3(unsigned(k_pad), unsigned(batch)), dim3(kPackThreads), 0, st, dim3(0, 0, 0),
+                    p, X.ld, X.bstride, X.cols, idx, k_keep, k_pad, o, ldo);
 }
 
 }  // namespace
 
 cudaError_t launch_pack_cols(const MatView& X, ElemKind e, int64_t batch, const int32_t* idx, int64_t k_keep,
-                             int64_t k_pad, void* out, cudaStream_t st) {
+                             int64_t k_pad, void* out, uint32_t* status, uint64_t wait_ns, cudaStream_t st) {
   if (batch == 0 || X.rows == 0) return cudaSuccess;
-  return e == kBF16 ? launch_pack_cols_t<uint16_t>(X, batch, idx, k_keep, k_pad, out, st)
-                    : launch_pack_cols_t<uint32_t>(X, batch, idx, k_keep, k_pad, out, st);
+  return e == kBF16 ? launch_pack_cols_t<uint16_t>(X, batch, idx, k_keep, k_pad, out, status, wait_ns, st)
+                    : launch_pack_cols_t<uint32_t>(X, batch, idx, k_keep, k_pad, out, status, wait_ns, st);
 }
 
-cudaError_t launch_pack_rows_t(const MatView& X, ElemKind e, int64_t batch, const int32_t* idx, int64_t k_keep,
-                               int64_t k_pad, void* out, cudaStream_t st) {
-  if (batch == 0 || X.cols == 0) return cudaSuccess;
-  return e == kBF16 ? launch_pack_rows_t_t<uint16_t>(X, batch, idx, k_keep, k_pad, out, st)
-                    : launch_pack_rows_t_t<uint32_t>(X, batch, idx, k_keep, k_pad, out, st);
+cudaError_t launch_pack_rows(const MatView& X, ElemKind e, int64_t batch, const int32_t* idx, int64_t k_keep,
+                             int64_t k_pad, void* out, int64_t ldo, uint32_t* status, uint64_t wait_ns,
+                             cudaStream_t st) {
+  if (batch == 0) return cudaSuccess;
+  return e == kBF16 ? launch_pack_rows_t<uint16_t>(X, batch, idx, k_keep, k_pad, out, ldo, status, wait_ns, st)
+                    : launch_pack_rows_t<uint32_t>(X, batch, idx, k_keep, k_pad, out, ldo, status, wait_ns, st);
 }
 
 }  // namespace rmm

@@ -21,18 +21,44 @@ struct MatView {
 };
 
 void count_launch();
+
+// Launch `kernel` on `st` with programmatic stream serialisation (the kernel
+// calls pdl_wait before touching global memory) and, if cluster.x > 0, that
+// thread-block cluster shape.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       dim3 cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster.x > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster.x;
+    attr[n].val.clusterDim.y = cluster.y;
+    attr[n].val.clusterDim.z = cluster.z;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 // Sets the message rmm_last_error_string() returns on the calling thread.
 void set_last_error(const char* msg);
 
 // score.cu
-//  Column sums of squares of X (rows × cols, per batch item), combined per
-//  `finalize`: 0 = store the sum in out; 1 = out = sqrt(sum) * sqrt(out);
-//  2 = out = sqrt(sum).
-cudaError_t launch_colsq(const MatView& X, ElemKind e, int64_t batch, float* out, int64_t out_bstride,
-                         int finalize, uint32_t* status, cudaStream_t st);
-//  Row sums of squares of X stored in out (one per row).
-cudaError_t launch_rowsq(const MatView& X, ElemKind e, int64_t batch, float* out, int64_t out_bstride,
-                         cudaStream_t st);
+//  s[b][k] = sqrt(sum_i A[b][i][k]^2) · (bmode 1: sqrt(sum_j B[b][k][j]^2) with B
+//  row-major [K][N]; bmode 2: sqrt(sum_j B[b][j][k]^2) with B = Kmat [N][K];
+//  bmode 0: 1). One launch.
+cudaError_t launch_score(const MatView& A, const MatView& B, int bmode, ElemKind e, int64_t batch, float* s,
+                         uint32_t* status, cudaStream_t st);
 
 // select.cu
 cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,
@@ -41,22 +67,29 @@ cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_ke
 // pack.cu
 //  out[b][r][t] = X[b][r][idx[b][t]] for t < k_keep, 0 for k_keep <= t < k_pad.
 cudaError_t launch_pack_cols(const MatView& X, ElemKind e, int64_t batch, const int32_t* idx,
-                             int64_t k_keep, int64_t k_pad, void* out, cudaStream_t st);
-//  out[b][n][t] = X[b][idx[b][t]][n] (kept rows, transposed), zero padded to k_pad.
-cudaError_t launch_pack_rows_t(const MatView& X, ElemKind e, int64_t batch, const int32_t* idx,
-                               int64_t k_keep, int64_t k_pad, void* out, cudaStream_t st);
+                             int64_t k_keep, int64_t k_pad, void* out, uint32_t* status, uint64_t wait_ns,
+                             cudaStream_t st);
+//  out[b][t][:] = X[b][idx[b][t]][:] (kept rows, row pitch ldo >= cols, zero
+//  padded to ldo columns and k_pad rows).
+cudaError_t launch_pack_rows(const MatView& X, ElemKind e, int64_t batch, const int32_t* idx,
+                             int64_t k_keep, int64_t k_pad, void* out, int64_t ldo, uint32_t* status,
+                             uint64_t wait_ns, cudaStream_t st);
 
 // gemm_tc.cu (bf16 tensor cores) / gemm_simt.cu (f32 CUDA cores)
 struct GemmArgs {
   const void* a;  // [batch][M][k_pad]
-  const void* b;  // [batch][N][k_pad]
+  const void* b;  // b_kmajor: [batch][N][k_pad]; else [batch][k_pad][ldb]
+  int b_kmajor;
+  int64_t ldb;    // row pitch of the N-major B operand (elements)
   void* c;        // [batch][M][N] (ldc, strideC)
   int64_t batch, M, N, k_pad, ldc, strideC;
   ElemKind out;
   uint32_t* status;
   uint64_t wait_limit_ns;
   int stall_producer;
+  int cta_group;
 };
+//  cta_group: 2 = 2-SM MMAs on CTA pairs (default), 1 = one SM per tile.
 cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st, const char** why);
 cudaError_t launch_gemm_simt(const GemmArgs& g, cudaStream_t st);
 

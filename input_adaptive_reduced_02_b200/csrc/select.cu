@@ -6,10 +6,11 @@
 // One 1024-thread CTA per batch item. Scores become order-preserving 32-bit
 // keys in shared memory (up to 32768 of them; larger K re-reads the scores
 // from global memory, which stays in L2). A 4-pass MSB-first radix select
-// (8-bit digits) finds the exact key T of the k-th largest score and how many
-// keys equal to T must be kept; per-warp histograms with match-any
-// aggregation avoid hot-bin atomic contention. Two block-wide scans then
-// compact the kept indices in index order. Integer work only: the result
+// (8-bit digits; per-warp histograms built from ballot-based peer masks, one
+// leader lane per digit, no atomics) finds the digit
+// string of the k-th largest score, stopping early once the threshold bin is
+// kept whole, and how many keys equal to it must be kept. Two block-wide
+// scans then compact the kept indices in index order. Integer work only: the result
 // depends on the order of the scores, never on rounding.
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
@@ -17,8 +18,6 @@
 namespace rmm {
 namespace {
 
-constexpr int kSelThreads = 1024;
-constexpr int kSelWarps = kSelThreads / 32;
 constexpr int64_t kSelSmemKeys = 32768;
 
 // Order-preserving map from f32 to u32 (larger score -> larger key), with
@@ -30,7 +29,9 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 }
 
 // Exclusive scan of one value per thread over the block; *total receives the sum.
+template <int THREADS>
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
+  constexpr int kWarps = THREADS / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
 #pragma unroll
@@ -41,132 +42,156 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   if (lane == 31) warp_sums[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    uint32_t w = warp_sums[lane];
+    uint32_t w = lane < kWarps ? warp_sums[lane] : 0u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += y;
     }
-    warp_sums[lane] = w;
+    if (lane < kWarps) warp_sums[lane] = w;
   }
   __syncthreads();
   const uint32_t before = (warp ? warp_sums[warp - 1] : 0u) + x - v;
-  *total = warp_sums[kSelWarps - 1];
+  *total = warp_sums[kWarps - 1];
   __syncthreads();
   return before;
 }
 
-__global__ void __launch_bounds__(kSelThreads, 1)
-select_kernel(const float* __restrict__ s, int64_t K, int64_t k_keep, int32_t* __restrict__ idx,
-              uint32_t* status, int keys_in_smem) {
-  extern __shared__ uint32_t keys[];
-  __shared__ uint32_t hist[kSelWarps][256];
+constexpr int kSelThreads = 1024;
+constexpr int kBins = 2048;  // 11-bit digits: passes cover bits 31-21, 20-10, 9-0
+
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS, 1)
+select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t* __restrict__ idx,
+              uint32_t* status, int keys_in_smem, int hist_copies) {
+  const int K = int(K64);  // K < 2^31 (checked on the host)
+  // dynamic shared memory: [keys: K words if keys_in_smem][histograms: hist_copies x 1024 words]
+  // Each histogram word packs two 16-bit bin counters (bins 2w and 2w+1); a
+  // copy is shared by THREADS/32/hist_copies warps, so a bin never exceeds
+  // K·hist_warps/32 <= 2^16 - 1 for the sizes the host allows.
+  extern __shared__ uint32_t dyn[];
+  uint32_t* keys = dyn;
+  uint32_t* hist = dyn + (keys_in_smem ? K : 0);
+  __shared__ uint32_t tot[kBins];
   __shared__ uint32_t warp_sums[32];
-  __shared__ uint32_t sh_digit, sh_above;
+  __shared__ uint32_t sh_digit, sh_above, sh_count;
   __shared__ int sh_nan;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const float* sb = s + int64_t(blockIdx.x) * K;
   int32_t* ib = idx + int64_t(blockIdx.x) * k_keep;
+  uint32_t* my_hist = hist + (warp % hist_copies) * (kBins / 2);
 
+  pdl_trigger();
+  pdl_wait();
   if (tid == 0) sh_nan = 0;
   __syncthreads();
   bool nan_seen = false;
-  for (int64_t i = tid; i < K; i += kSelThreads) {
-    const float x = sb[i];
-    nan_seen |= (x != x);
-    if (keys_in_smem) keys[i] = order_key(x);
+  if (keys_in_smem && (K & 3) == 0 && (reinterpret_cast<uintptr_t>(sb) & 15u) == 0) {
+    const float4* s4 = reinterpret_cast<const float4*>(sb);
+    for (int i = tid; i < K / 4; i += THREADS) {
+      const float4 x = s4[i];
+      nan_seen |= (x.x != x.x) | (x.y != x.y) | (x.z != x.z) | (x.w != x.w);
+      reinterpret_cast<uint4*>(keys)[i] = make_uint4(order_key(x.x), order_key(x.y), order_key(x.z), order_key(x.w));
+    }
+  } else {
+    for (int i = tid; i < K; i += THREADS) {
+      const float x = sb[i];
+      nan_seen |= (x != x);
+      if (keys_in_smem) keys[i] = order_key(x);
+    }
   }
   if (nan_seen) sh_nan = 1;
   __syncthreads();
   if (tid == 0 && sh_nan) status_or(status, RMM_NONFINITE_BIT);
 
   if (k_keep >= K) {  // everything is kept
-    for (int64_t i = tid; i < K; i += kSelThreads) ib[i] = int32_t(i);
+    for (int i = tid; i < K; i += THREADS) ib[i] = i;
     return;
   }
 
-  uint32_t prefix = 0, mask = 0, remaining = uint32_t(k_keep);
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < kSelWarps * 256; i += kSelThreads) (&hist[0][0])[i] = 0u;
+  // MSB-first radix select. After each pass, `prefix` (under `mask`) is the
+  // digit string of the k-th largest key so far, `remaining` the number of
+  // keys still to take among those matching it.
+  uint32_t prefix = 0, mask = 0, remaining = uint32_t(k_keep), bin_count = 0;
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
+    for (int w = tid; w < hist_copies * (kBins / 2); w += THREADS) hist[w] = 0u;
     __syncthreads();
-    for (int64_t i0 = int64_t(warp) * 32; i0 < K; i0 += kSelThreads) {
-      const int64_t i = i0 + lane;
-      uint32_t key = 0;
-      bool active = false;
-      if (i < K) {
-        key = keys_in_smem ? keys[i] : order_key(sb[i]);
-        active = (key & mask) == prefix;
-      }
-      const unsigned am = __ballot_sync(0xffffffffu, active);
-      if (active) {
-        const uint32_t d = (key >> shift) & 0xFFu;
-        const unsigned peers = __match_any_sync(am, d);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hist[warp][d], uint32_t(__popc(peers)));
+    for (int i = tid; i < K; i += THREADS) {
+      const uint32_t key = keys_in_smem ? keys[i] : order_key(sb[i]);
+      if ((key & mask) == prefix) {
+        const uint32_t d = (key >> shift) & dmask;
+        atomicAdd(&my_hist[d >> 1], (d & 1u) ? 0x10000u : 1u);
       }
     }
     __syncthreads();
-    if (tid < 256) {
-      uint32_t t = 0;
-      for (int w = 0; w < kSelWarps; ++w) t += hist[w][tid];
-      hist[0][tid] = t;
+    // totals per bin, then a descending scan to find the bin of the k-th key:
+    // thread t owns bins 2047-2t and 2046-2t
+    for (int w = tid; w < kBins / 2; w += THREADS) {
+      uint32_t lo = 0, hi = 0;
+      for (int c = 0; c < hist_copies; ++c) {
+        const uint32_t v = hist[c * (kBins / 2) + w];
+        lo += v & 0xFFFFu;
+        hi += v >> 16;
+      }
+      tot[2 * w] = lo;
+      tot[2 * w + 1] = hi;
     }
     __syncthreads();
-    if (warp == 0) {
-      // lane l owns digits 255-8l .. 248-8l, scanned from the top digit down
-      uint32_t c[8], local = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        c[j] = hist[0][255 - 8 * lane - j];
-        local += c[j];
-      }
-      uint32_t incl = local;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const uint32_t excl = incl - local;
-      if (excl < remaining && remaining <= incl) {
-        uint32_t run = excl;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (run + c[j] >= remaining) {
-            sh_digit = uint32_t(255 - 8 * lane - j);
-            sh_above = run;
-            break;
-          }
-          run += c[j];
-        }
+    uint32_t c0 = 0, c1 = 0;
+    if (tid < kBins / 2) {
+      c0 = tot[kBins - 1 - 2 * tid];
+      c1 = tot[kBins - 2 - 2 * tid];
+    }
+    uint32_t all;
+    const uint32_t excl = block_exclusive_scan<THREADS>(c0 + c1, warp_sums, &all);
+    if (tid < kBins / 2 && excl < remaining && remaining <= excl + c0 + c1) {
+      if (excl + c0 >= remaining) {
+        sh_digit = uint32_t(kBins - 1 - 2 * tid);
+        sh_above = excl;
+        sh_count = c0;
+      } else {
+        sh_digit = uint32_t(kBins - 2 - 2 * tid);
+        sh_above = excl + c0;
+        sh_count = c1;
       }
     }
     __syncthreads();
     prefix |= sh_digit << shift;
-    mask |= 0xFFu << shift;
+    mask |= dmask << shift;
     remaining -= sh_above;
+    bin_count = sh_count;
+    // every key in the chosen bin is kept: no finer threshold is needed
+    if (remaining == bin_count) break;
   }
-  // prefix is now the exact key T of the k-th largest score; `remaining` keys
-  // equal to T are kept (the lowest-indexed ones), plus every key above T.
+  // Kept: keys whose masked digits exceed `prefix`, plus the `remaining`
+  // lowest-indexed keys whose masked digits equal it (all of them when the
+  // bin is taken whole).
   const uint32_t T = prefix, need_eq = remaining;
-  const int64_t per = (K + kSelThreads - 1) / kSelThreads;
-  const int64_t lo = min(K, int64_t(tid) * per), hi = min(K, lo + per);
+  const bool take_all_eq = remaining == bin_count;
+  const int per = (K + THREADS - 1) / THREADS;
+  const int lo = min(K, tid * per), hi = min(K, lo + per);
   uint32_t n_gt = 0, n_eq = 0;
-  for (int64_t i = lo; i < hi; ++i) {
-    const uint32_t k = keys_in_smem ? keys[i] : order_key(sb[i]);
+  for (int i = lo; i < hi; ++i) {
+    const uint32_t k = (keys_in_smem ? keys[i] : order_key(sb[i])) & mask;
     n_gt += (k > T);
     n_eq += (k == T);
   }
-  uint32_t total;
-  const uint32_t eq_before = block_exclusive_scan(n_eq, warp_sums, &total);
-  const uint32_t eq_take = eq_before >= need_eq ? 0u : min(n_eq, need_eq - eq_before);
-  uint32_t pos = block_exclusive_scan(n_gt + eq_take, warp_sums, &total);
+  uint32_t total, eq_take = n_eq;
+  if (!take_all_eq) {
+    const uint32_t eq_before = block_exclusive_scan<THREADS>(n_eq, warp_sums, &total);
+    eq_take = eq_before >= need_eq ? 0u : min(n_eq, need_eq - eq_before);
+  }
+  uint32_t pos = block_exclusive_scan<THREADS>(n_gt + eq_take, warp_sums, &total);
   uint32_t taken_eq = 0;
-  for (int64_t i = lo; i < hi; ++i) {
-    const uint32_t k = keys_in_smem ? keys[i] : order_key(sb[i]);
+  for (int i = lo; i < hi; ++i) {
+    const uint32_t k = (keys_in_smem ? keys[i] : order_key(sb[i])) & mask;
     if (k > T) {
-      ib[pos++] = int32_t(i);
+      ib[pos++] = i;
     } else if (k == T && taken_eq < eq_take) {
-      ib[pos++] = int32_t(i);
+      ib[pos++] = i;
       ++taken_eq;
     }
   }
@@ -178,19 +203,23 @@ cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_ke
                           uint32_t* status, cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
   const int keys_in_smem = K <= kSelSmemKeys;
-  const size_t smem = keys_in_smem ? size_t(K) * 4 : 0;
+  // Histogram copies: one per warp while they fit next to the keys, else one
+  // per two warps (packed 16-bit bins stay below 2^16 for K <= 2^16).
+  const int copies = (K <= 16384 || !keys_in_smem) ? 32 : 16;
+  if (int64_t(copies) * kSelThreads / 32 > 0 && K * (32 / copies) > 65535 * 32)
+    return cudaErrorInvalidValue;
+  const size_t smem = (keys_in_smem ? size_t(K) * 4 : 0) + size_t(copies) * (kBins / 2) * 4;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(kSelSmemKeys * 4));
+    cudaError_t e = cudaFuncSetAttribute(select_kernel<kSelThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(kSelSmemKeys * 4 + 16 * (kBins / 2) * 4));
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-  count_launch();
-  select_kernel<<<unsigned(batch), kSelThreads, smem, st>>>(s, K, k_keep, idx, status, keys_in_smem);
-  return cudaGetLastError();
+  return launch_pdl(select_kernel<kSelThreads>, dim3(unsigned(batch)), dim3(kSelThreads), smem, st, dim3(0, 0, 0), s,
+                    K, k_keep, idx, status, keys_in_smem, copies);
 }
 
 }  // namespace rmm

@@ -38,13 +38,14 @@ _vp, _i64, _f64, _i32, _u64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_double, 
 _SIGS = {
     "rmm_keep_count": (_i64, [_f64, _i64]),
     "rmm_padded_keep": (_i64, [_i64]),
+    "rmm_packed_b_ld": (_i64, [_i64]),
     "rmm_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64, _i64, _i32]),
     "rmm_score": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i32, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp,
                          _vp]),
     "rmm_select": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "rmm_pack": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i32, _i64, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _vp,
-                        _vp]),
-    "rmm_gemm": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _i32, _vp, _i64, _i64, _i32, _vp, _vp]),
+                        _vp, _vp]),
+    "rmm_gemm": (_i32, [_vp, _vp, _i32, _i64, _i64, _i64, _i64, _i32, _vp, _i64, _i64, _i32, _vp, _vp]),
     "rmm_matmul_reduced": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _i64, _f64, _i32, _i32, _vp, _i64, _i32, _vp,
                                   _vp, ctypes.c_size_t, _vp]),
     "rmm_matmul_reduced_batched": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i32, _i64, _i64, _i64, _i64, _f64,
@@ -59,6 +60,7 @@ _SIGS = {
     "rmm_last_error_string": (ctypes.c_char_p, []),
     "rmm_set_wait_limit_ns": (None, [_u64]),
     "rmm_set_stall_producer_for_test": (None, [_i32]),
+    "rmm_set_gemm_cta_group": (_i32, [_i32]),
     "rmm_launch_count": (_u64, []),
 }
 
@@ -215,36 +217,51 @@ def select(s: torch.Tensor, k_keep: int, out: torch.Tensor | None = None,
     return out
 
 
-def pack(A: torch.Tensor, B: torch.Tensor, idx: torch.Tensor, b_kmajor: bool = False, out=None):
-    """A_S [b][M][k_pad] and B_St [b][N][k_pad] (kept slices, contraction dim contiguous, zero padded).
-    `out` may supply the (A_S, B_St) pair."""
+def packed_b_ld(N: int) -> int:
+    return int(lib().rmm_packed_b_ld(int(N)))
+
+
+def packed_b_shape(batched: bool, batch: int, N: int, k_pad: int, b_kmajor: bool):
+    """Shape of the packed B operand: [(b)][N][k_pad] (b_kmajor) or [(b)][k_pad][packed_b_ld(N)]."""
+    shp = (N, k_pad) if b_kmajor else (k_pad, packed_b_ld(N))
+    return (batch, *shp) if batched else shp
+
+
+def pack(A: torch.Tensor, B: torch.Tensor, idx: torch.Tensor, b_kmajor: bool = False, out=None,
+         status: torch.Tensor | None = None):
+    """A_S [b][M][k_pad] (kept columns of A, zero padded) and the packed B
+    operand: the kept rows of B ([b][k_pad][packed_b_ld(N)]) or, with b_kmajor,
+    the kept columns of Kmat ([b][N][k_pad]). `out` may supply the pair."""
     ba, M, K, lda, sA = _mat(A, "A")
     bb, r, c, ldb, sB = _mat(B, "B")
     N = r if b_kmajor else c
     k_keep = idx.shape[-1]
     kp = padded_keep(k_keep)
+    bshape = packed_b_shape(A.dim() == 3, ba, N, kp, b_kmajor)
     if out is None:
-        shp = (lambda rows: (ba, rows, kp)) if A.dim() == 3 else (lambda rows: (rows, kp))
-        A_S = torch.empty(shp(M), dtype=A.dtype, device=A.device)
-        B_St = torch.empty(shp(N), dtype=A.dtype, device=A.device)
+        A_S = torch.empty((ba, M, kp) if A.dim() == 3 else (M, kp), dtype=A.dtype, device=A.device)
+        B_S = torch.empty(bshape, dtype=A.dtype, device=A.device)
     else:
-        A_S, B_St = out
-        if A_S.numel() != ba * M * kp or B_St.numel() != ba * N * kp:
+        A_S, B_S = out
+        if A_S.numel() != ba * M * kp or B_S.numel() != int(torch.tensor(bshape).prod()):
             raise ValueError("pack: output buffers have the wrong size")
     _check(lib().rmm_pack(_ptr(A), lda, sA, _ptr(B), ldb, sB, int(b_kmajor), ba, M, K, N, _ptr(idx), k_keep,
-                          _dtype(A), _ptr(A_S), _ptr(B_St), _stream(A)))
-    return A_S, B_St
+                          _dtype(A), _ptr(A_S), _ptr(B_S), _ptr(status), _stream(A)))
+    return A_S, B_S
 
 
-def gemm(A_S: torch.Tensor, B_St: torch.Tensor, k_keep: int, out_dtype=torch.float32,
-         out: torch.Tensor | None = None, status: torch.Tensor | None = None) -> torch.Tensor:
-    """C = A_S · B_Stᵀ over the first k_keep (of k_pad) slices."""
+def gemm(A_S: torch.Tensor, B_S: torch.Tensor, k_keep: int, out_dtype=torch.float32, b_kmajor: bool = False,
+         N: int | None = None, out: torch.Tensor | None = None, status: torch.Tensor | None = None) -> torch.Tensor:
+    """C = A_S · B_S over the first k_keep (of k_pad) slices; B_S as written by pack()."""
     ba, M, kp, _, _ = _mat(A_S, "A_S")
-    _, N, _, _, _ = _mat(B_St, "B_St")
+    if b_kmajor:
+        N = B_S.shape[-2]
+    elif N is None:
+        N = B_S.shape[-1]
     if out is None:
         out = torch.empty((ba, M, N) if A_S.dim() == 3 else (M, N), dtype=out_dtype, device=A_S.device)
     _, _, _, ldc, sC = _mat(out, "C")
-    _check(lib().rmm_gemm(_ptr(A_S), _ptr(B_St), ba, M, N, k_keep, _dtype(A_S), _ptr(out), ldc, sC,
+    _check(lib().rmm_gemm(_ptr(A_S), _ptr(B_S), int(b_kmajor), ba, M, N, k_keep, _dtype(A_S), _ptr(out), ldc, sC,
                           _out_code(out.dtype), _ptr(status), _stream(A_S)))
     return out
 
@@ -310,6 +327,11 @@ def set_wait_limit_ns(ns: int):
 
 def set_stall_producer_for_test(on: bool):
     lib().rmm_set_stall_producer_for_test(int(bool(on)))
+
+
+def set_gemm_cta_group(cta_group: int) -> int:
+    """2 = 2-SM MMAs on CTA pairs (default), 1 = one SM per tile; returns the previous value."""
+    return int(lib().rmm_set_gemm_cta_group(int(cta_group)))
 
 
 def launch_count() -> int:

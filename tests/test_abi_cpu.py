@@ -47,11 +47,11 @@ def test_keep_count_matches_exact_ceiling():
 def test_padded_keep_and_workspace_layout():
     assert rmm.padded_keep(1) == 64 and rmm.padded_keep(64) == 64 and rmm.padded_keep(65) == 128
     ws = rmm.workspace_size(1, 4096, 4096, 4096, 2048, rmm.torch.bfloat16)
-    # status + scores + indices + A_S + B_St, each 1 KiB aligned
+    # status + scores + indices + A_S + packed B, each 1 KiB aligned
     expect = 1024 + 4096 * 4 + 2048 * 4 + 4096 * 2048 * 2 + 4096 * 2048 * 2
     assert ws == expect
     ws32 = rmm.workspace_size(2, 3, 5, 7, 3, rmm.torch.float32)
-    # A_S: 2*3*64*4 = 1536 -> 2048; B_St: 2*7*64*4 = 3584 -> 4096
+    # A_S: 2*3*64*4 = 1536 -> 2048; packed B: 2*64*8*4 = 4096 (row pitch 7 -> 8)
     assert ws32 == 1024 + 1024 + 1024 + 2048 + 4096
 
 

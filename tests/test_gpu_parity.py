@@ -39,9 +39,18 @@ SHAPES = [
 ]
 
 
+@pytest.fixture(params=[2, 1], ids=["cta_pair", "one_sm"])
+def gemm_cta_group(request):
+    prev = rmm.set_gemm_cta_group(request.param)
+    yield request.param
+    rmm.set_gemm_cta_group(prev)
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
-def test_stages_match_oracle(shape, dtype):
+def test_stages_match_oracle(shape, dtype, gemm_cta_group):
+    if dtype == torch.float32 and gemm_cta_group == 1:
+        pytest.skip("the f32 path does not use the tensor-core GEMM")
     M, K, N = shape
     A, B = _ab(M, K, N, dtype, seed=M * 7 + K)
     A64, B64 = f64(A), f64(B)
@@ -54,21 +63,29 @@ def test_stages_match_oracle(shape, dtype):
             idx = rmm.select(s, k)
             # integer stage: bit-exact against the oracle's selection on the same f32 scores
             assert idx.cpu().numpy().tolist() == O.select_top(s.cpu().numpy(), k).tolist()
-            A_S, B_St = rmm.pack(A, B, idx)
             kp = rmm.padded_keep(k)
             ii = idx.long()
-            assert torch.equal(A_S[:, :k], A[:, ii]) and torch.equal(B_St[:, :k], B[ii, :].t())
-            assert not A_S[:, k:].any() and not B_St[:, k:].any()
-            assert A_S.shape == (M, kp) and B_St.shape == (N, kp)
+            # B given row-major: kept rows copied as they are (N-major operand)
+            A_S, B_S = rmm.pack(A, B, idx)
+            assert A_S.shape == (M, kp) and B_S.shape == (kp, rmm.packed_b_ld(N))
+            assert torch.equal(A_S[:, :k], A[:, ii]) and torch.equal(B_S[:k, :N], B[ii, :])
+            assert not A_S[:, k:].any() and not B_S[k:].any() and not B_S[:, N:].any()
+            # B given as Bᵀ (the Kmat form): kept columns, K-major operand
+            Bt = B.t().contiguous()
+            A_S2, B_St = rmm.pack(A, Bt, idx, b_kmajor=True)
+            assert torch.equal(A_S2, A_S) and B_St.shape == (N, kp)
+            assert torch.equal(B_St[:, :k], Bt[:, ii]) and not B_St[:, k:].any()
             for out_dtype in (torch.float32, torch.bfloat16):
-                C = rmm.gemm(A_S, B_St, k, out_dtype)
-                torch.cuda.synchronize()
-                check_product(f64(C), A64, B64, idx.cpu().numpy(), product_tol(dtype, out_dtype))
+                tol = product_tol(dtype, out_dtype)
+                C = rmm.gemm(A_S, B_S, k, out_dtype, N=N)
+                check_product(f64(C), A64, B64, idx.cpu().numpy(), tol)
+                C2 = rmm.gemm(A_S2, B_St, k, out_dtype, b_kmajor=True)
+                check_product(f64(C2), A64, B64, idx.cpu().numpy(), tol)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
 @pytest.mark.parametrize("rho", [0.3, 0.5, 0.7, 1.0])
-def test_fused_matmul_reduced(dtype, rho):
+def test_fused_matmul_reduced(dtype, rho, gemm_cta_group):
     A, B = _ab(300, 1000, 520, dtype, seed=11)
     k = rmm.keep_count(rho, 1000)
     idx = torch.empty(k, dtype=torch.int32, device=DEV)
@@ -86,7 +103,7 @@ def test_config_f32_64x256x64_end_to_end():
     assert err <= 1e-5
 
 
-def test_batched_qk_small():
+def test_batched_qk_small(gemm_cta_group):
     Q, Km = inputs.attention_qk(bh=3, S=300, d=128, seed=1, device=DEV)
     Q = Q[:, :200].contiguous()  # S_q != S_k
     k = rmm.keep_count(0.5, 128)
@@ -100,7 +117,7 @@ def test_batched_qk_small():
         check_product(f64(S16[h]), f64(Q[h]), f64(Km[h]).T, idx[h].cpu().numpy(), 1e-2)
 
 
-def test_batched_pv_small():
+def test_batched_pv_small(gemm_cta_group):
     P, V = inputs.attention_pv(bh=2, S=700, d=128, seed=2, device=DEV)
     for rho in (0.3, 0.5, 0.7):
         k = rmm.keep_count(rho, 700)
@@ -194,5 +211,5 @@ def test_launch_counter_counts_kernels():
     n0 = rmm.launch_count()
     rmm.matmul_reduced(A, B, 0.5)
     torch.cuda.synchronize()
-    # score (B rows, A columns), select, pack (A, B), gemm
-    assert rmm.launch_count() - n0 == 6
+    # score (one launch for A's and B's norms), select, pack (A, B), gemm
+    assert rmm.launch_count() - n0 == 5

@@ -22,14 +22,14 @@ def test_stalled_producer_times_out_and_context_survives():
     s = rmm.score(A, B)
     k = rmm.keep_count(0.5, 256)
     idx = rmm.select(s, k)
-    A_S, B_St = rmm.pack(A, B, idx)
+    A_S, B_S = rmm.pack(A, B, idx)
     torch.cuda.synchronize()
 
     status = rmm.status_word()
     rmm.set_wait_limit_ns(20_000_000)  # 20 ms per wait
     rmm.set_stall_producer_for_test(True)
     try:
-        rmm.gemm(A_S, B_St, k, status=status)
+        rmm.gemm(A_S, B_S, k, status=status)
         torch.cuda.synchronize()
     finally:
         rmm.set_stall_producer_for_test(False)
@@ -38,6 +38,6 @@ def test_stalled_producer_times_out_and_context_survives():
         rmm.check(status)
     assert e.value.status == rmm.RMM_ERR_TIMEOUT
 
-    C = rmm.gemm(A_S, B_St, k, status=status)
+    C = rmm.gemm(A_S, B_S, k, status=status)
     rmm.check(status)
     check_product(f64(C), f64(A), f64(B), idx.cpu().numpy(), 1e-2)
