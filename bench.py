@@ -144,24 +144,28 @@ class Pipeline:
             A_S = self.a_store[: p.M * kp].view(p.M, kp)
         return k, idx, A_S, B_S
 
-    def step(self, rho, ev=None):
-        """One pass of score -> select -> pack -> gemm; ev: 5 events bracketing the stages."""
+    def step(self, rho, ev=None, breakdown=False):
+        """One pass of score -> select -> pack -> gemm.
+
+        ev: events to record. With breakdown, 5 events bracket every stage
+        (the events break programmatic-launch overlap between stages);
+        otherwise 3 events: before score, before gemm, after gemm."""
         p = self.p
         k, idx, A_S, B_S = self.views(rho)
         if ev:
             ev[0].record()
         rmm.score(p.A, p.B, "product", p.b_kmajor, out=self.s, status=self.status)
-        if ev:
+        if ev and breakdown:
             ev[1].record()
         rmm.select(self.s, k, out=idx, status=self.status)
-        if ev:
+        if ev and breakdown:
             ev[2].record()
         rmm.pack(p.A, p.B, idx, p.b_kmajor, out=(A_S, B_S), status=self.status)
         if ev:
-            ev[3].record()
+            ev[3 if breakdown else 1].record()
         rmm.gemm(A_S, B_S, k, b_kmajor=p.b_kmajor, N=p.N, out=self.C, status=self.status)
         if ev:
-            ev[4].record()
+            ev[4 if breakdown else 2].record()
 
 
 STAGES = ("score", "select", "pack", "gemm")
@@ -181,16 +185,21 @@ class L2Flush:
         self.r.sum()
 
 
-def timed_steps(pipe: Pipeline, rho: float, steps: int, flush):
-    """Run `steps` steps; returns (per-step ms list, per-stage ms lists)."""
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+def timed_steps(pipe: Pipeline, rho: float, steps: int, flush, breakdown=False):
+    """Run `steps` steps (L2 flushed and the host queued ahead before each).
+
+    Returns (per-step ms, per-stage ms lists). Without breakdown the stages
+    are {"pre_gemm": score+select+pack, "gemm": gemm}."""
+    n_ev = 5 if breakdown else 3
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)]
     for i in range(steps):
         flush()
         torch.cuda._sleep(SLEEP_CYCLES)
-        pipe.step(rho, evs[i])
+        pipe.step(rho, evs[i], breakdown)
     torch.cuda.synchronize()
-    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
-    stage_ms = {s: [e[j].elapsed_time(e[j + 1]) for e in evs] for j, s in enumerate(STAGES)}
+    step_ms = [e[0].elapsed_time(e[-1]) for e in evs]
+    names = STAGES if breakdown else ("pre_gemm", "gemm")
+    stage_ms = {s: [e[j].elapsed_time(e[j + 1]) for e in evs] for j, s in enumerate(names)}
     return step_ms, stage_ms
 
 
@@ -364,11 +373,22 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Largest value of x over the ranks (a no-op for one rank)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(step_ms_local_total: float, steps: int, flops_per_rank_step: float, world: int):
+    """Whole-job throughput of `world` replicas: every rank processed its own
+    steps; the job took as long as the slowest rank. Returns (ms per step,
+    TFLOP/s over all ranks)."""
+    total = max_over_ranks(step_ms_local_total, world)
+    ms = total / steps
+    return ms, world * flops_per_rank_step / (ms * 1e-3) / 1e12
 
 
 def run_reference(args):
@@ -423,10 +443,7 @@ def run_ours(args):
         rmm.check(pipe.status)
     clk = clocks.summary()
 
-    total_ms = sum(step_ms)
-    total_ms_max = max_over_ranks(total_ms, world)
-    ms_per_step = total_ms_max / args.steps
-    value = world * p.kept_flops(rho) / (ms_per_step * 1e-3) / 1e12
+    ms_per_step, value = job_throughput(sum(step_ms), args.steps, p.kept_flops(rho), world)
 
     # rho sweep: the same staged pipeline, speedup against rho = 1
     sweep = {}
@@ -448,7 +465,10 @@ def run_ours(args):
         sweep = {f"{r:g}": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in d.items()}
                  for r, d in sweep.items()}
 
-    stage_mean = {s: statistics.mean(v) for s, v in stage_ms.items()}
+    gemm_ms_timed = statistics.mean(stage_ms["gemm"])
+    # per-stage breakdown (separate pass: events between stages cost the overlap)
+    _, bd = timed_steps(pipe, rho, max(10, args.steps // 2), flush, breakdown=True)
+    stage_mean = {s: statistics.mean(v) for s, v in bd.items()}
     del pipe
     torch.cuda.empty_cache()
     # fused C-ABI call (one user call, same kernels)
@@ -460,10 +480,13 @@ def run_ours(args):
         e2e = run_e2e(p, rho, max(5, min(20, args.steps)), world)
 
     peaks, peak_src = measured_peaks()
-    gemm_ms = statistics.mean(stage_ms["gemm"])
-    gemm_ms_max = max_over_ranks(gemm_ms, world)
+    gemm_ms_max = max_over_ranks(gemm_ms_timed, world)
     dominant = max(stage_mean, key=stage_mean.get)
-    roof = roofline(p, rho, stage_mean, dominant, peaks, peak_src)
+    # the dominant kernel's duration is taken from the timed region itself
+    roof_ms = dict(stage_mean)
+    if dominant == "gemm":
+        roof_ms["gemm"] = gemm_ms_timed
+    roof = roofline(p, rho, roof_ms, dominant, peaks, peak_src)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -481,9 +504,12 @@ def run_ours(args):
                        "out_dtype": str(p.out_dtype).replace("torch.", ""),
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed before every timed step (256 MiB written, then another 256 MiB read)",
-                       "timing": "CUDA events around each stage call on the launching stream; device sleep "
+                       "timing": "CUDA events on the launching stream before score, before gemm and after "
+                                 "gemm of each step (stage breakdown from a separate pass); a device sleep "
                                  "before each step hides host launch overhead"},
             "stages_ms": {s: round(v, 5) for s, v in stage_mean.items()},
+            "timed_region_ms": {"pre_gemm": round(statistics.mean(stage_ms["pre_gemm"]), 5),
+                                "gemm": round(gemm_ms_timed, 5)},
             "fused_call_ms": round(fused, 5),
             "wall_s_timed_region": round(wall_s, 4),
             "gemm_ms_max_over_ranks": round(gemm_ms_max, 5),

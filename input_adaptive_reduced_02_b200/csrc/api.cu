@@ -77,8 +77,8 @@ static bool layout_ok(int64_t batch, int64_t rows, int64_t cols, int64_t ld, int
 }
 
 constexpr int64_t kMaxGridBatch = 65535;
-// The select kernel's packed 16-bit histogram counters hold up to 2^16 - 1
-// keys per bin and histogram copy (32 copies): 2^21 slices per selection.
+// Slices per selection: the select kernel indexes keys with 32-bit integers
+// and re-reads them from global memory beyond 32768; 2^21 bounds its work.
 constexpr int64_t kMaxSelectK = int64_t(1) << 21;
 
 struct Workspace {

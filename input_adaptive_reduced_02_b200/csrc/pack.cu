@@ -25,6 +25,7 @@ namespace {
 constexpr int kPackThreads = 256;
 constexpr size_t kStageBytes = 32 * 1024;   // shared-memory rows per CTA (short rows)
 constexpr size_t kStageMax = 112 * 1024;    // one long row per CTA, two CTAs per SM
+constexpr size_t kSmemAttr = kStageMax + kStageBytes;  // + staged kept indices
 
 template <typename T>
 union Vec16 {
@@ -55,9 +56,11 @@ __device__ __forceinline__ bool wait_loads(uint64_t* bar, uint64_t limit_ns, uin
   return false;
 }
 
+// Gather kept columns of nr staged rows; ib points at the kept indices (in
+// shared memory or global memory, 16-byte aligned).
 template <typename T>
-__device__ __forceinline__ void gather_rows(const T* srow, int nr, int64_t C, const int32_t* __restrict__ ib,
-                                            int64_t k_keep, int64_t k_pad, T* dst) {
+__device__ __forceinline__ void gather_rows(const T* srow, int nr, int64_t C, const int32_t* ib, int64_t k_keep,
+                                            int64_t k_pad, T* dst) {
   constexpr int V = 16 / sizeof(T);
   const int64_t ng = k_pad / V;
   for (int rr = 0; rr < nr; ++rr) {
@@ -66,9 +69,9 @@ __device__ __forceinline__ void gather_rows(const T* srow, int nr, int64_t C, co
       const int64_t t0 = g * V;
       Vec16<T> v;
       if (t0 + V <= k_keep) {
-        const int4 i0 = __ldg(reinterpret_cast<const int4*>(ib + t0));
+        const int4 i0 = *reinterpret_cast<const int4*>(ib + t0);
         if constexpr (V == 8) {
-          const int4 i1 = __ldg(reinterpret_cast<const int4*>(ib + t0 + 4));
+          const int4 i1 = *reinterpret_cast<const int4*>(ib + t0 + 4);
           v.e[0] = row[i0.x]; v.e[1] = row[i0.y]; v.e[2] = row[i0.z]; v.e[3] = row[i0.w];
           v.e[4] = row[i1.x]; v.e[5] = row[i1.y]; v.e[6] = row[i1.z]; v.e[7] = row[i1.w];
         } else {
@@ -78,7 +81,7 @@ __device__ __forceinline__ void gather_rows(const T* srow, int nr, int64_t C, co
 #pragma unroll
         for (int j = 0; j < V; ++j) {
           const int64_t t = t0 + j;
-          v.e[j] = t < k_keep ? row[__ldg(ib + t)] : T(0);
+          v.e[j] = t < k_keep ? row[ib[t]] : T(0);
         }
       }
       reinterpret_cast<uint4*>(dst + rr * k_pad)[g] = v.u;
@@ -86,21 +89,24 @@ __device__ __forceinline__ void gather_rows(const T* srow, int nr, int64_t C, co
   }
 }
 
-// Rows staged by bulk-async copies (rows 16-byte aligned, C·e a multiple of 16;
-// idx 16-byte aligned so that it can be read four at a time).
+// Rows (and, when idx_in_smem, the kept indices) staged by bulk-async copies
+// (rows 16-byte aligned, C·e a multiple of 16; idx 16-byte aligned).
 template <typename T>
 __global__ void __launch_bounds__(kPackThreads)
 pack_cols_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t R, int64_t C,
                       const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
-                      int rows_per_cta, uint32_t* status, uint64_t wait_ns) {
+                      int rows_per_cta, int idx_in_smem, uint32_t* status, uint64_t wait_ns) {
   extern __shared__ __align__(128) unsigned char pack_smem[];
   __shared__ uint64_t bar;
   __shared__ int never;
   T* srow = reinterpret_cast<T*>(pack_smem);
+  int32_t* sidx = reinterpret_cast<int32_t*>(pack_smem + size_t(rows_per_cta) * C * sizeof(T));
   const int64_t b = blockIdx.y;
   const int64_t r0 = int64_t(blockIdx.x) * rows_per_cta;
   const int nr = int(min(int64_t(rows_per_cta), R - r0));
   const T* src = X + b * bstride + r0 * ld;
+  const int32_t* gidx = idx + b * k_keep;
+  const int64_t idx_bulk = idx_in_smem ? (k_keep & ~int64_t(3)) : 0;  // whole 16-byte groups
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     never = 0;
@@ -111,11 +117,15 @@ pack_cols_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int6
   __syncthreads();
   if (threadIdx.x == 0) {
     const uint32_t row_bytes = uint32_t(C * sizeof(T));
-    mbar_arrive_expect_tx(&bar, row_bytes * uint32_t(nr));
+    mbar_arrive_expect_tx(&bar, row_bytes * uint32_t(nr) + uint32_t(idx_bulk * 4));
     for (int rr = 0; rr < nr; ++rr) bulk_load(srow + rr * C, src + rr * ld, row_bytes, &bar);
+    if (idx_bulk > 0) bulk_load(sidx, gidx, uint32_t(idx_bulk * 4), &bar);
   }
+  if (idx_in_smem)
+    for (int64_t t = idx_bulk + threadIdx.x; t < k_keep; t += kPackThreads) sidx[t] = gidx[t];
   wait_loads(&bar, wait_ns, status, &never);
-  gather_rows(srow, nr, C, idx + b * k_keep, k_keep, k_pad, out + (b * R + r0) * k_pad);
+  __syncthreads();
+  gather_rows(srow, nr, C, idx_in_smem ? sidx : gidx, k_keep, k_pad, out + (b * R + r0) * k_pad);
 }
 
 // Any alignment: rows staged with plain loads (eight in flight per thread).
@@ -263,7 +273,7 @@ void set_smem_attr_once(K kernel) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !done[dev]) {
-    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kStageMax));
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemAttr));
     done[dev] = true;
   }
 }
@@ -280,15 +290,17 @@ cudaError_t launch_pack_cols_t(const MatView& X, int64_t batch, const int32_t* i
   }
   const int rows_per_cta =
       row_bytes <= kStageBytes ? int(std::min<size_t>(64, kStageBytes / std::max<size_t>(row_bytes, 1))) : 1;
-  const size_t smem = size_t(rows_per_cta) * row_bytes;
+  const size_t idx_bytes = size_t(k_keep) * 4;
+  const int idx_in_smem = idx_bytes <= kStageBytes;
+  const size_t smem = size_t(rows_per_cta) * row_bytes + (idx_in_smem ? (idx_bytes + 15) / 16 * 16 : 0);
   const dim3 grid(unsigned((X.rows + rows_per_cta - 1) / rows_per_cta), unsigned(batch), 1u);
   const bool bulk = aligned16(X.ptr) && row_bytes % 16 == 0 && (X.ld * int64_t(sizeof(T))) % 16 == 0 &&
                     (batch == 1 || (X.bstride * int64_t(sizeof(T))) % 16 == 0) && aligned16(idx) &&
                     (batch == 1 || k_keep % 4 == 0);
   if (bulk) {
     set_smem_attr_once(pack_cols_bulk_kernel<T>);
-    return launch_pdl(pack_cols_bulk_kernel<T>, grid, dim3(kPackThreads), smem, st, dim3(0, 0, 0), p, X.ld, X.bstride, X.rows,
-                      X.cols, idx, k_keep, k_pad, o, rows_per_cta, status, wait_ns);
+    return launch_pdl(pack_cols_bulk_kernel<T>, grid, dim3(kPackThreads), smem, st, dim3(0, 0, 0), p, X.ld,
+                      X.bstride, X.rows, X.cols, idx, k_keep, k_pad, o, rows_per_cta, idx_in_smem, status, wait_ns);
   }
   set_smem_attr_once(pack_cols_plain_kernel<T>);
   return launch_pdl(pack_cols_plain_kernel<T>, grid, dim3(kPackThreads), smem, st, dim3(0, 0, 0), p, X.ld, X.bstride, X.rows,

@@ -58,92 +58,103 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
 }
 
 constexpr int kSelThreads = 1024;
-constexpr int kBins = 2048;  // 11-bit digits: passes cover bits 31-21, 20-10, 9-0
+constexpr int kDigitBits = 11;
+constexpr int kBins = 1 << kDigitBits;
 
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS, 1)
 select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t* __restrict__ idx,
-              uint32_t* status, int keys_in_smem, int hist_copies) {
-  const int K = int(K64);  // K < 2^31 (checked on the host)
-  // dynamic shared memory: [keys: K words if keys_in_smem][histograms: hist_copies x 1024 words]
-  // Each histogram word packs two 16-bit bin counters (bins 2w and 2w+1); a
-  // copy is shared by THREADS/32/hist_copies warps, so a bin never exceeds
-  // K·hist_warps/32 <= 2^16 - 1 for the sizes the host allows.
-  extern __shared__ uint32_t dyn[];
-  uint32_t* keys = dyn;
-  uint32_t* hist = dyn + (keys_in_smem ? K : 0);
-  __shared__ uint32_t tot[kBins];
+              uint32_t* status, int keys_in_smem) {
+  constexpr int kWarps = THREADS / 32;
+  const int K = int(K64);  // K <= 2^21 (checked on the host)
+  extern __shared__ uint32_t keys[];  // K keys when keys_in_smem
+  __shared__ uint32_t hist[kBins];
   __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t warp_min[kWarps], warp_max[kWarps];
   __shared__ uint32_t sh_digit, sh_above, sh_count;
   __shared__ int sh_nan;
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* sb = s + int64_t(blockIdx.x) * K;
   int32_t* ib = idx + int64_t(blockIdx.x) * k_keep;
-  uint32_t* my_hist = hist + (warp % hist_copies) * (kBins / 2);
 
   pdl_trigger();
   pdl_wait();
   if (tid == 0) sh_nan = 0;
   __syncthreads();
   bool nan_seen = false;
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
   if (keys_in_smem && (K & 3) == 0 && (reinterpret_cast<uintptr_t>(sb) & 15u) == 0) {
     const float4* s4 = reinterpret_cast<const float4*>(sb);
     for (int i = tid; i < K / 4; i += THREADS) {
       const float4 x = s4[i];
       nan_seen |= (x.x != x.x) | (x.y != x.y) | (x.z != x.z) | (x.w != x.w);
-      reinterpret_cast<uint4*>(keys)[i] = make_uint4(order_key(x.x), order_key(x.y), order_key(x.z), order_key(x.w));
+      const uint4 k4 = make_uint4(order_key(x.x), order_key(x.y), order_key(x.z), order_key(x.w));
+      kmin = min(min(kmin, min(k4.x, k4.y)), min(k4.z, k4.w));
+      kmax = max(max(kmax, max(k4.x, k4.y)), max(k4.z, k4.w));
+      reinterpret_cast<uint4*>(keys)[i] = k4;
     }
   } else {
     for (int i = tid; i < K; i += THREADS) {
       const float x = sb[i];
       nan_seen |= (x != x);
-      if (keys_in_smem) keys[i] = order_key(x);
+      const uint32_t k = order_key(x);
+      kmin = min(kmin, k);
+      kmax = max(kmax, k);
+      if (keys_in_smem) keys[i] = k;
     }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    warp_min[warp] = kmin;
+    warp_max[warp] = kmax;
   }
   if (nan_seen) sh_nan = 1;
   __syncthreads();
   if (tid == 0 && sh_nan) status_or(status, RMM_NONFINITE_BIT);
+  kmin = warp_min[0];
+  kmax = warp_max[0];
+  for (int w = 1; w < kWarps; ++w) {
+    kmin = min(kmin, warp_min[w]);
+    kmax = max(kmax, warp_max[w]);
+  }
 
   if (k_keep >= K) {  // everything is kept
     for (int i = tid; i < K; i += THREADS) ib[i] = i;
     return;
   }
 
-  // MSB-first radix select. After each pass, `prefix` (under `mask`) is the
-  // digit string of the k-th largest key so far, `remaining` the number of
-  // keys still to take among those matching it.
-  uint32_t prefix = 0, mask = 0, remaining = uint32_t(k_keep), bin_count = 0;
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-    const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
-    for (int w = tid; w < hist_copies * (kBins / 2); w += THREADS) hist[w] = 0u;
+  // MSB-first radix select over the bits in which the keys differ: every key
+  // shares the bits of kmin above the highest bit where kmin and kmax differ,
+  // so the first histogram already spreads the keys over many bins. After
+  // each pass, `prefix` (under `mask`) is the digit string of the k-th largest
+  // key so far and `remaining` the number of keys still to take among those
+  // matching it.
+  const uint32_t diff = kmin ^ kmax;
+  int hi = diff ? 31 - __clz(diff) : -1;  // highest unresolved bit
+  uint32_t mask = hi >= 0 ? uint32_t(~((uint64_t(2) << hi) - 1)) : 0xFFFFFFFFu;
+  uint32_t prefix = kmin & mask, remaining = uint32_t(k_keep), bin_count = uint32_t(K);
+  while (hi >= 0) {
+    const int width = min(kDigitBits, hi + 1);
+    const int shift = hi - width + 1;
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int b = tid; b < kBins; b += THREADS) hist[b] = 0u;
     __syncthreads();
     for (int i = tid; i < K; i += THREADS) {
       const uint32_t key = keys_in_smem ? keys[i] : order_key(sb[i]);
-      if ((key & mask) == prefix) {
-        const uint32_t d = (key >> shift) & dmask;
-        atomicAdd(&my_hist[d >> 1], (d & 1u) ? 0x10000u : 1u);
-      }
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
     }
     __syncthreads();
-    // totals per bin, then a descending scan to find the bin of the k-th key:
-    // thread t owns bins 2047-2t and 2046-2t
-    for (int w = tid; w < kBins / 2; w += THREADS) {
-      uint32_t lo = 0, hi = 0;
-      for (int c = 0; c < hist_copies; ++c) {
-        const uint32_t v = hist[c * (kBins / 2) + w];
-        lo += v & 0xFFFFu;
-        hi += v >> 16;
-      }
-      tot[2 * w] = lo;
-      tot[2 * w + 1] = hi;
-    }
-    __syncthreads();
+    // descending scan to find the bin of the k-th key: thread t owns bins
+    // kBins-1-2t and kBins-2-2t
     uint32_t c0 = 0, c1 = 0;
     if (tid < kBins / 2) {
-      c0 = tot[kBins - 1 - 2 * tid];
-      c1 = tot[kBins - 2 - 2 * tid];
+      c0 = hist[kBins - 1 - 2 * tid];
+      c1 = hist[kBins - 2 - 2 * tid];
     }
     uint32_t all;
     const uint32_t excl = block_exclusive_scan<THREADS>(c0 + c1, warp_sums, &all);
@@ -165,16 +176,17 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
     bin_count = sh_count;
     // every key in the chosen bin is kept: no finer threshold is needed
     if (remaining == bin_count) break;
+    hi = shift - 1;
   }
-  // Kept: keys whose masked digits exceed `prefix`, plus the `remaining`
-  // lowest-indexed keys whose masked digits equal it (all of them when the
-  // bin is taken whole).
+  // Kept: keys whose masked bits exceed `prefix`, plus the `remaining`
+  // lowest-indexed keys whose masked bits equal it (all of them when the bin
+  // is taken whole).
   const uint32_t T = prefix, need_eq = remaining;
   const bool take_all_eq = remaining == bin_count;
   const int per = (K + THREADS - 1) / THREADS;
-  const int lo = min(K, tid * per), hi = min(K, lo + per);
+  const int lo = min(K, tid * per), hi_i = min(K, lo + per);
   uint32_t n_gt = 0, n_eq = 0;
-  for (int i = lo; i < hi; ++i) {
+  for (int i = lo; i < hi_i; ++i) {
     const uint32_t k = (keys_in_smem ? keys[i] : order_key(sb[i])) & mask;
     n_gt += (k > T);
     n_eq += (k == T);
@@ -186,7 +198,7 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
   }
   uint32_t pos = block_exclusive_scan<THREADS>(n_gt + eq_take, warp_sums, &total);
   uint32_t taken_eq = 0;
-  for (int i = lo; i < hi; ++i) {
+  for (int i = lo; i < hi_i; ++i) {
     const uint32_t k = (keys_in_smem ? keys[i] : order_key(sb[i])) & mask;
     if (k > T) {
       ib[pos++] = i;
@@ -203,23 +215,18 @@ cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_ke
                           uint32_t* status, cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
   const int keys_in_smem = K <= kSelSmemKeys;
-  // Histogram copies: one per warp while they fit next to the keys, else one
-  // per two warps (packed 16-bit bins stay below 2^16 for K <= 2^16).
-  const int copies = (K <= 16384 || !keys_in_smem) ? 32 : 16;
-  if (int64_t(copies) * kSelThreads / 32 > 0 && K * (32 / copies) > 65535 * 32)
-    return cudaErrorInvalidValue;
-  const size_t smem = (keys_in_smem ? size_t(K) * 4 : 0) + size_t(copies) * (kBins / 2) * 4;
+  const size_t smem = keys_in_smem ? size_t(K) * 4 : 0;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel<kSelThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(kSelSmemKeys * 4 + 16 * (kBins / 2) * 4));
+                                         int(kSelSmemKeys * 4));
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
   return launch_pdl(select_kernel<kSelThreads>, dim3(unsigned(batch)), dim3(kSelThreads), smem, st, dim3(0, 0, 0), s,
-                    K, k_keep, idx, status, keys_in_smem, copies);
+                    K, k_keep, idx, status, keys_in_smem);
 }
 
 }  // namespace rmm
