@@ -20,7 +20,9 @@
 //               rounding, swizzled staging in shared memory, TMA tile store
 // Two accumulators let the epilogue of tile i overlap the mainloop of tile
 // i+1. Tiles are visited m-fastest so a column block of B is shared through
-// L2 by the pairs working on it at the same time.
+// L2 by the pairs working on it at the same time. When the tile count leaves
+// the last round less than half full, those tiles are split in two along K
+// and both halves reduce-add (f32) into C, which a small kernel zeroes first.
 //
 // Every mbarrier wait is bounded (rmm_set_wait_limit_ns). A role whose wait
 // runs out records RMM_STATUS_BIT_TIMEOUT, raises its CTA's abort flag, and
@@ -65,6 +67,11 @@ static_assert(TcCfg<128, 2>::STAGES * 2 + 6 <= 32, "barrier area");
 struct TcParams {
   int32_t M, N, num_kb, tiles_m, tiles_n;
   int64_t total_tiles;
+  // Work units: units [0, full_units) are whole tiles; when the last round
+  // would leave pairs idle, its tiles are split at k-block kb_mid into two
+  // units each (same tile, two halves of K) that add into a zeroed C.
+  int64_t full_units, total_units;
+  int32_t kb_mid;
   uint32_t* status;
   uint64_t wait_limit_ns;
   int stall_producer;
@@ -81,6 +88,30 @@ __device__ __forceinline__ void decode_tile(int64_t t, const TcParams& p, int32_
   const int64_t r = t - int64_t(b) * per;
   nb = int32_t(r / p.tiles_m);
   mb = int32_t(r - int64_t(nb) * p.tiles_m);
+}
+
+struct Unit {
+  int64_t tile;
+  int32_t kb0, kb1;
+  bool split;
+};
+
+__device__ __forceinline__ Unit unit_info(int64_t u, const TcParams& p) {
+  Unit w;
+  if (u < p.full_units) {
+    w.tile = u;
+    w.kb0 = 0;
+    w.kb1 = p.num_kb;
+    w.split = false;
+  } else {
+    const int64_t j = u - p.full_units;
+    w.tile = p.full_units + (j >> 1);
+    const bool second = (j & 1) != 0;
+    w.kb0 = second ? p.kb_mid : 0;
+    w.kb1 = second ? p.num_kb : p.kb_mid;
+    w.split = true;
+  }
+  return w;
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t* status) {
@@ -157,12 +188,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       uint32_t issued = 0;      // bit s: this CTA loaded stage s
       uint32_t issued_par = 0;  // bit s: parity of that stage's last phase
       bool ok = true;
-      for (int64_t t = pair; ok && t < p.total_tiles; t += npairs) {
+      for (int64_t u = pair; ok && u < p.total_units; u += npairs) {
+        const Unit w = unit_info(u, p);
         int32_t b, mb, nb;
-        decode_tile(t, p, b, mb, nb);
+        decode_tile(w.tile, p, b, mb, nb);
         const int32_t m_row = mb * BM * CG + int32_t(rank) * BM;
         const int32_t n_col = nb * BN + int32_t(rank) * BN_CTA;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, limit, abort_v)) {
             ok = false;
             break;
@@ -223,14 +255,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       uint32_t stage = 0, phase = 0;
       uint32_t acc = 0, acc_phase = 0;
       bool ok = true;
-      for (int64_t t = pair; ok && t < p.total_tiles; t += npairs) {
+      for (int64_t u = pair; ok && u < p.total_units; u += npairs) {
+        const Unit w = unit_info(u, p);
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, limit, abort_v)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, limit, abort_v)) {
             ok = false;
             break;
@@ -243,7 +276,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             // K-major: 16 elements = 32 bytes along the swizzled row;
             // N-major: 16 K-rows of 128 bytes
             const uint64_t bdesc = BMN ? umma_desc_mn_sw128(b0 + kk * 2048, 8192) : umma_desc_k_sw128(b0 + kk * 32);
-            umma_bf16<CG>(d_tmem, umma_desc_k_sw128(a0 + kk * 32), bdesc, idesc, (kb | kk) != 0);
+            umma_bf16<CG>(d_tmem, umma_desc_k_sw128(a0 + kk * 32), bdesc, idesc, (kb > w.kb0) || kk != 0);
           }
           // this stage's smem is free in both CTAs once these MMAs are done
           umma_commit<CG>(smem_addr(&empty[stage]));
@@ -273,9 +306,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     bool ok = true;
     const int cols_per_chunk = p.out_bf16 ? 64 : 32;
     const int chunks = BN / cols_per_chunk;
-    for (int64_t t = pair; ok && t < p.total_tiles; t += npairs) {
+    for (int64_t u = pair; ok && u < p.total_units; u += npairs) {
+      const Unit unit = unit_info(u, p);
       int32_t b, mb, nb;
-      decode_tile(t, p, b, mb, nb);
+      decode_tile(unit.tile, p, b, mb, nb);
       int w = 1;
       if (lane == 0) w = mbar_wait_bounded(&tfull[acc], acc_phase, limit, abort_v);
       w = __shfl_sync(0xffffffffu, w, 0);
@@ -327,7 +361,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&tmC, buf, col0, row0, b);
+            if (unit.split)
+              tma_reduce_add_3d(&tmC, buf, col0, row0, b);  // the tile's other K half adds too
+            else
+              tma_store_3d(&tmC, buf, col0, row0, b);
             tma_store_commit();
           }
           __syncwarp();
@@ -364,6 +401,39 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if constexpr (CG == 2) cluster_sync_all();  // the pair is done with each other's barriers and TMEM
   tc_fence_after();
   if (warp == 1) tmem_dealloc<CG>(tmem_base, Cfg::TMEM_COLS);
+}
+
+// Zero the f32 C tiles [first_tile, first_tile + gridDim.x) that receive two
+// reduce-adds (split K). Waits for its predecessor first: C may still be
+// written by earlier work on the stream, and the GEMM launched after this
+// kernel relies on it having waited.
+__global__ void __launch_bounds__(256)
+zero_split_tiles_kernel(float* __restrict__ C, int64_t ldc, int64_t strideC, TcParams p, int64_t first_tile,
+                        int32_t tile_rows, int32_t tile_cols) {
+  pdl_trigger();
+  pdl_wait();
+  int32_t b, mb, nb;
+  decode_tile(first_tile + blockIdx.x, p, b, mb, nb);
+  const int64_t r0 = int64_t(mb) * tile_rows, c0 = int64_t(nb) * tile_cols;
+  const int64_t r1 = min(int64_t(p.M), r0 + tile_rows), c1 = min(int64_t(p.N), c0 + tile_cols);
+  const int64_t rows_per = (tile_rows + gridDim.y - 1) / gridDim.y;
+  const int64_t ra = r0 + int64_t(blockIdx.y) * rows_per, rb = min(r1, ra + rows_per);
+  if (ra >= rb) return;
+  float* base = C + int64_t(b) * strideC;
+  const int vec_per_row = (tile_cols + 3) / 4;  // 16-byte slots per tile row
+  const int64_t n = (rb - ra) * vec_per_row;
+  // consecutive threads write consecutive 16 bytes of a row; rows start 16-byte
+  // aligned (ldc, strideC and c0 are multiples of 4)
+  for (int64_t v = threadIdx.x; v < n; v += 256) {
+    const int64_t r = ra + v / vec_per_row;
+    const int64_t c = c0 + (v % vec_per_row) * 4;
+    float* dst = base + r * ldc + c;
+    if (c + 4 <= c1) {
+      *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      for (int64_t j = c; j < c1; ++j) base[r * ldc + j] = 0.f;
+    }
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -478,7 +548,22 @@ cudaError_t launch_cfg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, co
   p.ldc = g.ldc;
   p.strideC = g.strideC;
   const int64_t units = std::max<int64_t>(1, (di.sms > 0 ? di.sms : 148) / CG);
-  const int64_t grid = CG * std::min<int64_t>(p.total_tiles, units);
+  // Split the K range of the last round's tiles when that round would leave
+  // more than half the pairs idle (f32 output through TMA only: the two halves
+  // reduce-add into C, and with C zeroed first a + b == b + a keeps the
+  // result independent of which half lands first).
+  const int64_t rem = p.total_tiles % units;
+  const bool split = g.out == kF32 && tma_store && p.num_kb >= 2 && rem > 0 && 2 * rem <= units;
+  p.full_units = split ? p.total_tiles - rem : p.total_tiles;
+  p.total_units = split ? p.full_units + 2 * rem : p.total_tiles;
+  p.kb_mid = p.num_kb / 2;
+  if (split) {
+    cudaError_t e = launch_pdl(zero_split_tiles_kernel, dim3(unsigned(rem), 8u), dim3(256), 0, st, dim3(0, 0, 0),
+                               static_cast<float*>(g.c), g.ldc, g.batch == 1 ? int64_t(0) : g.strideC, p,
+                               p.full_units, int32_t(BM * CG), int32_t(BN));
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t grid = CG * std::min<int64_t>(p.total_units, units);
   return launch_pdl(gemm_tc_kernel<BN, BMN, CG>, dim3(unsigned(grid)), dim3(kTcThreads), Cfg::SMEM, st,
                     CG == 2 ? dim3(2, 1, 1) : dim3(0, 0, 0), tmA, tmB, tmC, p);
 }
