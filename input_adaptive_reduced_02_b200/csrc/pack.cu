@@ -199,50 +199,97 @@ pack_cols_direct_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, in
   }
 }
 
-// Kept rows of B (N·e a multiple of 16, rows 16-byte aligned): bulk-async row
-// copies through shared memory. CTA x covers kept rows [x·rows, (x+1)·rows).
+// Kept rows of B (N·e a multiple of 16, rows 16-byte aligned): a persistent
+// CTA streams its share of the kept rows through a ring of shared-memory
+// buffers, one thread keeping bulk-async loads and bulk-async stores in
+// flight at once; the other threads write the zero padding rows.
+constexpr int kRowRing = 4;
+constexpr int64_t kRowIdxStage = 8192;  // kept-row indices a CTA stages in shared memory
+
 template <typename T>
 __global__ void __launch_bounds__(kPackThreads)
 pack_rows_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t N,
                       const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
-                      int64_t ldo, int rows_per_cta, uint32_t* status, uint64_t wait_ns) {
+                      int64_t ldo, int rows_per_buf, int64_t seg, uint32_t* status, uint64_t wait_ns) {
+  // A chunk is rows_per_buf whole rows (seg == N) or one `seg`-element segment
+  // of one row (rows_per_buf == 1, long rows).
   extern __shared__ __align__(128) unsigned char pack_smem[];
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar[kRowRing];
   __shared__ int never;
-  T* srow = reinterpret_cast<T*>(pack_smem);
   const int64_t b = blockIdx.y;
-  const int64_t t0 = int64_t(blockIdx.x) * rows_per_cta;
-  const int nr = int(min(int64_t(rows_per_cta), k_pad - t0));
-  const int nload = int(max(int64_t(0), min(int64_t(nr), k_keep - t0)));  // kept rows in this CTA
-  const uint32_t row_bytes = uint32_t(N * sizeof(T));
-  T* dst = out + (b * k_pad + t0) * ldo;
+  const int64_t segs = (N + seg - 1) / seg;
+  const size_t buf_elems = size_t(rows_per_buf) * seg;
+  T* ring = reinterpret_cast<T*>(pack_smem);
+  int32_t* sidx = reinterpret_cast<int32_t*>(pack_smem + kRowRing * buf_elems * sizeof(T));
+  // this CTA's kept rows: a contiguous range of [0, k_keep), at most kRowIdxStage long
+  const int64_t per = (k_keep + gridDim.x - 1) / gridDim.x;
+  const int64_t t_begin = min(k_keep, int64_t(blockIdx.x) * per), t_end = min(k_keep, t_begin + per);
+  const int64_t nchunks = (t_end - t_begin + rows_per_buf - 1) / rows_per_buf * segs;
+  T* outb = out + b * k_pad * ldo;
   if (threadIdx.x == 0) {
-    mbar_init(&bar, 1);
+    for (int i = 0; i < kRowRing; ++i) mbar_init(&bar[i], 1);
     never = 0;
     fence_mbar_init();
   }
   pdl_trigger();
   pdl_wait();
+  for (int64_t t = t_begin + threadIdx.x; t < t_end; t += kPackThreads) sidx[t - t_begin] = idx[b * k_keep + t];
   __syncthreads();
-  if (threadIdx.x == 0 && nload > 0) {
-    const int32_t* ib = idx + b * k_keep + t0;
-    const T* src = X + b * bstride;
-    mbar_arrive_expect_tx(&bar, row_bytes * uint32_t(nload));
-    for (int rr = 0; rr < nload; ++rr) bulk_load(srow + rr * N, src + int64_t(__ldg(ib + rr)) * ld, row_bytes, &bar);
+  // zero padding: rows k_keep <= t < k_pad (split across CTAs), and columns N <= c < ldo
+  {
+    const int64_t pad_rows = k_pad - k_keep;
+    const int64_t pr = (pad_rows + gridDim.x - 1) / gridDim.x;
+    const int64_t pa = k_keep + min(pad_rows, int64_t(blockIdx.x) * pr), pb = min(k_pad, pa + pr);
+    for (int64_t t = pa; t < pb; ++t)
+      for (int64_t c = threadIdx.x; c < ldo; c += kPackThreads) outb[t * ldo + c] = T(0);
+    if (ldo > N)
+      for (int64_t t = t_begin; t < t_end; ++t)
+        for (int64_t c = N + threadIdx.x; c < ldo; c += kPackThreads) outb[t * ldo + c] = T(0);
   }
-  // padding rows (t >= k_keep) are zeros; padding columns N <= c < ldo too
-  for (int rr = nload; rr < nr; ++rr)
-    for (int64_t c = threadIdx.x; c < ldo; c += kPackThreads) dst[rr * ldo + c] = T(0);
-  if (ldo > N)
-    for (int rr = 0; rr < nload; ++rr)
-      for (int64_t c = N + threadIdx.x; c < ldo; c += kPackThreads) dst[rr * ldo + c] = T(0);
-  if (nload > 0) {
-    wait_loads(&bar, wait_ns, status, &never);
-    if (threadIdx.x == 0) {
-      for (int rr = 0; rr < nload; ++rr) bulk_store(dst + rr * ldo, srow + rr * N, row_bytes);
+  if (threadIdx.x == 0 && nchunks > 0) {
+    const T* src = X + b * bstride;
+    // chunk c: rows [t_begin + (c / segs)·rows_per_buf, ...), columns of
+    // segment c % segs, through buffer c % kRowRing
+    auto chunk = [&](int64_t c, int64_t& r0, int& nr, int64_t& c0, uint32_t& bytes) {
+      r0 = (c / segs) * rows_per_buf;
+      nr = int(min(int64_t(rows_per_buf), t_end - t_begin - r0));
+      c0 = (c % segs) * seg;
+      bytes = uint32_t(min(seg, N - c0) * int64_t(sizeof(T)));
+    };
+    auto issue_load = [&](int64_t c) {
+      int64_t r0, c0;
+      int nr;
+      uint32_t bytes;
+      chunk(c, r0, nr, c0, bytes);
+      T* buf = ring + (c % kRowRing) * buf_elems;
+      mbar_arrive_expect_tx(&bar[c % kRowRing], bytes * uint32_t(nr));
+      for (int r = 0; r < nr; ++r)
+        bulk_load(buf + r * seg, src + int64_t(sidx[r0 + r]) * ld + c0, bytes, &bar[c % kRowRing]);
+    };
+    int64_t issued = min(int64_t(kRowRing - 1), nchunks);
+    for (int64_t c = 0; c < issued; ++c) issue_load(c);
+    int64_t c = 0;
+    for (; c < nchunks; ++c) {
+      if (!mbar_wait_bounded(&bar[c % kRowRing], uint32_t((c / kRowRing) & 1), wait_ns, &never)) break;
+      int64_t r0, c0;
+      int nr;
+      uint32_t bytes;
+      chunk(c, r0, nr, c0, bytes);
+      T* buf = ring + (c % kRowRing) * buf_elems;
+      for (int r = 0; r < nr; ++r) bulk_store(outb + (t_begin + r0 + r) * ldo + c0, buf + r * seg, bytes);
       asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // smem stays live until read
+      if (issued < nchunks) {
+        // the buffer of chunk `issued` was last read by chunk c - 1's store
+        asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        issue_load(issued++);
+      }
     }
+    if (c < nchunks) {  // a wait ran out: record it, then let the loads in flight land
+      status_or(status, RMM_TIMEOUT_BIT);
+      for (int64_t d = c; d < issued; ++d)
+        mbar_wait_bounded(&bar[d % kRowRing], uint32_t((d / kRowRing) & 1), wait_ns, &never);
+    }
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // smem stays live until read
   }
 }
 
@@ -317,13 +364,26 @@ cudaError_t launch_pack_rows_t(const MatView& X, int64_t batch, const int32_t* i
                     aligned16(out) && (X.ld * int64_t(sizeof(T))) % 16 == 0 &&
                     (batch == 1 || (X.bstride * int64_t(sizeof(T))) % 16 == 0) && (ldo * int64_t(sizeof(T))) % 16 == 0;
   if (bulk) {
-    const int rows_per_cta =
-        row_bytes <= kStageBytes ? int(std::min<size_t>(64, kStageBytes / row_bytes)) : 1;
-    const size_t smem = size_t(rows_per_cta) * row_bytes;
-    set_smem_attr_once(pack_rows_bulk_kernel<T>);
-    const dim3 grid(unsigned((k_pad + rows_per_cta - 1) / rows_per_cta), unsigned(batch), 1u);
-    return launch_pdl(pack_rows_bulk_kernel<T>, grid, dim3(kPackThreads), smem, st, dim3(0, 0, 0), p, X.ld, X.bstride, X.cols, idx,
-                      k_keep, k_pad, o, ldo, rows_per_cta, status, wait_ns);
+    // ring of kRowRing buffers of up to 16 KB (at least one row each)
+    // ring of kRowRing buffers of 16 KB: several whole rows, or a segment of a long row
+    const int rows_per_buf = row_bytes <= 16384 ? int(std::min<size_t>(32, 16384 / row_bytes)) : 1;
+    const int64_t seg = row_bytes <= 16384 ? X.cols : int64_t(16384 / sizeof(T));
+    const size_t smem = size_t(kRowRing) * rows_per_buf * size_t(seg) * sizeof(T) + size_t(kRowIdxStage) * 4;
+    if (smem <= kSmemAttr) {
+      set_smem_attr_once(pack_rows_bulk_kernel<T>);
+      int dev = 0, sms = 148;
+      cudaGetDevice(&dev);
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      // about two CTAs per SM over the whole batch, each streaming >= 4 buffers,
+      // and few enough kept rows per CTA for its index stage
+      const int64_t want = std::max<int64_t>(1, 2 * int64_t(sms) / std::max<int64_t>(1, batch));
+      const int64_t segs = (X.cols + seg - 1) / seg;
+      const int64_t by_work = std::max<int64_t>(1, k_keep * segs / (4 * rows_per_buf));
+      const int64_t ctas = std::max(std::min(want, by_work), (k_keep + kRowIdxStage - 1) / kRowIdxStage);
+      const dim3 grid(unsigned(ctas), unsigned(batch), 1u);
+      return launch_pdl(pack_rows_bulk_kernel<T>, grid, dim3(kPackThreads), smem, st, dim3(0, 0, 0), p, X.ld,
+                        X.bstride, X.cols, idx, k_keep, k_pad, o, ldo, rows_per_buf, seg, status, wait_ns);
+    }
   }
   return launch_pdl(pack_rows_plain_kernel<T>, dim3(unsigned(k_pad), unsigned(batch)), dim3(kPackThreads), 0, st, dim3(0, 0, 0),
                     p, X.ld, X.bstride, X.cols, idx, k_keep, k_pad, o, ldo);

@@ -26,6 +26,7 @@ namespace rmm {
 namespace {
 
 constexpr int kScoreThreads = 256;
+constexpr unsigned kMaxCluster = 8;  // CTAs sharing one strip (portable cluster size; 16 measured slower)
 constexpr int kUnroll = 8;
 
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
@@ -220,7 +221,7 @@ cudaError_t launch_t(const MatView& A, const MatView& B, int64_t batch, float* s
   const int64_t work_rows =
       A.rows + (BMODE == 2 ? B.rows : 0) + (BMODE == 1 ? CW * B.cols * int64_t(sizeof(T)) / 128 : 0);
   unsigned cs = 1;
-  while (cs < 8 && work_rows >= int64_t(cs) * 2 * 256) cs *= 2;
+  while (cs < kMaxCluster && work_rows >= int64_t(cs) * 2 * 256) cs *= 2;
   const int a_vec = aligned16(A.ptr) && (A.ld * int64_t(sizeof(T))) % 16 == 0 &&
                     (batch == 1 || (A.bstride * int64_t(sizeof(T))) % 16 == 0);
   const int b_vec = BMODE == 0 ? 0
