@@ -255,6 +255,17 @@ int rmm_set_gemm_cta_group(int cta_group);
 /* Number of kernels this library has launched in this process. */
 uint64_t rmm_launch_count(void);
 
+/* Timing hook (diagnostics; no counterpart in the method). While set, every
+ * GEMM launch of this process records `start` on its stream immediately
+ * before the GEMM kernel and `stop` immediately after it, so that
+ * cudaEventElapsedTime(start, stop) is that kernel alone (a split-K zeroing
+ * kernel of rmm_gemm runs before `start`). The events are created and owned
+ * by the caller; pass NULL, NULL to clear. Recording an event between two
+ * kernels ends their programmatic launch overlap, so the hook perturbs the
+ * timing of whatever surrounds the GEMM. Process-wide; not for concurrent
+ * callers. */
+void rmm_set_gemm_events(cudaEvent_t start, cudaEvent_t stop);
+
 #ifdef __cplusplus
 }
 #endif

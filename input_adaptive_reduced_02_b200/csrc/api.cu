@@ -19,6 +19,7 @@ static std::atomic<uint64_t> g_launches{0};
 static std::atomic<uint64_t> g_wait_limit_ns{0};
 static std::atomic<int> g_stall_producer{0};
 static std::atomic<int> g_cta_group{2};
+static std::atomic<cudaEvent_t> g_ev_start{nullptr}, g_ev_stop{nullptr};
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -139,9 +140,8 @@ static rmm_status do_pack(const void* A, int64_t lda, int64_t sA, const void* B,
   return RMM_OK;
 }
 
-static rmm_status do_gemm(const void* A_S, const void* B_S, int b_kmajor, int64_t batch, int64_t M, int64_t N,
-                          int64_t k_keep, rmm_dtype in, void* C, int64_t ldc, int64_t sC, rmm_dtype out,
-                          uint32_t* status, cudaStream_t st) {
+static GemmArgs gemm_args(const void* A_S, const void* B_S, int b_kmajor, int64_t batch, int64_t M, int64_t N,
+                          int64_t k_keep, void* C, int64_t ldc, int64_t sC, rmm_dtype out, uint32_t* status) {
   GemmArgs g;
   g.a = A_S;
   g.b = B_S;
@@ -159,6 +159,13 @@ static rmm_status do_gemm(const void* A_S, const void* B_S, int b_kmajor, int64_
   g.wait_limit_ns = wait_limit();
   g.stall_producer = g_stall_producer.load();
   g.cta_group = g_cta_group.load();
+  g.c_zeroed = 0;
+  g.ev_start = g_ev_start.load();
+  g.ev_stop = g_ev_stop.load();
+  return g;
+}
+
+static rmm_status do_gemm(const GemmArgs& g, rmm_dtype in, cudaStream_t st) {
   cudaError_t ce;
   const char* why = nullptr;
   if (in == RMM_BF16)
@@ -273,7 +280,7 @@ rmm_status rmm_gemm(const void* A_S, const void* B_S, int b_kmajor, int64_t batc
   if (!A_S || !B_S || !C) return fail(RMM_ERR_INVALID, "A_S, B_S or C is NULL");
   rmm_status r = bind_device(stream);
   if (r) return r;
-  return do_gemm(A_S, B_S, b_kmajor, batch, M, N, k_keep, in, C, ldc, strideC, out, status_word, stream);
+  return do_gemm(gemm_args(A_S, B_S, b_kmajor, batch, M, N, k_keep, C, ldc, strideC, out, status_word), in, stream);
 }
 
 rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb,
@@ -303,13 +310,20 @@ rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t stride
   int32_t* idx = idx_out ? idx_out : w.idx;
   if ((r = do_score(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, in, mode, w.s, w.status, stream)))
     return r;
-  ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream);
+  // The select runs on one SM per batch item; the C tiles that the GEMM's
+  // split-K round adds into are zeroed meanwhile by helper blocks of the same
+  // launch instead of by a launch of their own.
+  GemmArgs g = gemm_args(w.a_s, w.b_st, b_kmajor, batch, M, N, k_keep, C, ldc, strideC, out, w.status);
+  SplitZero z;
+  const bool zero = in == RMM_BF16 && gemm_tc_split_zero(g, &z);
+  ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr);
   if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
+  g.c_zeroed = zero ? 1 : 0;
   if (M == 0 || N == 0) return RMM_OK;
   if ((r = do_pack(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, idx, k_keep, in, w.a_s, w.b_st,
                    w.status, stream)))
     return r;
-  return do_gemm(w.a_s, w.b_st, b_kmajor, batch, M, N, k_keep, in, C, ldc, strideC, out, w.status, stream);
+  return do_gemm(g, in, stream);
 }
 
 rmm_status rmm_matmul_reduced(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t M, int64_t K, int64_t N,
@@ -364,3 +378,8 @@ int rmm_set_gemm_cta_group(int cta_group) {
 uint64_t rmm_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"
+
+void rmm_set_gemm_events(cudaEvent_t start, cudaEvent_t stop) {
+  g_ev_start.store(start);
+  g_ev_stop.store(stop);
+}

@@ -94,9 +94,15 @@ gemm_simt_kernel(const float* __restrict__ A, const float* __restrict__ Bp, int 
 cudaError_t launch_gemm_simt(const GemmArgs& g, cudaStream_t st) {
   if (g.batch == 0 || g.M == 0 || g.N == 0) return cudaSuccess;
   dim3 grid(unsigned((g.N + ST - 1) / ST), unsigned((g.M + ST - 1) / ST), unsigned(g.batch));
-  return launch_pdl(gemm_simt_kernel, grid, dim3(256), 0, st, dim3(0, 0, 0), static_cast<const float*>(g.a),
-                    static_cast<const float*>(g.b), g.b_kmajor, g.ldb, g.c, g.M, g.N, g.k_pad, g.ldc, g.strideC,
-                    int(g.out == kBF16));
+  if (g.ev_start) {
+    cudaError_t e = cudaEventRecord(g.ev_start, st);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = launch_pdl(gemm_simt_kernel, grid, dim3(256), 0, st, dim3(0, 0, 0),
+                             static_cast<const float*>(g.a), static_cast<const float*>(g.b), g.b_kmajor, g.ldb, g.c,
+                             g.M, g.N, g.k_pad, g.ldc, g.strideC, int(g.out == kBF16));
+  if (e == cudaSuccess && g.ev_stop) e = cudaEventRecord(g.ev_stop, st);
+  return e;
 }
 
 }  // namespace rmm

@@ -22,7 +22,9 @@
 // i+1. Tiles are visited m-fastest so a column block of B is shared through
 // L2 by the pairs working on it at the same time. When the tile count leaves
 // the last round less than half full, those tiles are split in two along K
-// and both halves reduce-add (f32) into C, which a small kernel zeroes first.
+// and both halves reduce-add (f32) into C, whose tiles are zeroed beforehand
+// (by a small kernel, or within the fused call by spare blocks of the select
+// launch, which leaves all but one SM per batch item idle).
 //
 // Every mbarrier wait is bounded (rmm_set_wait_limit_ns). A role whose wait
 // runs out records RMM_STATUS_BIT_TIMEOUT, raises its CTA's abort flag, and
@@ -403,37 +405,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 1) tmem_dealloc<CG>(tmem_base, Cfg::TMEM_COLS);
 }
 
-// Zero the f32 C tiles [first_tile, first_tile + gridDim.x) that receive two
-// reduce-adds (split K). Waits for its predecessor first: C may still be
-// written by earlier work on the stream, and the GEMM launched after this
-// kernel relies on it having waited.
-__global__ void __launch_bounds__(256)
-zero_split_tiles_kernel(float* __restrict__ C, int64_t ldc, int64_t strideC, TcParams p, int64_t first_tile,
-                        int32_t tile_rows, int32_t tile_cols) {
+// Zero the f32 C tiles that the split-K round reduce-adds into. Waits for its
+// predecessor first: C may still be written by earlier work on the stream, and
+// the GEMM launched after this kernel relies on it having waited.
+__global__ void __launch_bounds__(256) zero_split_tiles_kernel(const SplitZero z) {
   pdl_trigger();
   pdl_wait();
-  int32_t b, mb, nb;
-  decode_tile(first_tile + blockIdx.x, p, b, mb, nb);
-  const int64_t r0 = int64_t(mb) * tile_rows, c0 = int64_t(nb) * tile_cols;
-  const int64_t r1 = min(int64_t(p.M), r0 + tile_rows), c1 = min(int64_t(p.N), c0 + tile_cols);
-  const int64_t rows_per = (tile_rows + gridDim.y - 1) / gridDim.y;
-  const int64_t ra = r0 + int64_t(blockIdx.y) * rows_per, rb = min(r1, ra + rows_per);
-  if (ra >= rb) return;
-  float* base = C + int64_t(b) * strideC;
-  const int vec_per_row = (tile_cols + 3) / 4;  // 16-byte slots per tile row
-  const int64_t n = (rb - ra) * vec_per_row;
-  // consecutive threads write consecutive 16 bytes of a row; rows start 16-byte
-  // aligned (ldc, strideC and c0 are multiples of 4)
-  for (int64_t v = threadIdx.x; v < n; v += 256) {
-    const int64_t r = ra + v / vec_per_row;
-    const int64_t c = c0 + (v % vec_per_row) * 4;
-    float* dst = base + r * ldc + c;
-    if (c + 4 <= c1) {
-      *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
-    } else {
-      for (int64_t j = c; j < c1; ++j) base[r * ldc + j] = 0.f;
-    }
-  }
+  zero_split_tiles(z, blockIdx.x, gridDim.x, threadIdx.x, 256);
 }
 
 // ------------------------------------------------------------------ host side
@@ -499,6 +477,60 @@ DevInfo& dev_info(int dev) {
   return d;
 }
 
+// C through TMA tile stores: rows 16-byte aligned and a tensor map that encodes.
+bool encode_c(const GemmArgs& g, CUtensorMap* tmC) {
+  const uint64_t eb = g.out == kBF16 ? 2 : 4;
+  const bool c_ok = (reinterpret_cast<uintptr_t>(g.c) & 15u) == 0 && (uint64_t(g.ldc) * eb) % 16 == 0 &&
+                    (g.batch == 1 || (uint64_t(g.strideC) * eb) % 16 == 0);
+  if (!c_ok) return false;
+  const uint64_t s2 = g.batch == 1 ? uint64_t(g.ldc) * eb * uint64_t(g.M) : uint64_t(g.strideC) * eb;
+  return encode_3d(tmC, g.out == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.c,
+                   uint64_t(g.N), uint64_t(g.M), uint64_t(g.batch), uint64_t(g.ldc) * eb, s2 == 0 ? 16 : s2,
+                   uint32_t(128 / eb), 32);
+}
+
+// Tile grid and K split of one launch. Tiles are visited m-fastest; the pairs
+// (units) take them round-robin. When the last round would leave more than
+// half the pairs idle, its tiles are split along K into two halves that
+// reduce-add (f32, TMA) into C zeroed beforehand; with C zero, a + b == b + a
+// keeps the result independent of which half lands first.
+struct Plan {
+  int32_t tiles_m, tiles_n, num_kb, bn, bm;
+  int64_t total_tiles, units, rem;
+  bool split;
+};
+
+Plan make_plan(const GemmArgs& g, int sms, bool c_tma) {
+  Plan q;
+  const int cg = g.cta_group == 1 ? 1 : 2;
+  q.bn = g.N <= 128 ? 128 : 256;
+  q.bm = BM * cg;
+  q.tiles_m = int32_t((g.M + q.bm - 1) / q.bm);
+  q.tiles_n = int32_t((g.N + q.bn - 1) / q.bn);
+  q.num_kb = int32_t(g.k_pad / BK);
+  q.total_tiles = int64_t(q.tiles_m) * q.tiles_n * g.batch;
+  q.units = std::max<int64_t>(1, (sms > 0 ? sms : 148) / cg);
+  q.rem = q.total_tiles % q.units;
+  q.split = g.out == kF32 && c_tma && q.num_kb >= 2 && q.rem > 0 && 2 * q.rem <= q.units;
+  return q;
+}
+
+SplitZero split_zero(const GemmArgs& g, const Plan& q) {
+  SplitZero z;
+  z.c = static_cast<float*>(g.c);
+  z.ldc = g.ldc;
+  z.strideC = g.batch == 1 ? 0 : g.strideC;
+  z.M = g.M;
+  z.N = g.N;
+  z.first_tile = q.total_tiles - q.rem;
+  z.count = q.split ? q.rem : 0;
+  z.tiles_m = q.tiles_m;
+  z.tiles_n = q.tiles_n;
+  z.tile_rows = q.bm;
+  z.tile_cols = q.bn;
+  return z;
+}
+
 template <int BN, bool BMN, int CG>
 cudaError_t launch_cfg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, const char** why) {
   using Cfg = TcCfg<BN, CG>;
@@ -518,27 +550,21 @@ cudaError_t launch_cfg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, co
     *why = "cuTensorMapEncodeTiled failed for a packed operand";
     return cudaErrorInvalidValue;
   }
-  const uint64_t eb = g.out == kBF16 ? 2 : 4;
-  const bool c_ok = (reinterpret_cast<uintptr_t>(g.c) & 15u) == 0 && (uint64_t(g.ldc) * eb) % 16 == 0 &&
-                    (g.batch == 1 || (uint64_t(g.strideC) * eb) % 16 == 0);
-  int tma_store = 0;
-  if (c_ok) {
-    const uint64_t s2 = g.batch == 1 ? uint64_t(g.ldc) * eb * uint64_t(g.M) : uint64_t(g.strideC) * eb;
-    tma_store = encode_3d(&tmC, g.out == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                          g.c, uint64_t(g.N), uint64_t(g.M), uint64_t(g.batch), uint64_t(g.ldc) * eb,
-                          s2 == 0 ? 16 : s2, uint32_t(128 / eb), 32)
-                    ? 1
-                    : 0;
-  }
+  const int tma_store = encode_c(g, &tmC) ? 1 : 0;
   if (!tma_store) tmC = tmA;  // never dereferenced when tma_store == 0
+  const Plan q = make_plan(g, di.sms, tma_store != 0);
+  if (q.bn != BN || q.bm != BM * CG) {
+    *why = "internal: tile plan does not match the launched configuration";
+    return cudaErrorInvalidValue;
+  }
 
   TcParams p;
   p.M = int32_t(g.M);
   p.N = int32_t(g.N);
-  p.num_kb = int32_t(g.k_pad / BK);
-  p.tiles_m = int32_t((g.M + BM * CG - 1) / (BM * CG));
-  p.tiles_n = int32_t((g.N + BN - 1) / BN);
-  p.total_tiles = int64_t(p.tiles_m) * p.tiles_n * g.batch;
+  p.num_kb = q.num_kb;
+  p.tiles_m = q.tiles_m;
+  p.tiles_n = q.tiles_n;
+  p.total_tiles = q.total_tiles;
   p.status = g.status;
   p.wait_limit_ns = g.wait_limit_ns;
   p.stall_producer = g.stall_producer;
@@ -547,25 +573,25 @@ cudaError_t launch_cfg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, co
   p.c = g.c;
   p.ldc = g.ldc;
   p.strideC = g.strideC;
-  const int64_t units = std::max<int64_t>(1, (di.sms > 0 ? di.sms : 148) / CG);
-  // Split the K range of the last round's tiles when that round would leave
-  // more than half the pairs idle (f32 output through TMA only: the two halves
-  // reduce-add into C, and with C zeroed first a + b == b + a keeps the
-  // result independent of which half lands first).
-  const int64_t rem = p.total_tiles % units;
-  const bool split = g.out == kF32 && tma_store && p.num_kb >= 2 && rem > 0 && 2 * rem <= units;
-  p.full_units = split ? p.total_tiles - rem : p.total_tiles;
-  p.total_units = split ? p.full_units + 2 * rem : p.total_tiles;
+  const int64_t units = q.units;
+  p.full_units = q.split ? p.total_tiles - q.rem : p.total_tiles;
+  p.total_units = q.split ? p.full_units + 2 * q.rem : p.total_tiles;
   p.kb_mid = p.num_kb / 2;
-  if (split) {
-    cudaError_t e = launch_pdl(zero_split_tiles_kernel, dim3(unsigned(rem), 8u), dim3(256), 0, st, dim3(0, 0, 0),
-                               static_cast<float*>(g.c), g.ldc, g.batch == 1 ? int64_t(0) : g.strideC, p,
-                               p.full_units, int32_t(BM * CG), int32_t(BN));
+  if (q.split && !g.c_zeroed) {
+    const SplitZero z = split_zero(g, q);
+    cudaError_t e = launch_pdl(zero_split_tiles_kernel, dim3(unsigned(std::min<int64_t>(z.count * 8, 1184))),
+                               dim3(256), 0, st, dim3(0, 0, 0), z);
     if (e != cudaSuccess) return e;
   }
   const int64_t grid = CG * std::min<int64_t>(p.total_units, units);
-  return launch_pdl(gemm_tc_kernel<BN, BMN, CG>, dim3(unsigned(grid)), dim3(kTcThreads), Cfg::SMEM, st,
-                    CG == 2 ? dim3(2, 1, 1) : dim3(0, 0, 0), tmA, tmB, tmC, p);
+  if (g.ev_start) {
+    cudaError_t e = cudaEventRecord(g.ev_start, st);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = launch_pdl(gemm_tc_kernel<BN, BMN, CG>, dim3(unsigned(grid)), dim3(kTcThreads), Cfg::SMEM, st,
+                             CG == 2 ? dim3(2, 1, 1) : dim3(0, 0, 0), tmA, tmB, tmC, p);
+  if (e == cudaSuccess && g.ev_stop) e = cudaEventRecord(g.ev_stop, st);
+  return e;
 }
 
 template <int CG>
@@ -576,6 +602,18 @@ cudaError_t launch_cg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, con
 }
 
 }  // namespace
+
+bool gemm_tc_split_zero(const GemmArgs& g, SplitZero* z) {
+  if (g.batch == 0 || g.M == 0 || g.N == 0) return false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const DevInfo& di = dev_info(dev);
+  CUtensorMap tmC;
+  const Plan q = make_plan(g, di.sms, encode_c(g, &tmC));
+  if (!q.split) return false;
+  *z = split_zero(g, q);
+  return true;
+}
 
 cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st, const char** why) {
   if (g.batch == 0 || g.M == 0 || g.N == 0) return cudaSuccess;

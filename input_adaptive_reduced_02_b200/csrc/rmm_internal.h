@@ -60,9 +60,23 @@ void set_last_error(const char* msg);
 cudaError_t launch_score(const MatView& A, const MatView& B, int bmode, ElemKind e, int64_t batch, float* s,
                          uint32_t* status, cudaStream_t st);
 
+// f32 C tiles that the tensor-core GEMM's split-K round reduce-adds into, and
+// which must therefore hold zeros before it starts: `count` tiles of
+// tile_rows x tile_cols starting at tile `first_tile` of the m-fastest tile
+// order (tiles_m x tiles_n per batch item), clipped to M x N.
+struct SplitZero {
+  float* c;
+  int64_t ldc, strideC;
+  int64_t M, N;
+  int64_t first_tile, count;
+  int32_t tiles_m, tiles_n, tile_rows, tile_cols;
+};
+
 // select.cu
+//  Blocks [batch, batch + zero_blocks) of the launch zero `zero`'s tiles
+//  meanwhile (zero may be null); the select itself uses one block per item.
 cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,
-                          uint32_t* status, cudaStream_t st);
+                          uint32_t* status, cudaStream_t st, const SplitZero* zero = nullptr);
 
 // pack.cu
 //  out[b][r][t] = X[b][r][idx[b][t]] for t < k_keep, 0 for k_keep <= t < k_pad.
@@ -88,9 +102,13 @@ struct GemmArgs {
   uint64_t wait_limit_ns;
   int stall_producer;
   int cta_group;
+  int c_zeroed;  // 1: the tiles gemm_tc_split_zero names are already zero
+  cudaEvent_t ev_start, ev_stop;  // recorded around the GEMM kernel when non-null
 };
 //  cta_group: 2 = 2-SM MMAs on CTA pairs (default), 1 = one SM per tile.
 cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st, const char** why);
+//  The tiles launch_gemm_tc(g) splits along K (false: it splits none).
+bool gemm_tc_split_zero(const GemmArgs& g, SplitZero* z);
 cudaError_t launch_gemm_simt(const GemmArgs& g, cudaStream_t st);
 
 }  // namespace rmm

@@ -12,6 +12,8 @@
 // kept whole, and how many keys equal to it must be kept. Two block-wide
 // scans then compact the kept indices in index order. Integer work only: the result
 // depends on the order of the scores, never on rounding.
+#include <algorithm>
+
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
 
@@ -64,7 +66,7 @@ constexpr int kBins = 1 << kDigitBits;
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS, 1)
 select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t* __restrict__ idx,
-              uint32_t* status, int keys_in_smem) {
+              uint32_t* status, int keys_in_smem, int64_t items, const SplitZero zero) {
   constexpr int kWarps = THREADS / 32;
   const int K = int(K64);  // K <= 2^21 (checked on the host)
   extern __shared__ uint32_t keys[];  // K keys when keys_in_smem
@@ -80,6 +82,10 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
 
   pdl_trigger();
   pdl_wait();
+  if (blockIdx.x >= items) {  // helper block: zero C tiles for the GEMM later on the stream
+    zero_split_tiles(zero, blockIdx.x - items, gridDim.x - items, tid, THREADS);
+    return;
+  }
   if (tid == 0) sh_nan = 0;
   __syncthreads();
   bool nan_seen = false;
@@ -212,8 +218,15 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
 }  // namespace
 
 cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,
-                          uint32_t* status, cudaStream_t st) {
+                          uint32_t* status, cudaStream_t st, const SplitZero* zero) {
   if (batch == 0) return cudaSuccess;
+  SplitZero z = {};
+  int64_t helpers = 0;
+  if (zero && zero->count > 0) {
+    z = *zero;
+    const int64_t vecs = z.count * z.tile_rows * (z.tile_cols / 4);
+    helpers = std::min<int64_t>(147, (vecs + 8 * kSelThreads - 1) / (8 * kSelThreads));
+  }
   const int keys_in_smem = K <= kSelSmemKeys;
   const size_t smem = keys_in_smem ? size_t(K) * 4 : 0;
   static bool attr_done[64] = {};
@@ -225,8 +238,8 @@ cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_ke
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-  return launch_pdl(select_kernel<kSelThreads>, dim3(unsigned(batch)), dim3(kSelThreads), smem, st, dim3(0, 0, 0), s,
-                    K, k_keep, idx, status, keys_in_smem);
+  return launch_pdl(select_kernel<kSelThreads>, dim3(unsigned(batch + helpers)), dim3(kSelThreads), smem, st,
+                    dim3(0, 0, 0), s, K, k_keep, idx, status, keys_in_smem, batch, z);
 }
 
 }  // namespace rmm

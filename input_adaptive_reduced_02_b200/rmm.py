@@ -62,6 +62,7 @@ _SIGS = {
     "rmm_set_stall_producer_for_test": (None, [_i32]),
     "rmm_set_gemm_cta_group": (_i32, [_i32]),
     "rmm_launch_count": (_u64, []),
+    "rmm_set_gemm_events": (None, [ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 
@@ -336,6 +337,18 @@ def set_gemm_cta_group(cta_group: int) -> int:
 
 def launch_count() -> int:
     return int(lib().rmm_launch_count())
+
+
+def set_gemm_events(start: torch.cuda.Event | None, stop: torch.cuda.Event | None):
+    """Record `start`/`stop` immediately around every GEMM kernel launch (None, None clears)."""
+    def handle(e):
+        if e is None:
+            return ctypes.c_void_p(0)
+        if not e.cuda_event:  # torch creates the CUDA event on its first record
+            e.record()
+        return ctypes.c_void_p(e.cuda_event)
+
+    lib().rmm_set_gemm_events(handle(start), handle(stop))
 
 
 def matmul_reduced_noalloc(A: torch.Tensor, B: torch.Tensor, rho: float, mode: str = "product",

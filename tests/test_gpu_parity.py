@@ -213,3 +213,53 @@ def test_launch_counter_counts_kernels():
     torch.cuda.synchronize()
     # score (one launch for A's and B's norms), select, pack (A, B), gemm
     assert rmm.launch_count() - n0 == 5
+
+
+@pytest.mark.parametrize("batch", [1, 3])
+def test_split_k_tiles_zeroed_inside_the_select_launch(batch, gemm_cta_group):
+    """A shape whose last GEMM round is split along K (f32 C): in the fused call
+    the select launch's spare blocks zero those C tiles, so no separate zeroing
+    kernel runs; C is filled with NaN first, so a tile left unzeroed shows."""
+    M, K, N = 2048, 512, 1024
+    g = torch.Generator(device=DEV)
+    g.manual_seed(71 + batch)
+    A = torch.randn(batch, M, K, generator=g, device=DEV).to(torch.bfloat16)
+    B = torch.randn(batch, K, N, generator=g, device=DEV).to(torch.bfloat16)
+    out = torch.full((batch, M, N), float("nan"), device=DEV)
+    idx = torch.empty(batch, rmm.keep_count(0.5, K), dtype=torch.int32, device=DEV)
+    n0 = rmm.launch_count()
+    C, ws = rmm.matmul_reduced(A, B, 0.5, out=out, idx_out=idx)
+    torch.cuda.synchronize()
+    rmm.check(ws)
+    assert rmm.launch_count() - n0 == 5  # score, select (+ zeroing), pack A, pack B, gemm
+    for b in range(batch):
+        check_product(f64(C[b]), f64(A[b]), f64(B[b]), idx[b].cpu().numpy(), product_tol(torch.bfloat16, torch.float32))
+    # the stage-by-stage GEMM zeroes them with a kernel of its own
+    A_S, B_S = rmm.pack(A, B, idx)
+    out2 = torch.full((batch, M, N), float("nan"), device=DEV)
+    C2 = rmm.gemm(A_S, B_S, idx.shape[-1], N=N, out=out2)
+    assert torch.equal(C2, C)
+
+
+def test_gemm_event_hook_brackets_the_gemm_kernel():
+    """rmm_set_gemm_events: the events land around the GEMM kernel only (the
+    split-K zeroing kernel of the stage call runs before the first one)."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(81)
+    A_S = torch.randn(2048, 256, generator=g, device=DEV).to(torch.bfloat16)
+    B_S = torch.randn(256, 1024, generator=g, device=DEV).to(torch.bfloat16)
+    outer0, outer1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    C_ref = rmm.gemm(A_S, B_S, 256, N=1024)
+    outer0.record()
+    rmm.set_gemm_events(e0, e1)
+    try:
+        C = rmm.gemm(A_S, B_S, 256, N=1024)
+    finally:
+        rmm.set_gemm_events(None, None)
+    outer1.record()
+    torch.cuda.synchronize()
+    assert torch.equal(C, C_ref)
+    inner, outer = e0.elapsed_time(e1), outer0.elapsed_time(outer1)
+    assert 0 < inner <= outer
+    assert outer0.elapsed_time(e0) >= 0 and e1.elapsed_time(outer1) >= 0
