@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 from input_adaptive_reduced_02_b200 import inputs, rmm  # noqa: E402
 
 RHOS = (0.3, 0.5, 0.7, 0.9, 1.0)
+METRIC = "reduced-matmul effective TFLOP/s (kept FLOPs 2*M*N*k) and speedup vs rho=1"
 FLUSH_BYTES = 256 << 20
 SLEEP_CYCLES = 1_000_000  # ~0.5-0.8 ms: lets the host queue a whole step ahead of the GPU
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "gemm_tc_linear_4096_rho0.5.txt")
@@ -59,6 +60,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-sweep", action="store_true", help="skip the rho sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--score-mode", choices=["product", "a_only"], default="product",
+                    help="slice score: ||A[:,k]||·||B[k,:]|| (library default) or the pages' ||A[:,k]||")
+    ap.add_argument("--no-quality", action="store_true",
+                    help="skip the error check of top-k against random selection")
     return ap.parse_args(argv)
 
 
@@ -69,6 +74,7 @@ class Problem:
     def __init__(self, name, A, B, b_kmajor, out_dtype, rho, descr):
         self.name, self.A, self.B, self.b_kmajor = name, A, B, b_kmajor
         self.out_dtype, self.rho, self.descr = out_dtype, rho, descr
+        self.mode = "product"
         A3 = A if A.dim() == 3 else A.unsqueeze(0)
         B3 = B if B.dim() == 3 else B.unsqueeze(0)
         self.batch, self.M, self.K = A3.shape
@@ -155,7 +161,7 @@ class Pipeline:
         k, idx, A_S, B_S = self.views(rho)
         if ev:
             ev[0].record()
-        rmm.score(p.A, p.B, "product", p.b_kmajor, out=self.s, status=self.status)
+        rmm.score(p.A, p.B, p.mode, p.b_kmajor, out=self.s, status=self.status)
         if ev and breakdown:
             ev[1].record()
         rmm.select(self.s, k, out=idx, status=self.status)
@@ -180,19 +186,26 @@ STAGES = ("score", "select", "pack", "gemm")
 
 class Fused:
     """The one-call public path: rmm_matmul_reduced into a preallocated C with a
-    reusable workspace (sized for rho_max)."""
+    reusable workspace (sized for rho_max). With b_norm, the call with B's
+    norms cached (rmm_matmul_reduced_b_norms; the norms are computed once,
+    outside the timed steps, as a caller would for a weight)."""
 
-    def __init__(self, p: Problem, rho_max: float):
+    def __init__(self, p: Problem, rho_max: float, b_norm=None):
         self.p = p
         dev = p.A.device
         self.C = torch.empty((p.batch, p.M, p.N) if p.A.dim() == 3 else (p.M, p.N), dtype=p.out_dtype, device=dev)
         self.ws = rmm.Workspace(rmm.workspace_size(p.batch, p.M, p.K, p.N, p.k_keep(rho_max), p.A.dtype), dev)
+        self.b_norm = b_norm
 
     def step(self, rho, ev=None, breakdown=False):
         p = self.p
         if ev:
             ev[0].record()
-        rmm.matmul_reduced(p.A, p.B, rho, out=self.C, workspace=self.ws, b_kmajor=p.b_kmajor)
+        if self.b_norm is not None:
+            rmm.matmul_reduced_b_norms(p.A, p.B, self.b_norm, rho, out=self.C, workspace=self.ws,
+                                       b_kmajor=p.b_kmajor)
+        else:
+            rmm.matmul_reduced(p.A, p.B, rho, p.mode, out=self.C, workspace=self.ws, b_kmajor=p.b_kmajor)
         if ev:
             ev[1].record()
 
@@ -347,7 +360,7 @@ def oracle_cpu_timing(p: Problem, rho: float, budget_s: float, max_steps: int):
     while len(times) < max_steps and (not times or time.perf_counter() - t_start < budget_s):
         t0 = time.perf_counter()
         for b in range(A64.shape[0]):
-            O.matmul_reduced(A64[b], B64[b], rho, O.SCORE_PRODUCT)
+            O.matmul_reduced(A64[b], B64[b], rho, O.SCORE_A_ONLY if p.mode == "a_only" else O.SCORE_PRODUCT)
             if time.perf_counter() - t_start > 4 * budget_s:
                 break
         else:
@@ -410,15 +423,18 @@ def run_reference(args):
         return 0
     name = args.workload
     p = make_problem(name, "cpu", 0, args.rho)
+    p.mode = args.score_mode
     rho = p.rho
     from oracle import rmm_oracle as O  # noqa: F401
     budget = 150.0
     res = oracle_cpu_timing(p, rho, budget_s=budget, max_steps=max(1, args.steps))
-    line = {"impl": "reference", "metric": "reduced-matmul effective TFLOP/s (kept FLOPs)",
+    line = {"impl": "reference", "metric": METRIC,
             "value": res["value"] if res else None, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": 0, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": name, "rho": rho, "M": p.M, "K": p.K, "N": p.N,
-                                              "batch": p.batch, "k_keep": p.k_keep(rho)},
+            "data": "synthetic", "config": {"workload": name, "descr": p.descr, "batch": p.batch, "M": p.M,
+                                              "K": p.K, "N": p.N, "rho": rho, "k_keep": p.k_keep(rho),
+                                              "score_mode": p.mode,
+                                              "out_dtype": str(p.out_dtype).replace("torch.", "")},
             "cpu_baseline": res,
             "e2e": {"value": res["value"] if res else None, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -431,6 +447,7 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device(f"cuda:{local}")
     p = make_problem(args.workload, dev, seed=rank, rho=args.rho)
+    p.mode = args.score_mode
     rho = p.rho
     rho_max = rho if args.no_sweep else 1.0
     call = Fused(p, rho_max)
@@ -494,6 +511,24 @@ def run_ours(args):
     del pipe, call
     torch.cuda.empty_cache()
 
+    # the same call with B's norms cached (a weight's norms are computed once)
+    cached = None
+    if p.mode == "product":
+        bn = rmm.b_norms(p.B, p.b_kmajor)
+        ccall = Fused(p, rho, b_norm=bn)
+        for _ in range(3):
+            ccall.step(rho)
+        cms, _ = timed_steps(ccall, rho, max(10, args.steps // 2), flush)
+        rmm.check(ccall.ws)
+        cached = {"ms": round(statistics.median(cms), 5),
+                  "effective_tflops": round(p.kept_flops(rho) / (statistics.median(cms) * 1e-3) / 1e12, 3),
+                  "note": "rmm_matmul_reduced_b_norms with ||B[k,:]|| from rmm_b_norms computed once "
+                          "outside the timed steps; the score then reads A only"}
+        del ccall, bn
+        torch.cuda.empty_cache()
+
+    quality = None if args.no_quality else quality_check(p, rho, seed=rank)
+
     # end to end through the public call with host buffers
     e2e = None
     if not args.no_e2e:
@@ -514,13 +549,13 @@ def run_ours(args):
 
     if rank == 0:
         line = {
-            "metric": "reduced-matmul effective TFLOP/s (kept FLOPs 2*M*N*k) and speedup vs rho=1",
+            "metric": METRIC,
             "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if p.A.dtype == torch.bfloat16 else "f32",
             "data": "synthetic",
             "config": {"workload": p.name, "descr": p.descr, "batch": p.batch, "M": p.M, "K": p.K, "N": p.N,
-                       "rho": rho, "k_keep": p.k_keep(rho), "score_mode": "product",
+                       "rho": rho, "k_keep": p.k_keep(rho), "score_mode": p.mode,
                        "out_dtype": str(p.out_dtype).replace("torch.", ""),
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed before every timed step (256 MiB written, then another 256 MiB read)",
@@ -531,6 +566,9 @@ def run_ours(args):
                                  "calls, with events before and after the GEMM launch; the stage breakdown "
                                  "from a third pass with events between all stages"},
             "stages_ms": {s: round(v, 5) for s, v in stage_mean.items()},
+            "stages_gbs": stage_gbs(p, rho, stage_mean),
+            "cached_b_norm_call": cached,
+            "quality": quality,
             "staged_region_ms": {"step": round(statistics.mean(staged_ms), 5),
                                  "pre_gemm": round(statistics.mean(stage_ms["pre_gemm"]), 5),
                                  "gemm": round(gemm_ms_timed, 5)},
@@ -550,10 +588,66 @@ def run_ours(args):
     return 0
 
 
+def stage_bytes(p: Problem, rho):
+    """Algorithmic HBM bytes of each stage for one step (all batch items)."""
+    k = p.k_keep(rho)
+    kp = rmm.padded_keep(k)
+    eb = p.A.element_size()
+    ob = torch.tensor([], dtype=p.out_dtype).element_size()
+    b_read = 0 if p.mode == "a_only" else p.K * p.N * eb
+    ldb = p.N if p.b_kmajor else rmm.packed_b_ld(p.N)
+    return {
+        "score": (p.M * p.K * eb + b_read + 4 * p.K) * p.batch,
+        "select": (4 * p.K + 4 * k) * p.batch,
+        "pack": (p.M * p.K * eb + k * p.N * eb + p.M * kp * eb + kp * ldb * eb) * p.batch,
+        "gemm": ((p.M + p.N) * kp * eb + p.M * p.N * ob) * p.batch,
+    }
+
+
+def stage_gbs(p: Problem, rho, stage_mean):
+    by = stage_bytes(p, rho)
+    return {s: round(by[s] / (stage_mean[s] * 1e-3) / 1e9, 1) for s in stage_mean}
+
+
+def quality_check(p: Problem, rho, seed):
+    """Relative Frobenius error against the dense product (torch f32 matmul on
+    the GPU, a measurement reference only) of the library's top-k selection and
+    of a seeded random selection of the same size (the pages' baseline), both
+    through the library's pack and GEMM; first batch item only."""
+    A = p.A[0] if p.A.dim() == 3 else p.A
+    B = p.B[0] if p.B.dim() == 3 else p.B
+    k = p.k_keep(rho)
+    Bf = (B.t() if p.b_kmajor else B).float()
+    dense = A.float() @ Bf
+    nd = torch.linalg.norm(dense).item()
+    idx = torch.empty(k, dtype=torch.int32, device=A.device)
+    C, _ = rmm.matmul_reduced(A, B, rho, p.mode, torch.float32, idx_out=idx, b_kmajor=p.b_kmajor)
+    g = torch.Generator(device=A.device)
+    g.manual_seed(1000 + seed)
+    ridx = torch.randperm(p.K, generator=g, device=A.device)[:k].sort().values.to(torch.int32).contiguous()
+    A_S, B_S = rmm.pack(A, B, ridx, p.b_kmajor)
+    Cr = rmm.gemm(A_S, B_S, k, b_kmajor=p.b_kmajor, N=p.N)
+    torch.cuda.synchronize()
+    e_top = torch.linalg.norm(C - dense).item() / nd
+    e_rand = torch.linalg.norm(Cr - dense).item() / nd
+    return {"rel_fro_err_topk": round(e_top, 6), "rel_fro_err_random": round(e_rand, 6),
+            "score_mode": p.mode, "item": 0, "reference": "dense f32 product (torch matmul on the GPU)"}
+
+
 def roofline(p: Problem, rho, stage_mean, dominant, peaks, peak_src):
     k = p.k_keep(rho)
     eb = p.A.element_size()
     ob = torch.tensor([], dtype=p.out_dtype).element_size()
+    gemm_bytes = stage_bytes(p, rho)["gemm"]
+    ridge = (peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9)
+    if dominant == "gemm" and p.A.dtype == torch.bfloat16 and p.kept_flops(rho) / gemm_bytes < ridge:
+        # below the ridge (P·V, Q·Kᵀ's output write): the GEMM is bound by HBM
+        ach = gemm_bytes / (stage_mean["gemm"] * 1e-3) / 1e9
+        return {"kernel": "gemm_tc_kernel", "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
+                "algorithmic_bytes_per_launch": gemm_bytes,
+                "arithmetic_intensity": round(p.kept_flops(rho) / gemm_bytes, 1), "ridge": round(ridge, 1),
+                "peak_source": f"{peak_src} HBM copy bandwidth"}
     if dominant == "gemm" and p.M >= 128 and p.N >= 128:
         flops = p.kept_flops(rho)
         ach = flops / (stage_mean["gemm"] * 1e-3) / 1e12
@@ -564,12 +658,7 @@ def roofline(p: Problem, rho, stage_mean, dominant, peaks, peak_src):
                 "algorithmic_flops_per_launch": flops,
                 "peak_source": f"{peak_src} bf16 dense burst (cuBLAS)" if peak else "n/a (f32 CUDA-core path)"}
     # bandwidth-bound stage: algorithmic bytes per launch
-    by = {
-        "score": (p.M * p.K + p.K * p.N) * eb * p.batch + 4 * p.K * p.batch,
-        "select": (4 * p.K + 4 * k) * p.batch,
-        "pack": ((p.M * p.K + k * p.N) * eb + (p.M + p.N) * rmm.padded_keep(k) * eb) * p.batch,
-        "gemm": ((p.M + p.N) * rmm.padded_keep(k) * eb + p.M * p.N * ob) * p.batch,
-    }[dominant]
+    by = stage_bytes(p, rho)[dominant]
     ach = by / (stage_mean[dominant] * 1e-3) / 1e9
     return {"kernel": dominant, "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None, "algorithmic_bytes_per_launch": by,

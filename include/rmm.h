@@ -94,6 +94,9 @@ size_t rmm_workspace_size(int64_t batch, int64_t M, int64_t K, int64_t N, int64_
  *      if b_kmajor == 1, B is given transposed as [batch][N][K] (ld ldb), so
  *      "row k of B" is column k of that matrix (the Q·Kᵀ case, Kmat).
  *      B is not read in RMM_SCORE_A_ONLY mode and may be NULL there.
+ *      strideA / strideB may be 0 to use one matrix for every batch item (a
+ *      read-only input such as a weight); otherwise batch items must not
+ *      overlap. The same holds for every call that takes A and B.
  *   s: [batch][K] f32 output: s_k = sqrt(sum_i A[i,k]^2) · sqrt(sum_j B[k,j]^2)
  *      (product) or sqrt(sum_i A[i,k]^2) (a_only); sums in f32 in a fixed order,
  *      so repeated calls give identical bits.
@@ -172,6 +175,44 @@ rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t stride
                                       int64_t batch, int64_t M, int64_t K, int64_t N, double rho,
                                       rmm_dtype in, rmm_score_mode mode,
                                       void* C, int64_t ldc, int64_t strideC, rmm_dtype out,
+                                      int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream);
+
+/* ---------------------------------------------------------------- cached B norms
+ * B's factor of the product score, ||B[k,:]||_2, depends on B alone. When B is
+ * a weight that is reused across calls, it can be computed once with
+ * rmm_b_norms and passed to rmm_score_b_norms / rmm_matmul_reduced_b_norms,
+ * which then read only A to score (the selection and the product are
+ * computed as before). The cached scores agree with rmm_score's product
+ * scores to f32 rounding (B's norms are the same f32 sums for b_kmajor == 0;
+ * A's column sums may be grouped differently), so a near-tie can order
+ * differently; the result is deterministic either way. This is an
+ * implementation convenience; the pages' method has no separate step for it. */
+
+/* b_norm[b][k] = sqrt(sum_j B[b][k][j]^2) (b_kmajor == 0, B [batch][K][N]) or
+ * sqrt(sum_j Kmat[b][j][k]^2) (b_kmajor == 1, B = Kmat [batch][N][K]); f32,
+ * [batch][K] contiguous. status_word (nullable) receives
+ * RMM_STATUS_BIT_NONFINITE for a NaN/Inf norm. */
+rmm_status rmm_b_norms(const void* B, int64_t ldb, int64_t strideB, int b_kmajor,
+                       int64_t batch, int64_t K, int64_t N, rmm_dtype in, float* b_norm,
+                       uint32_t* status_word, cudaStream_t stream);
+
+/* rmm_score (product form) with B's norms given: s[b][k] = sqrt(sum_i A[b][i][k]^2)
+ * · b_norm[b·b_norm_stride + k]. b_norm_stride = 0 shares one [K] vector among
+ * all batch items (one weight for the whole batch), K when b_norm is
+ * [batch][K]. */
+rmm_status rmm_score_b_norms(const void* A, int64_t lda, int64_t strideA, const float* b_norm,
+                             int64_t b_norm_stride, int64_t batch, int64_t M, int64_t K,
+                             rmm_dtype in, float* s, uint32_t* status_word, cudaStream_t stream);
+
+/* rmm_matmul_reduced_batched in product mode with cached B norms (the score
+ * reads only A). Arguments as there, plus b_norm / b_norm_stride as in
+ * rmm_score_b_norms; workspace sized by rmm_workspace_size as before. */
+rmm_status rmm_matmul_reduced_b_norms(const void* A, int64_t lda, int64_t strideA,
+                                      const void* B, int64_t ldb, int64_t strideB, int b_kmajor,
+                                      const float* b_norm, int64_t b_norm_stride,
+                                      int64_t batch, int64_t M, int64_t K, int64_t N, double rho,
+                                      rmm_dtype in, void* C, int64_t ldc, int64_t strideC, rmm_dtype out,
                                       int32_t* idx_out, void* workspace, size_t workspace_bytes,
                                       cudaStream_t stream);
 

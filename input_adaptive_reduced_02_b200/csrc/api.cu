@@ -70,10 +70,13 @@ static ElemKind kind(rmm_dtype d) { return d == RMM_BF16 ? kBF16 : kF32; }
 
 // A batch of row-major matrices (rows x cols, leading dimension ld, batch
 // stride bstride) must fit its own declared layout.
-static bool layout_ok(int64_t batch, int64_t rows, int64_t cols, int64_t ld, int64_t bstride) {
+// Batch items must not overlap, except that a read-only input may repeat one
+// matrix for every item (bstride == 0, e.g. one weight for a batch).
+static bool layout_ok(int64_t batch, int64_t rows, int64_t cols, int64_t ld, int64_t bstride,
+                      bool broadcast_ok = false) {
   if (rows < 0 || cols < 0 || ld < 0 || bstride < 0) return false;
   if (rows > 1 && ld < cols) return false;
-  if (batch > 1 && rows > 0 && bstride < (rows - 1) * ld + cols) return false;
+  if (batch > 1 && rows > 0 && !(broadcast_ok && bstride == 0) && bstride < (rows - 1) * ld + cols) return false;
   return true;
 }
 
@@ -113,13 +116,15 @@ static Workspace carve(void* base, int64_t batch, int64_t M, int64_t K, int64_t 
 }
 
 // ---------------------------------------------------------------- stage bodies
+// bn non-null: product scores with B's norms given (B is not read).
 static rmm_status do_score(const void* A, int64_t lda, int64_t sA, const void* B, int64_t ldb, int64_t sB,
                            int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N, rmm_dtype in,
-                           rmm_score_mode mode, float* s, uint32_t* status, cudaStream_t st) {
+                           rmm_score_mode mode, float* s, uint32_t* status, cudaStream_t st,
+                           const float* bn = nullptr, int64_t bn_stride = 0) {
   const MatView a{A, lda, sA, M, K};
-  const int bmode = mode == RMM_SCORE_A_ONLY ? 0 : (b_kmajor ? 2 : 1);
+  const int bmode = bn ? 3 : (mode == RMM_SCORE_A_ONLY ? 0 : (b_kmajor ? 2 : 1));
   const MatView b = b_kmajor ? MatView{B, ldb, sB, N, K} : MatView{B, ldb, sB, K, N};
-  const cudaError_t ce = launch_score(a, b, bmode, kind(in), batch, s, status, st);
+  const cudaError_t ce = launch_score(a, b, bmode, kind(in), batch, s, status, st, bn, bn_stride);
   if (ce != cudaSuccess) return cuda_fail(ce, "score kernel");
   return RMM_OK;
 }
@@ -189,10 +194,10 @@ static rmm_status check_common(int64_t batch, int64_t M, int64_t K, int64_t N, r
 static rmm_status check_ab(const void* A, int64_t lda, int64_t sA, const void* B, int64_t ldb, int64_t sB,
                            int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N, bool need_b) {
   if (batch > 0 && M > 0 && !A) return fail(RMM_ERR_INVALID, "A is NULL");
-  if (!layout_ok(batch, M, K, lda, sA)) return fail(RMM_ERR_INVALID, "A layout (lda/strideA) is too small");
+  if (!layout_ok(batch, M, K, lda, sA, true)) return fail(RMM_ERR_INVALID, "A layout (lda/strideA) is too small");
   if (need_b) {
     if (batch > 0 && N > 0 && !B) return fail(RMM_ERR_INVALID, "B is NULL");
-    const bool ok = b_kmajor ? layout_ok(batch, N, K, ldb, sB) : layout_ok(batch, K, N, ldb, sB);
+    const bool ok = b_kmajor ? layout_ok(batch, N, K, ldb, sB, true) : layout_ok(batch, K, N, ldb, sB, true);
     if (!ok) return fail(RMM_ERR_INVALID, "B layout (ldb/strideB) is too small");
   }
   return RMM_OK;
@@ -283,11 +288,11 @@ rmm_status rmm_gemm(const void* A_S, const void* B_S, int b_kmajor, int64_t batc
   return do_gemm(gemm_args(A_S, B_S, b_kmajor, batch, M, N, k_keep, C, ldc, strideC, out, status_word), in, stream);
 }
 
-rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb,
-                                      int64_t strideB, int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N,
-                                      double rho, rmm_dtype in, rmm_score_mode mode, void* C, int64_t ldc,
-                                      int64_t strideC, rmm_dtype out, int32_t* idx_out, void* workspace,
-                                      size_t workspace_bytes, cudaStream_t stream) {
+static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb,
+                             int64_t strideB, int b_kmajor, const float* bn, int64_t bn_stride, int64_t batch,
+                             int64_t M, int64_t K, int64_t N, double rho, rmm_dtype in, rmm_score_mode mode, void* C,
+                             int64_t ldc, int64_t strideC, rmm_dtype out, int32_t* idx_out, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
   rmm_status r = check_common(batch, M, K, N, in);
   if (r) return r;
   if (!dtype_ok(out)) return fail(RMM_ERR_INVALID, "unknown output dtype");
@@ -308,7 +313,8 @@ rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t stride
   if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemsetAsync(status)");
   if (batch == 0) return RMM_OK;
   int32_t* idx = idx_out ? idx_out : w.idx;
-  if ((r = do_score(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, in, mode, w.s, w.status, stream)))
+  if ((r = do_score(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, in, mode, w.s, w.status, stream,
+                    bn, bn_stride)))
     return r;
   // The select runs on one SM per batch item; the C tiles that the GEMM's
   // split-K round adds into are zeroed meanwhile by helper blocks of the same
@@ -324,6 +330,13 @@ rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t stride
                    w.status, stream)))
     return r;
   return do_gemm(g, in, stream);
+}
+
+static rmm_status check_bn(const float* bn, int64_t bn_stride, int64_t batch, int64_t K) {
+  if (batch > 0 && !bn) return fail(RMM_ERR_INVALID, "b_norm is NULL");
+  if (bn_stride < 0 || (batch > 1 && bn_stride != 0 && bn_stride < K))
+    return fail(RMM_ERR_INVALID, "b_norm_stride must be 0 (shared) or >= K");
+  return RMM_OK;
 }
 
 rmm_status rmm_matmul_reduced(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t M, int64_t K, int64_t N,
@@ -382,4 +395,63 @@ uint64_t rmm_launch_count(void) { return g_launches.load(); }
 void rmm_set_gemm_events(cudaEvent_t start, cudaEvent_t stop) {
   g_ev_start.store(start);
   g_ev_stop.store(stop);
+}
+
+rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb,
+                                      int64_t strideB, int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N,
+                                      double rho, rmm_dtype in, rmm_score_mode mode, void* C, int64_t ldc,
+                                      int64_t strideC, rmm_dtype out, int32_t* idx_out, void* workspace,
+                                      size_t workspace_bytes, cudaStream_t stream) {
+  return fused_call(A, lda, strideA, B, ldb, strideB, b_kmajor, nullptr, 0, batch, M, K, N, rho, in, mode, C, ldc,
+                    strideC, out, idx_out, workspace, workspace_bytes, stream);
+}
+
+rmm_status rmm_b_norms(const void* B, int64_t ldb, int64_t strideB, int b_kmajor, int64_t batch, int64_t K, int64_t N,
+                       rmm_dtype in, float* b_norm, uint32_t* status_word, cudaStream_t stream) {
+  rmm_status r = check_common(batch, 1, K, N, in);
+  if (r) return r;
+  const int64_t rows = b_kmajor ? N : K, cols = b_kmajor ? K : N;
+  if (batch > 0 && (!B || !b_norm)) return fail(RMM_ERR_INVALID, "B or b_norm is NULL");
+  if (!layout_ok(batch, rows, cols, ldb, strideB, true))
+    return fail(RMM_ERR_INVALID, "B layout (ldb/strideB) is too small");
+  if (batch == 0 || N == 0) {
+    if (batch > 0 && N == 0 && b_norm) {
+      if ((r = bind_device(stream))) return r;
+      cudaError_t ce = cudaMemsetAsync(b_norm, 0, size_t(batch * K) * 4, stream);
+      if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemsetAsync(b_norm)");
+    }
+    return RMM_OK;
+  }
+  if ((r = bind_device(stream))) return r;
+  const cudaError_t ce = launch_b_norms(MatView{B, ldb, strideB, rows, cols}, b_kmajor, kind(in), batch, b_norm,
+                                        status_word, stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "b_norms kernel");
+  return RMM_OK;
+}
+
+rmm_status rmm_score_b_norms(const void* A, int64_t lda, int64_t strideA, const float* b_norm, int64_t b_norm_stride,
+                             int64_t batch, int64_t M, int64_t K, rmm_dtype in, float* s, uint32_t* status_word,
+                             cudaStream_t stream) {
+  rmm_status r = check_common(batch, M, K, 1, in);
+  if (r) return r;
+  if ((r = check_bn(b_norm, b_norm_stride, batch, K))) return r;
+  if (batch > 0 && M > 0 && !A) return fail(RMM_ERR_INVALID, "A is NULL");
+  if (!layout_ok(batch, M, K, lda, strideA, true))
+    return fail(RMM_ERR_INVALID, "A layout (lda/strideA) is too small");
+  if (batch > 0 && !s) return fail(RMM_ERR_INVALID, "s is NULL");
+  if (batch == 0) return RMM_OK;
+  if ((r = bind_device(stream))) return r;
+  return do_score(A, lda, strideA, nullptr, 0, 0, 0, batch, M, K, 0, in, RMM_SCORE_PRODUCT, s, status_word, stream,
+                  b_norm, b_norm_stride);
+}
+
+rmm_status rmm_matmul_reduced_b_norms(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb,
+                                      int64_t strideB, int b_kmajor, const float* b_norm, int64_t b_norm_stride,
+                                      int64_t batch, int64_t M, int64_t K, int64_t N, double rho, rmm_dtype in,
+                                      void* C, int64_t ldc, int64_t strideC, rmm_dtype out, int32_t* idx_out,
+                                      void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  rmm_status r = check_bn(b_norm, b_norm_stride, batch, K);
+  if (r) return r;
+  return fused_call(A, lda, strideA, B, ldb, strideB, b_kmajor, b_norm, b_norm_stride, batch, M, K, N, rho, in,
+                    RMM_SCORE_PRODUCT, C, ldc, strideC, out, idx_out, workspace, workspace_bytes, stream);
 }

@@ -26,6 +26,7 @@ constexpr int kPackThreads = 256;
 constexpr size_t kStageBytes = 32 * 1024;   // shared-memory rows per CTA (short rows)
 constexpr size_t kStageMax = 112 * 1024;    // one long row per CTA, two CTAs per SM
 constexpr size_t kSmemAttr = kStageMax + kStageBytes;  // + staged kept indices
+constexpr size_t kIdxStageMax = 64 * 1024;             // kept indices a pack_cols CTA stages
 
 template <typename T>
 union Vec16 {
@@ -57,10 +58,11 @@ __device__ __forceinline__ bool wait_loads(uint64_t* bar, uint64_t limit_ns, uin
 }
 
 // Gather kept columns of nr staged rows; ib points at the kept indices (in
-// shared memory or global memory, 16-byte aligned).
+// shared memory or global memory; read as 16-byte vectors when ib_vec, i.e.
+// ib is 16-byte aligned, else one by one).
 template <typename T>
-__device__ __forceinline__ void gather_rows(const T* srow, int nr, int64_t C, const int32_t* ib, int64_t k_keep,
-                                            int64_t k_pad, T* dst) {
+__device__ __forceinline__ void gather_rows(const T* srow, int nr, int64_t C, const int32_t* ib, bool ib_vec,
+                                            int64_t k_keep, int64_t k_pad, T* dst) {
   constexpr int V = 16 / sizeof(T);
   const int64_t ng = k_pad / V;
   for (int rr = 0; rr < nr; ++rr) {
@@ -68,7 +70,7 @@ __device__ __forceinline__ void gather_rows(const T* srow, int nr, int64_t C, co
     for (int64_t g = threadIdx.x; g < ng; g += kPackThreads) {
       const int64_t t0 = g * V;
       Vec16<T> v;
-      if (t0 + V <= k_keep) {
+      if (ib_vec && t0 + V <= k_keep) {
         const int4 i0 = *reinterpret_cast<const int4*>(ib + t0);
         if constexpr (V == 8) {
           const int4 i1 = *reinterpret_cast<const int4*>(ib + t0 + 4);
@@ -106,7 +108,9 @@ pack_cols_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int6
   const int nr = int(min(int64_t(rows_per_cta), R - r0));
   const T* src = X + b * bstride + r0 * ld;
   const int32_t* gidx = idx + b * k_keep;
-  const int64_t idx_bulk = idx_in_smem ? (k_keep & ~int64_t(3)) : 0;  // whole 16-byte groups
+  const bool gidx_vec = (reinterpret_cast<uintptr_t>(gidx) & 15u) == 0;
+  // whole 16-byte groups of indices by bulk copy when this item's list is aligned
+  const int64_t idx_bulk = (idx_in_smem && gidx_vec) ? (k_keep & ~int64_t(3)) : 0;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     never = 0;
@@ -118,14 +122,18 @@ pack_cols_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int6
   if (threadIdx.x == 0) {
     const uint32_t row_bytes = uint32_t(C * sizeof(T));
     mbar_arrive_expect_tx(&bar, row_bytes * uint32_t(nr) + uint32_t(idx_bulk * 4));
-    for (int rr = 0; rr < nr; ++rr) bulk_load(srow + rr * C, src + rr * ld, row_bytes, &bar);
+    if (ld == C)  // contiguous rows: one copy (each copy has a fixed cost; rows can be short)
+      bulk_load(srow, src, row_bytes * uint32_t(nr), &bar);
+    else
+      for (int rr = 0; rr < nr; ++rr) bulk_load(srow + rr * C, src + rr * ld, row_bytes, &bar);
     if (idx_bulk > 0) bulk_load(sidx, gidx, uint32_t(idx_bulk * 4), &bar);
   }
   if (idx_in_smem)
     for (int64_t t = idx_bulk + threadIdx.x; t < k_keep; t += kPackThreads) sidx[t] = gidx[t];
   wait_loads(&bar, wait_ns, status, &never);
   __syncthreads();
-  gather_rows(srow, nr, C, idx_in_smem ? sidx : gidx, k_keep, k_pad, out + (b * R + r0) * k_pad);
+  gather_rows(srow, nr, C, idx_in_smem ? sidx : gidx, idx_in_smem || gidx_vec, k_keep, k_pad,
+              out + (b * R + r0) * k_pad);
 }
 
 // Any alignment: rows staged with plain loads (eight in flight per thread).
@@ -337,13 +345,15 @@ cudaError_t launch_pack_cols_t(const MatView& X, int64_t batch, const int32_t* i
   }
   const int rows_per_cta =
       row_bytes <= kStageBytes ? int(std::min<size_t>(64, kStageBytes / std::max<size_t>(row_bytes, 1))) : 1;
-  const size_t idx_bytes = size_t(k_keep) * 4;
-  const int idx_in_smem = idx_bytes <= kStageBytes;
-  const size_t smem = size_t(rows_per_cta) * row_bytes + (idx_in_smem ? (idx_bytes + 15) / 16 * 16 : 0);
+  // kept indices in shared memory when they fit beside the rows (up to 64 KB;
+  // beyond that the gather reads them from global memory, through L1)
+  const size_t idx_bytes = (size_t(k_keep) * 4 + 15) / 16 * 16;
+  const int idx_in_smem = idx_bytes <= kIdxStageMax && size_t(rows_per_cta) * row_bytes + idx_bytes <= kSmemAttr;
+  const size_t smem = size_t(rows_per_cta) * row_bytes + (idx_in_smem ? idx_bytes : 0);
   const dim3 grid(unsigned((X.rows + rows_per_cta - 1) / rows_per_cta), unsigned(batch), 1u);
+  // any index alignment: each CTA stages or reads its item's list as aligned allows
   const bool bulk = aligned16(X.ptr) && row_bytes % 16 == 0 && (X.ld * int64_t(sizeof(T))) % 16 == 0 &&
-                    (batch == 1 || (X.bstride * int64_t(sizeof(T))) % 16 == 0) && aligned16(idx) &&
-                    (batch == 1 || k_keep % 4 == 0);
+                    (batch == 1 || (X.bstride * int64_t(sizeof(T))) % 16 == 0);
   if (bulk) {
     set_smem_attr_once(pack_cols_bulk_kernel<T>);
     return launch_pdl(pack_cols_bulk_kernel<T>, grid, dim3(kPackThreads), smem, st, dim3(0, 0, 0), p, X.ld,

@@ -57,8 +57,13 @@ void set_last_error(const char* msg);
 //  s[b][k] = sqrt(sum_i A[b][i][k]^2) · (bmode 1: sqrt(sum_j B[b][k][j]^2) with B
 //  row-major [K][N]; bmode 2: sqrt(sum_j B[b][j][k]^2) with B = Kmat [N][K];
 //  bmode 0: 1). One launch.
+//  bmode 3: s[b][k] = sqrt(sum_i A[b][i][k]^2) · bn[b * bn_stride + k] (B not read).
 cudaError_t launch_score(const MatView& A, const MatView& B, int bmode, ElemKind e, int64_t batch, float* s,
-                         uint32_t* status, cudaStream_t st);
+                         uint32_t* status, cudaStream_t st, const float* bn = nullptr, int64_t bn_stride = 0);
+//  out[b][k] = sqrt(sum_j B[b][k][j]^2) (B row-major [K][N], view rows = K) or, with
+//  b_kmajor, sqrt(sum_j B[b][j][k]^2) (B = Kmat [N][K], view rows = N, cols = K).
+cudaError_t launch_b_norms(const MatView& B, int b_kmajor, ElemKind e, int64_t batch, float* out, uint32_t* status,
+                           cudaStream_t st);
 
 // f32 C tiles that the tensor-core GEMM's split-K round reduce-adds into, and
 // which must therefore hold zeros before it starts: `count` tiles of

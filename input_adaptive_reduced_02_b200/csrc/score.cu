@@ -15,6 +15,7 @@
 //    through distributed shared memory and writes
 //    s_k = sqrt(sum_i A[i,k]^2) · sqrt(sum_j B[k,j]^2)  (or sqrt of A's sum).
 // Fixed summation order everywhere: bit-reproducible, no atomics, no scratch.
+#include <algorithm>
 #include <cooperative_groups.h>
 
 #include "rmm_device.cuh"
@@ -121,11 +122,13 @@ __device__ __forceinline__ float rowsq_warp(const T* __restrict__ row, int64_t C
 }
 
 // BMODE: 0 = A-only score; 1 = B row-major [K][N] (rows of the strip);
-//        2 = B given as Kmat [N][K] (columns of the strip).
+//        2 = B given as Kmat [N][K] (columns of the strip);
+//        3 = B's norms given (bn[b * bn_stride + k]).
 template <typename T, int BMODE>
 __global__ void __launch_bounds__(kScoreThreads)
 score_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, int64_t M, int64_t K,
              const T* __restrict__ B, int64_t ldb, int64_t sB, int64_t N,
+             const float* __restrict__ bn, int64_t bn_stride,
              float* __restrict__ s, uint32_t* status, int a_vec, int b_vec) {
   constexpr int V = 16 / sizeof(T);
   constexpr int CW = 8 * V;
@@ -196,11 +199,12 @@ score_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, int64_t M, int64_
     float ssa = 0.f, ssb = 0.f;
     for (unsigned q = 0; q < cs; ++q) {
       ssa += cluster.map_shared_rank(partA, q)[tid];
-      if constexpr (BMODE != 0) ssb += cluster.map_shared_rank(partB, q)[tid];
+      if constexpr (BMODE == 1 || BMODE == 2) ssb += cluster.map_shared_rank(partB, q)[tid];
     }
     if (c < K) {
       float sc = sqrtf(ssa);
-      if constexpr (BMODE != 0) sc *= sqrtf(ssb);
+      if constexpr (BMODE == 1 || BMODE == 2) sc *= sqrtf(ssb);
+      if constexpr (BMODE == 3) sc *= bn[b * bn_stride + c];
       s[b * K + c] = sc;
       if (!isfinite(sc)) status_or(status, RMM_NONFINITE_BIT);
     }
@@ -208,11 +212,39 @@ score_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, int64_t M, int64_
   cluster.sync();  // keep shared memory alive until rank 0 has read it
 }
 
+// b_norm[b][k] = sqrt(sum_j B[b][k][j]^2) for a row-major B: one warp per row,
+// the same per-row sum as the score kernel's product mode (bit-identical).
+template <typename T>
+__global__ void __launch_bounds__(kScoreThreads)
+bnorm_rows_kernel(const T* __restrict__ B, int64_t ldb, int64_t sB, int64_t K, int64_t N, int b_vec,
+                  float* __restrict__ out, uint32_t* status) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t b = blockIdx.y;
+  constexpr int kWarps = kScoreThreads / 32;
+  for (int64_t k = int64_t(blockIdx.x) * kWarps + warp; k < K; k += int64_t(gridDim.x) * kWarps) {
+    const float t = rowsq_warp<T>(B + b * sB + k * ldb, N, b_vec != 0, lane);
+    if (lane == 0) {
+      const float v = sqrtf(t);
+      out[b * K + k] = v;
+      if (!isfinite(v)) status_or(status, RMM_NONFINITE_BIT);
+    }
+  }
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 16-byte loads for B: base, rows and batch items 16-byte aligned.
+template <typename T>
+int b_vec_ok(const MatView& B, int64_t batch) {
+  return aligned16(B.ptr) && (B.ld * int64_t(sizeof(T))) % 16 == 0 &&
+         (batch == 1 || (B.bstride * int64_t(sizeof(T))) % 16 == 0);
+}
 
 template <typename T, int BMODE>
 cudaError_t launch_t(const MatView& A, const MatView& B, int64_t batch, float* s, uint32_t* status,
-                     cudaStream_t st) {
+                     cudaStream_t st, const float* bn = nullptr, int64_t bn_stride = 0) {
   constexpr int V = 16 / sizeof(T);
   constexpr int CW = 8 * V;
   const int64_t K = A.cols;
@@ -224,32 +256,53 @@ cudaError_t launch_t(const MatView& A, const MatView& B, int64_t batch, float* s
   while (cs < kMaxCluster && work_rows >= int64_t(cs) * 2 * 256) cs *= 2;
   const int a_vec = aligned16(A.ptr) && (A.ld * int64_t(sizeof(T))) % 16 == 0 &&
                     (batch == 1 || (A.bstride * int64_t(sizeof(T))) % 16 == 0);
-  const int b_vec = BMODE == 0 ? 0
-                    : aligned16(B.ptr) && (B.ld * int64_t(sizeof(T))) % 16 == 0 &&
-                          (batch == 1 || (B.bstride * int64_t(sizeof(T))) % 16 == 0);
+  const int b_vec = (BMODE == 0 || BMODE == 3) ? 0 : b_vec_ok<T>(B, batch);
   const int64_t N = BMODE == 2 ? B.rows : B.cols;
   return launch_pdl(score_kernel<T, BMODE>, dim3(unsigned((K + CW - 1) / CW), cs, unsigned(batch)),
                     dim3(kScoreThreads), 0, st, dim3(1, cs, 1), static_cast<const T*>(A.ptr), A.ld, A.bstride, A.rows, K,
-                    static_cast<const T*>(B.ptr), B.ld, B.bstride, N, s, status, a_vec, b_vec);
+                    static_cast<const T*>(B.ptr), B.ld, B.bstride, N, bn, bn_stride, s, status, a_vec, b_vec);
+}
+
+template <typename T>
+cudaError_t launch_bnorm_rows(const MatView& B, int64_t batch, float* out, uint32_t* status, cudaStream_t st) {
+  constexpr int kWarps = kScoreThreads / 32;
+  const int64_t ctas = std::min<int64_t>((B.rows + kWarps - 1) / kWarps, 148 * 8);
+  return launch_pdl(bnorm_rows_kernel<T>, dim3(unsigned(ctas), unsigned(batch)), dim3(kScoreThreads), 0, st,
+                    dim3(0, 0, 0), static_cast<const T*>(B.ptr), B.ld, B.bstride, B.rows, B.cols,
+                    b_vec_ok<T>(B, batch), out, status);
 }
 
 }  // namespace
 
 cudaError_t launch_score(const MatView& A, const MatView& B, int bmode, ElemKind e, int64_t batch, float* s,
-                         uint32_t* status, cudaStream_t st) {
+                         uint32_t* status, cudaStream_t st, const float* bn, int64_t bn_stride) {
   if (batch == 0 || A.cols == 0) return cudaSuccess;
   if (e == kBF16) {
     switch (bmode) {
       case 0: return launch_t<uint16_t, 0>(A, B, batch, s, status, st);
       case 1: return launch_t<uint16_t, 1>(A, B, batch, s, status, st);
-      default: return launch_t<uint16_t, 2>(A, B, batch, s, status, st);
+      case 2: return launch_t<uint16_t, 2>(A, B, batch, s, status, st);
+      default: return launch_t<uint16_t, 3>(A, B, batch, s, status, st, bn, bn_stride);
     }
   }
   switch (bmode) {
     case 0: return launch_t<uint32_t, 0>(A, B, batch, s, status, st);
     case 1: return launch_t<uint32_t, 1>(A, B, batch, s, status, st);
-    default: return launch_t<uint32_t, 2>(A, B, batch, s, status, st);
+    case 2: return launch_t<uint32_t, 2>(A, B, batch, s, status, st);
+    default: return launch_t<uint32_t, 3>(A, B, batch, s, status, st, bn, bn_stride);
   }
+}
+
+cudaError_t launch_b_norms(const MatView& B, int b_kmajor, ElemKind e, int64_t batch, float* out, uint32_t* status,
+                           cudaStream_t st) {
+  if (batch == 0 || B.rows == 0 || B.cols == 0) return cudaSuccess;
+  if (b_kmajor) {  // column norms of Kmat [N][K]: the A-only score of Kmat
+    const MatView none{nullptr, 0, 0, 0, 0};
+    return e == kBF16 ? launch_t<uint16_t, 0>(B, none, batch, out, status, st)
+                      : launch_t<uint32_t, 0>(B, none, batch, out, status, st);
+  }
+  return e == kBF16 ? launch_bnorm_rows<uint16_t>(B, batch, out, status, st)
+                    : launch_bnorm_rows<uint32_t>(B, batch, out, status, st);
 }
 
 }  // namespace rmm

@@ -56,6 +56,11 @@ _SIGS = {
                               ctypes.c_size_t, _vp]),
     "rmm_matmul_reduced_noalloc": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _i64, _f64, _i32, _i32, _vp, _i64, _i32,
                                           _vp, _vp, _vp]),
+    "rmm_b_norms": (_i32, [_vp, _i64, _i64, _i32, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "rmm_score_b_norms": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "rmm_matmul_reduced_b_norms": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i32, _vp, _i64, _i64, _i64, _i64,
+                                          _i64, _f64, _i32, _vp, _i64, _i64, _i32, _vp, _vp, ctypes.c_size_t,
+                                          _vp]),
     "rmm_check": (_i32, [_vp, _vp]),
     "rmm_last_error_string": (ctypes.c_char_p, []),
     "rmm_set_wait_limit_ns": (None, [_u64]),
@@ -206,6 +211,43 @@ def score(A: torch.Tensor, B: torch.Tensor | None, mode: str = "product", b_kmaj
     return out
 
 
+def b_norms(B: torch.Tensor, b_kmajor: bool = False, out: torch.Tensor | None = None,
+            status: torch.Tensor | None = None) -> torch.Tensor:
+    """B's factor of the product score, ||B[k,:]||_2 per slice k (f32 [batch][K] or [K]),
+    for reuse across calls while B is unchanged. B [b][K][N] (or Kmat [b][N][K] with b_kmajor)."""
+    bb, r, c, ldb, sB = _mat(B, "B")
+    K, N = (c, r) if b_kmajor else (r, c)
+    if out is None:
+        out = torch.empty((bb, K) if B.dim() == 3 else (K,), dtype=torch.float32, device=B.device)
+    _check(lib().rmm_b_norms(_ptr(B), ldb, sB, int(b_kmajor), bb, K, N, _dtype(B), _ptr(out), _ptr(status),
+                             _stream(B)))
+    return out
+
+
+def _bn_stride(b_norm: torch.Tensor, batch: int, K: int) -> int:
+    if b_norm.dtype != torch.float32 or not b_norm.is_cuda or not b_norm.is_contiguous():
+        raise ValueError("b_norm must be a contiguous float32 CUDA tensor")
+    if b_norm.dim() == 1:
+        if b_norm.shape[0] != K:
+            raise ValueError("b_norm must hold K values")
+        return 0  # one vector shared by every batch item
+    if tuple(b_norm.shape) != (batch, K):
+        raise ValueError("b_norm must be [K] or [batch][K]")
+    return K
+
+
+def score_b_norms(A: torch.Tensor, b_norm: torch.Tensor, out: torch.Tensor | None = None,
+                  status: torch.Tensor | None = None) -> torch.Tensor:
+    """Product-form slice scores with B's norms given: s[k] = ||A[:,k]||_2 · b_norm[k]."""
+    ba, M, K, lda, sA = _mat(A, "A")
+    stride = _bn_stride(b_norm, ba, K)
+    if out is None:
+        out = torch.empty((ba, K) if A.dim() == 3 else (K,), dtype=torch.float32, device=A.device)
+    _check(lib().rmm_score_b_norms(_ptr(A), lda, sA, _ptr(b_norm), stride, ba, M, K, _dtype(A), _ptr(out),
+                                   _ptr(status), _stream(A)))
+    return out
+
+
 def select(s: torch.Tensor, k_keep: int, out: torch.Tensor | None = None,
            status: torch.Tensor | None = None) -> torch.Tensor:
     """Ascending int32 indices of the k_keep largest scores per row of s (ties -> lower index)."""
@@ -285,6 +327,27 @@ def matmul_reduced(A: torch.Tensor, B: torch.Tensor, rho: float, mode: str = "pr
     _, _, _, ldc, sC = _mat(out, "C")
     _check(lib().rmm_matmul_reduced_batched(_ptr(A), lda, sA, _ptr(B), ldb, sB, int(b_kmajor), ba, M, K, N,
                                             float(rho), _dtype(A), SCORE_MODES[mode], _ptr(out), ldc, sC,
+                                            _out_code(out.dtype), _ptr(idx_out), ctypes.c_void_p(ws.ptr),
+                                            ws.nbytes, _stream(A)))
+    return out, ws
+
+
+def matmul_reduced_b_norms(A: torch.Tensor, B: torch.Tensor, b_norm: torch.Tensor, rho: float,
+                           out_dtype=torch.float32, out: torch.Tensor | None = None,
+                           workspace: Workspace | None = None, idx_out: torch.Tensor | None = None,
+                           b_kmajor: bool = False):
+    """matmul_reduced in product mode with B's norms cached (see b_norms): the score reads only A."""
+    ba, M, K, lda, sA = _mat(A, "A")
+    bb, r, c, ldb, sB = _mat(B, "B")
+    N = r if b_kmajor else c
+    stride = _bn_stride(b_norm, ba, K)
+    k = keep_count(rho, K)
+    ws = _ensure_ws(workspace, workspace_size(ba, M, K, N, k, A.dtype), A.device)
+    if out is None:
+        out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
+    _, _, _, ldc, sC = _mat(out, "C")
+    _check(lib().rmm_matmul_reduced_b_norms(_ptr(A), lda, sA, _ptr(B), ldb, sB, int(b_kmajor), _ptr(b_norm),
+                                            stride, ba, M, K, N, float(rho), _dtype(A), _ptr(out), ldc, sC,
                                             _out_code(out.dtype), _ptr(idx_out), ctypes.c_void_p(ws.ptr),
                                             ws.nbytes, _stream(A)))
     return out, ws

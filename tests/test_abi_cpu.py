@@ -89,6 +89,23 @@ def test_validation_errors_need_no_gpu():
     assert L.rmm_select(null, 0, 10, 3, null, null, null) == rmm.RMM_OK
 
 
+def test_cached_b_norm_calls_validate_without_gpu():
+    L = rmm.lib()
+    null = V(0)
+    # rmm_b_norms: B or the output missing; ld smaller than a row
+    assert L.rmm_b_norms(null, 8, 0, 0, 1, 8, 8, 0, V(16), null, null) == rmm.RMM_ERR_INVALID
+    assert L.rmm_b_norms(V(16), 8, 0, 0, 1, 8, 8, 0, null, null, null) == rmm.RMM_ERR_INVALID
+    assert L.rmm_b_norms(V(16), 4, 0, 0, 1, 8, 8, 0, V(16), null, null) == rmm.RMM_ERR_INVALID
+    # rmm_score_b_norms: norms missing; a batch stride between 0 and K
+    assert L.rmm_score_b_norms(V(16), 8, 64, null, 0, 2, 4, 8, 0, V(16), null, null) == rmm.RMM_ERR_INVALID
+    st = L.rmm_score_b_norms(V(16), 8, 64, V(16), 3, 2, 4, 8, 0, V(16), null, null)
+    assert st == rmm.RMM_ERR_INVALID and b"b_norm_stride" in L.rmm_last_error_string()
+    # fused: rho outside (0, 1] is still caught
+    st = L.rmm_matmul_reduced_b_norms(V(16), 8, 0, V(16), 8, 0, 0, V(16), 0, 1, 4, 8, 8, 0.0, 0, V(16), 8, 0, 1,
+                                      null, V(1024), 1 << 20, null)
+    assert st == rmm.RMM_ERR_INVALID and b"rho" in L.rmm_last_error_string()
+
+
 def test_binding_refuses_cpu_tensors():
     A = rmm.torch.zeros(4, 8, dtype=rmm.torch.bfloat16)
     with pytest.raises(ValueError):

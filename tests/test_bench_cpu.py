@@ -67,3 +67,13 @@ def test_reference_arm_times_the_oracle_on_the_host():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"] == "f32_64x256x64" and line["config"]["k_keep"] == 128
+
+
+def test_reference_arm_follows_the_score_mode():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0",
+                        "--workload", "f32_64x256x64", "--score-mode", "a_only"], cwd=ROOT, capture_output=True,
+                       text=True, timeout=600, env={**os.environ, "CUDA_VISIBLE_DEVICES": ""})
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["config"]["score_mode"] == "a_only" and line["value"] > 0
+

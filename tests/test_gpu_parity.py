@@ -263,3 +263,70 @@ def test_gemm_event_hook_brackets_the_gemm_kernel():
     inner, outer = e0.elapsed_time(e1), outer0.elapsed_time(outer1)
     assert 0 < inner <= outer
     assert outer0.elapsed_time(e0) >= 0 and e1.elapsed_time(outer1) >= 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("b_kmajor", [False, True], ids=["rows", "kmat"])
+def test_cached_b_norms(dtype, b_kmajor):
+    """rmm_b_norms against the fp64 row norms of B; scores and the fused call
+    with cached norms against the oracle's product-mode scores and product."""
+    M, K, N = 300, 1000, 520
+    A, B = _ab(M, K, N, dtype, seed=91)
+    Bg = B.t().contiguous() if b_kmajor else B  # Kmat [N][K] when b_kmajor
+    B64 = f64(B)
+    bn = rmm.b_norms(Bg, b_kmajor=b_kmajor)
+    check_scores(bn.cpu().numpy(), O.row_norms(B64))
+    s = rmm.score_b_norms(A, bn)
+    check_scores(s.cpu().numpy(), O.slice_scores(f64(A), B64, "product"))
+    if not b_kmajor:  # B's norms are the same f32 sums as in rmm_score's product mode
+        ref = rmm.score(A, B, "product")
+        assert torch.allclose(s, ref, rtol=1e-6, atol=0)
+    for rho in (0.3, 0.5):
+        idx = torch.empty(rmm.keep_count(rho, K), dtype=torch.int32, device=DEV)
+        C, ws = rmm.matmul_reduced_b_norms(A, Bg, bn, rho, idx_out=idx, b_kmajor=b_kmajor)
+        rmm.check(ws)
+        check_single(A, B, rho, "product", C, idx)
+
+
+def test_cached_b_norms_shared_across_batch():
+    """One weight for a batch of activations: b_norm [K] shared (stride 0)."""
+    batch, M, K, N = 3, 256, 512, 384
+    g = torch.Generator(device=DEV)
+    g.manual_seed(93)
+    A = torch.randn(batch, M, K, generator=g, device=DEV).to(torch.bfloat16)
+    W = torch.randn(K, N, generator=g, device=DEV).to(torch.bfloat16)
+    Wb = W.unsqueeze(0).expand(batch, K, N)  # batch stride 0
+    bn = rmm.b_norms(W)
+    idx = torch.empty(batch, rmm.keep_count(0.5, K), dtype=torch.int32, device=DEV)
+    C, ws = rmm.matmul_reduced_b_norms(A, Wb, bn, 0.5, idx_out=idx)
+    rmm.check(ws)
+    for b in range(batch):
+        check_single(A[b], W, 0.5, "product", C[b], idx[b])
+
+
+@pytest.mark.parametrize("shape,rho", [((4, 100, 128, 90), 0.3),       # k = 39: odd-length index lists, in smem
+                                       ((3, 40, 40000, 24), 0.50001)],  # k = 20001 > 16384: lists read from global
+                         ids=["k39", "k20001"])
+def test_pack_batched_unaligned_index_lists(shape, rho):
+    """Batched packs whose per-item index lists start off 16-byte boundaries
+    (k_keep not a multiple of 4) take the bulk path and copy bits exactly."""
+    batch, M, K, N = shape
+    g = torch.Generator(device=DEV)
+    g.manual_seed(97)
+    A = torch.randn(batch, M, K, generator=g, device=DEV).to(torch.bfloat16)
+    B = torch.randn(batch, K, N, generator=g, device=DEV).to(torch.bfloat16)
+    k = rmm.keep_count(rho, K)
+    assert k % 4 != 0
+    s = rmm.score(A, B)
+    idx = rmm.select(s, k)
+    A_S, B_S = rmm.pack(A, B, idx)
+    Kt = B.transpose(1, 2).contiguous()
+    A_S2, Kt_S = rmm.pack(A, Kt, idx, b_kmajor=True)
+    kp = rmm.padded_keep(k)
+    for b in range(batch):
+        I = idx[b].cpu().numpy().astype(np.int64)
+        a_ref = np.zeros((M, kp)); a_ref[:, :k] = f64(A[b])[:, I]
+        b_ref = np.zeros((kp, rmm.packed_b_ld(N))); b_ref[:k, :N] = f64(B[b])[I, :]
+        assert np.array_equal(f64(A_S[b]), a_ref) and np.array_equal(f64(A_S2[b]), a_ref)
+        assert np.array_equal(f64(B_S[b]), b_ref)
+        assert np.array_equal(f64(Kt_S[b]), b_ref[:, :N].T)
