@@ -55,7 +55,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="linear_4096",
                     choices=["linear_4096", "f32_64x256x64", "qk_32x4096x128", "pv_8192", "pv_16384", "pv_32768",
-                             "mlp_up", "mlp_down"])
+                             "mlp_up", "mlp_down", "decode_4096", "decode_mlp_up", "decode_mlp_up_m1"])
     ap.add_argument("--rho", type=float, default=None, help="retention ratio of the headline step")
     ap.add_argument("--no-sweep", action="store_true", help="skip the rho sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -79,6 +79,12 @@ class Problem:
         B3 = B if B.dim() == 3 else B.unsqueeze(0)
         self.batch, self.M, self.K = A3.shape
         self.N = B3.shape[1] if b_kmajor else B3.shape[2]
+        self.b_norm = None  # B's cached norms: the step uses them (decode: B is a resident weight)
+
+    @property
+    def gemv(self):
+        """Decode shape: the library streams B's kept rows without packing."""
+        return self.M <= 16 and not self.b_kmajor
 
     def k_keep(self, rho):
         return rmm.keep_count(rho, self.K)
@@ -109,6 +115,19 @@ def make_problem(name, device, seed, rho):
         X, W = inputs.mlp_up(seed=seed, device=device)
         return Problem(name, X, W, False, torch.float32, rho or 0.5,
                        "X[2048x8192] (0.5% outliers x20) · W[8192x28672] bf16 N(0,0.01^2)")
+    if name == "decode_4096":
+        X, W = inputs.linear_projection(M=16, seed=seed, device=device)
+        p = Problem(name, X[:1].contiguous(), W, False, torch.float32, rho or 0.5,
+                    "decode: x[1x4096] (1% outlier channels x20) · W[4096x4096] bf16, W's norms cached")
+        p.b_norm = rmm.b_norms(W) if str(device) != "cpu" else None
+        return p
+    if name in ("decode_mlp_up", "decode_mlp_up_m1"):
+        X, W = inputs.mlp_up(seed=seed, device=device)
+        m = 1 if name.endswith("_m1") else 16
+        p = Problem(name, X[:m].contiguous(), W, False, torch.float32, rho or 0.5,
+                    f"decode: x[{m}x8192] (0.5% outliers x20) · W[8192x28672] bf16 N(0,0.01^2), W's norms cached")
+        p.b_norm = rmm.b_norms(W) if str(device) != "cpu" else None
+        return p
     if name == "mlp_down":
         X, W = inputs.mlp_down(seed=seed, device=device)
         return Problem(name, X, W, False, torch.float32, rho or 0.5,
@@ -161,12 +180,24 @@ class Pipeline:
         k, idx, A_S, B_S = self.views(rho)
         if ev:
             ev[0].record()
-        rmm.score(p.A, p.B, p.mode, p.b_kmajor, out=self.s, status=self.status)
+        if p.b_norm is not None:
+            rmm.score_b_norms(p.A, p.b_norm, out=self.s, status=self.status)
+        else:
+            rmm.score(p.A, p.B, p.mode, p.b_kmajor, out=self.s, status=self.status)
         if ev and breakdown:
             ev[1].record()
         rmm.select(self.s, k, out=idx, status=self.status)
         if ev and breakdown:
             ev[2].record()
+        if p.gemv:  # decode shape: no pack; the GEMV reads B's kept rows through idx
+            if ev and breakdown:
+                ev[3].record()
+            elif ev:
+                ev[1].record()
+            rmm.gemv_gather(p.A, p.B, idx, out=self.C)
+            if ev:
+                ev[4 if breakdown else 2].record()
+            return
         rmm.pack(p.A, p.B, idx, p.b_kmajor, out=(A_S, B_S), status=self.status)
         if ev and breakdown:
             ev[3].record()
@@ -195,7 +226,7 @@ class Fused:
         dev = p.A.device
         self.C = torch.empty((p.batch, p.M, p.N) if p.A.dim() == 3 else (p.M, p.N), dtype=p.out_dtype, device=dev)
         self.ws = rmm.Workspace(rmm.workspace_size(p.batch, p.M, p.K, p.N, p.k_keep(rho_max), p.A.dtype), dev)
-        self.b_norm = b_norm
+        self.b_norm = b_norm if b_norm is not None else p.b_norm
 
     def step(self, rho, ev=None, breakdown=False):
         p = self.p
@@ -513,7 +544,7 @@ def run_ours(args):
 
     # the same call with B's norms cached (a weight's norms are computed once)
     cached = None
-    if p.mode == "product":
+    if p.mode == "product" and p.b_norm is None:
         bn = rmm.b_norms(p.B, p.b_kmajor)
         ccall = Fused(p, rho, b_norm=bn)
         for _ in range(3):
@@ -594,8 +625,15 @@ def stage_bytes(p: Problem, rho):
     kp = rmm.padded_keep(k)
     eb = p.A.element_size()
     ob = torch.tensor([], dtype=p.out_dtype).element_size()
-    b_read = 0 if p.mode == "a_only" else p.K * p.N * eb
+    b_read = 0 if (p.mode == "a_only" or p.b_norm is not None) else p.K * p.N * eb
     ldb = p.N if p.b_kmajor else rmm.packed_b_ld(p.N)
+    if p.gemv:  # no pack; the GEMV reads k rows of B, k columns of A, writes C
+        return {
+            "score": (p.M * p.K * eb + b_read + 4 * p.K) * p.batch,
+            "select": (4 * p.K + 4 * k) * p.batch,
+            "pack": 0,
+            "gemm": (k * p.N * eb + p.M * k * eb + 4 * k + p.M * p.N * ob) * p.batch,
+        }
     return {
         "score": (p.M * p.K * eb + b_read + 4 * p.K) * p.batch,
         "select": (4 * p.K + 4 * k) * p.batch,
@@ -606,7 +644,7 @@ def stage_bytes(p: Problem, rho):
 
 def stage_gbs(p: Problem, rho, stage_mean):
     by = stage_bytes(p, rho)
-    return {s: round(by[s] / (stage_mean[s] * 1e-3) / 1e9, 1) for s in stage_mean}
+    return {s: round(by[s] / (stage_mean[s] * 1e-3) / 1e9, 1) for s in stage_mean if by[s] > 0}
 
 
 def quality_check(p: Problem, rho, seed):
@@ -640,10 +678,11 @@ def roofline(p: Problem, rho, stage_mean, dominant, peaks, peak_src):
     ob = torch.tensor([], dtype=p.out_dtype).element_size()
     gemm_bytes = stage_bytes(p, rho)["gemm"]
     ridge = (peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9)
-    if dominant == "gemm" and p.A.dtype == torch.bfloat16 and p.kept_flops(rho) / gemm_bytes < ridge:
+    if dominant == "gemm" and (p.gemv or p.A.dtype == torch.bfloat16) and p.kept_flops(rho) / gemm_bytes < ridge:
         # below the ridge (P·V, Q·Kᵀ's output write): the GEMM is bound by HBM
         ach = gemm_bytes / (stage_mean["gemm"] * 1e-3) / 1e9
-        return {"kernel": "gemm_tc_kernel", "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+        return {"kernel": "gemv_gather_kernel" if p.gemv else "gemm_tc_kernel", "bound": "hbm",
+                "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
                 "algorithmic_bytes_per_launch": gemm_bytes,
                 "arithmetic_intensity": round(p.kept_flops(rho) / gemm_bytes, 1), "ridge": round(ridge, 1),
@@ -668,21 +707,33 @@ def roofline(p: Problem, rho, stage_mean, dominant, peaks, peak_src):
 def run_e2e(p: Problem, rho, steps, world):
     """Same metric through the public fused call with pinned host buffers:
     H2D of A and B, rmm_matmul_reduced, D2H of C, all inside the timed region."""
+    resident_b = p.b_norm is not None  # decode: the weight and its norms stay on the device
     hA = p.A.to("cpu").pin_memory()
-    hB = p.B.to("cpu").pin_memory()
-    dA, dB = torch.empty_like(p.A), torch.empty_like(p.B)
+    hB = None if resident_b else p.B.to("cpu").pin_memory()
+    dA = torch.empty_like(p.A)
+    dB = p.B if resident_b else torch.empty_like(p.B)
     shape = (p.batch, p.M, p.N) if p.A.dim() == 3 else (p.M, p.N)
     dC = torch.empty(shape, dtype=p.out_dtype, device=p.A.device)
     hC = torch.empty(shape, dtype=p.out_dtype).pin_memory()
-    _, ws = rmm.matmul_reduced(p.A, p.B, rho, out=dC, b_kmajor=p.b_kmajor)
+
+    def call(ws=None):
+        if resident_b:
+            return rmm.matmul_reduced_b_norms(dA, dB, p.b_norm, rho, out=dC, workspace=ws)
+        return rmm.matmul_reduced(dA, dB, rho, p.mode, out=dC, workspace=ws, b_kmajor=p.b_kmajor)
+
+    dA.copy_(p.A)
+    if not resident_b:
+        dB.copy_(p.B)
+    _, ws = call()
     torch.cuda.synchronize()
     ts = []
     for _ in range(steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         dA.copy_(hA, non_blocking=True)
-        dB.copy_(hB, non_blocking=True)
-        rmm.matmul_reduced(dA, dB, rho, out=dC, workspace=ws, b_kmajor=p.b_kmajor)
+        if not resident_b:
+            dB.copy_(hB, non_blocking=True)
+        call(ws)
         hC.copy_(dC, non_blocking=True)
         e1.record()
         e1.synchronize()
@@ -691,7 +742,8 @@ def run_e2e(p: Problem, rho, steps, world):
     ms = max_over_ranks(statistics.mean(ts), world)
     return {"value": round(world * p.kept_flops(rho) / (ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 4),
-            "h2d_bytes_per_step": int(hA.numel() * hA.element_size() + hB.numel() * hB.element_size()),
+            "h2d_bytes_per_step": int(hA.numel() * hA.element_size()
+                                      + (0 if hB is None else hB.numel() * hB.element_size())),
             "d2h_bytes_per_step": int(hC.numel() * hC.element_size())}
 
 

@@ -178,6 +178,22 @@ rmm_status rmm_matmul_reduced_batched(const void* A, int64_t lda, int64_t stride
                                       int32_t* idx_out, void* workspace, size_t workspace_bytes,
                                       cudaStream_t stream);
 
+/* Decode-shaped reduced product without packing: C[b] = A[b][:, idx[b]] ·
+ * B[b][idx[b], :] for M <= 16 rows of A (a few tokens, "Escopo de
+ * Aplicação": autoregressive use), B row-major [batch][K][N]. Reads A and B
+ * directly through idx (as written by rmm_select), streaming only the kept
+ * rows of B; f32 products and fixed-order f32 sums (bit-reproducible); C as
+ * in rmm_gemm. The fused calls take this route by themselves when M <= 16
+ * and B is row-major (they then skip rmm_pack); combine with cached B norms
+ * (below) or the A-only score so that scoring does not read all of B either.
+ * M > 16 is RMM_ERR_INVALID. */
+rmm_status rmm_gemv_gather(const void* A, int64_t lda, int64_t strideA,
+                           const void* B, int64_t ldb, int64_t strideB,
+                           int64_t batch, int64_t M, int64_t K, int64_t N,
+                           const int32_t* idx, int64_t k_keep, rmm_dtype in,
+                           void* C, int64_t ldc, int64_t strideC, rmm_dtype out,
+                           cudaStream_t stream);
+
 /* ---------------------------------------------------------------- cached B norms
  * B's factor of the product score, ||B[k,:]||_2, depends on B alone. When B is
  * a weight that is reused across calls, it can be computed once with

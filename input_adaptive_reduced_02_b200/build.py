@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "librmm.so")
-SOURCES = ["api.cu", "score.cu", "select.cu", "pack.cu", "gemm_tc.cu", "gemm_simt.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "score.cu", "select.cu", "pack.cu", "gemm_tc.cu", "gemm_simt.cu", "gemv.cu", "noalloc.cu"]
 HEADERS = ["rmm_device.cuh", "rmm_internal.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

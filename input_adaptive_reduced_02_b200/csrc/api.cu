@@ -170,6 +170,31 @@ static GemmArgs gemm_args(const void* A_S, const void* B_S, int b_kmajor, int64_
   return g;
 }
 
+static rmm_status do_gemv(const void* A, int64_t lda, int64_t sA, const void* B, int64_t ldb, int64_t sB,
+                          int64_t batch, int64_t M, int64_t N, const int32_t* idx, int64_t k_keep, rmm_dtype in,
+                          void* C, int64_t ldc, int64_t sC, rmm_dtype out, cudaStream_t st) {
+  GemvArgs g;
+  g.a = A;
+  g.b = B;
+  g.lda = lda;
+  g.strideA = sA;
+  g.ldb = ldb;
+  g.strideB = sB;
+  g.idx = idx;
+  g.k_keep = k_keep;
+  g.c = C;
+  g.ldc = ldc;
+  g.strideC = sC;
+  g.batch = batch;
+  g.M = M;
+  g.N = N;
+  g.in = kind(in);
+  g.out = kind(out);
+  const cudaError_t ce = launch_gemv_gather(g, st);
+  if (ce != cudaSuccess) return cuda_fail(ce, "gemv kernel");
+  return RMM_OK;
+}
+
 static rmm_status do_gemm(const GemmArgs& g, rmm_dtype in, cudaStream_t st) {
   cudaError_t ce;
   const char* why = nullptr;
@@ -320,12 +345,16 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
   // split-K round adds into are zeroed meanwhile by helper blocks of the same
   // launch instead of by a launch of their own.
   GemmArgs g = gemm_args(w.a_s, w.b_st, b_kmajor, batch, M, N, k_keep, C, ldc, strideC, out, w.status);
+  // A few rows of A (decode): the product streams B's kept rows straight
+  // through idx, with no packed copy.
+  const bool gemv = M <= kGemvMaxRows && !b_kmajor;
   SplitZero z;
-  const bool zero = in == RMM_BF16 && gemm_tc_split_zero(g, &z);
+  const bool zero = !gemv && in == RMM_BF16 && gemm_tc_split_zero(g, &z);
   ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr);
   if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
   g.c_zeroed = zero ? 1 : 0;
   if (M == 0 || N == 0) return RMM_OK;
+  if (gemv) return do_gemv(A, lda, strideA, B, ldb, strideB, batch, M, N, idx, k_keep, in, C, ldc, strideC, out, stream);
   if ((r = do_pack(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, idx, k_keep, in, w.a_s, w.b_st,
                    w.status, stream)))
     return r;
@@ -454,4 +483,22 @@ rmm_status rmm_matmul_reduced_b_norms(const void* A, int64_t lda, int64_t stride
   if (r) return r;
   return fused_call(A, lda, strideA, B, ldb, strideB, b_kmajor, b_norm, b_norm_stride, batch, M, K, N, rho, in,
                     RMM_SCORE_PRODUCT, C, ldc, strideC, out, idx_out, workspace, workspace_bytes, stream);
+}
+
+rmm_status rmm_gemv_gather(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb, int64_t strideB,
+                           int64_t batch, int64_t M, int64_t K, int64_t N, const int32_t* idx, int64_t k_keep,
+                           rmm_dtype in, void* C, int64_t ldc, int64_t strideC, rmm_dtype out,
+                           cudaStream_t stream) {
+  rmm_status r = check_common(batch, M, K, N, in);
+  if (r) return r;
+  if (!dtype_ok(out)) return fail(RMM_ERR_INVALID, "unknown output dtype");
+  if (M > kGemvMaxRows) return fail(RMM_ERR_INVALID, "M must be at most %lld", (long long)kGemvMaxRows);
+  if (k_keep < 1 || k_keep > K) return fail(RMM_ERR_INVALID, "k_keep must be in [1, K]");
+  r = check_ab(A, lda, strideA, B, ldb, strideB, 0, batch, M, K, N, true);
+  if (r) return r;
+  if (!layout_ok(batch, M, N, ldc, strideC)) return fail(RMM_ERR_INVALID, "C layout (ldc/strideC) is too small");
+  if (batch == 0 || M == 0 || N == 0) return RMM_OK;
+  if (!idx || !C) return fail(RMM_ERR_INVALID, "idx or C is NULL");
+  if ((r = bind_device(stream))) return r;
+  return do_gemv(A, lda, strideA, B, ldb, strideB, batch, M, N, idx, k_keep, in, C, ldc, strideC, out, stream);
 }

@@ -116,4 +116,20 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st, const char** why)
 bool gemm_tc_split_zero(const GemmArgs& g, SplitZero* z);
 cudaError_t launch_gemm_simt(const GemmArgs& g, cudaStream_t st);
 
+// gemv.cu: C[b] = A[b][:, idx[b]] · B[b][idx[b], :] read straight from A and
+// B (no packed copy) for M <= kGemvMaxRows rows of A; B row-major [K][N].
+constexpr int64_t kGemvMaxRows = 16;
+struct GemvArgs {
+  const void* a;  // [batch][M][K] (lda, strideA)
+  const void* b;  // [batch][K][N] (ldb, strideB)
+  int64_t lda, strideA, ldb, strideB;
+  const int32_t* idx;  // [batch][k_keep]
+  int64_t k_keep;
+  void* c;  // [batch][M][N] (ldc, strideC)
+  int64_t ldc, strideC;
+  int64_t batch, M, N;
+  ElemKind in, out;
+};
+cudaError_t launch_gemv_gather(const GemvArgs& g, cudaStream_t st);
+
 }  // namespace rmm

@@ -61,6 +61,8 @@ _SIGS = {
     "rmm_matmul_reduced_b_norms": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i32, _vp, _i64, _i64, _i64, _i64,
                                           _i64, _f64, _i32, _vp, _i64, _i64, _i32, _vp, _vp, ctypes.c_size_t,
                                           _vp]),
+    "rmm_gemv_gather": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _vp, _i64, _i32, _vp,
+                               _i64, _i64, _i32, _vp]),
     "rmm_check": (_i32, [_vp, _vp]),
     "rmm_last_error_string": (ctypes.c_char_p, []),
     "rmm_set_wait_limit_ns": (None, [_u64]),
@@ -306,6 +308,22 @@ def gemm(A_S: torch.Tensor, B_S: torch.Tensor, k_keep: int, out_dtype=torch.floa
     _, _, _, ldc, sC = _mat(out, "C")
     _check(lib().rmm_gemm(_ptr(A_S), _ptr(B_S), int(b_kmajor), ba, M, N, k_keep, _dtype(A_S), _ptr(out), ldc, sC,
                           _out_code(out.dtype), _ptr(status), _stream(A_S)))
+    return out
+
+
+def gemv_gather(A: torch.Tensor, B: torch.Tensor, idx: torch.Tensor, out_dtype=torch.float32,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+    """C = A[:, idx] · B[idx, :] straight from A (M <= 16 rows) and row-major B, no packing."""
+    ba, M, K, lda, sA = _mat(A, "A")
+    bb, r, N, ldb, sB = _mat(B, "B")
+    if r != K or bb != ba:
+        raise ValueError("A and B disagree on the contraction dimension or batch")
+    k = idx.shape[-1]
+    if out is None:
+        out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
+    _, _, _, ldc, sC = _mat(out, "C")
+    _check(lib().rmm_gemv_gather(_ptr(A), lda, sA, _ptr(B), ldb, sB, ba, M, K, N, _ptr(idx), k, _dtype(A),
+                                 _ptr(out), ldc, sC, _out_code(out.dtype), _stream(A)))
     return out
 
 

@@ -330,3 +330,60 @@ def test_pack_batched_unaligned_index_lists(shape, rho):
         assert np.array_equal(f64(A_S[b]), a_ref) and np.array_equal(f64(A_S2[b]), a_ref)
         assert np.array_equal(f64(B_S[b]), b_ref)
         assert np.array_equal(f64(Kt_S[b]), b_ref[:, :N].T)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("shape", [(1, 1000, 130), (3, 4096, 1000), (8, 777, 4100), (16, 2048, 257), (2, 64, 1)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_gemv_gather_matches_oracle(shape, dtype):
+    """Decode-shaped product read straight from A and B through idx: ragged
+    and unaligned N, 1 to 16 rows, both output dtypes."""
+    M, K, N = shape
+    A, B = _ab(M, K, N, dtype, seed=M + K + N)
+    A64, B64 = f64(A), f64(B)
+    for rho in (0.3, 1.0):
+        k = rmm.keep_count(rho, K)
+        idx = rmm.select(rmm.score(A, B), k)
+        for out_dtype in (torch.float32, torch.bfloat16):
+            C = rmm.gemv_gather(A, B, idx, out_dtype)
+            check_product(f64(C), A64, B64, idx.cpu().numpy(), product_tol(dtype, out_dtype))
+        C1 = rmm.gemv_gather(A, B, idx)
+        C2 = rmm.gemv_gather(A, B, idx)
+        assert torch.equal(C1, C2)  # fixed summation order
+
+
+def test_gemv_gather_unaligned_rows():
+    """B rows that are not 16-byte aligned (odd N, a strided view) take the
+    element-wise loads."""
+    M, K, N = 4, 600, 333
+    A, Bfull = _ab(M, K, N + 3, torch.bfloat16, seed=5)
+    B = Bfull[:, 1:N + 1]  # ld N + 3, base off by 2 bytes
+    idx = rmm.select(rmm.score(A, B.contiguous()), rmm.keep_count(0.5, K))
+    C = rmm.gemv_gather(A, B, idx)
+    check_product(f64(C), f64(A), f64(B), idx.cpu().numpy(), 1e-2)
+
+
+def test_fused_decode_shape_skips_the_pack():
+    """The fused call with M <= 16 (and cached B norms, the decode setting)
+    runs score, select and the gather-GEMV: 3 launches, oracle parity, one
+    weight shared by a batch of sequences."""
+    batch, M, K, N = 3, 4, 2048, 1536
+    g = torch.Generator(device=DEV)
+    g.manual_seed(101)
+    X = torch.randn(batch, M, K, generator=g, device=DEV).to(torch.bfloat16)
+    W = torch.randn(K, N, generator=g, device=DEV).to(torch.bfloat16)
+    Wb = W.unsqueeze(0).expand(batch, K, N)
+    bn = rmm.b_norms(W)
+    idx = torch.empty(batch, rmm.keep_count(0.5, K), dtype=torch.int32, device=DEV)
+    torch.cuda.synchronize()
+    n0 = rmm.launch_count()
+    C, ws = rmm.matmul_reduced_b_norms(X, Wb, bn, 0.5, idx_out=idx)
+    torch.cuda.synchronize()
+    assert rmm.launch_count() - n0 == 3
+    rmm.check(ws)
+    for b in range(batch):
+        check_single(X[b], W, 0.5, "product", C[b], idx[b])
+    idx2 = torch.empty_like(idx)
+    C2, _ = rmm.matmul_reduced(X, Wb, 0.5, idx_out=idx2)  # product score reading W, same route
+    for b in range(batch):
+        check_single(X[b], W, 0.5, "product", C2[b], idx2[b])
