@@ -20,6 +20,7 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <cmath>
 
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
@@ -328,6 +329,191 @@ gemv_gather_async_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, const
 }
 static_assert(size_t(kGvWarps) * 16 * kGvCols * 4 <= size_t(2) * kGvPass * 32 * 8, "warp partials fit in the ring");
 
+// ---------------------------------------------------------------- bf16 tensor-core path
+// Same data movement idea as the async path, but the products run on the
+// tensor cores as warp-level mma.sync m16n8k16 (bf16 x bf16 -> f32): A is x_S
+// padded to 16 rows; each warp owns 16 of the CTA's 128 columns (two n8 tiles)
+// and walks every kept slice, so warps never share an output and no warp
+// reduction is needed.
+//  * The CTA's slices are taken in chunks of up to kMmaChunk: one step loads
+//    the chunk's row numbers and A values (bf16) into shared memory, so the
+//    copies of B never wait on a global load inside the loop.
+//  * B's rows stream by cp.async through a ring of kMmaBufs passes of
+//    kMmaPass rows; kMmaBufs - 1 passes are in flight while one is summed.
+//  * Ring rows (256 bytes) and A rows are XOR-swizzled in 16-byte chunks so
+//    that ldmatrix reads are free of bank conflicts; slices past the end are
+//    zero in both.
+constexpr int kMmaPass = 32;                  // kept slices per ring buffer
+constexpr int kMmaBufs = 4;                   // ring buffers (kMmaBufs - 1 in flight)
+constexpr int kMmaChunk = 1024;               // slices whose indices and A values are staged at once
+constexpr int kMmaCols = 256;                 // columns of C per CTA: 8 per lane, 16-byte copies
+constexpr int kMmaRow = kMmaCols * 2;         // bytes of one slice of B in the ring
+
+__device__ __forceinline__ uint32_t swz(int row, int row_bytes, int chunk) {
+  return uint32_t(row) * uint32_t(row_bytes) + (uint32_t(chunk ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void cp_async16_zfill(uint32_t smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_dst), "l"(gsrc), "r"(src_bytes)
+               : "memory");
+}
+
+constexpr size_t gv_mma_smem_bytes() {
+  return size_t(kMmaBufs) * kMmaPass * kMmaRow  // ring (then the CTA's partial)
+         + size_t(16) * kMmaChunk * 2           // A: 16 rows of kMmaChunk bf16
+         + size_t(kMmaChunk) * 4;               // row numbers
+}
+static_assert(size_t(16) * kMmaCols * 4 <= size_t(kMmaBufs) * kMmaPass * kMmaRow, "the partial fits in the ring");
+static_assert(kMmaPass % kGvWarps == 0 && kMmaPass % 16 == 0 && kMmaChunk % kMmaPass == 0, "pass shape");
+static_assert(kMmaCols == 32 * 8 && kMmaCols == kGvWarps * 32, "8 columns per lane, 32 per warp");
+
+// Requires B's rows (and its base) 16-byte aligned.
+__global__ void __launch_bounds__(kGvThreads)
+gemv_gather_mma_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t sA, const uint16_t* __restrict__ B,
+                       int64_t ldb, int64_t sB, int64_t M, int64_t N, const int32_t* __restrict__ idx, int64_t k_keep,
+                       void* __restrict__ C, int64_t ldc, int64_t sC, int out_bf16) {
+  constexpr int RPW = kMmaPass / kGvWarps;  // slices each warp copies per pass
+  constexpr int AROW = kMmaChunk * 2;       // bytes per row of A in shared memory
+  extern __shared__ __align__(128) unsigned char gvm_smem[];
+  unsigned char* ring = gvm_smem;                                   // [kMmaBufs][kMmaPass][kMmaRow]
+  unsigned char* as = ring + size_t(kMmaBufs) * kMmaPass * kMmaRow;  // [16][AROW]
+  int32_t* rows = reinterpret_cast<int32_t*>(as + 16 * AROW);       // [kMmaChunk]
+  float* cta = reinterpret_cast<float*>(ring);                      // [16][kMmaCols], once the ring is drained
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const unsigned cs = cluster.num_blocks();
+  const unsigned crank = cluster.block_rank();
+  const int64_t b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t n0 = int64_t(blockIdx.x) * kMmaCols;
+  const int64_t c = n0 + 8 * lane;  // this lane's 8 columns in the copies
+  const uint32_t src_bytes = c >= N ? 0u : uint32_t(min(int64_t(8), N - c) * 2);
+  const uint16_t* Ab = A + b * sA;
+  const uint16_t* Bc = B + b * sB + (src_bytes ? c : 0);  // this lane's column start in row 0
+  const int32_t* ib = idx + b * k_keep;
+  const int64_t per = (k_keep + cs - 1) / cs;
+  const int64_t t_begin = min(k_keep, int64_t(crank) * per), t_end = min(k_keep, t_begin + per);
+  const uint32_t ring_s = smem_addr(ring), as_s = smem_addr(as);
+  // this lane's copy destinations within a ring buffer (slice warp + 8j, 16-byte chunk `lane`)
+  uint32_t dst[RPW];
+#pragma unroll
+  for (int j = 0; j < RPW; ++j) dst[j] = ring_s + swz(warp + kGvWarps * j, kMmaRow, lane);
+  // ldmatrix lane roles: A x4 = (m 0-7 | 8-15) x (k 0-7 | 8-15) of a 16-slice step;
+  // B x4.trans = (k 0-7 | 8-15) x (two of this warp's four 8-column tiles)
+  const int a_m = (lane & 7) + ((lane >> 3) & 1) * 8, a_kc = lane >> 4;
+  const int b_k = (lane & 7) + ((lane >> 3) & 1) * 8, b_nt = lane >> 4;
+
+  // rows m >= M of A stay zero for the whole kernel
+  for (int e = tid; e < 16 * AROW / 16; e += kGvThreads)
+    reinterpret_cast<uint4*>(as)[e] = make_uint4(0u, 0u, 0u, 0u);
+
+  float d[4][4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+
+  pdl_trigger();
+  pdl_wait();
+#pragma unroll 1
+  for (int64_t c0 = t_begin; c0 < t_end; c0 += kMmaChunk) {
+    const int nc = int(min(int64_t(kMmaChunk), t_end - c0));
+    const int np = (nc + kMmaPass - 1) / kMmaPass;
+    __syncthreads();  // the previous chunk is done with rows and A (and the zero fill is done)
+    // row numbers, and A[m][idx] as bf16 bits for m < M (zero past the chunk end)
+    for (int i = tid; i < np * kMmaPass; i += kGvThreads) {
+      const int32_t r = i < nc ? ib[c0 + i] : 0;
+      rows[i] = r;
+      uint16_t v[16];  // all loads first, then the stores: independent round trips
+#pragma unroll
+      for (int m = 0; m < 16; ++m) v[m] = (m < M && i < nc) ? __ldg(Ab + int64_t(m) * lda + r) : uint16_t(0);
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+        if (m < M) *reinterpret_cast<uint16_t*>(as + swz(m, AROW, i >> 3) + (i & 7) * 2) = v[m];
+    }
+    __syncthreads();
+    // copies of pass p's slices of B (zeros past the chunk end); one commit
+    // group per call in every thread, so that group counts stay uniform
+    auto issue = [&](int p) {
+      if (p < np) {
+        const uint32_t boff = uint32_t(p % kMmaBufs) * kMmaPass * kMmaRow;
+#pragma unroll
+        for (int j = 0; j < RPW; ++j) {
+          const int i = p * kMmaPass + warp + kGvWarps * j;
+          const bool live = i < nc && src_bytes != 0;
+          cp_async16_zfill(dst[j] + boff, live ? Bc + int64_t(rows[i]) * ldb : Bc, live ? src_bytes : 0u);
+        }
+      }
+      cp_async_commit();
+    };
+#pragma unroll 1
+    for (int q = 0; q < kMmaBufs - 1; ++q) issue(q);
+#pragma unroll 1
+    for (int p = 0; p < np; ++p) {
+      cp_async_wait<kMmaBufs - 2>();  // this thread's copies of pass p have landed
+      __syncthreads();                // and everyone's are visible to all warps
+      const uint32_t rb = ring_s + uint32_t(p % kMmaBufs) * kMmaPass * kMmaRow;
+#pragma unroll
+      for (int kc = 0; kc < kMmaPass / 16; ++kc) {
+        uint32_t a0, a1, a2, a3, b0, b1, b2, b3, b4, b5, b6, b7;
+        ldsm_x4(as_s + swz(a_m, AROW, (p * kMmaPass + kc * 16) / 8 + a_kc), a0, a1, a2, a3);
+        ldsm_x4_t(rb + swz(kc * 16 + b_k, kMmaRow, warp * 4 + b_nt), b0, b1, b2, b3);
+        ldsm_x4_t(rb + swz(kc * 16 + b_k, kMmaRow, warp * 4 + 2 + b_nt), b4, b5, b6, b7);
+        mma_bf16_16816(d[0], a0, a1, a2, a3, b0, b1);
+        mma_bf16_16816(d[1], a0, a1, a2, a3, b2, b3);
+        mma_bf16_16816(d[2], a0, a1, a2, a3, b4, b5);
+        mma_bf16_16816(d[3], a0, a1, a2, a3, b6, b7);
+      }
+      __syncthreads();  // every warp is done with this buffer
+      issue(p + kMmaBufs - 1);
+    }
+    cp_async_wait<0>();
+  }
+  __syncthreads();  // every warp is done with the ring: the partial takes its place
+  // accumulator fragment: rows lane/4 and lane/4 + 8, columns 2·(lane%4) + {0, 1} of each tile
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int col = warp * 32 + t * 8 + (lane & 3) * 2;
+    const int m = lane >> 2;
+    cta[m * kMmaCols + col] = d[t][0];
+    cta[m * kMmaCols + col + 1] = d[t][1];
+    cta[(m + 8) * kMmaCols + col] = d[t][2];
+    cta[(m + 8) * kMmaCols + col + 1] = d[t][3];
+  }
+  cluster.sync();
+  if (crank == 0) {
+    for (int e = tid; e < 16 * kMmaCols; e += kGvThreads) {
+      const int m = e / kMmaCols;
+      const int64_t col = n0 + (e % kMmaCols);
+      if (m >= M || col >= N) continue;
+      float t = 0.f;
+      for (unsigned q = 0; q < cs; ++q) t += cluster.map_shared_rank(cta, q)[e];
+      const int64_t off = b * sC + int64_t(m) * ldc + col;
+      if (out_bf16)
+        static_cast<uint16_t*>(C)[off] = uint16_t(pack_bf16x2(t, 0.f) & 0xFFFFu);
+      else
+        static_cast<float*>(C)[off] = t;
+    }
+  }
+  cluster.sync();
+}
+
 template <typename T, int MT>
 cudaError_t launch_mt(const GemvArgs& g, cudaStream_t st) {
   const size_t smem = gv_smem_bytes<MT>();
@@ -351,6 +537,34 @@ cudaError_t launch_mt(const GemvArgs& g, cudaStream_t st) {
   const T* bp = static_cast<const T*>(g.b);
   const int b_vec = (reinterpret_cast<uintptr_t>(g.b) % 16 == 0) && (g.ldb * int64_t(sizeof(T))) % 16 == 0 &&
                     (g.batch == 1 || (g.strideB * int64_t(sizeof(T))) % 16 == 0);
+  if (b_vec && sizeof(T) == 2) {
+    const size_t msmem = gv_mma_smem_bytes();
+    const int64_t mblk = (g.N + kMmaCols - 1) / kMmaCols;
+    // cluster size (slices split over 1..8 CTAs): the one whose grid fills
+    // whole waves of two CTAs per SM best, each CTA keeping >= 64 slices
+    unsigned mcs = 1;
+    double best = -1.0;
+    for (unsigned q = 1; q <= kGvMaxCluster; ++q) {
+      if (q > 1 && g.k_keep < int64_t(q) * 64) break;
+      const double waves = double(mblk * g.batch * q) / double(2 * sms);
+      const double eff = waves / std::max(1.0, std::ceil(waves));
+      if (eff > best + 1e-9) {
+        best = eff;
+        mcs = q;
+      }
+    }
+    static bool mma_attr[64] = {};
+    if (dev >= 0 && dev < 64 && !mma_attr[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(gemv_gather_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           int(msmem));
+      if (e != cudaSuccess) return e;
+      mma_attr[dev] = true;
+    }
+    return launch_pdl(gemv_gather_mma_kernel, dim3(unsigned(mblk), mcs, unsigned(g.batch)), dim3(kGvThreads), msmem,
+                      st, dim3(1, mcs, 1), static_cast<const uint16_t*>(g.a), g.lda, g.strideA,
+                      static_cast<const uint16_t*>(g.b), g.ldb, g.strideB, g.M, g.N, g.idx, g.k_keep, g.c, g.ldc,
+                      g.strideC, int(g.out == kBF16));
+  }
   if (b_vec) {
     const size_t asmem = gv_async_smem_bytes<T, MT>();
     static bool async_attr[64] = {};
