@@ -5,13 +5,18 @@
 //
 // One 1024-thread CTA per batch item. Scores become order-preserving 32-bit
 // keys in shared memory (up to 32768 of them; larger K re-reads the scores
-// from global memory, which stays in L2). A 4-pass MSB-first radix select
-// (8-bit digits; per-warp histograms built from ballot-based peer masks, one
-// leader lane per digit, no atomics) finds the digit
-// string of the k-th largest score, stopping early once the threshold bin is
-// kept whole, and how many keys equal to it must be kept. Two block-wide
-// scans then compact the kept indices in index order. Integer work only: the result
-// depends on the order of the scores, never on rounding.
+// from global memory, which stays in L2). The block's smallest and largest
+// keys share every bit above the highest bit where they differ, so an
+// MSB-first radix select starts there: 11-bit digits counted into one shared
+// histogram with shared-memory atomics, a block scan to find the bin of the
+// k-th largest key, and an early stop as soon as that bin is kept whole. Two
+// block-wide scans then compact the kept indices in index order (ties: the
+// lowest indices among keys equal to the threshold). Integer work only: the
+// result depends on the order of the scores, never on rounding.
+//
+// Spare blocks of the same launch (in the fused call) zero the f32 C tiles
+// that the GEMM's split-K round reduce-adds into, while one SM per batch item
+// selects.
 #include <algorithm>
 
 #include "rmm_device.cuh"
