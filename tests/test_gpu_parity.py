@@ -387,3 +387,23 @@ def test_fused_decode_shape_skips_the_pack():
     C2, _ = rmm.matmul_reduced(X, Wb, 0.5, idx_out=idx2)  # product score reading W, same route
     for b in range(batch):
         check_single(X[b], W, 0.5, "product", C2[b], idx2[b])
+
+
+@pytest.mark.parametrize("shape", [(300, 1000, 520), (2048, 512, 1024), (256, 4096, 200), (130, 777, 1000)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_fused_call_bit_identical_to_stage_calls(shape, gemm_cta_group):
+    """The fused call equals, bit for bit, the stage calls pack + GEMM on its
+    own kept set, for both output dtypes (ragged N, split-K last rounds whose
+    C tiles the select launch zeroes, N <= 256)."""
+    M, K, N = shape
+    A, B = _ab(M, K, N, torch.bfloat16, seed=M + N)
+    k = rmm.keep_count(0.5, K)
+    idx = torch.empty(k, dtype=torch.int32, device=DEV)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        C, ws = rmm.matmul_reduced(A, B, 0.5, out_dtype=out_dtype, idx_out=idx)
+        torch.cuda.synchronize()
+        rmm.check(ws)
+        A_S, B_S = rmm.pack(A, B, idx)
+        C_ref = rmm.gemm(A_S, B_S, k, out_dtype, N=N)
+        assert torch.equal(C, C_ref)
+        check_product(f64(C), f64(A), f64(B), idx.cpu().numpy(), product_tol(torch.bfloat16, out_dtype))
