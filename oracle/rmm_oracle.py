@@ -148,6 +148,24 @@ def pv_reduced(P: np.ndarray, V: np.ndarray, rho: float, mode: str = SCORE_PRODU
     return matmul_reduced_batched(P, V, rho, mode)
 
 
+def dequantize_w8(Wq: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """INT8 weight with one scale per output channel ("Resultados
+    Experimentais" › "Compatibilidade": the method works with INT8 weight
+    quantization; the scheme is not given, so the plainest symmetric
+    per-column form is read): W[k, n] = Wq[k, n] · scale[n], Wq in [-127, 127]."""
+    Wq = np.asarray(Wq)
+    if Wq.dtype != np.int8:
+        raise TypeError("Wq must be int8")
+    return Wq.astype(np.float64) * np.asarray(scale, dtype=np.float64)[None, :]
+
+
+def matmul_reduced_w8(A: np.ndarray, Wq: np.ndarray, scale: np.ndarray, rho: float, mode: str = SCORE_PRODUCT):
+    """RMM on an INT8 weight: the method applied to the dequantized weight, so
+    the score is ‖A[:, k]‖₂ · ‖W[k, :]‖₂ of the dequantized W and the product
+    is A[:, I] · W[I, :]. Returns (C, idx, s)."""
+    return matmul_reduced(A, dequantize_w8(Wq, scale), rho, mode)
+
+
 def frobenius_rel_error(C_test: np.ndarray, C_ref: np.ndarray) -> float:
     """‖C_test − C_ref‖_F / ‖C_ref‖_F (0 when both are zero)."""
     C_test = np.asarray(C_test, dtype=np.float64)

@@ -306,3 +306,44 @@ def test_frobenius_rel_error():
     a = np.array([[3.0, 4.0]])
     assert O.frobenius_rel_error(a, a) == 0.0
     assert abs(O.frobenius_rel_error(np.zeros_like(a), a) - 1.0) < 1e-15
+
+
+# ---------------------------------------------------------------- INT8 weights
+def test_w8_hand_worked_example():
+    """Per-output-channel INT8 weight, worked by hand: W = Wq · diag(scale) =
+    [[1, 2], [1.5, -8], [-0.5, 0]]; column norms of A are (5, 0, 1), row norms
+    of W (√5, √66.25, 0.5); product scores (5√5, 0, 0.5); ρ = 2/3 keeps {0, 2}
+    and C = A[:, {0,2}]·W[{0,2}, :] = [[2.5, 6], [4, 8]]."""
+    A = np.array([[3.0, 0.0, 1.0], [4.0, 0.0, 0.0]])
+    Wq = np.array([[2, 1], [3, -4], [-1, 0]], dtype=np.int8)
+    scale = np.array([0.5, 2.0])
+    W = O.dequantize_w8(Wq, scale)
+    assert np.array_equal(W, np.array([[1.0, 2.0], [1.5, -8.0], [-0.5, 0.0]]))
+    s = O.slice_scores(A, W)
+    assert np.allclose(s, [5.0 * math.sqrt(5.0), 0.0, 0.5], rtol=0, atol=1e-15)
+    C, idx, _ = O.matmul_reduced_w8(A, Wq, scale, 2.0 / 3.0)
+    assert idx.tolist() == [0, 2]
+    assert np.array_equal(C, np.array([[2.5, 6.0], [4.0, 8.0]]))
+
+
+def test_w8_unit_scales_reduce_to_the_integer_weight():
+    rng = np.random.default_rng(7)
+    A = rng.integers(-9, 10, size=(5, 12)).astype(np.float64)
+    Wq = rng.integers(-127, 128, size=(12, 7)).astype(np.int8)
+    C8, i8, _ = O.matmul_reduced_w8(A, Wq, np.ones(7), 0.5)
+    C, i, _ = O.matmul_reduced(A, Wq.astype(np.float64), 0.5)
+    assert np.array_equal(i8, i) and np.array_equal(C8, C)
+
+
+def test_w8_uniform_scale_keeps_the_selection_and_scales_the_product():
+    rng = np.random.default_rng(8)
+    A = rng.standard_normal((6, 20))
+    Wq = rng.integers(-127, 128, size=(20, 9)).astype(np.int8)
+    C1, i1, _ = O.matmul_reduced_w8(A, Wq, np.full(9, 1.0), 0.4)
+    C4, i4, _ = O.matmul_reduced_w8(A, Wq, np.full(9, 4.0), 0.4)  # a power of two: exact
+    assert np.array_equal(i1, i4) and np.array_equal(C4, 4.0 * C1)
+
+
+def test_w8_rejects_non_int8_weights():
+    with pytest.raises(TypeError):
+        O.dequantize_w8(np.zeros((2, 2), dtype=np.int16), np.ones(2))
