@@ -55,7 +55,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="linear_4096",
                     choices=["linear_4096", "f32_64x256x64", "qk_32x4096x128", "pv_8192", "pv_16384", "pv_32768",
-                             "mlp_up", "mlp_down", "decode_4096", "decode_mlp_up", "decode_mlp_up_m1"])
+                             "mlp_up", "mlp_down", "decode_4096", "decode_mlp_up", "decode_mlp_up_m1",
+                             "w8_linear_4096", "w8_decode_mlp_up_m1"])
     ap.add_argument("--rho", type=float, default=None, help="retention ratio of the headline step")
     ap.add_argument("--no-sweep", action="store_true", help="skip the rho sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -80,6 +81,7 @@ class Problem:
         self.batch, self.M, self.K = A3.shape
         self.N = B3.shape[1] if b_kmajor else B3.shape[2]
         self.b_norm = None  # B's cached norms: the step uses them (decode: B is a resident weight)
+        self.scale = None   # INT8 weight: B holds the int8 codes, W = B · diag(scale)
 
     @property
     def gemv(self):
@@ -127,6 +129,20 @@ def make_problem(name, device, seed, rho):
         p = Problem(name, X[:m].contiguous(), W, False, torch.float32, rho or 0.5,
                     f"decode: x[{m}x8192] (0.5% outliers x20) · W[8192x28672] bf16 N(0,0.01^2), W's norms cached")
         p.b_norm = rmm.b_norms(W) if str(device) != "cpu" else None
+        return p
+    if name in ("w8_linear_4096", "w8_decode_mlp_up_m1"):
+        if name == "w8_linear_4096":
+            X, _ = inputs.linear_projection(seed=seed, device=device)
+            Wq, sc = inputs.int8_weight(4096, 4096, std=0.02, seed=seed + 1, device=device)
+            descr = "X[4096x4096] bf16 (1% outliers x20) · INT8 W[4096x4096] with per-column scales, W's norms cached"
+        else:
+            X, _ = inputs.mlp_up(seed=seed, device=device)
+            X = X[:1].contiguous()
+            Wq, sc = inputs.int8_weight(8192, 28672, std=0.01, seed=seed + 1, device=device)
+            descr = "decode: x[1x8192] · INT8 W[8192x28672] with per-column scales, W's norms cached"
+        p = Problem(name, X, Wq, False, torch.float32, rho or 0.5, descr)
+        p.scale = sc
+        p.b_norm = rmm.b_norms_w8(Wq, sc) if str(device) != "cpu" else None
         return p
     if name == "mlp_down":
         X, W = inputs.mlp_down(seed=seed, device=device)
@@ -194,11 +210,17 @@ class Pipeline:
                 ev[3].record()
             elif ev:
                 ev[1].record()
-            rmm.gemv_gather(p.A, p.B, idx, out=self.C)
+            if p.scale is not None:
+                rmm.gemv_gather_w8(p.A, p.B, p.scale, idx, out=self.C)
+            else:
+                rmm.gemv_gather(p.A, p.B, idx, out=self.C)
             if ev:
                 ev[4 if breakdown else 2].record()
             return
-        rmm.pack(p.A, p.B, idx, p.b_kmajor, out=(A_S, B_S), status=self.status)
+        if p.scale is not None:
+            rmm.pack_w8(p.A, p.B, p.scale, idx, out=(A_S, B_S), status=self.status)
+        else:
+            rmm.pack(p.A, p.B, idx, p.b_kmajor, out=(A_S, B_S), status=self.status)
         if ev and breakdown:
             ev[3].record()
         elif ev:
@@ -232,7 +254,10 @@ class Fused:
         p = self.p
         if ev:
             ev[0].record()
-        if self.b_norm is not None:
+        if p.scale is not None:
+            rmm.matmul_reduced_w8(p.A, p.B, p.scale, rho, b_norm=p.b_norm, mode=p.mode, out=self.C,
+                                  workspace=self.ws)
+        elif self.b_norm is not None:
             rmm.matmul_reduced_b_norms(p.A, p.B, self.b_norm, rho, out=self.C, workspace=self.ws,
                                        b_kmajor=p.b_kmajor)
         else:
@@ -381,7 +406,10 @@ def oracle_cpu_timing(p: Problem, rho: float, budget_s: float, max_steps: int):
     except Exception:
         cores = os.cpu_count()
     A64 = p.A.to("cpu", torch.float32).numpy().astype(np.float64)
-    B64 = p.B.to("cpu", torch.float32).numpy().astype(np.float64)
+    if p.scale is not None:
+        B64 = O.dequantize_w8(p.B.to("cpu").numpy(), p.scale.to("cpu").numpy())
+    else:
+        B64 = p.B.to("cpu", torch.float32).numpy().astype(np.float64)
     if p.A.dim() == 2:
         A64, B64 = A64[None], B64[None]
     if p.b_kmajor:
@@ -625,19 +653,20 @@ def stage_bytes(p: Problem, rho):
     kp = rmm.padded_keep(k)
     eb = p.A.element_size()
     ob = torch.tensor([], dtype=p.out_dtype).element_size()
-    b_read = 0 if (p.mode == "a_only" or p.b_norm is not None) else p.K * p.N * eb
+    wb = 1 if p.scale is not None else eb  # bytes per element of B as stored (INT8 codes)
+    b_read = 0 if (p.mode == "a_only" or p.b_norm is not None) else p.K * p.N * wb
     ldb = p.N if p.b_kmajor else rmm.packed_b_ld(p.N)
     if p.gemv:  # no pack; the GEMV reads k rows of B, k columns of A, writes C
         return {
             "score": (p.M * p.K * eb + b_read + 4 * p.K) * p.batch,
             "select": (4 * p.K + 4 * k) * p.batch,
             "pack": 0,
-            "gemm": (k * p.N * eb + p.M * k * eb + 4 * k + p.M * p.N * ob) * p.batch,
+            "gemm": (k * p.N * wb + p.M * k * eb + 4 * k + p.M * p.N * ob) * p.batch,
         }
     return {
         "score": (p.M * p.K * eb + b_read + 4 * p.K) * p.batch,
         "select": (4 * p.K + 4 * k) * p.batch,
-        "pack": (p.M * p.K * eb + k * p.N * eb + p.M * kp * eb + kp * ldb * eb) * p.batch,
+        "pack": (p.M * p.K * eb + k * p.N * wb + p.M * kp * eb + kp * ldb * eb) * p.batch,
         "gemm": ((p.M + p.N) * kp * eb + p.M * p.N * ob) * p.batch,
     }
 
@@ -656,15 +685,26 @@ def quality_check(p: Problem, rho, seed):
     B = p.B[0] if p.B.dim() == 3 else p.B
     k = p.k_keep(rho)
     Bf = (B.t() if p.b_kmajor else B).float()
+    if p.scale is not None:
+        Bf = Bf * p.scale[None, :]
     dense = A.float() @ Bf
     nd = torch.linalg.norm(dense).item()
     idx = torch.empty(k, dtype=torch.int32, device=A.device)
-    C, _ = rmm.matmul_reduced(A, B, rho, p.mode, torch.float32, idx_out=idx, b_kmajor=p.b_kmajor)
     g = torch.Generator(device=A.device)
     g.manual_seed(1000 + seed)
     ridx = torch.randperm(p.K, generator=g, device=A.device)[:k].sort().values.to(torch.int32).contiguous()
-    A_S, B_S = rmm.pack(A, B, ridx, p.b_kmajor)
-    Cr = rmm.gemm(A_S, B_S, k, b_kmajor=p.b_kmajor, N=p.N)
+    if p.scale is not None:
+        bn = p.b_norm if p.b_norm is not None else rmm.b_norms_w8(B, p.scale)
+        C, _ = rmm.matmul_reduced_w8(A, B, p.scale, rho, b_norm=bn, mode=p.mode, idx_out=idx)
+        if p.gemv:
+            Cr = rmm.gemv_gather_w8(A, B, p.scale, ridx)
+        else:
+            A_S, B_S = rmm.pack_w8(A, B, p.scale, ridx)
+            Cr = rmm.gemm(A_S, B_S, k, N=p.N)
+    else:
+        C, _ = rmm.matmul_reduced(A, B, rho, p.mode, torch.float32, idx_out=idx, b_kmajor=p.b_kmajor)
+        A_S, B_S = rmm.pack(A, B, ridx, p.b_kmajor)
+        Cr = rmm.gemm(A_S, B_S, k, b_kmajor=p.b_kmajor, N=p.N)
     torch.cuda.synchronize()
     e_top = torch.linalg.norm(C - dense).item() / nd
     e_rand = torch.linalg.norm(Cr - dense).item() / nd
@@ -717,6 +757,8 @@ def run_e2e(p: Problem, rho, steps, world):
     hC = torch.empty(shape, dtype=p.out_dtype).pin_memory()
 
     def call(ws=None):
+        if p.scale is not None:
+            return rmm.matmul_reduced_w8(dA, dB, p.scale, rho, b_norm=p.b_norm, mode=p.mode, out=dC, workspace=ws)
         if resident_b:
             return rmm.matmul_reduced_b_norms(dA, dB, p.b_norm, rho, out=dC, workspace=ws)
         return rmm.matmul_reduced(dA, dB, rho, p.mode, out=dC, workspace=ws, b_kmajor=p.b_kmajor)

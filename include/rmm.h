@@ -232,6 +232,53 @@ rmm_status rmm_matmul_reduced_b_norms(const void* A, int64_t lda, int64_t stride
                                       int32_t* idx_out, void* workspace, size_t workspace_bytes,
                                       cudaStream_t stream);
 
+/* ---------------------------------------------------------------- INT8 weights
+ * "Resultados Experimentais" › "Compatibilidade": the method works with INT8
+ * weight quantization. Read as symmetric per-output-channel quantization: the
+ * weight W [K][N] is given as Wq (int8, [batch][K][ldw], batch stride strideW;
+ * values in [-127, 127]) and scale (f32 [N] per batch item, scale_stride apart,
+ * 0 = one vector for all items), W[k][j] = Wq[k][j] · scale[j]; the method runs
+ * on that W. A stays bf16. The gather-GEMV (M <= 16) needs Wq's rows and
+ * base 4-byte aligned (RMM_ERR_UNSUPPORTED otherwise); the other calls take
+ * any alignment. */
+
+/* b_norm[b][k] = ||W[b][k][:]||_2 of the dequantized weight (f32 sums), the
+ * B factor of the product score, for caching while the weight is unchanged. */
+rmm_status rmm_b_norms_w8(const int8_t* Wq, int64_t ldw, int64_t strideW, const float* scale,
+                          int64_t scale_stride, int64_t batch, int64_t K, int64_t N, float* b_norm,
+                          uint32_t* status_word, cudaStream_t stream);
+
+/* rmm_pack for an INT8 weight: A_S as in rmm_pack; B_S [batch][k_pad][ldbs]
+ * (ldbs = rmm_packed_b_ld(N)) holds bf16(Wq[idx[t]][j] · scale[j]) (round to
+ * nearest even), zero padded — the operand rmm_gemm takes with b_kmajor = 0. */
+rmm_status rmm_pack_w8(const void* A, int64_t lda, int64_t strideA, const int8_t* Wq, int64_t ldw,
+                       int64_t strideW, const float* scale, int64_t scale_stride, int64_t batch, int64_t M,
+                       int64_t K, int64_t N, const int32_t* idx, int64_t k_keep, void* A_S, void* B_S,
+                       uint32_t* status_word, cudaStream_t stream);
+
+/* rmm_gemv_gather on an INT8 weight (M <= 16): C = A[:, idx] · W[idx, :] with
+ * W = Wq · diag(scale), Wq's kept rows read directly (int8), products and sums
+ * in f32, the column scale applied to the sums. */
+rmm_status rmm_gemv_gather_w8(const void* A, int64_t lda, int64_t strideA, const int8_t* Wq, int64_t ldw,
+                              int64_t strideW, const float* scale, int64_t scale_stride, int64_t batch,
+                              int64_t M, int64_t K, int64_t N, const int32_t* idx, int64_t k_keep, void* C,
+                              int64_t ldc, int64_t strideC, rmm_dtype out, cudaStream_t stream);
+
+/* The fused call on an INT8 weight: score with cached b_norm (product mode,
+ * b_norm from rmm_b_norms_w8, b_norm_stride as in rmm_score_b_norms) or
+ * A-only (mode RMM_SCORE_A_ONLY, b_norm may be NULL), select, then for
+ * M <= 16 the gather-GEMV reading Wq's kept rows directly (int8 loads, f32
+ * products, the column scale applied to the sums) and otherwise rmm_pack_w8 +
+ * the tensor-core GEMM. in must be RMM_BF16 (A). Other arguments as in
+ * rmm_matmul_reduced_batched; workspace sized by rmm_workspace_size(...,
+ * RMM_BF16). */
+rmm_status rmm_matmul_reduced_w8(const void* A, int64_t lda, int64_t strideA, const int8_t* Wq, int64_t ldw,
+                                 int64_t strideW, const float* scale, int64_t scale_stride,
+                                 const float* b_norm, int64_t b_norm_stride, int64_t batch, int64_t M,
+                                 int64_t K, int64_t N, double rho, rmm_dtype in, rmm_score_mode mode,
+                                 void* C, int64_t ldc, int64_t strideC, rmm_dtype out, int32_t* idx_out,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Attention scores S = Q·Kᵀ per head, reduced over the head dimension
  * ("Escopo de Aplicação": the feature dimension of QKᵀ).
  *   Q [bh][S_q][d], Kmat [bh][S_k][d] (contiguous); S_out [bh][S_q][S_k]

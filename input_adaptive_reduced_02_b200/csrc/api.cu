@@ -502,3 +502,162 @@ rmm_status rmm_gemv_gather(const void* A, int64_t lda, int64_t strideA, const vo
   if ((r = bind_device(stream))) return r;
   return do_gemv(A, lda, strideA, B, ldb, strideB, batch, M, N, idx, k_keep, in, C, ldc, strideC, out, stream);
 }
+
+// ---------------------------------------------------------------- INT8 weights
+// need_align: the gather-GEMV copies 4 int8 at a time and needs Wq's rows
+// 4-byte aligned; the norm and pack kernels take any alignment.
+static rmm_status check_w8(const int8_t* Wq, int64_t ldw, int64_t strideW, const float* scale, int64_t scale_stride,
+                           int64_t batch, int64_t K, int64_t N, bool need_align) {
+  if (batch > 0 && N > 0 && (!Wq || !scale)) return fail(RMM_ERR_INVALID, "Wq or scale is NULL");
+  if (!layout_ok(batch, K, N, ldw, strideW, true)) return fail(RMM_ERR_INVALID, "Wq layout (ldw/strideW) is too small");
+  if (scale_stride < 0 || (batch > 1 && scale_stride != 0 && scale_stride < N))
+    return fail(RMM_ERR_INVALID, "scale_stride must be 0 (shared) or >= N");
+  if (need_align && ((reinterpret_cast<uintptr_t>(Wq) & 3u) || (ldw & 3) || (batch > 1 && (strideW & 3))))
+    return fail(RMM_ERR_UNSUPPORTED, "Wq's rows must be 4-byte aligned for M <= 16 (the gather-GEMV)");
+  return RMM_OK;
+}
+
+rmm_status rmm_b_norms_w8(const int8_t* Wq, int64_t ldw, int64_t strideW, const float* scale, int64_t scale_stride,
+                          int64_t batch, int64_t K, int64_t N, float* b_norm, uint32_t* status_word,
+                          cudaStream_t stream) {
+  rmm_status r = check_common(batch, 1, K, N, RMM_BF16);
+  if (r) return r;
+  if ((r = check_w8(Wq, ldw, strideW, scale, scale_stride, batch, K, N, false))) return r;
+  if (batch > 0 && !b_norm) return fail(RMM_ERR_INVALID, "b_norm is NULL");
+  if (batch == 0) return RMM_OK;
+  if ((r = bind_device(stream))) return r;
+  cudaError_t ce = N == 0 ? cudaMemsetAsync(b_norm, 0, size_t(batch * K) * 4, stream)
+                          : launch_b_norms_w8(Wq, ldw, strideW, scale, scale_stride, batch, K, N, b_norm,
+                                              status_word, stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "b_norms_w8 kernel");
+  return RMM_OK;
+}
+
+static rmm_status do_pack_w8(const void* A, int64_t lda, int64_t sA, const int8_t* Wq, int64_t ldw, int64_t sW,
+                             const float* scale, int64_t s_stride, int64_t batch, int64_t M, int64_t K, int64_t N,
+                             const int32_t* idx, int64_t k_keep, void* A_S, void* B_S, uint32_t* status,
+                             cudaStream_t st) {
+  const int64_t kp = round_up(k_keep, 64);
+  cudaError_t ce = launch_pack_cols(MatView{A, lda, sA, M, K}, kBF16, batch, idx, k_keep, kp, A_S, status,
+                                    wait_limit(), st);
+  if (ce != cudaSuccess) return cuda_fail(ce, "pack kernel (A)");
+  ce = launch_pack_rows_w8(Wq, ldw, sW, scale, s_stride, batch, N, idx, k_keep, kp, B_S, packed_b_ld(N), st);
+  if (ce != cudaSuccess) return cuda_fail(ce, "pack kernel (INT8 weight)");
+  return RMM_OK;
+}
+
+rmm_status rmm_pack_w8(const void* A, int64_t lda, int64_t strideA, const int8_t* Wq, int64_t ldw, int64_t strideW,
+                       const float* scale, int64_t scale_stride, int64_t batch, int64_t M, int64_t K, int64_t N,
+                       const int32_t* idx, int64_t k_keep, void* A_S, void* B_S, uint32_t* status_word,
+                       cudaStream_t stream) {
+  rmm_status r = check_common(batch, M, K, N, RMM_BF16);
+  if (r) return r;
+  if (k_keep < 1 || k_keep > K) return fail(RMM_ERR_INVALID, "k_keep must be in [1, K]");
+  r = check_ab(A, lda, strideA, nullptr, 0, 0, 0, batch, M, K, N, false);
+  if (r) return r;
+  if ((r = check_w8(Wq, ldw, strideW, scale, scale_stride, batch, K, N, false))) return r;
+  if (batch == 0) return RMM_OK;
+  if (!idx || (M > 0 && !A_S) || !B_S) return fail(RMM_ERR_INVALID, "idx, A_S or B_S is NULL");
+  if ((r = bind_device(stream))) return r;
+  return do_pack_w8(A, lda, strideA, Wq, ldw, strideW, scale, scale_stride, batch, M, K, N, idx, k_keep, A_S, B_S,
+                    status_word, stream);
+}
+
+static rmm_status do_gemv_w8(const void* A, int64_t lda, int64_t strideA, const int8_t* Wq, int64_t ldw,
+                             int64_t strideW, const float* scale, int64_t scale_stride, int64_t batch, int64_t M,
+                             int64_t N, const int32_t* idx, int64_t k_keep, void* C, int64_t ldc, int64_t strideC,
+                             rmm_dtype out, cudaStream_t stream);
+
+rmm_status rmm_matmul_reduced_w8(const void* A, int64_t lda, int64_t strideA, const int8_t* Wq, int64_t ldw,
+                                 int64_t strideW, const float* scale, int64_t scale_stride, const float* b_norm,
+                                 int64_t b_norm_stride, int64_t batch, int64_t M, int64_t K, int64_t N, double rho,
+                                 rmm_dtype in, rmm_score_mode mode, void* C, int64_t ldc, int64_t strideC,
+                                 rmm_dtype out, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream) {
+  rmm_status r = check_common(batch, M, K, N, in);
+  if (r) return r;
+  if (in != RMM_BF16) return fail(RMM_ERR_INVALID, "the INT8-weight path takes bf16 activations");
+  if (!dtype_ok(out)) return fail(RMM_ERR_INVALID, "unknown output dtype");
+  if (mode != RMM_SCORE_PRODUCT && mode != RMM_SCORE_A_ONLY) return fail(RMM_ERR_INVALID, "unknown score mode");
+  if (mode == RMM_SCORE_PRODUCT && (r = check_bn(b_norm, b_norm_stride, batch, K))) return r;
+  const int64_t k_keep = rmm_keep_count(rho, K);
+  if (k_keep < 1) return fail(RMM_ERR_INVALID, "rho must lie in (0, 1] (got %g)", rho);
+  r = check_ab(A, lda, strideA, nullptr, 0, 0, 0, batch, M, K, N, false);
+  if (r) return r;
+  if ((r = check_w8(Wq, ldw, strideW, scale, scale_stride, batch, K, N, M <= kGemvMaxRows))) return r;
+  if (!layout_ok(batch, M, N, ldc, strideC)) return fail(RMM_ERR_INVALID, "C layout (ldc/strideC) is too small");
+  if (batch > 0 && M > 0 && N > 0 && !C) return fail(RMM_ERR_INVALID, "C is NULL");
+  if (!workspace) return fail(RMM_ERR_INVALID, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(workspace) & 1023u) return fail(RMM_ERR_INVALID, "workspace must be 1 KiB aligned");
+  const Workspace w = carve(workspace, batch, M, K, N, k_keep, in);
+  if (workspace_bytes < w.bytes)
+    return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, w.bytes);
+  if ((r = bind_device(stream))) return r;
+  cudaError_t ce = cudaMemsetAsync(w.status, 0, 4, stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemsetAsync(status)");
+  if (batch == 0) return RMM_OK;
+  int32_t* idx = idx_out ? idx_out : w.idx;
+  if ((r = do_score(A, lda, strideA, nullptr, 0, 0, 0, batch, M, K, N, in, mode, w.s, w.status, stream,
+                    mode == RMM_SCORE_PRODUCT ? b_norm : nullptr, b_norm_stride)))
+    return r;
+  GemmArgs g = gemm_args(w.a_s, w.b_st, 0, batch, M, N, k_keep, C, ldc, strideC, out, w.status);
+  const bool gemv = M <= kGemvMaxRows;
+  SplitZero z;
+  const bool zero = !gemv && gemm_tc_split_zero(g, &z);
+  ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr);
+  if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
+  g.c_zeroed = zero ? 1 : 0;
+  if (M == 0 || N == 0) return RMM_OK;
+  if (gemv) return do_gemv_w8(A, lda, strideA, Wq, ldw, strideW, scale, scale_stride, batch, M, N, idx, k_keep, C,
+                              ldc, strideC, out, stream);
+  if ((r = do_pack_w8(A, lda, strideA, Wq, ldw, strideW, scale, scale_stride, batch, M, K, N, idx, k_keep, w.a_s,
+                      w.b_st, w.status, stream)))
+    return r;
+  return do_gemm(g, in, stream);
+}
+
+static rmm_status do_gemv_w8(const void* A, int64_t lda, int64_t strideA, const int8_t* Wq, int64_t ldw,
+                             int64_t strideW, const float* scale, int64_t scale_stride, int64_t batch, int64_t M,
+                             int64_t N, const int32_t* idx, int64_t k_keep, void* C, int64_t ldc, int64_t strideC,
+                             rmm_dtype out, cudaStream_t stream) {
+  GemvArgs v;
+  v.a = A;
+  v.b = Wq;
+  v.lda = lda;
+  v.strideA = strideA;
+  v.ldb = ldw;
+  v.strideB = strideW;
+  v.idx = idx;
+  v.k_keep = k_keep;
+  v.c = C;
+  v.ldc = ldc;
+  v.strideC = strideC;
+  v.batch = batch;
+  v.M = M;
+  v.N = N;
+  v.in = kBF16;
+  v.out = kind(out);
+  const cudaError_t ce = launch_gemv_gather_w8(v, scale, scale_stride, stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "gemv kernel (INT8 weight)");
+  return RMM_OK;
+}
+
+rmm_status rmm_gemv_gather_w8(const void* A, int64_t lda, int64_t strideA, const int8_t* Wq, int64_t ldw,
+                              int64_t strideW, const float* scale, int64_t scale_stride, int64_t batch, int64_t M,
+                              int64_t K, int64_t N, const int32_t* idx, int64_t k_keep, void* C, int64_t ldc,
+                              int64_t strideC, rmm_dtype out, cudaStream_t stream) {
+  rmm_status r = check_common(batch, M, K, N, RMM_BF16);
+  if (r) return r;
+  if (!dtype_ok(out)) return fail(RMM_ERR_INVALID, "unknown output dtype");
+  if (M > kGemvMaxRows) return fail(RMM_ERR_INVALID, "M must be at most %lld", (long long)kGemvMaxRows);
+  if (k_keep < 1 || k_keep > K) return fail(RMM_ERR_INVALID, "k_keep must be in [1, K]");
+  if ((r = check_ab(A, lda, strideA, nullptr, 0, 0, 0, batch, M, K, N, false))) return r;
+  if ((r = check_w8(Wq, ldw, strideW, scale, scale_stride, batch, K, N, true))) return r;
+  if (!layout_ok(batch, M, N, ldc, strideC)) return fail(RMM_ERR_INVALID, "C layout (ldc/strideC) is too small");
+  if (batch == 0 || M == 0 || N == 0) return RMM_OK;
+  if (!idx || !C) return fail(RMM_ERR_INVALID, "idx or C is NULL");
+  if ((r = bind_device(stream))) return r;
+  return do_gemv_w8(A, lda, strideA, Wq, ldw, strideW, scale, scale_stride, batch, M, N, idx, k_keep, C, ldc,
+                    strideC, out, stream);
+}
+

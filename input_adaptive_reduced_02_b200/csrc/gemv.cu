@@ -180,7 +180,7 @@ constexpr int lane_bytes() { return 4 * int(sizeof(T)); }  // 4 columns
 
 template <typename T, int MT>
 constexpr size_t gv_async_smem_bytes() {
-  return size_t(2) * kGvPass * 32 * lane_bytes<T>()  // ring (the warp partials reuse it afterwards)
+  return size_t(2) * kGvPass * 32 * (lane_bytes<T>() < 8 ? 8 : lane_bytes<T>())  // ring (then the warp partials)
          + size_t(2) * kGvPass * MT * 4               // A values
          + size_t(2) * kGvPass * 4                    // row numbers
          + size_t(MT) * kGvCols * 4;                  // the CTA's partial
@@ -191,8 +191,11 @@ __device__ __forceinline__ void cp_async_zfill(void* smem_dst, const void* gsrc,
   if constexpr (BYTES == 16)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(smem_dst)), "l"(gsrc),
                  "r"(src_bytes) : "memory");
-  else
+  else if constexpr (BYTES == 8)
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_addr(smem_dst)), "l"(gsrc),
+                 "r"(src_bytes) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_addr(smem_dst)), "l"(gsrc),
                  "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -207,14 +210,22 @@ __device__ __forceinline__ float4 slot_to_f32(const uint16_t*, const unsigned ch
 __device__ __forceinline__ float4 slot_to_f32(const uint32_t*, const unsigned char* slot) {
   return *reinterpret_cast<const float4*>(slot);
 }
+__device__ __forceinline__ float4 slot_to_f32(const int8_t*, const unsigned char* slot) {
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(slot);
+  return make_float4(float(int8_t(u & 0xFF)), float(int8_t((u >> 8) & 0xFF)), float(int8_t((u >> 16) & 0xFF)),
+                     float(int8_t(u >> 24)));
+}
 
-// Requires B's rows (and its base) aligned to lane_bytes<T>().
-template <typename T, int MT>
+// Requires B's rows (and its base) aligned to lane_bytes<TB>(). TB is B's
+// element type (T's, or int8_t for an INT8 weight whose column j is scaled by
+// col_scale[b * s_stride + j] at the end; col_scale null: no scale).
+template <typename T, int MT, typename TB = T>
 __global__ void __launch_bounds__(kGvThreads)
-gemv_gather_async_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, const T* __restrict__ B, int64_t ldb,
+gemv_gather_async_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, const TB* __restrict__ B, int64_t ldb,
                          int64_t sB, int64_t M, int64_t N, const int32_t* __restrict__ idx, int64_t k_keep,
-                         void* __restrict__ C, int64_t ldc, int64_t sC, int out_bf16) {
-  constexpr int LB = lane_bytes<T>();
+                         void* __restrict__ C, int64_t ldc, int64_t sC, int out_bf16,
+                         const float* __restrict__ col_scale, int64_t s_stride) {
+  constexpr int LB = lane_bytes<TB>() < 8 ? 8 : lane_bytes<TB>();  // slot bytes (int8: 4 used of 8)
   constexpr int RPW = kGvPass / kGvWarps;  // slices per warp per pass
   extern __shared__ __align__(16) unsigned char gva_smem[];
   unsigned char* ring = gva_smem;                                              // [2][kGvPass][32][LB]
@@ -230,9 +241,9 @@ gemv_gather_async_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, const
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n0 = int64_t(blockIdx.x) * kGvCols;
   const int64_t c = n0 + 4 * lane;
-  const uint32_t src_bytes = c >= N ? 0u : uint32_t(min(int64_t(4), N - c) * int64_t(sizeof(T)));
+  const uint32_t src_bytes = c >= N ? 0u : uint32_t(min(int64_t(4), N - c) * int64_t(sizeof(TB)));
   const T* Ab = A + b * sA;
-  const T* Bb = B + b * sB;
+  const TB* Bb = B + b * sB;
   const int32_t* ib = idx + b * k_keep;
   const int64_t per = (k_keep + cs - 1) / cs;
   const int64_t t_begin = min(k_keep, int64_t(crank) * per), t_end = min(k_keep, t_begin + per);
@@ -255,8 +266,8 @@ gemv_gather_async_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, const
     for (int j = 0; j < RPW; ++j) {
       const int i = warp + kGvWarps * j;
       if (i < n) {
-        const T* src = src_bytes ? Bb + int64_t(rows[buf * kGvPass + i]) * ldb + c : Bb;
-        cp_async_zfill<LB>(ring + (size_t(buf * kGvPass + i) * 32 + lane) * LB, src, src_bytes);
+        const TB* src = src_bytes ? Bb + int64_t(rows[buf * kGvPass + i]) * ldb + c : Bb;
+        cp_async_zfill<lane_bytes<TB>()>(ring + (size_t(buf * kGvPass + i) * 32 + lane) * LB, src, src_bytes);
       }
     }
     cp_async_commit();  // one group per pass in every thread, empty or not
@@ -289,7 +300,7 @@ gemv_gather_async_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, const
       const int i = warp + kGvWarps * j;
       if (i < n)
         fma_row<MT>(acc, xs + (buf * kGvPass + i) * MT,
-                    slot_to_f32(static_cast<const T*>(nullptr), ring + (size_t(buf * kGvPass + i) * 32 + lane) * LB));
+                    slot_to_f32(static_cast<const TB*>(nullptr), ring + (size_t(buf * kGvPass + i) * 32 + lane) * LB));
     }
     __syncthreads();  // every warp is done with buffer `buf`
     if (p + 2 < np) {
@@ -318,6 +329,7 @@ gemv_gather_async_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, const
       if (m >= M || col >= N) continue;
       float t = 0.f;
       for (unsigned q = 0; q < cs; ++q) t += cluster.map_shared_rank(cta, q)[e];
+      if (col_scale) t *= col_scale[b * s_stride + col];
       const int64_t off = b * sC + int64_t(m) * ldc + col;
       if (out_bf16)
         static_cast<uint16_t*>(C)[off] = uint16_t(pack_bf16x2(t, 0.f) & 0xFFFFu);
@@ -576,7 +588,8 @@ cudaError_t launch_mt(const GemvArgs& g, cudaStream_t st) {
     }
     return launch_pdl(gemv_gather_async_kernel<T, MT>, dim3(unsigned(nblk), cs, unsigned(g.batch)),
                       dim3(kGvThreads), asmem, st, dim3(1, cs, 1), a, g.lda, g.strideA, bp, g.ldb, g.strideB, g.M,
-                      g.N, g.idx, g.k_keep, g.c, g.ldc, g.strideC, int(g.out == kBF16));
+                      g.N, g.idx, g.k_keep, g.c, g.ldc, g.strideC, int(g.out == kBF16),
+                      static_cast<const float*>(nullptr), int64_t(0));
   }
   return launch_pdl(gemv_gather_kernel<T, MT>, dim3(unsigned(nblk), cs, unsigned(g.batch)), dim3(kGvThreads), smem,
                     st, dim3(1, cs, 1), a, g.lda, g.strideA, bp, g.ldb, g.strideB, g.M, g.N, g.idx, g.k_keep, g.c,
@@ -592,7 +605,40 @@ cudaError_t launch_t(const GemvArgs& g, cudaStream_t st) {
   return launch_mt<T, 16>(g, st);
 }
 
+template <int MT>
+cudaError_t launch_w8_mt(const GemvArgs& g, const float* scale, int64_t s_stride, cudaStream_t st) {
+  const size_t smem = gv_async_smem_bytes<int8_t, MT>();
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_gather_async_kernel<uint16_t, MT, int8_t>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t nblk = (g.N + kGvCols - 1) / kGvCols;
+  unsigned cs = 1;
+  while (cs < kGvMaxCluster && nblk * g.batch * cs < 2 * int64_t(sms) && g.k_keep >= int64_t(cs) * 2 * 64) cs *= 2;
+  return launch_pdl(gemv_gather_async_kernel<uint16_t, MT, int8_t>, dim3(unsigned(nblk), cs, unsigned(g.batch)),
+                    dim3(kGvThreads), smem, st, dim3(1, cs, 1), static_cast<const uint16_t*>(g.a), g.lda, g.strideA,
+                    static_cast<const int8_t*>(g.b), g.ldb, g.strideB, g.M, g.N, g.idx, g.k_keep, g.c, g.ldc,
+                    g.strideC, int(g.out == kBF16), scale, s_stride);
+}
+
 }  // namespace
+
+cudaError_t launch_gemv_gather_w8(const GemvArgs& g, const float* scale, int64_t s_stride, cudaStream_t st) {
+  if (g.batch == 0 || g.M == 0 || g.N == 0) return cudaSuccess;
+  if (g.M > kGemvMaxRows) return cudaErrorInvalidValue;
+  if (g.M <= 1) return launch_w8_mt<1>(g, scale, s_stride, st);
+  if (g.M <= 2) return launch_w8_mt<2>(g, scale, s_stride, st);
+  if (g.M <= 4) return launch_w8_mt<4>(g, scale, s_stride, st);
+  if (g.M <= 8) return launch_w8_mt<8>(g, scale, s_stride, st);
+  return launch_w8_mt<16>(g, scale, s_stride, st);
+}
 
 cudaError_t launch_gemv_gather(const GemvArgs& g, cudaStream_t st) {
   if (g.batch == 0 || g.M == 0 || g.N == 0) return cudaSuccess;

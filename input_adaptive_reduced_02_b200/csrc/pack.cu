@@ -416,4 +416,64 @@ cudaError_t launch_pack_rows(const MatView& X, ElemKind e, int64_t batch, const 
                     : launch_pack_rows_t<uint32_t>(X, batch, idx, k_keep, k_pad, out, ldo, status, wait_ns, st);
 }
 
+namespace {
+
+// out[b][t][j] = bf16(Wq[b][idx[b][t]][j] · scale[b][j]) for t < k_keep and
+// j < N; zero for k_keep <= t < k_pad and N <= j < ldo. A CTA per kept row
+// (grid-stride), 8 weights per thread step (8-byte load, 16-byte store) when
+// aligned.
+__global__ void __launch_bounds__(kPackThreads)
+pack_rows_w8_kernel(const int8_t* __restrict__ Wq, int64_t ldw, int64_t sW, const float* __restrict__ scale,
+                    int64_t s_stride, int64_t N, const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad,
+                    uint16_t* __restrict__ out, int64_t ldo, int vec) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t b = blockIdx.y;
+  const float* sc = scale + b * s_stride;
+  for (int64_t t = blockIdx.x; t < k_pad; t += gridDim.x) {
+    uint16_t* dst = out + (b * k_pad + t) * ldo;
+    if (t >= k_keep) {
+      for (int64_t c = threadIdx.x; c < ldo; c += kPackThreads) dst[c] = 0;
+      continue;
+    }
+    const int8_t* src = Wq + b * sW + int64_t(idx[b * k_keep + t]) * ldw;
+    int64_t c0 = 0;
+    if (vec) {
+      const int64_t n8 = N / 8;
+      for (int64_t g = threadIdx.x; g < n8; g += kPackThreads) {
+        const uint2 q = *reinterpret_cast<const uint2*>(src + 8 * g);
+        const float4 s0 = *reinterpret_cast<const float4*>(sc + 8 * g);
+        const float4 s1 = *reinterpret_cast<const float4*>(sc + 8 * g + 4);
+        const float v[8] = {float(int8_t(q.x & 0xFF)) * s0.x,         float(int8_t((q.x >> 8) & 0xFF)) * s0.y,
+                            float(int8_t((q.x >> 16) & 0xFF)) * s0.z, float(int8_t(q.x >> 24)) * s0.w,
+                            float(int8_t(q.y & 0xFF)) * s1.x,         float(int8_t((q.y >> 8) & 0xFF)) * s1.y,
+                            float(int8_t((q.y >> 16) & 0xFF)) * s1.z, float(int8_t(q.y >> 24)) * s1.w};
+        *reinterpret_cast<uint4*>(dst + 8 * g) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+      }
+      c0 = n8 * 8;
+    }
+    for (int64_t c = c0 + threadIdx.x; c < ldo; c += kPackThreads)
+      dst[c] = c < N ? uint16_t(pack_bf16x2(float(src[c]) * sc[c], 0.f) & 0xFFFFu) : uint16_t(0);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pack_rows_w8(const int8_t* Wq, int64_t ldw, int64_t sW, const float* scale, int64_t s_stride,
+                                int64_t batch, int64_t N, const int32_t* idx, int64_t k_keep, int64_t k_pad,
+                                void* out, int64_t ldo, cudaStream_t st) {
+  if (batch == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int vec = (reinterpret_cast<uintptr_t>(Wq) % 8 == 0) && ldw % 8 == 0 && (batch == 1 || sW % 8 == 0) &&
+                  (reinterpret_cast<uintptr_t>(scale) % 16 == 0) && (batch == 1 || s_stride % 4 == 0) &&
+                  (reinterpret_cast<uintptr_t>(out) % 16 == 0) && ldo % 8 == 0;
+  const int64_t ctas = std::min<int64_t>(k_pad, std::max<int64_t>(1, 8 * int64_t(sms) / std::max<int64_t>(1, batch)));
+  return launch_pdl(pack_rows_w8_kernel, dim3(unsigned(ctas), unsigned(batch)), dim3(kPackThreads), 0, st,
+                    dim3(0, 0, 0), Wq, ldw, sW, scale, s_stride, N, idx, k_keep, k_pad, static_cast<uint16_t*>(out),
+                    ldo, vec);
+}
+
 }  // namespace rmm

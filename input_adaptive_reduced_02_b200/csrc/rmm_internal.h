@@ -94,6 +94,15 @@ cudaError_t launch_pack_rows(const MatView& X, ElemKind e, int64_t batch, const 
                              int64_t k_keep, int64_t k_pad, void* out, int64_t ldo, uint32_t* status,
                              uint64_t wait_ns, cudaStream_t st);
 
+// INT8 weights with one f32 scale per output column (scale[b * s_stride + j]):
+//  b_norm[b][k] = ||Wq[b][k][:] · scale||_2 (score.cu) and
+//  out[b][t][j] = bf16(Wq[b][idx[b][t]][j] · scale[j]) (pack.cu, zero padded).
+cudaError_t launch_b_norms_w8(const int8_t* Wq, int64_t ldw, int64_t sW, const float* scale, int64_t s_stride,
+                              int64_t batch, int64_t K, int64_t N, float* out, uint32_t* status, cudaStream_t st);
+cudaError_t launch_pack_rows_w8(const int8_t* Wq, int64_t ldw, int64_t sW, const float* scale, int64_t s_stride,
+                                int64_t batch, int64_t N, const int32_t* idx, int64_t k_keep, int64_t k_pad,
+                                void* out, int64_t ldo, cudaStream_t st);
+
 // gemm_tc.cu (bf16 tensor cores) / gemm_simt.cu (f32 CUDA cores)
 struct GemmArgs {
   const void* a;  // [batch][M][k_pad]
@@ -131,5 +140,8 @@ struct GemvArgs {
   ElemKind in, out;
 };
 cudaError_t launch_gemv_gather(const GemvArgs& g, cudaStream_t st);
+//  B = an INT8 weight (g.b int8, rows 4-byte aligned) whose column j is scaled
+//  by scale[b * s_stride + j]; A bf16.
+cudaError_t launch_gemv_gather_w8(const GemvArgs& g, const float* scale, int64_t s_stride, cudaStream_t st);
 
 }  // namespace rmm

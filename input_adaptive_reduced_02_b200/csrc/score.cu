@@ -233,6 +233,55 @@ bnorm_rows_kernel(const T* __restrict__ B, int64_t ldb, int64_t sB, int64_t K, i
   }
 }
 
+// b_norm[b][k] = sqrt(sum_j (Wq[b][k][j] · scale[j])^2): the row norms of a
+// per-column-scaled INT8 weight (one warp per row; 16 weights per load when
+// the rows and the scales are 16-byte aligned).
+__global__ void __launch_bounds__(kScoreThreads)
+bnorm_rows_w8_kernel(const int8_t* __restrict__ Wq, int64_t ldw, int64_t sW, const float* __restrict__ scale,
+                     int64_t s_stride, int64_t K, int64_t N, int vec, float* __restrict__ out, uint32_t* status) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t b = blockIdx.y;
+  constexpr int kWarps = kScoreThreads / 32;
+  const float* sc = scale + b * s_stride;
+  for (int64_t k = int64_t(blockIdx.x) * kWarps + warp; k < K; k += int64_t(gridDim.x) * kWarps) {
+    const int8_t* row = Wq + b * sW + k * ldw;
+    float acc = 0.f;
+    int64_t tail = 0;
+    if (vec) {
+      const int64_t nv = N / 16;
+      for (int64_t j = lane; j < nv; j += 32) {
+        const int4 q = *reinterpret_cast<const int4*>(row + 16 * j);
+        const float4* s4 = reinterpret_cast<const float4*>(sc + 16 * j);
+        const uint32_t w[4] = {uint32_t(q.x), uint32_t(q.y), uint32_t(q.z), uint32_t(q.w)};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float4 sv = s4[h];
+          const float v0 = float(int8_t(w[h] & 0xFF)) * sv.x, v1 = float(int8_t((w[h] >> 8) & 0xFF)) * sv.y;
+          const float v2 = float(int8_t((w[h] >> 16) & 0xFF)) * sv.z, v3 = float(int8_t(w[h] >> 24)) * sv.w;
+          acc = fmaf(v0, v0, acc);
+          acc = fmaf(v1, v1, acc);
+          acc = fmaf(v2, v2, acc);
+          acc = fmaf(v3, v3, acc);
+        }
+      }
+      tail = nv * 16;
+    }
+    for (int64_t c = tail + lane; c < N; c += 32) {
+      const float v = float(row[c]) * sc[c];
+      acc = fmaf(v, v, acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      const float v = sqrtf(acc);
+      out[b * K + k] = v;
+      if (!isfinite(v)) status_or(status, RMM_NONFINITE_BIT);
+    }
+  }
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // 16-byte loads for B: base, rows and batch items 16-byte aligned.
@@ -303,6 +352,17 @@ cudaError_t launch_b_norms(const MatView& B, int b_kmajor, ElemKind e, int64_t b
   }
   return e == kBF16 ? launch_bnorm_rows<uint16_t>(B, batch, out, status, st)
                     : launch_bnorm_rows<uint32_t>(B, batch, out, status, st);
+}
+
+cudaError_t launch_b_norms_w8(const int8_t* Wq, int64_t ldw, int64_t sW, const float* scale, int64_t s_stride,
+                              int64_t batch, int64_t K, int64_t N, float* out, uint32_t* status, cudaStream_t st) {
+  if (batch == 0 || K == 0 || N == 0) return cudaSuccess;
+  constexpr int kWarps = kScoreThreads / 32;
+  const int64_t ctas = std::min<int64_t>((K + kWarps - 1) / kWarps, 148 * 8);
+  const int vec = aligned16(Wq) && ldw % 16 == 0 && (batch == 1 || sW % 16 == 0) && aligned16(scale) &&
+                  (batch == 1 || s_stride % 4 == 0);
+  return launch_pdl(bnorm_rows_w8_kernel, dim3(unsigned(ctas), unsigned(batch)), dim3(kScoreThreads), 0, st,
+                    dim3(0, 0, 0), Wq, ldw, sW, scale, s_stride, K, N, vec, out, status);
 }
 
 }  // namespace rmm

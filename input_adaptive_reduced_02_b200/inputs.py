@@ -53,6 +53,17 @@ def outlier_activations(M: int, K: int, outlier_frac: float, factor: float,
     return X.to(dtype).contiguous(), ch
 
 
+def int8_weight(K: int, N: int, std: float = 0.02, seed: int = 0, device="cpu"):
+    """A weight given as INT8 codes and one f32 scale per output column:
+    Wq [K][N] int8 = round(N(0, 40²)) clipped to [-127, 127]; scale [N] =
+    std/40 · (1 + 0.1·N(0,1)), so Wq · scale has entries of about N(0, std²)."""
+    g = _gen(seed, device)
+    q = torch.randn(K, N, generator=g, device=device, dtype=torch.float32) * 40.0
+    Wq = q.round().clamp(-127, 127).to(torch.int8).contiguous()
+    scale = (std / 40.0) * (1.0 + 0.1 * torch.randn(N, generator=g, device=device, dtype=torch.float32))
+    return Wq, scale.contiguous()
+
+
 def gaussian(shape, std: float, seed: int, device="cpu", dtype=torch.bfloat16):
     """N(0, std²) entries of the given shape."""
     g = _gen(seed, device)

@@ -63,6 +63,14 @@ _SIGS = {
                                           _vp]),
     "rmm_gemv_gather": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _vp, _i64, _i32, _vp,
                                _i64, _i64, _i32, _vp]),
+    "rmm_b_norms_w8": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "rmm_pack_w8": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _i64, _vp,
+                           _vp, _vp, _vp]),
+    "rmm_matmul_reduced_w8": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _i64, _vp, _i64, _i64, _i64, _i64,
+                                     _i64, _f64, _i32, _i32, _vp, _i64, _i64, _i32, _vp, _vp, ctypes.c_size_t,
+                                     _vp]),
+    "rmm_gemv_gather_w8": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _i64,
+                                  _vp, _i64, _i64, _i32, _vp]),
     "rmm_check": (_i32, [_vp, _vp]),
     "rmm_last_error_string": (ctypes.c_char_p, []),
     "rmm_set_wait_limit_ns": (None, [_u64]),
@@ -368,6 +376,93 @@ def matmul_reduced_b_norms(A: torch.Tensor, B: torch.Tensor, b_norm: torch.Tenso
                                             stride, ba, M, K, N, float(rho), _dtype(A), _ptr(out), ldc, sC,
                                             _out_code(out.dtype), _ptr(idx_out), ctypes.c_void_p(ws.ptr),
                                             ws.nbytes, _stream(A)))
+    return out, ws
+
+
+def _w8(Wq: torch.Tensor, scale: torch.Tensor):
+    """(batch, K, N, ldw, strideW, scale_stride) of an INT8 weight and its column scales."""
+    if Wq.dtype != torch.int8:
+        raise ValueError("Wq must be int8")
+    bw, K, N, ldw, sW = _mat(Wq, "Wq")
+    if scale.dtype != torch.float32 or not scale.is_cuda or not scale.is_contiguous():
+        raise ValueError("scale must be a contiguous float32 CUDA tensor")
+    if scale.dim() == 1:
+        if scale.shape[0] != N:
+            raise ValueError("scale must hold N values")
+        return bw, K, N, ldw, sW, 0
+    if tuple(scale.shape) != (bw, N):
+        raise ValueError("scale must be [N] or [batch][N]")
+    return bw, K, N, ldw, sW, N
+
+
+def b_norms_w8(Wq: torch.Tensor, scale: torch.Tensor, out: torch.Tensor | None = None,
+               status: torch.Tensor | None = None) -> torch.Tensor:
+    """||W[k,:]||_2 of the dequantized INT8 weight W = Wq · diag(scale) (f32 [batch][K] or [K])."""
+    bw, K, N, ldw, sW, ss = _w8(Wq, scale)
+    if out is None:
+        out = torch.empty((bw, K) if Wq.dim() == 3 else (K,), dtype=torch.float32, device=Wq.device)
+    _check(lib().rmm_b_norms_w8(_ptr(Wq), ldw, sW, _ptr(scale), ss, bw, K, N, _ptr(out), _ptr(status), _stream(Wq)))
+    return out
+
+
+def pack_w8(A: torch.Tensor, Wq: torch.Tensor, scale: torch.Tensor, idx: torch.Tensor, out=None,
+            status: torch.Tensor | None = None):
+    """(A_S, B_S): A's kept columns and bf16(Wq[idx] · scale) — the operands rmm.gemm takes."""
+    ba, M, K, lda, sA = _mat(A, "A")
+    bw, K2, N, ldw, sW, ss = _w8(Wq, scale)
+    if K2 != K:
+        raise ValueError("A and Wq disagree on the contraction dimension")
+    k = idx.shape[-1]
+    kp = padded_keep(k)
+    if out is None:
+        A_S = torch.empty((ba, M, kp) if A.dim() == 3 else (M, kp), dtype=A.dtype, device=A.device)
+        B_S = torch.empty(packed_b_shape(A.dim() == 3, ba, N, kp, False), dtype=A.dtype, device=A.device)
+    else:
+        A_S, B_S = out
+    _check(lib().rmm_pack_w8(_ptr(A), lda, sA, _ptr(Wq), ldw, sW, _ptr(scale), ss, ba, M, K, N, _ptr(idx), k,
+                             _ptr(A_S), _ptr(B_S), _ptr(status), _stream(A)))
+    return A_S, B_S
+
+
+def gemv_gather_w8(A: torch.Tensor, Wq: torch.Tensor, scale: torch.Tensor, idx: torch.Tensor,
+                   out_dtype=torch.float32, out: torch.Tensor | None = None) -> torch.Tensor:
+    """C = A[:, idx] · (Wq · diag(scale))[idx, :] straight from A (M <= 16 rows) and the INT8 weight."""
+    ba, M, K, lda, sA = _mat(A, "A")
+    bw, K2, N, ldw, sW, ss = _w8(Wq, scale)
+    if K2 != K:
+        raise ValueError("A and Wq disagree on the contraction dimension")
+    k = idx.shape[-1]
+    if out is None:
+        out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
+    _, _, _, ldc, sC = _mat(out, "C")
+    _check(lib().rmm_gemv_gather_w8(_ptr(A), lda, sA, _ptr(Wq), ldw, sW, _ptr(scale), ss, ba, M, K, N, _ptr(idx), k,
+                                    _ptr(out), ldc, sC, _out_code(out.dtype), _stream(A)))
+    return out
+
+
+def matmul_reduced_w8(A: torch.Tensor, Wq: torch.Tensor, scale: torch.Tensor, rho: float,
+                      b_norm: torch.Tensor | None = None, mode: str = "product", out_dtype=torch.float32,
+                      out: torch.Tensor | None = None, workspace: Workspace | None = None,
+                      idx_out: torch.Tensor | None = None):
+    """matmul_reduced on an INT8 weight W = Wq · diag(scale); product mode needs b_norm (b_norms_w8)."""
+    ba, M, K, lda, sA = _mat(A, "A")
+    bw, K2, N, ldw, sW, ss = _w8(Wq, scale)
+    if K2 != K:
+        raise ValueError("A and Wq disagree on the contraction dimension")
+    bn_stride = 0
+    if b_norm is not None:
+        bn_stride = _bn_stride(b_norm, ba, K)
+    elif SCORE_MODES[mode] == 0:
+        raise ValueError("product mode needs b_norm (b_norms_w8)")
+    k = keep_count(rho, K)
+    ws = _ensure_ws(workspace, workspace_size(ba, M, K, N, k, A.dtype), A.device)
+    if out is None:
+        out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
+    _, _, _, ldc, sC = _mat(out, "C")
+    _check(lib().rmm_matmul_reduced_w8(_ptr(A), lda, sA, _ptr(Wq), ldw, sW, _ptr(scale), ss, _ptr(b_norm), bn_stride,
+                                       ba, M, K, N, float(rho), _dtype(A), SCORE_MODES[mode], _ptr(out), ldc, sC,
+                                       _out_code(out.dtype), _ptr(idx_out), ctypes.c_void_p(ws.ptr), ws.nbytes,
+                                       _stream(A)))
     return out, ws
 
 
