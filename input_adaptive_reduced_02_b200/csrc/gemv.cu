@@ -605,6 +605,177 @@ cudaError_t launch_t(const GemvArgs& g, cudaStream_t st) {
   return launch_mt<T, 16>(g, st);
 }
 
+// ---------------------------------------------------------------- INT8 weight, tensor cores
+// The mma path for an INT8 weight: each pass's int8 rows (256 columns = 256
+// bytes per slice, one 16-byte cp.async per 16 weights) are converted exactly
+// to bf16 into a swizzled staging buffer, which the same ldmatrix + mma.sync
+// loop reads; column j of the sums is scaled by scale[j] at the end.
+constexpr size_t gv_mma_w8_smem_bytes() {
+  return size_t(kMmaBufs) * kMmaPass * kMmaCols  // int8 ring (then the CTA's partial)
+         + size_t(kMmaPass) * kMmaRow            // bf16 staging of one pass
+         + size_t(16) * kMmaChunk * 2            // A
+         + size_t(kMmaChunk) * 4;                // row numbers
+}
+static_assert(size_t(16) * kMmaCols * 4 <= size_t(kMmaBufs) * kMmaPass * kMmaCols, "the partial fits in the ring");
+static_assert(kMmaPass * (kMmaCols / 16) == 2 * kGvThreads, "two 16-byte copies per thread per pass");
+
+// Requires Wq's rows (and its base) 16-byte aligned.
+__global__ void __launch_bounds__(kGvThreads)
+gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t sA, const int8_t* __restrict__ B,
+                          int64_t ldb, int64_t sB, int64_t M, int64_t N, const int32_t* __restrict__ idx,
+                          int64_t k_keep, void* __restrict__ C, int64_t ldc, int64_t sC, int out_bf16,
+                          const float* __restrict__ scale, int64_t s_stride) {
+  constexpr int AROW = kMmaChunk * 2;
+  constexpr int R8 = kMmaCols;  // bytes per slice in the int8 ring
+  extern __shared__ __align__(128) unsigned char gvw_smem[];
+  unsigned char* ring = gvw_smem;                                    // [kMmaBufs][kMmaPass][R8]
+  unsigned char* cvt = ring + size_t(kMmaBufs) * kMmaPass * R8;       // [kMmaPass][kMmaRow], swizzled bf16
+  unsigned char* as = cvt + size_t(kMmaPass) * kMmaRow;               // [16][AROW]
+  int32_t* rows = reinterpret_cast<int32_t*>(as + 16 * AROW);        // [kMmaChunk]
+  float* cta = reinterpret_cast<float*>(ring);                       // [16][kMmaCols], once the ring is drained
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const unsigned cs = cluster.num_blocks();
+  const unsigned crank = cluster.block_rank();
+  const int64_t b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t n0 = int64_t(blockIdx.x) * kMmaCols;
+  const int cchunk = tid & 15;                   // this thread's 16 columns in the copies
+  const int64_t c = n0 + 16 * cchunk;
+  const uint32_t src_bytes = c >= N ? 0u : uint32_t(min(int64_t(16), N - c));
+  const uint16_t* Ab = A + b * sA;
+  const int8_t* Bc = B + b * sB + (src_bytes ? c : 0);
+  const int32_t* ib = idx + b * k_keep;
+  const int64_t per = (k_keep + cs - 1) / cs;
+  const int64_t t_begin = min(k_keep, int64_t(crank) * per), t_end = min(k_keep, t_begin + per);
+  const uint32_t ring_s = smem_addr(ring), cvt_s = smem_addr(cvt), as_s = smem_addr(as);
+  const int a_m = (lane & 7) + ((lane >> 3) & 1) * 8, a_kc = lane >> 4;
+  const int b_k = (lane & 7) + ((lane >> 3) & 1) * 8, b_nt = lane >> 4;
+
+  for (int e = tid; e < 16 * AROW / 16; e += kGvThreads) reinterpret_cast<uint4*>(as)[e] = make_uint4(0u, 0u, 0u, 0u);
+
+  float d[4][4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+
+  pdl_trigger();
+  pdl_wait();
+#pragma unroll 1
+  for (int64_t c0 = t_begin; c0 < t_end; c0 += kMmaChunk) {
+    const int nc = int(min(int64_t(kMmaChunk), t_end - c0));
+    const int np = (nc + kMmaPass - 1) / kMmaPass;
+    __syncthreads();
+    for (int i = tid; i < np * kMmaPass; i += kGvThreads) {
+      const int32_t r = i < nc ? ib[c0 + i] : 0;
+      rows[i] = r;
+      uint16_t v[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) v[m] = (m < M && i < nc) ? __ldg(Ab + int64_t(m) * lda + r) : uint16_t(0);
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+        if (m < M) *reinterpret_cast<uint16_t*>(as + swz(m, AROW, i >> 3) + (i & 7) * 2) = v[m];
+    }
+    __syncthreads();
+    auto issue = [&](int p) {
+      if (p < np) {
+        const uint32_t boff = uint32_t(p % kMmaBufs) * kMmaPass * R8;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int il = (tid >> 4) + 16 * j;  // slice within the pass
+          const int i = p * kMmaPass + il;
+          const bool live = i < nc && src_bytes != 0;
+          cp_async16_zfill(ring_s + boff + uint32_t(il) * R8 + uint32_t(cchunk) * 16u,
+                           live ? Bc + int64_t(rows[i]) * ldb : Bc, live ? src_bytes : 0u);
+        }
+      }
+      cp_async_commit();
+    };
+#pragma unroll 1
+    for (int q = 0; q < kMmaBufs - 1; ++q) issue(q);
+#pragma unroll 1
+    for (int p = 0; p < np; ++p) {
+      cp_async_wait<kMmaBufs - 2>();
+      __syncthreads();  // pass p's int8 rows are visible; the previous pass is done with the staging
+      {
+        const unsigned char* src = ring + size_t(p % kMmaBufs) * kMmaPass * R8;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int il = (tid >> 4) + 16 * j;
+          const uint4 q = *reinterpret_cast<const uint4*>(src + il * R8 + cchunk * 16);
+          const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            o[2 * h] = pack_bf16x2(float(int8_t(w[h] & 0xFF)), float(int8_t((w[h] >> 8) & 0xFF)));
+            o[2 * h + 1] = pack_bf16x2(float(int8_t((w[h] >> 16) & 0xFF)), float(int8_t(w[h] >> 24)));
+          }
+          *reinterpret_cast<uint4*>(cvt + swz(il, kMmaRow, 2 * cchunk)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(cvt + swz(il, kMmaRow, 2 * cchunk + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+      }
+      __syncthreads();  // the bf16 staging of pass p is complete
+#pragma unroll
+      for (int kc = 0; kc < kMmaPass / 16; ++kc) {
+        uint32_t a0, a1, a2, a3, b0, b1, b2, b3, b4, b5, b6, b7;
+        ldsm_x4(as_s + swz(a_m, AROW, (p * kMmaPass + kc * 16) / 8 + a_kc), a0, a1, a2, a3);
+        ldsm_x4_t(cvt_s + swz(kc * 16 + b_k, kMmaRow, warp * 4 + b_nt), b0, b1, b2, b3);
+        ldsm_x4_t(cvt_s + swz(kc * 16 + b_k, kMmaRow, warp * 4 + 2 + b_nt), b4, b5, b6, b7);
+        mma_bf16_16816(d[0], a0, a1, a2, a3, b0, b1);
+        mma_bf16_16816(d[1], a0, a1, a2, a3, b2, b3);
+        mma_bf16_16816(d[2], a0, a1, a2, a3, b4, b5);
+        mma_bf16_16816(d[3], a0, a1, a2, a3, b6, b7);
+      }
+      __syncthreads();  // every warp is done with the staging and with ring buffer p
+      issue(p + kMmaBufs - 1);
+    }
+    cp_async_wait<0>();
+  }
+  __syncthreads();
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int col = warp * 32 + t * 8 + (lane & 3) * 2;
+    const int m = lane >> 2;
+    cta[m * kMmaCols + col] = d[t][0];
+    cta[m * kMmaCols + col + 1] = d[t][1];
+    cta[(m + 8) * kMmaCols + col] = d[t][2];
+    cta[(m + 8) * kMmaCols + col + 1] = d[t][3];
+  }
+  cluster.sync();
+  if (crank == 0) {
+    for (int e = tid; e < 16 * kMmaCols; e += kGvThreads) {
+      const int m = e / kMmaCols;
+      const int64_t col = n0 + (e % kMmaCols);
+      if (m >= M || col >= N) continue;
+      float t = 0.f;
+      for (unsigned q = 0; q < cs; ++q) t += cluster.map_shared_rank(cta, q)[e];
+      t *= scale[b * s_stride + col];
+      const int64_t off = b * sC + int64_t(m) * ldc + col;
+      if (out_bf16)
+        static_cast<uint16_t*>(C)[off] = uint16_t(pack_bf16x2(t, 0.f) & 0xFFFFu);
+      else
+        static_cast<float*>(C)[off] = t;
+    }
+  }
+  cluster.sync();
+}
+
+// cluster size (1..8) whose grid fills whole waves of two CTAs per SM best,
+// each CTA keeping >= 64 slices
+unsigned wave_cluster(int64_t blocks, int64_t k_keep, int sms) {
+  unsigned best_q = 1;
+  double best = -1.0;
+  for (unsigned q = 1; q <= kGvMaxCluster; ++q) {
+    if (q > 1 && k_keep < int64_t(q) * 64) break;
+    const double waves = double(blocks * q) / double(2 * sms);
+    const double eff = waves / std::max(1.0, std::ceil(waves));
+    if (eff > best + 1e-9) {
+      best = eff;
+      best_q = q;
+    }
+  }
+  return best_q;
+}
+
 template <int MT>
 cudaError_t launch_w8_mt(const GemvArgs& g, const float* scale, int64_t s_stride, cudaStream_t st) {
   const size_t smem = gv_async_smem_bytes<int8_t, MT>();
@@ -633,6 +804,25 @@ cudaError_t launch_w8_mt(const GemvArgs& g, const float* scale, int64_t s_stride
 cudaError_t launch_gemv_gather_w8(const GemvArgs& g, const float* scale, int64_t s_stride, cudaStream_t st) {
   if (g.batch == 0 || g.M == 0 || g.N == 0) return cudaSuccess;
   if (g.M > kGemvMaxRows) return cudaErrorInvalidValue;
+  if ((reinterpret_cast<uintptr_t>(g.b) % 16 == 0) && g.ldb % 16 == 0 && (g.batch == 1 || g.strideB % 16 == 0)) {
+    const size_t smem = gv_mma_w8_smem_bytes();
+    static bool attr_done[64] = {};
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(gemv_gather_mma_w8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           int(smem));
+      if (e != cudaSuccess) return e;
+      attr_done[dev] = true;
+    }
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t mblk = (g.N + kMmaCols - 1) / kMmaCols;
+    const unsigned mcs = wave_cluster(mblk * g.batch, g.k_keep, sms);
+    return launch_pdl(gemv_gather_mma_w8_kernel, dim3(unsigned(mblk), mcs, unsigned(g.batch)), dim3(kGvThreads),
+                      smem, st, dim3(1, mcs, 1), static_cast<const uint16_t*>(g.a), g.lda, g.strideA,
+                      static_cast<const int8_t*>(g.b), g.ldb, g.strideB, g.M, g.N, g.idx, g.k_keep, g.c, g.ldc,
+                      g.strideC, int(g.out == kBF16), scale, s_stride);
+  }
   if (g.M <= 1) return launch_w8_mt<1>(g, scale, s_stride, st);
   if (g.M <= 2) return launch_w8_mt<2>(g, scale, s_stride, st);
   if (g.M <= 4) return launch_w8_mt<4>(g, scale, s_stride, st);

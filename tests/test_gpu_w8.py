@@ -100,3 +100,23 @@ def test_w8_rejects_misaligned_weights_and_missing_norms():
     with pytest.raises(rmm.RMMError) as e:  # the gather-GEMV copies 4 int8 at a time
         rmm.matmul_reduced_w8(X, Wodd, scale, 0.5, mode="a_only")
     assert e.value.status == rmm.RMM_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("N,ld", [(1000, 1024), (4096, 4096)], ids=["ragged", "full"])
+def test_w8_gemv_tensor_core_route(M, N, ld):
+    """16-byte aligned INT8 rows take the tensor-core gather-GEMV (int8 rows
+    converted exactly to bf16 per pass); a ragged N inside a wider row pitch
+    checks the column bounds."""
+    K = 3000
+    X = _x(M, K, 11 + M)
+    Wfull, sfull = inputs.int8_weight(K, ld, seed=12, device=DEV)
+    Wq, scale = Wfull[:, :N], sfull[:N].contiguous()
+    W64 = _deq(Wq, scale)
+    bn = rmm.b_norms_w8(Wq, scale)
+    k = rmm.keep_count(0.4, K)
+    idx = rmm.select(rmm.score_b_norms(X, bn), k)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        C = rmm.gemv_gather_w8(X, Wq, scale, idx, out_dtype)
+        check_product(f64(C), f64(X), W64, idx.cpu().numpy(), product_tol(torch.bfloat16, out_dtype))
+    assert torch.equal(rmm.gemv_gather_w8(X, Wq, scale, idx), rmm.gemv_gather_w8(X, Wq, scale, idx))
