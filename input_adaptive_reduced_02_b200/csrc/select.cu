@@ -191,32 +191,96 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
   }
   // Kept: keys whose masked bits exceed `prefix`, plus the `remaining`
   // lowest-indexed keys whose masked bits equal it (all of them when the bin
-  // is taken whole).
+  // is taken whole). Larger K: warp w compacts the contiguous chunk w of the
+  // keys, 32 consecutive keys per step (conflict-free shared-memory reads; a
+  // contiguous run per thread would read 32 runs in one bank), in two sweeps:
+  // counts, then writes at offsets from a scan over the warps' counts.
   const uint32_t T = prefix, need_eq = remaining;
   const bool take_all_eq = remaining == bin_count;
-  const int per = (K + THREADS - 1) / THREADS;
-  const int lo = min(K, tid * per), hi_i = min(K, lo + per);
-  uint32_t n_gt = 0, n_eq = 0;
-  for (int i = lo; i < hi_i; ++i) {
-    const uint32_t k = (keys_in_smem ? keys[i] : order_key(sb[i])) & mask;
-    n_gt += (k > T);
-    n_eq += (k == T);
-  }
-  uint32_t total, eq_take = n_eq;
-  if (!take_all_eq) {
-    const uint32_t eq_before = block_exclusive_scan<THREADS>(n_eq, warp_sums, &total);
-    eq_take = eq_before >= need_eq ? 0u : min(n_eq, need_eq - eq_before);
-  }
-  uint32_t pos = block_exclusive_scan<THREADS>(n_gt + eq_take, warp_sums, &total);
-  uint32_t taken_eq = 0;
-  for (int i = lo; i < hi_i; ++i) {
-    const uint32_t k = (keys_in_smem ? keys[i] : order_key(sb[i])) & mask;
-    if (k > T) {
-      ib[pos++] = i;
-    } else if (k == T && taken_eq < eq_take) {
-      ib[pos++] = i;
-      ++taken_eq;
+  if (K <= 4 * THREADS) {
+    // up to 4 keys per thread: a contiguous run each and two block scans
+    // (measured faster than the warp sweeps below at this size)
+    const int per = (K + THREADS - 1) / THREADS;
+    const int lo = min(K, tid * per), hi_i = min(K, lo + per);
+    uint32_t c_gt = 0, c_eq = 0;
+    for (int i = lo; i < hi_i; ++i) {
+      const uint32_t k = (keys_in_smem ? keys[i] : order_key(sb[i])) & mask;
+      c_gt += (k > T);
+      c_eq += (k == T);
     }
+    uint32_t total, eq_take = c_eq;
+    if (!take_all_eq) {
+      const uint32_t eq_before = block_exclusive_scan<THREADS>(c_eq, warp_sums, &total);
+      eq_take = eq_before >= need_eq ? 0u : min(c_eq, need_eq - eq_before);
+    }
+    uint32_t pos = block_exclusive_scan<THREADS>(c_gt + eq_take, warp_sums, &total);
+    uint32_t taken_eq = 0;
+    for (int i = lo; i < hi_i; ++i) {
+      const uint32_t k = (keys_in_smem ? keys[i] : order_key(sb[i])) & mask;
+      if (k > T) {
+        ib[pos++] = i;
+      } else if (k == T && taken_eq < eq_take) {
+        ib[pos++] = i;
+        ++taken_eq;
+      }
+    }
+    return;
+  }
+  const int chunk = (K + kWarps - 1) / kWarps;
+  const int w_lo = min(K, warp * chunk), w_hi = min(K, w_lo + chunk);
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int base = w_lo; base < w_hi; base += 32) {
+    const int i = base + lane;
+    const bool valid = i < w_hi;
+    const uint32_t k = valid ? ((keys_in_smem ? keys[i] : order_key(sb[i])) & mask) : 0u;
+    n_gt += __popc(__ballot_sync(0xffffffffu, valid && k > T));
+    n_eq += __popc(__ballot_sync(0xffffffffu, valid && k == T));
+  }
+  // exclusive scans over the warps (in warp order) of the equal counts and of
+  // the kept counts; warp_min/warp_max are free again (the barrier covers the
+  // case without radix passes, where they were last read for kmin/kmax)
+  __syncthreads();
+  if (lane == 0) {
+    warp_min[warp] = n_eq;
+    warp_max[warp] = n_gt;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t e = lane < kWarps ? warp_min[lane] : 0u, g = lane < kWarps ? warp_max[lane] : 0u;
+    uint32_t e_incl = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, e_incl, o);
+      if (lane >= o) e_incl += y;
+    }
+    const uint32_t e_before = e_incl - e;
+    const uint32_t take = take_all_eq ? e : (e_before >= need_eq ? 0u : min(e, need_eq - e_before));
+    uint32_t k_incl = g + take;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, k_incl, o);
+      if (lane >= o) k_incl += y;
+    }
+    if (lane < kWarps) {
+      warp_min[lane] = take;                  // equal keys this warp keeps
+      warp_max[lane] = k_incl - (g + take);   // first output slot of this warp
+    }
+  }
+  __syncthreads();
+  const uint32_t eq_take = warp_min[warp];
+  uint32_t pos = warp_max[warp], eq_seen = 0;
+  for (int base = w_lo; base < w_hi; base += 32) {
+    const int i = base + lane;
+    const bool valid = i < w_hi;
+    const uint32_t k = valid ? ((keys_in_smem ? keys[i] : order_key(sb[i])) & mask) : 0u;
+    const bool gt = valid && k > T, eq = valid && k == T;
+    const uint32_t eq_mask = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && eq_seen + __popc(eq_mask & lt_mask) < eq_take);
+    const uint32_t t_mask = __ballot_sync(0xffffffffu, take);
+    if (take) ib[pos + __popc(t_mask & lt_mask)] = i;
+    pos += __popc(t_mask);
+    eq_seen += __popc(eq_mask);
   }
 }
 

@@ -407,3 +407,19 @@ def test_fused_call_bit_identical_to_stage_calls(shape, gemm_cta_group):
         C_ref = rmm.gemm(A_S, B_S, k, out_dtype, N=N)
         assert torch.equal(C, C_ref)
         check_product(f64(C), f64(A), f64(B), idx.cpu().numpy(), product_tol(torch.bfloat16, out_dtype))
+
+
+@pytest.mark.parametrize("K", [4096, 4097, 8192, 50000])
+def test_select_large_k_with_heavy_ties(K):
+    """Both compaction schemes (up to 4 keys per thread, warp sweeps beyond):
+    scores drawn from 7 distinct values, so the threshold bin holds thousands
+    of equal keys and only the lowest-indexed ones may be kept; batch of 3."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(K)
+    vals = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 7.0], device=DEV)
+    s = vals[torch.randint(0, 7, (3, K), generator=g, device=DEV)].contiguous()
+    for rho in (0.1, 0.5, 0.93):
+        k = rmm.keep_count(rho, K)
+        idx = rmm.select(s, k)
+        for b in range(3):
+            assert idx[b].cpu().numpy().tolist() == O.select_top(s[b].cpu().numpy(), k).tolist()
