@@ -112,7 +112,8 @@ rmm_status rmm_score(const void* A, int64_t lda, int64_t strideA,
  *   s: [batch][K] f32 scores; idx: [batch][k_keep] i32 output, ascending.
  *   Ties go to the lower index; -0.0 equals +0.0. Exact: the result depends
  *   only on the order of the scores, never on rounding. 1 <= k_keep <= K.
- *   A NaN score sets RMM_STATUS_BIT_NONFINITE in status_word (nullable).
+ *   A NaN or infinite score sets RMM_STATUS_BIT_NONFINITE in status_word
+ *   (nullable).
  *   K is at most 2^21 (RMM_ERR_UNSUPPORTED above; the same limit applies to
  *   every call that selects). */
 rmm_status rmm_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,

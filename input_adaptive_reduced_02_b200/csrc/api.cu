@@ -120,11 +120,11 @@ static Workspace carve(void* base, int64_t batch, int64_t M, int64_t K, int64_t 
 static rmm_status do_score(const void* A, int64_t lda, int64_t sA, const void* B, int64_t ldb, int64_t sB,
                            int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N, rmm_dtype in,
                            rmm_score_mode mode, float* s, uint32_t* status, cudaStream_t st,
-                           const float* bn = nullptr, int64_t bn_stride = 0) {
+                           const float* bn = nullptr, int64_t bn_stride = 0, int clear_status = 0) {
   const MatView a{A, lda, sA, M, K};
   const int bmode = bn ? 3 : (mode == RMM_SCORE_A_ONLY ? 0 : (b_kmajor ? 2 : 1));
   const MatView b = b_kmajor ? MatView{B, ldb, sB, N, K} : MatView{B, ldb, sB, K, N};
-  const cudaError_t ce = launch_score(a, b, bmode, kind(in), batch, s, status, st, bn, bn_stride);
+  const cudaError_t ce = launch_score(a, b, bmode, kind(in), batch, s, status, st, bn, bn_stride, clear_status);
   if (ce != cudaSuccess) return cuda_fail(ce, "score kernel");
   return RMM_OK;
 }
@@ -334,12 +334,15 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
   if (workspace_bytes < w.bytes)
     return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, w.bytes);
   if ((r = bind_device(stream))) return r;
-  cudaError_t ce = cudaMemsetAsync(w.status, 0, 4, stream);
-  if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemsetAsync(status)");
-  if (batch == 0) return RMM_OK;
+  cudaError_t ce = cudaSuccess;
+  if (batch == 0) {  // no kernel runs: clear the status word here
+    ce = cudaMemsetAsync(w.status, 0, 4, stream);
+    return ce == cudaSuccess ? RMM_OK : cuda_fail(ce, "cudaMemsetAsync(status)");
+  }
   int32_t* idx = idx_out ? idx_out : w.idx;
+  // the score kernel clears the status word (it is the call's first kernel)
   if ((r = do_score(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, in, mode, w.s, w.status, stream,
-                    bn, bn_stride)))
+                    bn, bn_stride, 1)))
     return r;
   // The select runs on one SM per batch item; the C tiles that the GEMM's
   // split-K round adds into are zeroed meanwhile by helper blocks of the same
@@ -593,12 +596,14 @@ rmm_status rmm_matmul_reduced_w8(const void* A, int64_t lda, int64_t strideA, co
   if (workspace_bytes < w.bytes)
     return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, w.bytes);
   if ((r = bind_device(stream))) return r;
-  cudaError_t ce = cudaMemsetAsync(w.status, 0, 4, stream);
-  if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemsetAsync(status)");
-  if (batch == 0) return RMM_OK;
+  cudaError_t ce = cudaSuccess;
+  if (batch == 0) {
+    ce = cudaMemsetAsync(w.status, 0, 4, stream);
+    return ce == cudaSuccess ? RMM_OK : cuda_fail(ce, "cudaMemsetAsync(status)");
+  }
   int32_t* idx = idx_out ? idx_out : w.idx;
   if ((r = do_score(A, lda, strideA, nullptr, 0, 0, 0, batch, M, K, N, in, mode, w.s, w.status, stream,
-                    mode == RMM_SCORE_PRODUCT ? b_norm : nullptr, b_norm_stride)))
+                    mode == RMM_SCORE_PRODUCT ? b_norm : nullptr, b_norm_stride, 1)))
     return r;
   GemmArgs g = gemm_args(w.a_s, w.b_st, 0, batch, M, N, k_keep, C, ldc, strideC, out, w.status);
   const bool gemv = M <= kGemvMaxRows;

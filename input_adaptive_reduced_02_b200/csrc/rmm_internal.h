@@ -58,8 +58,11 @@ void set_last_error(const char* msg);
 //  row-major [K][N]; bmode 2: sqrt(sum_j B[b][j][k]^2) with B = Kmat [N][K];
 //  bmode 0: 1). One launch.
 //  bmode 3: s[b][k] = sqrt(sum_i A[b][i][k]^2) · bn[b * bn_stride + k] (B not read).
+//  clear_status: zero *status first (the fused calls' first kernel) and leave
+//  non-finite scores to the selection to report.
 cudaError_t launch_score(const MatView& A, const MatView& B, int bmode, ElemKind e, int64_t batch, float* s,
-                         uint32_t* status, cudaStream_t st, const float* bn = nullptr, int64_t bn_stride = 0);
+                         uint32_t* status, cudaStream_t st, const float* bn = nullptr, int64_t bn_stride = 0,
+                         int clear_status = 0);
 //  out[b][k] = sqrt(sum_j B[b][k][j]^2) (B row-major [K][N], view rows = K) or, with
 //  b_kmajor, sqrt(sum_j B[b][j][k]^2) (B = Kmat [N][K], view rows = N, cols = K).
 cudaError_t launch_b_norms(const MatView& B, int b_kmajor, ElemKind e, int64_t batch, float* out, uint32_t* status,

@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kScoreThreads)
 score_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, int64_t M, int64_t K,
              const T* __restrict__ B, int64_t ldb, int64_t sB, int64_t N,
              const float* __restrict__ bn, int64_t bn_stride,
-             float* __restrict__ s, uint32_t* status, int a_vec, int b_vec) {
+             float* __restrict__ s, uint32_t* status, int a_vec, int b_vec, int clear_status) {
   constexpr int V = 16 / sizeof(T);
   constexpr int CW = 8 * V;
   __shared__ float red[32][CW + 1];
@@ -146,6 +146,11 @@ score_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, int64_t M, int64_
   const int64_t c0 = strip0 + int64_t(cl) * V;
   pdl_trigger();
   pdl_wait();
+  // clear_status: the first kernel of a fused call clears the status word
+  // (every later kernel of the call waits for this one), and non-finite scores
+  // are then reported by the selection, which reads them all
+  if (clear_status && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0 && status)
+    *status = 0u;
 
   // ---- A: column sums over this CTA's rows
   {
@@ -206,7 +211,7 @@ score_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, int64_t M, int64_
       if constexpr (BMODE == 1 || BMODE == 2) sc *= sqrtf(ssb);
       if constexpr (BMODE == 3) sc *= bn[b * bn_stride + c];
       s[b * K + c] = sc;
-      if (!isfinite(sc)) status_or(status, RMM_NONFINITE_BIT);
+      if (!clear_status && !isfinite(sc)) status_or(status, RMM_NONFINITE_BIT);
     }
   }
   cluster.sync();  // keep shared memory alive until rank 0 has read it
@@ -293,7 +298,7 @@ int b_vec_ok(const MatView& B, int64_t batch) {
 
 template <typename T, int BMODE>
 cudaError_t launch_t(const MatView& A, const MatView& B, int64_t batch, float* s, uint32_t* status,
-                     cudaStream_t st, const float* bn = nullptr, int64_t bn_stride = 0) {
+                     cudaStream_t st, const float* bn = nullptr, int64_t bn_stride = 0, int clear_status = 0) {
   constexpr int V = 16 / sizeof(T);
   constexpr int CW = 8 * V;
   const int64_t K = A.cols;
@@ -309,7 +314,8 @@ cudaError_t launch_t(const MatView& A, const MatView& B, int64_t batch, float* s
   const int64_t N = BMODE == 2 ? B.rows : B.cols;
   return launch_pdl(score_kernel<T, BMODE>, dim3(unsigned((K + CW - 1) / CW), cs, unsigned(batch)),
                     dim3(kScoreThreads), 0, st, dim3(1, cs, 1), static_cast<const T*>(A.ptr), A.ld, A.bstride, A.rows, K,
-                    static_cast<const T*>(B.ptr), B.ld, B.bstride, N, bn, bn_stride, s, status, a_vec, b_vec);
+                    static_cast<const T*>(B.ptr), B.ld, B.bstride, N, bn, bn_stride, s, status, a_vec, b_vec,
+                    clear_status);
 }
 
 template <typename T>
@@ -324,21 +330,22 @@ cudaError_t launch_bnorm_rows(const MatView& B, int64_t batch, float* out, uint3
 }  // namespace
 
 cudaError_t launch_score(const MatView& A, const MatView& B, int bmode, ElemKind e, int64_t batch, float* s,
-                         uint32_t* status, cudaStream_t st, const float* bn, int64_t bn_stride) {
+                         uint32_t* status, cudaStream_t st, const float* bn, int64_t bn_stride, int clear_status) {
   if (batch == 0 || A.cols == 0) return cudaSuccess;
+  const int cs = clear_status;
   if (e == kBF16) {
     switch (bmode) {
-      case 0: return launch_t<uint16_t, 0>(A, B, batch, s, status, st);
-      case 1: return launch_t<uint16_t, 1>(A, B, batch, s, status, st);
-      case 2: return launch_t<uint16_t, 2>(A, B, batch, s, status, st);
-      default: return launch_t<uint16_t, 3>(A, B, batch, s, status, st, bn, bn_stride);
+      case 0: return launch_t<uint16_t, 0>(A, B, batch, s, status, st, nullptr, 0, cs);
+      case 1: return launch_t<uint16_t, 1>(A, B, batch, s, status, st, nullptr, 0, cs);
+      case 2: return launch_t<uint16_t, 2>(A, B, batch, s, status, st, nullptr, 0, cs);
+      default: return launch_t<uint16_t, 3>(A, B, batch, s, status, st, bn, bn_stride, cs);
     }
   }
   switch (bmode) {
-    case 0: return launch_t<uint32_t, 0>(A, B, batch, s, status, st);
-    case 1: return launch_t<uint32_t, 1>(A, B, batch, s, status, st);
-    case 2: return launch_t<uint32_t, 2>(A, B, batch, s, status, st);
-    default: return launch_t<uint32_t, 3>(A, B, batch, s, status, st, bn, bn_stride);
+    case 0: return launch_t<uint32_t, 0>(A, B, batch, s, status, st, nullptr, 0, cs);
+    case 1: return launch_t<uint32_t, 1>(A, B, batch, s, status, st, nullptr, 0, cs);
+    case 2: return launch_t<uint32_t, 2>(A, B, batch, s, status, st, nullptr, 0, cs);
+    default: return launch_t<uint32_t, 3>(A, B, batch, s, status, st, bn, bn_stride, cs);
   }
 }
 

@@ -99,7 +99,7 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
     const float4* s4 = reinterpret_cast<const float4*>(sb);
     for (int i = tid; i < K / 4; i += THREADS) {
       const float4 x = s4[i];
-      nan_seen |= (x.x != x.x) | (x.y != x.y) | (x.z != x.z) | (x.w != x.w);
+      nan_seen |= !isfinite(x.x) | !isfinite(x.y) | !isfinite(x.z) | !isfinite(x.w);
       const uint4 k4 = make_uint4(order_key(x.x), order_key(x.y), order_key(x.z), order_key(x.w));
       kmin = min(min(kmin, min(k4.x, k4.y)), min(k4.z, k4.w));
       kmax = max(max(kmax, max(k4.x, k4.y)), max(k4.z, k4.w));
@@ -108,7 +108,7 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
   } else {
     for (int i = tid; i < K; i += THREADS) {
       const float x = sb[i];
-      nan_seen |= (x != x);
+      nan_seen |= !isfinite(x);
       const uint32_t k = order_key(x);
       kmin = min(kmin, k);
       kmax = max(kmax, k);
