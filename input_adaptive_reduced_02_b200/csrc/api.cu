@@ -135,6 +135,13 @@ static rmm_status do_pack(const void* A, int64_t lda, int64_t sA, const void* B,
   const ElemKind e = kind(in);
   const int64_t kp = round_up(k_keep, 64);
   const uint64_t lim = wait_limit();
+  if (!b_kmajor) {
+    bool handled = false;
+    const cudaError_t be = launch_pack_both(MatView{A, lda, sA, M, K}, MatView{B, ldb, sB, K, N}, e, batch, idx, k_keep,
+                                            kp, A_S, B_S, packed_b_ld(N), status, lim, st, &handled);
+    if (be != cudaSuccess) return cuda_fail(be, "pack kernel (A and B)");
+    if (handled) return RMM_OK;
+  }
   cudaError_t ce = launch_pack_cols(MatView{A, lda, sA, M, K}, e, batch, idx, k_keep, kp, A_S, status, lim, st);
   if (ce != cudaSuccess) return cuda_fail(ce, "pack kernel (A)");
   if (b_kmajor)

@@ -94,17 +94,18 @@ __device__ __forceinline__ void gather_rows(const T* srow, int nr, int64_t C, co
 // Rows (and, when idx_in_smem, the kept indices) staged by bulk-async copies
 // (rows 16-byte aligned, C·e a multiple of 16; idx 16-byte aligned).
 template <typename T>
-__global__ void __launch_bounds__(kPackThreads)
-pack_cols_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t R, int64_t C,
-                      const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
-                      int rows_per_cta, int idx_in_smem, uint32_t* status, uint64_t wait_ns) {
+__device__ __forceinline__ void pack_cols_bulk_body(int64_t bx, const T* __restrict__ X, int64_t ld, int64_t bstride,
+                                                    int64_t R, int64_t C, const int32_t* __restrict__ idx,
+                                                    int64_t k_keep, int64_t k_pad, T* __restrict__ out,
+                                                    int rows_per_cta, int idx_in_smem, uint32_t* status,
+                                                    uint64_t wait_ns) {
   extern __shared__ __align__(128) unsigned char pack_smem[];
   __shared__ uint64_t bar;
   __shared__ int never;
   T* srow = reinterpret_cast<T*>(pack_smem);
   int32_t* sidx = reinterpret_cast<int32_t*>(pack_smem + size_t(rows_per_cta) * C * sizeof(T));
   const int64_t b = blockIdx.y;
-  const int64_t r0 = int64_t(blockIdx.x) * rows_per_cta;
+  const int64_t r0 = bx * rows_per_cta;
   const int nr = int(min(int64_t(rows_per_cta), R - r0));
   const T* src = X + b * bstride + r0 * ld;
   const int32_t* gidx = idx + b * k_keep;
@@ -134,6 +135,15 @@ pack_cols_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int6
   __syncthreads();
   gather_rows(srow, nr, C, idx_in_smem ? sidx : gidx, idx_in_smem || gidx_vec, k_keep, k_pad,
               out + (b * R + r0) * k_pad);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPackThreads)
+pack_cols_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t R, int64_t C,
+                      const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
+                      int rows_per_cta, int idx_in_smem, uint32_t* status, uint64_t wait_ns) {
+  pack_cols_bulk_body<T>(blockIdx.x, X, ld, bstride, R, C, idx, k_keep, k_pad, out, rows_per_cta, idx_in_smem,
+                         status, wait_ns);
 }
 
 // Any alignment: rows staged with plain loads (eight in flight per thread).
@@ -215,10 +225,11 @@ constexpr int kRowRing = 4;
 constexpr int64_t kRowIdxStage = 8192;  // kept-row indices a CTA stages in shared memory
 
 template <typename T>
-__global__ void __launch_bounds__(kPackThreads)
-pack_rows_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t N,
-                      const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
-                      int64_t ldo, int rows_per_buf, int64_t seg, uint32_t* status, uint64_t wait_ns) {
+__device__ __forceinline__ void pack_rows_bulk_body(int64_t bx, int64_t nbx, const T* __restrict__ X, int64_t ld,
+                                                    int64_t bstride, int64_t N, const int32_t* __restrict__ idx,
+                                                    int64_t k_keep, int64_t k_pad, T* __restrict__ out, int64_t ldo,
+                                                    int rows_per_buf, int64_t seg, uint32_t* status,
+                                                    uint64_t wait_ns) {
   // A chunk is rows_per_buf whole rows (seg == N) or one `seg`-element segment
   // of one row (rows_per_buf == 1, long rows).
   extern __shared__ __align__(128) unsigned char pack_smem[];
@@ -230,8 +241,8 @@ pack_rows_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int6
   T* ring = reinterpret_cast<T*>(pack_smem);
   int32_t* sidx = reinterpret_cast<int32_t*>(pack_smem + kRowRing * buf_elems * sizeof(T));
   // this CTA's kept rows: a contiguous range of [0, k_keep), at most kRowIdxStage long
-  const int64_t per = (k_keep + gridDim.x - 1) / gridDim.x;
-  const int64_t t_begin = min(k_keep, int64_t(blockIdx.x) * per), t_end = min(k_keep, t_begin + per);
+  const int64_t per = (k_keep + nbx - 1) / nbx;
+  const int64_t t_begin = min(k_keep, bx * per), t_end = min(k_keep, t_begin + per);
   const int64_t nchunks = (t_end - t_begin + rows_per_buf - 1) / rows_per_buf * segs;
   T* outb = out + b * k_pad * ldo;
   if (threadIdx.x == 0) {
@@ -246,8 +257,8 @@ pack_rows_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int6
   // zero padding: rows k_keep <= t < k_pad (split across CTAs), and columns N <= c < ldo
   {
     const int64_t pad_rows = k_pad - k_keep;
-    const int64_t pr = (pad_rows + gridDim.x - 1) / gridDim.x;
-    const int64_t pa = k_keep + min(pad_rows, int64_t(blockIdx.x) * pr), pb = min(k_pad, pa + pr);
+    const int64_t pr = (pad_rows + nbx - 1) / nbx;
+    const int64_t pa = k_keep + min(pad_rows, bx * pr), pb = min(k_pad, pa + pr);
     for (int64_t t = pa; t < pb; ++t)
       for (int64_t c = threadIdx.x; c < ldo; c += kPackThreads) outb[t * ldo + c] = T(0);
     if (ldo > N)
@@ -299,6 +310,33 @@ pack_rows_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int6
     }
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // smem stays live until read
   }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPackThreads)
+pack_rows_bulk_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t N,
+                      const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
+                      int64_t ldo, int rows_per_buf, int64_t seg, uint32_t* status, uint64_t wait_ns) {
+  pack_rows_bulk_body<T>(blockIdx.x, gridDim.x, X, ld, bstride, N, idx, k_keep, k_pad, out, ldo, rows_per_buf, seg,
+                         status, wait_ns);
+}
+
+// Both packs in one launch (B row-major, both on the bulk paths): CTAs
+// [0, nb) copy B's kept rows, the others gather A's columns; the two copy
+// streams overlap instead of meeting at a kernel boundary.
+template <typename T>
+__global__ void __launch_bounds__(kPackThreads)
+pack_both_bulk_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, int64_t M, int64_t K, T* __restrict__ a_out,
+                      int rows_per_cta, int idx_in_smem, const T* __restrict__ B, int64_t ldb, int64_t sB, int64_t N,
+                      T* __restrict__ b_out, int64_t ldo, int rows_per_buf, int64_t seg, int64_t nb,
+                      const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, uint32_t* status,
+                      uint64_t wait_ns) {
+  if (int64_t(blockIdx.x) < nb)
+    pack_rows_bulk_body<T>(blockIdx.x, nb, B, ldb, sB, N, idx, k_keep, k_pad, b_out, ldo, rows_per_buf, seg, status,
+                           wait_ns);
+  else
+    pack_cols_bulk_body<T>(int64_t(blockIdx.x) - nb, A, lda, sA, M, K, idx, k_keep, k_pad, a_out, rows_per_cta,
+                           idx_in_smem, status, wait_ns);
 }
 
 // Kept rows of B, any alignment: plain element copies.
@@ -399,7 +437,62 @@ cudaError_t launch_pack_rows_t(const MatView& X, int64_t batch, const int32_t* i
                     p, X.ld, X.bstride, X.cols, idx, k_keep, k_pad, o, ldo);
 }
 
+// Both packs in one launch when A's rows are short enough to stage several per
+// CTA and both operands take the bulk paths; *handled = false otherwise.
+template <typename T>
+cudaError_t launch_pack_both_t(const MatView& A, const MatView& B, int64_t batch, const int32_t* idx,
+                               int64_t k_keep, int64_t k_pad, void* a_out, void* b_out, int64_t ldo, uint32_t* status,
+                               uint64_t wait_ns, cudaStream_t st, bool* handled) {
+  *handled = false;
+  const size_t a_row = size_t(A.cols) * sizeof(T), b_row = size_t(B.cols) * sizeof(T);
+  const bool a_bulk = A.rows > 0 && a_row > 0 && a_row <= kStageBytes && a_row % 16 == 0 && aligned16(A.ptr) &&
+                      (A.ld * int64_t(sizeof(T))) % 16 == 0 &&
+                      (batch == 1 || (A.bstride * int64_t(sizeof(T))) % 16 == 0);
+  const bool b_bulk = b_row > 0 && b_row % 16 == 0 && b_row <= kStageMax && aligned16(B.ptr) && aligned16(b_out) &&
+                      (B.ld * int64_t(sizeof(T))) % 16 == 0 &&
+                      (batch == 1 || (B.bstride * int64_t(sizeof(T))) % 16 == 0) && (ldo * int64_t(sizeof(T))) % 16 == 0;
+  if (!a_bulk || !b_bulk) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // B: as in launch_pack_rows_t, with the index stage sized to the CTA's share
+  const int rows_per_buf = b_row <= 16384 ? int(std::min<size_t>(32, 16384 / b_row)) : 1;
+  const int64_t seg = b_row <= 16384 ? B.cols : int64_t(16384 / sizeof(T));
+  const int64_t want = std::max<int64_t>(1, 2 * int64_t(sms) / std::max<int64_t>(1, batch));
+  const int64_t segs = (B.cols + seg - 1) / seg;
+  const int64_t by_work = std::max<int64_t>(1, k_keep * segs / (4 * rows_per_buf));
+  const int64_t nb = std::max(std::min(want, by_work), (k_keep + kRowIdxStage - 1) / kRowIdxStage);
+  const int64_t per = (k_keep + nb - 1) / nb;
+  const size_t b_smem = size_t(kRowRing) * rows_per_buf * size_t(seg) * sizeof(T) + size_t((per * 4 + 15) / 16 * 16);
+  // A: as many whole rows per CTA as the same shared-memory size holds
+  const size_t idx_bytes = (size_t(k_keep) * 4 + 15) / 16 * 16;
+  const int idx_in_smem = idx_bytes <= kIdxStageMax && a_row + idx_bytes <= kSmemAttr;
+  const size_t a_fixed = idx_in_smem ? idx_bytes : 0;
+  const size_t budget = std::max(b_smem, a_row + a_fixed);
+  const int rows_per_cta = int(std::max<size_t>(1, std::min<size_t>(64, (budget - a_fixed) / a_row)));
+  const size_t smem = std::max(b_smem, size_t(rows_per_cta) * a_row + a_fixed);
+  if (smem > kSmemAttr) return cudaSuccess;
+  const int64_t na = (A.rows + rows_per_cta - 1) / rows_per_cta;
+  set_smem_attr_once(pack_both_bulk_kernel<T>);
+  *handled = true;
+  return launch_pdl(pack_both_bulk_kernel<T>, dim3(unsigned(nb + na), unsigned(batch)), dim3(kPackThreads), smem, st,
+                    dim3(0, 0, 0), static_cast<const T*>(A.ptr), A.ld, A.bstride, A.rows, A.cols,
+                    static_cast<T*>(a_out), rows_per_cta, idx_in_smem, static_cast<const T*>(B.ptr), B.ld, B.bstride,
+                    B.cols, static_cast<T*>(b_out), ldo, rows_per_buf, seg, nb, idx, k_keep, k_pad, status, wait_ns);
+}
+
 }  // namespace
+
+cudaError_t launch_pack_both(const MatView& A, const MatView& B, ElemKind e, int64_t batch, const int32_t* idx,
+                             int64_t k_keep, int64_t k_pad, void* a_out, void* b_out, int64_t ldo, uint32_t* status,
+                             uint64_t wait_ns, cudaStream_t st, bool* handled) {
+  *handled = false;
+  if (batch == 0) return cudaSuccess;
+  return e == kBF16 ? launch_pack_both_t<uint16_t>(A, B, batch, idx, k_keep, k_pad, a_out, b_out, ldo, status, wait_ns,
+                                                   st, handled)
+                    : launch_pack_both_t<uint32_t>(A, B, batch, idx, k_keep, k_pad, a_out, b_out, ldo, status, wait_ns,
+                                                   st, handled);
+}
 
 cudaError_t launch_pack_cols(const MatView& X, ElemKind e, int64_t batch, const int32_t* idx, int64_t k_keep,
                              int64_t k_pad, void* out, uint32_t* status, uint64_t wait_ns, cudaStream_t st) {

@@ -97,6 +97,12 @@ cudaError_t launch_pack_rows(const MatView& X, ElemKind e, int64_t batch, const 
                              int64_t k_keep, int64_t k_pad, void* out, int64_t ldo, uint32_t* status,
                              uint64_t wait_ns, cudaStream_t st);
 
+//  Both packs (A's columns, B's rows) in one launch when both take the bulk
+//  paths and A's rows are at most 32 KB; *handled reports whether it did.
+cudaError_t launch_pack_both(const MatView& A, const MatView& B, ElemKind e, int64_t batch, const int32_t* idx,
+                             int64_t k_keep, int64_t k_pad, void* a_out, void* b_out, int64_t ldo, uint32_t* status,
+                             uint64_t wait_ns, cudaStream_t st, bool* handled);
+
 // INT8 weights with one f32 scale per output column (scale[b * s_stride + j]):
 //  b_norm[b][k] = ||Wq[b][k][:] · scale||_2 (score.cu) and
 //  out[b][t][j] = bf16(Wq[b][idx[b][t]][j] · scale[j]) (pack.cu, zero padded).
