@@ -618,7 +618,7 @@ def run_ours(args):
                        "out_dtype": str(p.out_dtype).replace("torch.", ""),
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed before every timed step (256 MiB written, then another 256 MiB read)",
-                       "step": "one rmm_matmul_reduced call (score, select, pack, gemm: 5 kernels)",
+                       "step": "one rmm_matmul_reduced call (score, select, pack, gemm: 4 kernels)",
                        "timing": "CUDA events on the launching stream around each call; a device sleep before "
                                  "each step hides host launch overhead. The GEMM's duration for the roofline "
                                  "comes from a second timed loop of the same step made of the four stage "
