@@ -606,18 +606,25 @@ cudaError_t launch_t(const GemvArgs& g, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- INT8 weight, tensor cores
-// The mma path for an INT8 weight: each pass's int8 rows (256 columns = 256
-// bytes per slice, one 16-byte cp.async per 16 weights) are converted exactly
-// to bf16 into a swizzled staging buffer, which the same ldmatrix + mma.sync
-// loop reads; column j of the sums is scaled by scale[j] at the end.
+// The mma path for an INT8 weight: each pass's int8 rows (512 columns = 512
+// bytes per slice, one 16-byte cp.async per 16 weights, so a pass moves as
+// many bytes as the bf16 kernel's) are converted exactly to bf16 into a
+// swizzled staging buffer, which an ldmatrix + mma.sync loop reads (64 columns
+// per warp); column j of the sums is scaled by scale[j] at the end.
+constexpr int kW8Cols = 512;                  // columns of C per CTA
+constexpr int kW8Bufs = 3;                    // int8 ring buffers (kW8Bufs - 1 in flight)
+constexpr int kW8Chunk = 512;                 // slices whose indices and A values are staged at once
+constexpr int kW8Row = kW8Cols * 2;           // bytes of one staged bf16 slice
+
 constexpr size_t gv_mma_w8_smem_bytes() {
-  return size_t(kMmaBufs) * kMmaPass * kMmaCols  // int8 ring (then the CTA's partial)
-         + size_t(kMmaPass) * kMmaRow            // bf16 staging of one pass
-         + size_t(16) * kMmaChunk * 2            // A
-         + size_t(kMmaChunk) * 4;                // row numbers
+  return size_t(kW8Bufs) * kMmaPass * kW8Cols  // int8 ring (then the CTA's partial)
+         + size_t(kMmaPass) * kW8Row           // bf16 staging of one pass
+         + size_t(16) * kW8Chunk * 2           // A
+         + size_t(kW8Chunk) * 4;               // row numbers
 }
-static_assert(size_t(16) * kMmaCols * 4 <= size_t(kMmaBufs) * kMmaPass * kMmaCols, "the partial fits in the ring");
-static_assert(kMmaPass * (kMmaCols / 16) == 2 * kGvThreads, "two 16-byte copies per thread per pass");
+static_assert(size_t(16) * kW8Cols * 4 <= size_t(kW8Bufs) * kMmaPass * kW8Cols, "the partial fits in the ring");
+static_assert(kMmaPass * (kW8Cols / 16) == 4 * kGvThreads, "four 16-byte copies per thread per pass");
+static_assert(kW8Cols == kGvWarps * 64, "64 columns per warp");
 
 // Requires Wq's rows (and its base) 16-byte aligned.
 __global__ void __launch_bounds__(kGvThreads)
@@ -625,22 +632,22 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
                           int64_t ldb, int64_t sB, int64_t M, int64_t N, const int32_t* __restrict__ idx,
                           int64_t k_keep, void* __restrict__ C, int64_t ldc, int64_t sC, int out_bf16,
                           const float* __restrict__ scale, int64_t s_stride) {
-  constexpr int AROW = kMmaChunk * 2;
-  constexpr int R8 = kMmaCols;  // bytes per slice in the int8 ring
+  constexpr int AROW = kW8Chunk * 2;
+  constexpr int R8 = kW8Cols;  // bytes per slice in the int8 ring
   extern __shared__ __align__(128) unsigned char gvw_smem[];
-  unsigned char* ring = gvw_smem;                                    // [kMmaBufs][kMmaPass][R8]
-  unsigned char* cvt = ring + size_t(kMmaBufs) * kMmaPass * R8;       // [kMmaPass][kMmaRow], swizzled bf16
-  unsigned char* as = cvt + size_t(kMmaPass) * kMmaRow;               // [16][AROW]
-  int32_t* rows = reinterpret_cast<int32_t*>(as + 16 * AROW);        // [kMmaChunk]
-  float* cta = reinterpret_cast<float*>(ring);                       // [16][kMmaCols], once the ring is drained
+  unsigned char* ring = gvw_smem;                                    // [kW8Bufs][kMmaPass][R8]
+  unsigned char* cvt = ring + size_t(kW8Bufs) * kMmaPass * R8;        // [kMmaPass][kW8Row], swizzled bf16
+  unsigned char* as = cvt + size_t(kMmaPass) * kW8Row;                // [16][AROW]
+  int32_t* rows = reinterpret_cast<int32_t*>(as + 16 * AROW);        // [kW8Chunk]
+  float* cta = reinterpret_cast<float*>(ring);                       // [16][kW8Cols], once the ring is drained
 
   cg::cluster_group cluster = cg::this_cluster();
   const unsigned cs = cluster.num_blocks();
   const unsigned crank = cluster.block_rank();
   const int64_t b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t n0 = int64_t(blockIdx.x) * kMmaCols;
-  const int cchunk = tid & 15;                   // this thread's 16 columns in the copies
+  const int64_t n0 = int64_t(blockIdx.x) * kW8Cols;
+  const int cchunk = tid & 31;                   // this thread's 16 columns in the copies
   const int64_t c = n0 + 16 * cchunk;
   const uint32_t src_bytes = c >= N ? 0u : uint32_t(min(int64_t(16), N - c));
   const uint16_t* Ab = A + b * sA;
@@ -654,15 +661,15 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
 
   for (int e = tid; e < 16 * AROW / 16; e += kGvThreads) reinterpret_cast<uint4*>(as)[e] = make_uint4(0u, 0u, 0u, 0u);
 
-  float d[4][4];
+  float d[8][4];
 #pragma unroll
-  for (int t = 0; t < 4; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+  for (int t = 0; t < 8; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
 
   pdl_trigger();
   pdl_wait();
 #pragma unroll 1
-  for (int64_t c0 = t_begin; c0 < t_end; c0 += kMmaChunk) {
-    const int nc = int(min(int64_t(kMmaChunk), t_end - c0));
+  for (int64_t c0 = t_begin; c0 < t_end; c0 += kW8Chunk) {
+    const int nc = int(min(int64_t(kW8Chunk), t_end - c0));
     const int np = (nc + kMmaPass - 1) / kMmaPass;
     __syncthreads();
     for (int i = tid; i < np * kMmaPass; i += kGvThreads) {
@@ -678,10 +685,10 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
     __syncthreads();
     auto issue = [&](int p) {
       if (p < np) {
-        const uint32_t boff = uint32_t(p % kMmaBufs) * kMmaPass * R8;
+        const uint32_t boff = uint32_t(p % kW8Bufs) * kMmaPass * R8;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int il = (tid >> 4) + 16 * j;  // slice within the pass
+        for (int j = 0; j < 4; ++j) {
+          const int il = (tid >> 5) + 8 * j;  // slice within the pass
           const int i = p * kMmaPass + il;
           const bool live = i < nc && src_bytes != 0;
           cp_async16_zfill(ring_s + boff + uint32_t(il) * R8 + uint32_t(cchunk) * 16u,
@@ -691,16 +698,16 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
       cp_async_commit();
     };
 #pragma unroll 1
-    for (int q = 0; q < kMmaBufs - 1; ++q) issue(q);
+    for (int q = 0; q < kW8Bufs - 1; ++q) issue(q);
 #pragma unroll 1
     for (int p = 0; p < np; ++p) {
-      cp_async_wait<kMmaBufs - 2>();
+      cp_async_wait<kW8Bufs - 2>();
       __syncthreads();  // pass p's int8 rows are visible; the previous pass is done with the staging
       {
-        const unsigned char* src = ring + size_t(p % kMmaBufs) * kMmaPass * R8;
+        const unsigned char* src = ring + size_t(p % kW8Bufs) * kMmaPass * R8;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int il = (tid >> 4) + 16 * j;
+        for (int j = 0; j < 4; ++j) {
+          const int il = (tid >> 5) + 8 * j;
           const uint4 q = *reinterpret_cast<const uint4*>(src + il * R8 + cchunk * 16);
           const uint32_t w[4] = {q.x, q.y, q.z, q.w};
           uint32_t o[8];
@@ -709,42 +716,43 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
             o[2 * h] = pack_bf16x2(float(int8_t(w[h] & 0xFF)), float(int8_t((w[h] >> 8) & 0xFF)));
             o[2 * h + 1] = pack_bf16x2(float(int8_t((w[h] >> 16) & 0xFF)), float(int8_t(w[h] >> 24)));
           }
-          *reinterpret_cast<uint4*>(cvt + swz(il, kMmaRow, 2 * cchunk)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(cvt + swz(il, kMmaRow, 2 * cchunk + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+          *reinterpret_cast<uint4*>(cvt + swz(il, kW8Row, 2 * cchunk)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(cvt + swz(il, kW8Row, 2 * cchunk + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
         }
       }
       __syncthreads();  // the bf16 staging of pass p is complete
 #pragma unroll
       for (int kc = 0; kc < kMmaPass / 16; ++kc) {
-        uint32_t a0, a1, a2, a3, b0, b1, b2, b3, b4, b5, b6, b7;
+        uint32_t a0, a1, a2, a3;
         ldsm_x4(as_s + swz(a_m, AROW, (p * kMmaPass + kc * 16) / 8 + a_kc), a0, a1, a2, a3);
-        ldsm_x4_t(cvt_s + swz(kc * 16 + b_k, kMmaRow, warp * 4 + b_nt), b0, b1, b2, b3);
-        ldsm_x4_t(cvt_s + swz(kc * 16 + b_k, kMmaRow, warp * 4 + 2 + b_nt), b4, b5, b6, b7);
-        mma_bf16_16816(d[0], a0, a1, a2, a3, b0, b1);
-        mma_bf16_16816(d[1], a0, a1, a2, a3, b2, b3);
-        mma_bf16_16816(d[2], a0, a1, a2, a3, b4, b5);
-        mma_bf16_16816(d[3], a0, a1, a2, a3, b6, b7);
+#pragma unroll
+        for (int t2 = 0; t2 < 4; ++t2) {  // this warp's 8 tiles of 8 columns, two per ldmatrix
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(cvt_s + swz(kc * 16 + b_k, kW8Row, warp * 8 + 2 * t2 + b_nt), b0, b1, b2, b3);
+          mma_bf16_16816(d[2 * t2], a0, a1, a2, a3, b0, b1);
+          mma_bf16_16816(d[2 * t2 + 1], a0, a1, a2, a3, b2, b3);
+        }
       }
       __syncthreads();  // every warp is done with the staging and with ring buffer p
-      issue(p + kMmaBufs - 1);
+      issue(p + kW8Bufs - 1);
     }
     cp_async_wait<0>();
   }
   __syncthreads();
 #pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const int col = warp * 32 + t * 8 + (lane & 3) * 2;
+  for (int t = 0; t < 8; ++t) {
+    const int col = warp * 64 + t * 8 + (lane & 3) * 2;
     const int m = lane >> 2;
-    cta[m * kMmaCols + col] = d[t][0];
-    cta[m * kMmaCols + col + 1] = d[t][1];
-    cta[(m + 8) * kMmaCols + col] = d[t][2];
-    cta[(m + 8) * kMmaCols + col + 1] = d[t][3];
+    cta[m * kW8Cols + col] = d[t][0];
+    cta[m * kW8Cols + col + 1] = d[t][1];
+    cta[(m + 8) * kW8Cols + col] = d[t][2];
+    cta[(m + 8) * kW8Cols + col + 1] = d[t][3];
   }
   cluster.sync();
   if (crank == 0) {
-    for (int e = tid; e < 16 * kMmaCols; e += kGvThreads) {
-      const int m = e / kMmaCols;
-      const int64_t col = n0 + (e % kMmaCols);
+    for (int e = tid; e < 16 * kW8Cols; e += kGvThreads) {
+      const int m = e / kW8Cols;
+      const int64_t col = n0 + (e % kW8Cols);
       if (m >= M || col >= N) continue;
       float t = 0.f;
       for (unsigned q = 0; q < cs; ++q) t += cluster.map_shared_rank(cta, q)[e];
@@ -816,7 +824,7 @@ cudaError_t launch_gemv_gather_w8(const GemvArgs& g, const float* scale, int64_t
       attr_done[dev] = true;
     }
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t mblk = (g.N + kMmaCols - 1) / kMmaCols;
+    const int64_t mblk = (g.N + kW8Cols - 1) / kW8Cols;
     const unsigned mcs = wave_cluster(mblk * g.batch, g.k_keep, sms);
     return launch_pdl(gemv_gather_mma_w8_kernel, dim3(unsigned(mblk), mcs, unsigned(g.batch)), dim3(kGvThreads),
                       smem, st, dim3(1, mcs, 1), static_cast<const uint16_t*>(g.a), g.lda, g.strideA,
