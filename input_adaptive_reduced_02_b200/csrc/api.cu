@@ -360,7 +360,7 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
   const bool gemv = M <= kGemvMaxRows && !b_kmajor;
   SplitZero z;
   const bool zero = !gemv && in == RMM_BF16 && gemm_tc_split_zero(g, &z);
-  ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr);
+  ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr, gemv);
   if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
   g.c_zeroed = zero ? 1 : 0;
   if (M == 0 || N == 0) return RMM_OK;
@@ -616,7 +616,7 @@ rmm_status rmm_matmul_reduced_w8(const void* A, int64_t lda, int64_t strideA, co
   const bool gemv = M <= kGemvMaxRows;
   SplitZero z;
   const bool zero = !gemv && gemm_tc_split_zero(g, &z);
-  ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr);
+  ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr, gemv);
   if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
   g.c_zeroed = zero ? 1 : 0;
   if (M == 0 || N == 0) return RMM_OK;

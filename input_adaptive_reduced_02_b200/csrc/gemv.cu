@@ -448,17 +448,7 @@ gemv_gather_mma_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t sA, 
     const int nc = int(min(int64_t(kMmaChunk), t_end - c0));
     const int np = (nc + kMmaPass - 1) / kMmaPass;
     __syncthreads();  // the previous chunk is done with rows and A (and the zero fill is done)
-    // row numbers, and A[m][idx] as bf16 bits for m < M (zero past the chunk end)
-    for (int i = tid; i < np * kMmaPass; i += kGvThreads) {
-      const int32_t r = i < nc ? ib[c0 + i] : 0;
-      rows[i] = r;
-      uint16_t v[16];  // all loads first, then the stores: independent round trips
-#pragma unroll
-      for (int m = 0; m < 16; ++m) v[m] = (m < M && i < nc) ? __ldg(Ab + int64_t(m) * lda + r) : uint16_t(0);
-#pragma unroll
-      for (int m = 0; m < 16; ++m)
-        if (m < M) *reinterpret_cast<uint16_t*>(as + swz(m, AROW, i >> 3) + (i & 7) * 2) = v[m];
-    }
+    for (int i = tid; i < np * kMmaPass; i += kGvThreads) rows[i] = i < nc ? ib[c0 + i] : 0;
     __syncthreads();
     // copies of pass p's slices of B (zeros past the chunk end); one commit
     // group per call in every thread, so that group counts stay uniform
@@ -476,10 +466,21 @@ gemv_gather_mma_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t sA, 
     };
 #pragma unroll 1
     for (int q = 0; q < kMmaBufs - 1; ++q) issue(q);
+    // A[m][idx] as bf16 bits for m < M (zero past the chunk end), loaded while
+    // the first passes of B are in flight; all loads before the stores
+    for (int i = tid; i < np * kMmaPass; i += kGvThreads) {
+      const int32_t r = rows[i];
+      uint16_t v[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) v[m] = (m < M && i < nc) ? __ldg(Ab + int64_t(m) * lda + r) : uint16_t(0);
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+        if (m < M) *reinterpret_cast<uint16_t*>(as + swz(m, AROW, i >> 3) + (i & 7) * 2) = v[m];
+    }
 #pragma unroll 1
     for (int p = 0; p < np; ++p) {
       cp_async_wait<kMmaBufs - 2>();  // this thread's copies of pass p have landed
-      __syncthreads();                // and everyone's are visible to all warps
+      __syncthreads();                // and everyone's (and A's values) are visible to all warps
       const uint32_t rb = ring_s + uint32_t(p % kMmaBufs) * kMmaPass * kMmaRow;
 #pragma unroll
       for (int kc = 0; kc < kMmaPass / 16; ++kc) {
@@ -672,16 +673,7 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
     const int nc = int(min(int64_t(kW8Chunk), t_end - c0));
     const int np = (nc + kMmaPass - 1) / kMmaPass;
     __syncthreads();
-    for (int i = tid; i < np * kMmaPass; i += kGvThreads) {
-      const int32_t r = i < nc ? ib[c0 + i] : 0;
-      rows[i] = r;
-      uint16_t v[16];
-#pragma unroll
-      for (int m = 0; m < 16; ++m) v[m] = (m < M && i < nc) ? __ldg(Ab + int64_t(m) * lda + r) : uint16_t(0);
-#pragma unroll
-      for (int m = 0; m < 16; ++m)
-        if (m < M) *reinterpret_cast<uint16_t*>(as + swz(m, AROW, i >> 3) + (i & 7) * 2) = v[m];
-    }
+    for (int i = tid; i < np * kMmaPass; i += kGvThreads) rows[i] = i < nc ? ib[c0 + i] : 0;
     __syncthreads();
     auto issue = [&](int p) {
       if (p < np) {
@@ -699,6 +691,16 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
     };
 #pragma unroll 1
     for (int q = 0; q < kW8Bufs - 1; ++q) issue(q);
+    // A's values while the first passes of B are in flight (all loads before the stores)
+    for (int i = tid; i < np * kMmaPass; i += kGvThreads) {
+      const int32_t r = rows[i];
+      uint16_t v[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) v[m] = (m < M && i < nc) ? __ldg(Ab + int64_t(m) * lda + r) : uint16_t(0);
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+        if (m < M) *reinterpret_cast<uint16_t*>(as + swz(m, AROW, i >> 3) + (i & 7) * 2) = v[m];
+    }
 #pragma unroll 1
     for (int p = 0; p < np; ++p) {
       cp_async_wait<kW8Bufs - 2>();

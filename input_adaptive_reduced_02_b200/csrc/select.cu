@@ -71,7 +71,7 @@ constexpr int kBins = 1 << kDigitBits;
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS, 1)
 select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t* __restrict__ idx,
-              uint32_t* status, int keys_in_smem, int64_t items, const SplitZero zero) {
+              uint32_t* status, int keys_in_smem, int64_t items, const SplitZero zero, int late_launch) {
   constexpr int kWarps = THREADS / 32;
   const int K = int(K64);  // K <= 2^21 (checked on the host)
   extern __shared__ uint32_t keys[];  // K keys when keys_in_smem
@@ -85,7 +85,11 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
   const float* sb = s + int64_t(blockIdx.x) * K;
   int32_t* ib = idx + int64_t(blockIdx.x) * k_keep;
 
-  pdl_trigger();
+  // late_launch: the next kernel (a gather-GEMV in clusters of CTAs with
+  // large shared memory) launches only when this grid exits; launched early,
+  // it would be placed around the previous kernel's CTAs and part of it would
+  // run as a second wave
+  if (!late_launch) pdl_trigger();
   pdl_wait();
   if (blockIdx.x >= items) {  // helper block: zero C tiles for the GEMM later on the stream
     zero_split_tiles(zero, blockIdx.x - items, gridDim.x - items, tid, THREADS);
@@ -287,7 +291,7 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
 }  // namespace
 
 cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,
-                          uint32_t* status, cudaStream_t st, const SplitZero* zero) {
+                          uint32_t* status, cudaStream_t st, const SplitZero* zero, bool late_launch) {
   if (batch == 0) return cudaSuccess;
   SplitZero z = {};
   int64_t helpers = 0;
@@ -308,7 +312,7 @@ cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_ke
     attr_done[dev] = true;
   }
   return launch_pdl(select_kernel<kSelThreads>, dim3(unsigned(batch + helpers)), dim3(kSelThreads), smem, st,
-                    dim3(0, 0, 0), s, K, k_keep, idx, status, keys_in_smem, batch, z);
+                    dim3(0, 0, 0), s, K, k_keep, idx, status, keys_in_smem, batch, z, int(late_launch));
 }
 
 }  // namespace rmm
