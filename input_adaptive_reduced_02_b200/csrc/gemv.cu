@@ -211,9 +211,9 @@ __device__ __forceinline__ float4 slot_to_f32(const uint32_t*, const unsigned ch
   return *reinterpret_cast<const float4*>(slot);
 }
 __device__ __forceinline__ float4 slot_to_f32(const int8_t*, const unsigned char* slot) {
-  const uint32_t u = *reinterpret_cast<const uint32_t*>(slot);
-  return make_float4(float(int8_t(u & 0xFF)), float(int8_t((u >> 8) & 0xFF)), float(int8_t((u >> 16) & 0xFF)),
-                     float(int8_t(u >> 24)));
+  float4 f;
+  s8x4_to_f32(*reinterpret_cast<const uint32_t*>(slot), f.x, f.y, f.z, f.w);
+  return f;
 }
 
 // Requires B's rows (and its base) aligned to lane_bytes<TB>(). TB is B's
@@ -714,10 +714,7 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
           const uint32_t w[4] = {q.x, q.y, q.z, q.w};
           uint32_t o[8];
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            o[2 * h] = pack_bf16x2(float(int8_t(w[h] & 0xFF)), float(int8_t((w[h] >> 8) & 0xFF)));
-            o[2 * h + 1] = pack_bf16x2(float(int8_t((w[h] >> 16) & 0xFF)), float(int8_t(w[h] >> 24)));
-          }
+          for (int h = 0; h < 4; ++h) s8x4_to_bf16x4(w[h], o[2 * h], o[2 * h + 1]);
           *reinterpret_cast<uint4*>(cvt + swz(il, kW8Row, 2 * cchunk)) = make_uint4(o[0], o[1], o[2], o[3]);
           *reinterpret_cast<uint4*>(cvt + swz(il, kW8Row, 2 * cchunk + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
         }

@@ -537,10 +537,11 @@ pack_rows_w8_kernel(const int8_t* __restrict__ Wq, int64_t ldw, int64_t sW, cons
         const uint2 q = *reinterpret_cast<const uint2*>(src + 8 * g);
         const float4 s0 = *reinterpret_cast<const float4*>(sc + 8 * g);
         const float4 s1 = *reinterpret_cast<const float4*>(sc + 8 * g + 4);
-        const float v[8] = {float(int8_t(q.x & 0xFF)) * s0.x,         float(int8_t((q.x >> 8) & 0xFF)) * s0.y,
-                            float(int8_t((q.x >> 16) & 0xFF)) * s0.z, float(int8_t(q.x >> 24)) * s0.w,
-                            float(int8_t(q.y & 0xFF)) * s1.x,         float(int8_t((q.y >> 8) & 0xFF)) * s1.y,
-                            float(int8_t((q.y >> 16) & 0xFF)) * s1.z, float(int8_t(q.y >> 24)) * s1.w};
+        float v[8];
+        s8x4_to_f32(q.x, v[0], v[1], v[2], v[3]);
+        s8x4_to_f32(q.y, v[4], v[5], v[6], v[7]);
+        v[0] *= s0.x, v[1] *= s0.y, v[2] *= s0.z, v[3] *= s0.w;
+        v[4] *= s1.x, v[5] *= s1.y, v[6] *= s1.z, v[7] *= s1.w;
         *reinterpret_cast<uint4*>(dst + 8 * g) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
                                                             pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
       }

@@ -263,8 +263,9 @@ bnorm_rows_w8_kernel(const int8_t* __restrict__ Wq, int64_t ldw, int64_t sW, con
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
           const float4 sv = s4[h];
-          const float v0 = float(int8_t(w[h] & 0xFF)) * sv.x, v1 = float(int8_t((w[h] >> 8) & 0xFF)) * sv.y;
-          const float v2 = float(int8_t((w[h] >> 16) & 0xFF)) * sv.z, v3 = float(int8_t(w[h] >> 24)) * sv.w;
+          float v0, v1, v2, v3;
+          s8x4_to_f32(w[h], v0, v1, v2, v3);
+          v0 *= sv.x, v1 *= sv.y, v2 *= sv.z, v3 *= sv.w;
           acc = fmaf(v0, v0, acc);
           acc = fmaf(v1, v1, acc);
           acc = fmaf(v2, v2, acc);
