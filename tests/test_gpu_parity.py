@@ -363,6 +363,25 @@ def test_gemv_gather_unaligned_rows():
     check_product(f64(C), f64(A), f64(B), idx.cpu().numpy(), 1e-2)
 
 
+@pytest.mark.parametrize("M", [1, 16])
+@pytest.mark.parametrize("N,ld", [(1003, 1008), (4096, 4096)], ids=["ragged", "full"])
+def test_gemv_gather_tensor_core_route(M, N, ld):
+    """16-byte aligned bf16 rows take the tensor-core gather-GEMV: a ragged N
+    inside an aligned row pitch (the last 16-byte copy of a row is partial),
+    very few kept slices (a pass of mostly empty slots), bit-reproducible."""
+    K = 3000
+    A, Bfull = _ab(M, K, ld, torch.bfloat16, seed=40 + M)
+    B = Bfull[:, :N]
+    A64, B64 = f64(A), f64(B)
+    s = rmm.score(A, B.contiguous())
+    for k in (1, 33, rmm.keep_count(0.4, K)):
+        idx = rmm.select(s, k)
+        for out_dtype in (torch.float32, torch.bfloat16):
+            C = rmm.gemv_gather(A, B, idx, out_dtype)
+            check_product(f64(C), A64, B64, idx.cpu().numpy(), product_tol(torch.bfloat16, out_dtype))
+        assert torch.equal(rmm.gemv_gather(A, B, idx), rmm.gemv_gather(A, B, idx))
+
+
 def test_fused_decode_shape_skips_the_pack():
     """The fused call with M <= 16 (and cached B norms, the decode setting)
     runs score, select and the gather-GEMV: 3 launches, oracle parity, one

@@ -120,3 +120,7 @@ def test_w8_gemv_tensor_core_route(M, N, ld):
         C = rmm.gemv_gather_w8(X, Wq, scale, idx, out_dtype)
         check_product(f64(C), f64(X), W64, idx.cpu().numpy(), product_tol(torch.bfloat16, out_dtype))
     assert torch.equal(rmm.gemv_gather_w8(X, Wq, scale, idx), rmm.gemv_gather_w8(X, Wq, scale, idx))
+    for k_small in (1, 33):  # a pass of mostly empty slots
+        idx_s = rmm.select(rmm.score_b_norms(X, bn), k_small)
+        C = rmm.gemv_gather_w8(X, Wq, scale, idx_s)
+        check_product(f64(C), f64(X), W64, idx_s.cpu().numpy(), product_tol(torch.bfloat16, torch.float32))
