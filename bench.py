@@ -676,6 +676,9 @@ def stage_gbs(p: Problem, rho, stage_mean):
     return {s: round(by[s] / (stage_mean[s] * 1e-3) / 1e9, 1) for s in stage_mean if by[s] > 0}
 
 
+NEAR_TIE_REL = 1e-5  # relative score window around the k-th largest inside which the parity tests accept swaps
+
+
 def quality_check(p: Problem, rho, seed):
     """Relative Frobenius error against the dense product (torch f32 matmul on
     the GPU, a measurement reference only) of the library's top-k selection and
@@ -705,11 +708,26 @@ def quality_check(p: Problem, rho, seed):
         C, _ = rmm.matmul_reduced(A, B, rho, p.mode, torch.float32, idx_out=idx, b_kmajor=p.b_kmajor)
         A_S, B_S = rmm.pack(A, B, ridx, p.b_kmajor)
         Cr = rmm.gemm(A_S, B_S, k, b_kmajor=p.b_kmajor, N=p.N)
+    # the selection's shape: slices whose score lies within the parity tests'
+    # near-tie window of the k-th largest (where a rounding-order difference may
+    # swap kept and dropped slices), and how contiguous the kept indices are
+    if p.mode == "a_only":
+        s = rmm.score(A, None, "a_only")
+    elif p.b_norm is not None or p.scale is not None:
+        s = rmm.score_b_norms(A, p.b_norm if p.b_norm is not None else rmm.b_norms_w8(B, p.scale))
+    else:
+        s = rmm.score(A, B, p.mode, b_kmajor=p.b_kmajor)
+    s = s.reshape(-1)[:p.K].double()
+    t = torch.topk(s, k).values[-1].item()
+    in_window = int((torch.abs(s - t) <= NEAR_TIE_REL * t).sum().item())
+    runs = 1 + int((torch.diff(idx.long()) != 1).sum().item()) if k > 1 else 1
     torch.cuda.synchronize()
     e_top = torch.linalg.norm(C - dense).item() / nd
     e_rand = torch.linalg.norm(Cr - dense).item() / nd
     return {"rel_fro_err_topk": round(e_top, 6), "rel_fro_err_random": round(e_rand, 6),
-            "score_mode": p.mode, "item": 0, "reference": "dense f32 product (torch matmul on the GPU)"}
+            "score_mode": p.mode, "item": 0, "reference": "dense f32 product (torch matmul on the GPU)",
+            "selection": {"kept": k, "threshold_score": t, "near_tie_window_rel": NEAR_TIE_REL,
+                          "slices_in_window": in_window, "kept_runs": runs, "kept_per_run": round(k / runs, 3)}}
 
 
 def roofline(p: Problem, rho, stage_mean, dominant, peaks, peak_src):
