@@ -442,3 +442,28 @@ def test_select_large_k_with_heavy_ties(K):
         idx = rmm.select(s, k)
         for b in range(3):
             assert idx[b].cpu().numpy().tolist() == O.select_top(s[b].cpu().numpy(), k).tolist()
+
+
+@pytest.mark.parametrize("K,batch", [(2048, 1), (2049, 2), (8190, 18), (32768, 1), (32769, 1), (8192, 19)],
+                         ids=lambda v: str(v))
+def test_select_matches_definition_across_shapes(K, batch):
+    """The selection is the definition's (largest scores, ties to the lower
+    index, ascending) on the library's own f32 scores: K around the
+    shared-memory limit and the compaction switch, one to 19 items, keep
+    counts from 1 to K, for continuous, signed, tied and constant scores."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(K + batch)
+    dists = {
+        "lognormal": torch.exp(torch.randn(batch, K, generator=g, device=DEV)),
+        "signed": torch.randn(batch, K, generator=g, device=DEV),
+        "coarse": torch.randint(0, 40, (batch, K), generator=g, device=DEV).float() * 0.25,
+        "constant": torch.full((batch, K), 3.0, device=DEV),
+    }
+    for name, s in dists.items():
+        s = s.contiguous()
+        for k in sorted({1, K // 2, K - 1, K}):
+            idx = rmm.select(s, k)
+            for b in sorted({0, batch - 1}):
+                want = O.select_top(s[b].double().cpu().numpy(), k).tolist()
+                assert idx[b].cpu().numpy().tolist() == want, (name, k, b)
+
