@@ -83,8 +83,9 @@ struct SplitZero {
 // select.cu
 //  Blocks [batch, batch + zero_blocks) of the launch zero `zero`'s tiles
 //  meanwhile (zero may be null); the select itself uses one block per item.
-//  late_launch: let the next kernel launch only when the selection exits (the
-//  fused calls' decode route, whose GEMV needs whole free SMs for its clusters).
+//  late_launch: release the next kernel only once the kernel before the
+//  selection has completed (the fused calls' decode route, whose GEMV needs
+//  whole free SMs for its clusters).
 cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,
                           uint32_t* status, cudaStream_t st, const SplitZero* zero = nullptr,
                           bool late_launch = false);

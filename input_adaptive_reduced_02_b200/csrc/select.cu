@@ -86,11 +86,13 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
   int32_t* ib = idx + int64_t(blockIdx.x) * k_keep;
 
   // late_launch: the next kernel (a gather-GEMV in clusters of CTAs with
-  // large shared memory) launches only when this grid exits; launched early,
-  // it would be placed around the previous kernel's CTAs and part of it would
-  // run as a second wave
+  // large shared memory) is released only once the previous kernel has
+  // completed (pdl_wait returns after that); released before, it would be
+  // placed around the previous kernel's CTAs and part of it would run as a
+  // second wave
   if (!late_launch) pdl_trigger();
   pdl_wait();
+  if (late_launch) pdl_trigger();
   if (blockIdx.x >= items) {  // helper block: zero C tiles for the GEMM later on the stream
     zero_split_tiles(zero, blockIdx.x - items, gridDim.x - items, tid, THREADS);
     return;
