@@ -106,6 +106,53 @@ def test_cached_b_norm_calls_validate_without_gpu():
     assert st == rmm.RMM_ERR_INVALID and b"rho" in L.rmm_last_error_string()
 
 
+def test_gemv_and_int8_calls_validate_without_gpu():
+    L = rmm.lib()
+    null = V(0)
+    BF16, F32 = 0, 1
+    # rmm_gemv_gather(A, lda, sA, B, ldb, sB, batch, M, K, N, idx, k_keep, in, C, ldc, sC, out, stream)
+    gv = [V(16), 8, 0, V(16), 8, 0, 1, 4, 8, 8, V(16), 3, BF16, V(16), 8, 0, F32, null]
+
+    def with_(args, pos, value):
+        a = list(args)
+        a[pos] = value
+        return a
+
+    assert L.rmm_gemv_gather(*with_(gv, 7, 17)) == rmm.RMM_ERR_INVALID  # M above 16
+    assert b"16" in L.rmm_last_error_string()
+    assert L.rmm_gemv_gather(*with_(gv, 11, 0)) == rmm.RMM_ERR_INVALID  # k_keep outside [1, K]
+    assert L.rmm_gemv_gather(*with_(gv, 11, 9)) == rmm.RMM_ERR_INVALID
+    assert L.rmm_gemv_gather(*with_(gv, 10, null)) == rmm.RMM_ERR_INVALID  # idx missing
+    assert L.rmm_gemv_gather(*with_(gv, 14, 4)) == rmm.RMM_ERR_INVALID  # ldc smaller than N
+    assert L.rmm_gemv_gather(*with_(gv, 16, 7)) == rmm.RMM_ERR_INVALID  # unknown output dtype
+    assert L.rmm_gemv_gather(*with_(gv, 6, 0)) == rmm.RMM_OK  # empty batch: nothing to do, no device needed
+    # rmm_b_norms_w8(Wq, ldw, sW, scale, ss, batch, K, N, out, status, stream)
+    assert L.rmm_b_norms_w8(null, 8, 0, V(16), 0, 1, 8, 8, V(16), null, null) == rmm.RMM_ERR_INVALID
+    assert L.rmm_b_norms_w8(V(16), 8, 0, null, 0, 1, 8, 8, V(16), null, null) == rmm.RMM_ERR_INVALID
+    assert L.rmm_b_norms_w8(V(16), 4, 0, V(16), 0, 1, 8, 8, V(16), null, null) == rmm.RMM_ERR_INVALID
+    # a per-item scale stride that would overlap the items' scales
+    assert L.rmm_b_norms_w8(V(16), 8, 64, V(16), 3, 2, 8, 8, V(16), null, null) == rmm.RMM_ERR_INVALID
+    # rmm_gemv_gather_w8(A, lda, sA, Wq, ldw, sW, scale, ss, batch, M, K, N, idx, k, C, ldc, sC, out, stream)
+    w8 = [V(16), 8, 0, V(16), 8, 0, V(16), 0, 1, 4, 8, 8, V(16), 3, V(16), 8, 0, F32, null]
+    assert L.rmm_gemv_gather_w8(*with_(w8, 9, 17)) == rmm.RMM_ERR_INVALID  # M above 16
+    # int8 rows not 4-byte aligned (base, then row pitch)
+    assert L.rmm_gemv_gather_w8(*with_(w8, 3, V(17))) == rmm.RMM_ERR_UNSUPPORTED
+    assert L.rmm_gemv_gather_w8(*with_(w8, 4, 10)) == rmm.RMM_ERR_UNSUPPORTED
+    # rmm_matmul_reduced_w8(A, lda, sA, Wq, ldw, sW, scale, ss, b_norm, bns, batch, M, K, N, rho, in, mode,
+    #                       C, ldc, sC, out, idx_out, workspace, ws_bytes, stream)
+    f = [V(16), 8, 0, V(16), 8, 0, V(16), 0, V(16), 0, 1, 4, 8, 8, 0.5, BF16, 0, V(16), 8, 0, F32, null,
+         V(1024), 1 << 20, null]
+    assert L.rmm_matmul_reduced_w8(*with_(f, 15, F32)) == rmm.RMM_ERR_INVALID  # activations must be bf16
+    assert L.rmm_matmul_reduced_w8(*with_(f, 8, null)) == rmm.RMM_ERR_INVALID  # product score needs W's norms
+    assert L.rmm_matmul_reduced_w8(*with_(f, 16, 5)) == rmm.RMM_ERR_INVALID  # unknown score mode
+    assert L.rmm_matmul_reduced_w8(*with_(f, 14, 0.0)) == rmm.RMM_ERR_INVALID  # rho outside (0, 1]
+    assert L.rmm_matmul_reduced_w8(*with_(f, 23, 16)) == rmm.RMM_ERR_INVALID  # workspace too small
+    # rmm_pack_w8(A, lda, sA, Wq, ldw, sW, scale, ss, batch, M, K, N, idx, k, A_S, B_S, status, stream)
+    pk = [V(16), 8, 0, V(16), 8, 0, V(16), 0, 1, 4, 8, 8, V(16), 3, V(16), V(16), null, null]
+    assert L.rmm_pack_w8(*with_(pk, 12, null)) == rmm.RMM_ERR_INVALID  # idx missing
+    assert L.rmm_pack_w8(*with_(pk, 13, 9)) == rmm.RMM_ERR_INVALID  # k_keep above K
+
+
 def test_binding_refuses_cpu_tensors():
     A = rmm.torch.zeros(4, 8, dtype=rmm.torch.bfloat16)
     with pytest.raises(ValueError):
