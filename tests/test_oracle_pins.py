@@ -293,6 +293,38 @@ def test_batched_sites_select_per_item():
     assert C.shape == (2, 6, 4) and idx.shape == (2, 3)
 
 
+def test_pv_site_closed_form_with_permutation_attention():
+    """P·V reduces over keys: with each query q attending to key π(q) alone
+    (a permutation that is not its own inverse, so P ≠ Pᵀ) every key column
+    of P has norm 1, key k scores ‖V[k,:]‖, the kept keys are the rows of V
+    with the largest norms, and row q of the output is V[π(q)] when key π(q)
+    is kept and zero otherwise. Two heads with different V select
+    differently."""
+    S, d = 6, 3
+    perm = (np.arange(S) + 2) % S
+    P1 = np.zeros((S, S))
+    P1[np.arange(S), perm] = 1.0
+    P = np.stack([P1, P1])
+    V = np.zeros((2, S, d))
+    V[0, :, 0] = [1.0, 5.0, 2.0, 6.0, 3.0, 4.0]
+    V[1, :, 0] = [6.0, 1.0, 5.0, 2.0, 4.0, 3.0]
+    V[:, :, 2] = np.arange(S)
+    # row norms: head 0: 1, √26, √8, √45, 5, √41 -> keys {1, 3, 5};
+    #            head 1: 6, √2, √29, √13, √32, √34 -> keys {0, 4, 5}
+    norms = [np.sqrt([1.0, 26.0, 8.0, 45.0, 25.0, 41.0]), np.sqrt([36.0, 2.0, 29.0, 13.0, 32.0, 34.0])]
+    keep = [[1, 3, 5], [0, 4, 5]]
+    C, idx, s = O.pv_reduced(P, V, 0.5)
+    for h in range(2):
+        np.testing.assert_allclose(s[h], norms[h], rtol=1e-15)
+        assert idx[h].tolist() == keep[h]
+        expect = np.zeros((S, d))
+        for q in range(S):
+            if perm[q] in idx[h]:
+                expect[q] = V[h][perm[q]]
+        np.testing.assert_array_equal(C[h], expect)
+    assert idx[0].tolist() != idx[1].tolist()
+
+
 def test_selection_matches_window_rule():
     s = np.array([1.0, 2.0, 2.0 + 1e-7, 3.0])
     o = O.select_top(s, 2)  # {2, 3}
