@@ -332,6 +332,14 @@ def test_selection_matches_window_rule():
     assert ok and n == 2
     ok, _ = O.selection_matches(np.array([0, 3]), o, s)
     assert not ok
+    # the window is relative to the threshold score t: a gap of 1 at t = 1e6
+    # (1e-6 relative) is a near-tie, a gap of 1e-6 at t = 1e-3 (1e-3 relative) is not
+    big = np.array([5.0e5, 1.0e6, 1.0e6 + 1.0, 3.0e6])
+    ok, n = O.selection_matches(np.array([1, 3]), O.select_top(big, 2), big)
+    assert ok and n == 2
+    small = np.array([5.0e-4, 1.0e-3, 1.0e-3 + 1.0e-6, 3.0e-3])
+    ok, _ = O.selection_matches(np.array([1, 3]), O.select_top(small, 2), small)
+    assert not ok
 
 
 def test_frobenius_rel_error():
