@@ -1,6 +1,7 @@
 """Host-side checks of bench.py that need no GPU: the whole-job aggregation over
-ranks (two gloo ranks on the CPU, as under torchrun) and the reference arm,
-which times the fp64 oracle on the host."""
+ranks (two gloo ranks on the CPU, as under torchrun), the reference arm, which
+times the fp64 oracle on the host, and the roofline arithmetic (algorithmic
+bytes per stage, bound chosen by arithmetic intensity) on shape-only tensors."""
 from __future__ import annotations
 
 import json
@@ -77,3 +78,64 @@ def test_reference_arm_follows_the_score_mode():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["config"]["score_mode"] == "a_only" and line["value"] > 0
 
+
+
+# ---------------------------------------------------------------- roofline arithmetic
+PEAKS = {"hbm_gbs": 6548.2, "bf16_tflops": 1652.0}
+
+
+def _bench():
+    sys.path.insert(0, ROOT)
+    import bench
+    return bench
+
+
+def _meta(bench, name, a_shape, b_shape, dtype, b_kmajor=False, out=None):
+    import torch
+    A = torch.empty(a_shape, dtype=dtype, device="meta")
+    B = torch.empty(b_shape, dtype=dtype, device="meta")
+    return bench.Problem(name, A, B, b_kmajor, out or torch.float32, 0.5, "")
+
+
+def test_stage_bytes_of_the_linear_workload():
+    """Algorithmic bytes per stage at 4096³, rho 0.5 (k = 2048, bf16 in, f32 out)."""
+    import torch
+    bench = _bench()
+    p = _meta(bench, "linear_4096", (4096, 4096), (4096, 4096), torch.bfloat16)
+    by = bench.stage_bytes(p, 0.5)
+    n = 4096
+    assert by["score"] == 2 * n * n * 2 + 4 * n             # A and W read once, scores written
+    assert by["select"] == 4 * n + 4 * 2048                 # scores read, indices written
+    assert by["pack"] == n * n * 2 + 3 * n * 2048 * 2 == 83886080  # A whole, W's kept rows, A_S and B_S
+    assert by["gemm"] == 2 * n * 2048 * 2 + n * n * 4       # A_S, B_S, f32 C
+
+
+def test_roofline_bound_follows_arithmetic_intensity():
+    import torch
+    bench = _bench()
+    # tensor-bound GEMM: 2·4096·4096·2048 flops in 62.7 us
+    p = _meta(bench, "linear_4096", (4096, 4096), (4096, 4096), torch.bfloat16)
+    r = bench.roofline(p, 0.5, {"gemm": 0.0627}, "gemm", PEAKS, "measured")
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["achieved"] - 2 * 4096 * 4096 * 2048 / 62.7e-6 / 1e12) < 0.01
+    assert abs(r["frac"] - r["achieved"] / 1652.0) < 1e-4
+    # decode GEMV (M = 1, W's norms cached): HBM-bound on the kept rows of W
+    p = _meta(bench, "decode_mlp_up_m1", (1, 8192), (8192, 28672), torch.bfloat16)
+    p.b_norm = object()
+    r = bench.roofline(p, 0.5, {"gemm": 0.056}, "gemm", PEAKS, "measured")
+    assert r["bound"] == "hbm" and r["kernel"] == "gemv_gather_kernel"
+    assert r["algorithmic_bytes_per_launch"] == 4096 * 28672 * 2 + 4096 * 2 + 4 * 4096 + 28672 * 4 == 235020288
+    assert abs(r["achieved"] - 235020288 / 56e-6 / 1e9) < 0.1
+    # P·V (32 heads, S 16384, d 128): below the ridge, HBM-bound
+    p = _meta(bench, "pv_16384", (32, 16384, 16384), (32, 16384, 128), torch.bfloat16)
+    r = bench.roofline(p, 0.5, {"gemm": 3.0}, "gemm", PEAKS, "measured")
+    assert r["bound"] == "hbm" and r["arithmetic_intensity"] < r["ridge"]
+    # Q·Kᵀ (B = Kᵀ given K-major, bf16 out): the output write keeps it below the ridge
+    p = _meta(bench, "qk_32x4096x128", (32, 4096, 128), (32, 4096, 128), torch.bfloat16, b_kmajor=True,
+              out=torch.bfloat16)
+    r = bench.roofline(p, 0.5, {"gemm": 0.3}, "gemm", PEAKS, "measured")
+    assert r["bound"] == "hbm" and r["arithmetic_intensity"] < r["ridge"]
+    # a memory-bound stage as the dominant one reports its own bytes
+    p = _meta(bench, "linear_4096", (4096, 4096), (4096, 4096), torch.bfloat16)
+    r = bench.roofline(p, 0.5, {"pack": 0.02}, "pack", PEAKS, "measured")
+    assert r["bound"] == "hbm" and r["algorithmic_bytes_per_launch"] == 83886080
