@@ -247,7 +247,8 @@ class Fused:
         self.p = p
         dev = p.A.device
         self.C = torch.empty((p.batch, p.M, p.N) if p.A.dim() == 3 else (p.M, p.N), dtype=p.out_dtype, device=dev)
-        self.ws = rmm.Workspace(rmm.workspace_size(p.batch, p.M, p.K, p.N, p.k_keep(rho_max), p.A.dtype), dev)
+        self.ws = rmm.Workspace(rmm.workspace_size_for(p.batch, p.M, p.K, p.N, p.k_keep(rho_max), p.A.dtype,
+                                                       p.b_kmajor), dev)
         self.b_norm = b_norm if b_norm is not None else p.b_norm
 
     def step(self, rho, ev=None, breakdown=False):

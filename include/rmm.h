@@ -86,6 +86,17 @@ int64_t rmm_packed_b_ld(int64_t N);
 size_t rmm_workspace_size(int64_t batch, int64_t M, int64_t K, int64_t N, int64_t k_keep,
                           rmm_dtype in);
 
+/* The workspace a fused call needs for the route it takes with these sizes
+ * and B's layout (b_kmajor as in rmm_score; 0 for the INT8-weight call): with
+ * M <= 16 and B row-major the call streams B's kept rows through the
+ * gather-GEMV and packs nothing, so the status word, scores and indices are
+ * all it uses (for x[1][8192] · W[8192][28672] at rho = 0.5: 49 KiB instead
+ * of 224 MiB); otherwise it equals rmm_workspace_size. The fused calls accept
+ * any workspace of at least this size; the layout of what they use does not
+ * change. */
+size_t rmm_workspace_size_for(int64_t batch, int64_t M, int64_t K, int64_t N, int64_t k_keep,
+                              rmm_dtype in, int b_kmajor);
+
 /* ---------------------------------------------------------------- stage calls */
 
 /* Slice scores ("Estratégia de Seleção"; product form is the library default).
@@ -158,8 +169,9 @@ rmm_status rmm_gemm(const void* A_S, const void* B_S, int b_kmajor, int64_t batc
  * pack → gemm, all enqueued on `stream`.
  *   A [M][K] (ld lda), B [K][N] (ld ldb), C [M][N] (ld ldc); dtypes in/out.
  *   idx_out: nullable device [k_keep] i32 that receives the kept indices.
- *   workspace: device buffer of at least rmm_workspace_size(1, M, K, N, k, in)
- *   bytes, 1 KiB-aligned; its first 4 bytes are the status word, cleared at
+ *   workspace: device buffer of at least rmm_workspace_size_for(1, M, K, N, k,
+ *   in, 0) bytes (rmm_workspace_size always suffices), 1 KiB-aligned; its
+ *   first 4 bytes are the status word, cleared at
  *   the start of the call. Call rmm_check(workspace, stream) to learn of
  *   device-side errors. Workspace contents are scratch between calls. */
 rmm_status rmm_matmul_reduced(const void* A, int64_t lda, const void* B, int64_t ldb,

@@ -91,8 +91,13 @@ struct Workspace {
   int32_t* idx;
   void* a_s;
   void* b_st;
-  size_t bytes;
+  size_t bytes;          // every route
+  size_t bytes_no_pack;  // the decode route (no packed operands): status, scores, indices
 };
+
+// The fused calls stream B's kept rows straight into the gather-GEMV, with no
+// packed operands, for a few rows of A and a row-major B.
+static bool decode_route(int64_t M, int b_kmajor) { return M <= kGemvMaxRows && !b_kmajor; }
 
 static Workspace carve(void* base, int64_t batch, int64_t M, int64_t K, int64_t N, int64_t k_keep, rmm_dtype in) {
   const int64_t kp = round_up(k_keep, 64);
@@ -107,6 +112,7 @@ static Workspace carve(void* base, int64_t batch, int64_t M, int64_t K, int64_t 
   off += al(batch * K * 4);
   w.idx = reinterpret_cast<int32_t*>(p + off);
   off += al(batch * k_keep * 4);
+  w.bytes_no_pack = size_t(off);
   w.a_s = reinterpret_cast<void*>(p + off);
   off += al(batch * M * kp * eb);
   w.b_st = reinterpret_cast<void*>(p + off);
@@ -256,6 +262,13 @@ size_t rmm_workspace_size(int64_t batch, int64_t M, int64_t K, int64_t N, int64_
   return carve(nullptr, batch, M, K, N, k_keep, in).bytes;
 }
 
+size_t rmm_workspace_size_for(int64_t batch, int64_t M, int64_t K, int64_t N, int64_t k_keep, rmm_dtype in,
+                              int b_kmajor) {
+  if (batch < 0 || M < 0 || K < 0 || N < 0 || k_keep < 0 || !dtype_ok(in)) return 0;
+  const Workspace w = carve(nullptr, batch, M, K, N, k_keep, in);
+  return decode_route(M, b_kmajor) ? w.bytes_no_pack : w.bytes;
+}
+
 rmm_status rmm_score(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb, int64_t strideB,
                      int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N, rmm_dtype in, rmm_score_mode mode,
                      float* s, uint32_t* status_word, cudaStream_t stream) {
@@ -338,8 +351,9 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
   if (!workspace) return fail(RMM_ERR_INVALID, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(workspace) & 1023u) return fail(RMM_ERR_INVALID, "workspace must be 1 KiB aligned");
   const Workspace w = carve(workspace, batch, M, K, N, k_keep, in);
-  if (workspace_bytes < w.bytes)
-    return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, w.bytes);
+  const size_t need = decode_route(M, b_kmajor) ? w.bytes_no_pack : w.bytes;
+  if (workspace_bytes < need)
+    return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
   if ((r = bind_device(stream))) return r;
   cudaError_t ce = cudaSuccess;
   if (batch == 0) {  // no kernel runs: clear the status word here
@@ -357,7 +371,7 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
   GemmArgs g = gemm_args(w.a_s, w.b_st, b_kmajor, batch, M, N, k_keep, C, ldc, strideC, out, w.status);
   // A few rows of A (decode): the product streams B's kept rows straight
   // through idx, with no packed copy.
-  const bool gemv = M <= kGemvMaxRows && !b_kmajor;
+  const bool gemv = decode_route(M, b_kmajor);
   SplitZero z;
   const bool zero = !gemv && in == RMM_BF16 && gemm_tc_split_zero(g, &z);
   ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr, gemv);
@@ -600,8 +614,9 @@ rmm_status rmm_matmul_reduced_w8(const void* A, int64_t lda, int64_t strideA, co
   if (!workspace) return fail(RMM_ERR_INVALID, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(workspace) & 1023u) return fail(RMM_ERR_INVALID, "workspace must be 1 KiB aligned");
   const Workspace w = carve(workspace, batch, M, K, N, k_keep, in);
-  if (workspace_bytes < w.bytes)
-    return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, w.bytes);
+  const size_t need = decode_route(M, 0) ? w.bytes_no_pack : w.bytes;
+  if (workspace_bytes < need)
+    return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
   if ((r = bind_device(stream))) return r;
   cudaError_t ce = cudaSuccess;
   if (batch == 0) {
@@ -613,7 +628,7 @@ rmm_status rmm_matmul_reduced_w8(const void* A, int64_t lda, int64_t strideA, co
                     mode == RMM_SCORE_PRODUCT ? b_norm : nullptr, b_norm_stride, 1)))
     return r;
   GemmArgs g = gemm_args(w.a_s, w.b_st, 0, batch, M, N, k_keep, C, ldc, strideC, out, w.status);
-  const bool gemv = M <= kGemvMaxRows;
+  const bool gemv = decode_route(M, 0);
   SplitZero z;
   const bool zero = !gemv && gemm_tc_split_zero(g, &z);
   ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr, gemv);

@@ -39,7 +39,7 @@ extern "C" rmm_status rmm_matmul_reduced_noalloc(const void* A, int64_t lda, con
   char msg[256];
   const int64_t k = rmm_keep_count(rho, K);
   if (k >= 1) {
-    const size_t need = rmm_workspace_size(1, M, K, N, k, in);
+    const size_t need = rmm_workspace_size_for(1, M, K, N, k, in, 0);
     if (need > kScratchBytes) {
       snprintf(msg, sizeof(msg),
                "rmm_matmul_reduced_noalloc: this product needs %zu bytes of scratch, the static scratch holds "

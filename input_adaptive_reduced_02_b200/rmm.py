@@ -40,6 +40,7 @@ _SIGS = {
     "rmm_padded_keep": (_i64, [_i64]),
     "rmm_packed_b_ld": (_i64, [_i64]),
     "rmm_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64, _i64, _i32]),
+    "rmm_workspace_size_for": (ctypes.c_size_t, [_i64, _i64, _i64, _i64, _i64, _i32, _i32]),
     "rmm_score": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i32, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp,
                          _vp]),
     "rmm_select": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
@@ -160,7 +161,14 @@ def padded_keep(k_keep: int) -> int:
 
 
 def workspace_size(batch: int, M: int, K: int, N: int, k_keep: int, dtype: torch.dtype) -> int:
+    """Workspace bytes of a fused call on any route."""
     return int(lib().rmm_workspace_size(batch, M, K, N, k_keep, _out_code(dtype)))
+
+
+def workspace_size_for(batch: int, M: int, K: int, N: int, k_keep: int, dtype: torch.dtype,
+                       b_kmajor: bool = False) -> int:
+    """Workspace bytes of a fused call on the route it takes (no packed operands when M <= 16 and B is row-major)."""
+    return int(lib().rmm_workspace_size_for(batch, M, K, N, k_keep, _out_code(dtype), int(b_kmajor)))
 
 
 class Workspace:
@@ -347,7 +355,7 @@ def matmul_reduced(A: torch.Tensor, B: torch.Tensor, rho: float, mode: str = "pr
     bb, r, c, ldb, sB = _mat(B, "B")
     N = r if b_kmajor else c
     k = keep_count(rho, K)
-    ws = _ensure_ws(workspace, workspace_size(ba, M, K, N, k, A.dtype), A.device)
+    ws = _ensure_ws(workspace, workspace_size_for(ba, M, K, N, k, A.dtype, b_kmajor), A.device)
     if out is None:
         out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
     _, _, _, ldc, sC = _mat(out, "C")
@@ -368,7 +376,7 @@ def matmul_reduced_b_norms(A: torch.Tensor, B: torch.Tensor, b_norm: torch.Tenso
     N = r if b_kmajor else c
     stride = _bn_stride(b_norm, ba, K)
     k = keep_count(rho, K)
-    ws = _ensure_ws(workspace, workspace_size(ba, M, K, N, k, A.dtype), A.device)
+    ws = _ensure_ws(workspace, workspace_size_for(ba, M, K, N, k, A.dtype, b_kmajor), A.device)
     if out is None:
         out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
     _, _, _, ldc, sC = _mat(out, "C")
@@ -455,7 +463,7 @@ def matmul_reduced_w8(A: torch.Tensor, Wq: torch.Tensor, scale: torch.Tensor, rh
     elif SCORE_MODES[mode] == 0:
         raise ValueError("product mode needs b_norm (b_norms_w8)")
     k = keep_count(rho, K)
-    ws = _ensure_ws(workspace, workspace_size(ba, M, K, N, k, A.dtype), A.device)
+    ws = _ensure_ws(workspace, workspace_size_for(ba, M, K, N, k, A.dtype), A.device)
     if out is None:
         out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
     _, _, _, ldc, sC = _mat(out, "C")
@@ -473,7 +481,7 @@ def qk_reduced(Q: torch.Tensor, Kmat: torch.Tensor, rho: float, mode: str = "pro
     bh, S_q, d = Q.shape
     S_k = Kmat.shape[1]
     k = keep_count(rho, d)
-    ws = _ensure_ws(workspace, workspace_size(bh, S_q, d, S_k, k, Q.dtype), Q.device)
+    ws = _ensure_ws(workspace, workspace_size_for(bh, S_q, d, S_k, k, Q.dtype, True), Q.device)
     if out is None:
         out = torch.empty(bh, S_q, S_k, dtype=out_dtype, device=Q.device)
     _check(lib().rmm_qk_reduced(_ptr(Q), _ptr(Kmat), bh, S_q, S_k, d, float(rho), _dtype(Q), SCORE_MODES[mode],
@@ -489,7 +497,7 @@ def pv_reduced(P: torch.Tensor, V: torch.Tensor, rho: float, mode: str = "produc
     bh, S_q, S_k = P.shape
     d = V.shape[2]
     k = keep_count(rho, S_k)
-    ws = _ensure_ws(workspace, workspace_size(bh, S_q, S_k, d, k, P.dtype), P.device)
+    ws = _ensure_ws(workspace, workspace_size_for(bh, S_q, S_k, d, k, P.dtype), P.device)
     if out is None:
         out = torch.empty(bh, S_q, d, dtype=out_dtype, device=P.device)
     _check(lib().rmm_pv_reduced(_ptr(P), _ptr(V), bh, S_q, S_k, d, float(rho), _dtype(P), SCORE_MODES[mode],

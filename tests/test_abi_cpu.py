@@ -55,7 +55,50 @@ def test_padded_keep_and_workspace_layout():
     assert ws32 == 1024 + 1024 + 1024 + 2048 + 4096
 
 
+def test_workspace_size_for_the_decode_route():
+    """With M <= 16 and B row-major the fused calls pack nothing: the workspace
+    they need is the status word, scores and indices; other routes need the
+    packed operands too."""
+    al = lambda x: (x + 1023) // 1024 * 1024  # noqa: E731
+    K, N, k = 8192, 28672, 4096
+    decode = rmm.workspace_size_for(1, 1, K, N, k, rmm.torch.bfloat16)
+    assert decode == al(4) + al(K * 4) + al(k * 4) == 50176
+    full = rmm.workspace_size(1, 1, K, N, k, rmm.torch.bfloat16)
+    assert full > 200 * 2**20 and decode < full
+    assert rmm.workspace_size_for(1, 1, K, N, k, rmm.torch.bfloat16, b_kmajor=True) == full
+    assert rmm.workspace_size_for(1, 17, K, N, k, rmm.torch.bfloat16) == rmm.workspace_size(1, 17, K, N, k,
+                                                                                               rmm.torch.bfloat16)
+    assert rmm.workspace_size_for(3, 16, K, N, k, rmm.torch.float32) == al(4) + al(3 * K * 4) + al(3 * k * 4)
+
+
 V = ctypes.c_void_p
+
+
+def test_fused_calls_accept_the_route_workspace():
+    """The fused call's workspace check follows its route: a decode-shaped call
+    (M = 4, B row-major) passes it with exactly rmm_workspace_size_for bytes and
+    fails it with one byte less; a K-major B needs the full size."""
+    L = rmm.lib()
+    null = V(0)
+    M, K, N = 4, 64, 40
+    k = rmm.keep_count(0.5, K)
+    need = rmm.workspace_size_for(1, M, K, N, k, rmm.torch.bfloat16)
+    # rmm_matmul_reduced_batched(A, lda, sA, B, ldb, sB, b_kmajor, batch, M, K, N, rho, in, mode, C, ldc, sC, out,
+    #                            idx_out, workspace, bytes, stream)
+    def call(b_kmajor, ldb, nbytes):
+        return L.rmm_matmul_reduced_batched(V(1 << 20), K, 0, V(1 << 20), ldb, 0, b_kmajor, 1, M, K, N, 0.5, 0, 0,
+                                            V(1 << 20), N, 0, 1, null, V(1 << 30), nbytes, null)
+    assert call(0, N, need - 1) == rmm.RMM_ERR_INVALID
+    assert b"workspace too small" in L.rmm_last_error_string()
+    assert call(1, K, need) == rmm.RMM_ERR_INVALID  # K-major B: the pack route needs the packed operands
+    assert b"workspace too small" in L.rmm_last_error_string()
+    if not rmm.torch.cuda.is_available():
+        # Past the workspace check the call goes on to bind a device, which
+        # fails without a GPU. (With a GPU these pointers would reach kernels,
+        # so the accepting half runs only where there is none.)
+        full = rmm.workspace_size(1, M, K, N, k, rmm.torch.bfloat16)
+        assert call(0, N, need) == rmm.RMM_ERR_CUDA
+        assert call(1, K, full) == rmm.RMM_ERR_CUDA
 
 
 def test_validation_errors_need_no_gpu():

@@ -64,3 +64,27 @@ def test_noalloc_rejects_products_beyond_its_scratch():
     st = _call_noalloc(A, B, 0.5, C, idx, rmm.status_word())
     assert st == rmm.RMM_ERR_INVALID
     assert b"static scratch" in rmm.lib().rmm_last_error_string()
+
+
+def test_noalloc_takes_decode_products_beyond_its_scratch():
+    """A decode-shaped product (one row of A, B row-major) packs nothing, so its
+    scratch is scores and indices only: a weight whose packed rows alone would
+    take 64 MiB runs through the static 32 MiB scratch, bit-identical to the
+    workspace entry point (same route, same kernels)."""
+    M, K, N, rho = 1, 4096, 16384, 0.5
+    k = rmm.keep_count(rho, K)
+    assert rmm.workspace_size(1, M, K, N, k, torch.bfloat16) > 32 * 2**20
+    A, B = _inputs(M, K, N, 4)
+    idx_ref = torch.empty(k, dtype=torch.int32, device="cuda")
+    C_ref, ws = rmm.matmul_reduced(A, B, rho, idx_out=idx_ref)
+    assert ws.nbytes == rmm.workspace_size_for(1, M, K, N, k, torch.bfloat16)
+    rmm.check(ws)
+    C = torch.full((M, N), float("nan"), device="cuda")
+    idx = torch.full((k,), -1, dtype=torch.int32, device="cuda")
+    status = rmm.status_word()
+    assert _call_noalloc(A, B, rho, C, idx, status) == rmm.RMM_OK, rmm.lib().rmm_last_error_string()
+    rmm.check(status)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_ref)
+    assert torch.equal(C, C_ref)
+
