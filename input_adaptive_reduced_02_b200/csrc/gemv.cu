@@ -6,17 +6,23 @@
 //
 // With a handful of rows the product is a matrix-vector product that streams
 // the kept rows of B once; skipping a row of B saves its bytes outright, so
-// the kernel is built around HBM reads of B:
-//  * a CTA owns 128 columns of C (4 per lane: 8-byte loads of bf16, 16-byte
-//    of f32) and a share of the kept slices; its 8 warps take the slices in
-//    turn, up to 16 rows of B in flight per lane;
-//  * the A values it needs, A[m][idx[t]], and the row numbers idx[t] are
-//    staged in shared memory 256 slices at a time;
-//  * the CTAs of a thread-block cluster (up to 8) split the kept slices; each
-//    sums its warps' partial products in warp order, then rank 0 adds the
-//    CTAs' partials in rank order through distributed shared memory and
-//    writes C. Fixed order throughout: bit-reproducible, no atomics.
-// Products and sums in f32 (FFMA); C in f32 or bf16 (round to nearest even).
+// every kernel here is built around HBM reads of B, and in all of them the
+// CTAs of a thread-block cluster (up to 8) split the kept slices and rank 0
+// adds the CTAs' partials in rank order through distributed shared memory
+// (fixed order throughout: bit-reproducible, no atomics). By B:
+//  * bf16, rows 16-byte aligned: gemv_gather_mma_kernel (tensor-core path,
+//    below) — cp.async ring of 32-slice passes, mma.sync m16n8k16;
+//  * INT8 with per-column scales, rows 16-byte aligned:
+//    gemv_gather_mma_w8_kernel — the same, after an exact int8 -> bf16
+//    conversion of each pass;
+//  * f32, or rows aligned to the 4-column copy: gemv_gather_async_kernel
+//    (FFMA, cp.async into per-lane slots);
+//  * anything else: gemv_gather_kernel (FFMA, plain loads), sketched next —
+//    a CTA owns 128 columns of C (4 per lane) and a share of the kept slices;
+//    its 8 warps take the slices in turn, up to 16 rows of B in flight per
+//    lane; A[m][idx[t]] and idx[t] are staged in shared memory 256 slices at
+//    a time; each CTA sums its warps' partials in warp order.
+// Sums in f32; C in f32 or bf16 (round to nearest even).
 #include <cooperative_groups.h>
 
 #include <algorithm>
