@@ -15,9 +15,11 @@
 //  * INT8 with per-column scales, rows 16-byte aligned:
 //    gemv_gather_mma_w8_kernel — the same, after an exact int8 -> bf16
 //    conversion of each pass;
-//  * f32, or rows aligned to the 4-column copy: gemv_gather_async_kernel
-//    (FFMA, cp.async into per-lane slots);
-//  * anything else: gemv_gather_kernel (FFMA, plain loads), sketched next —
+//  * f32 with rows 16-byte aligned, or INT8 with rows only 4-byte aligned:
+//    gemv_gather_async_kernel (FFMA, cp.async of 4 columns into per-lane
+//    slots);
+//  * bf16 or f32 rows that are not 16-byte aligned: gemv_gather_kernel (FFMA,
+//    plain loads), sketched next —
 //    a CTA owns 128 columns of C (4 per lane) and a share of the kept slices;
 //    its 8 warps take the slices in turn, up to 16 rows of B in flight per
 //    lane; A[m][idx[t]] and idx[t] are staged in shared memory 256 slices at
