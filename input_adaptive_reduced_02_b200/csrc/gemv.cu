@@ -30,6 +30,7 @@
 #include <algorithm>
 #include <cmath>
 
+#include "int8_convert.cuh"
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
 

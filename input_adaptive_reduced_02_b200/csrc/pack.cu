@@ -16,6 +16,7 @@
 // Pure bit copies. Rows that are not 16-byte aligned take plain-load paths.
 #include <algorithm>
 
+#include "int8_convert.cuh"
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
 

@@ -28,36 +28,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// Four signed bytes -> f32, exactly, on the integer and FP32 pipes (the
-// int-to-float conversion unit issues at a fraction of their rate). With its
-// sign bit flipped, the byte of a value v in [-128, 127] reads v + 128 in
-// [0, 255]; placed in the low mantissa bits of 2^23 it makes the float
-// 2^23 + v + 128, and subtracting 2^23 + 128 leaves v. Every quantity is an
-// integer below 2^24, so the subtraction is exact.
-__device__ __forceinline__ void s8x4_to_f32(uint32_t w, float& f0, float& f1, float& f2, float& f3) {
-  const uint32_t u = w ^ 0x80808080u;
-  constexpr uint32_t kTwo23 = 0x4B000000u;  // 2^23
-  constexpr float kBias = 8388736.0f;       // 2^23 + 128
-  f0 = __uint_as_float(__byte_perm(u, kTwo23, 0x7650)) - kBias;
-  f1 = __uint_as_float(__byte_perm(u, kTwo23, 0x7651)) - kBias;
-  f2 = __uint_as_float(__byte_perm(u, kTwo23, 0x7652)) - kBias;
-  f3 = __uint_as_float(__byte_perm(u, kTwo23, 0x7653)) - kBias;
-}
-
-// f32 pair whose values are exact in bf16 (at most 8 significant bits, e.g.
-// integers of magnitude <= 256) -> bf16x2: the upper halves, no rounding needed.
-__device__ __forceinline__ uint32_t pack_bf16x2_exact(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x7632);
-}
-
-// Four signed bytes -> two bf16x2 words (bytes 0,1 in lo; 2,3 in hi), exactly.
-__device__ __forceinline__ void s8x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  float f0, f1, f2, f3;
-  s8x4_to_f32(w, f0, f1, f2, f3);
-  lo = pack_bf16x2_exact(f0, f1);
-  hi = pack_bf16x2_exact(f2, f3);
-}
-
 __device__ __forceinline__ void status_or(uint32_t* status, uint32_t bits) {
   if (status != nullptr) atomicOr(status, bits);
 }

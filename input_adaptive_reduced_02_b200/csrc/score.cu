@@ -18,6 +18,7 @@
 #include <algorithm>
 #include <cooperative_groups.h>
 
+#include "int8_convert.cuh"
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
 
