@@ -323,8 +323,9 @@ rmm_status rmm_pv_reduced(const void* P, const void* V, int64_t bh, int64_t S_q,
  * defines. Every device on which the call has run keeps that array until the
  * process exits (with eager module loading, every device that loads the
  * library does).
- *   - Products whose rmm_workspace_size(1, M, K, N, k, in) exceeds 32 MiB
- *     (33554432 bytes) are rejected with RMM_ERR_INVALID before any launch.
+ *   - Products whose rmm_workspace_size_for(1, M, K, N, k, in, 0) exceeds
+ *     32 MiB (33554432 bytes) are rejected with RMM_ERR_INVALID before any
+ *     launch (decode shapes, M <= 16, need only their scores and indices).
  *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
