@@ -28,6 +28,7 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 
 #include "int8_convert.cuh"
@@ -539,7 +540,7 @@ gemv_gather_mma_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t sA, 
 template <typename T, int MT>
 cudaError_t launch_mt(const GemvArgs& g, cudaStream_t st) {
   const size_t smem = gv_smem_bytes<MT>();
-  static bool attr_done[64] = {};
+  static std::atomic<bool> attr_done[64];  // per device; racing first calls both set the attribute
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
@@ -575,7 +576,7 @@ cudaError_t launch_mt(const GemvArgs& g, cudaStream_t st) {
         mcs = q;
       }
     }
-    static bool mma_attr[64] = {};
+    static std::atomic<bool> mma_attr[64];  // per device; racing first calls both set the attribute
     if (dev >= 0 && dev < 64 && !mma_attr[dev]) {
       cudaError_t e = cudaFuncSetAttribute(gemv_gather_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            int(msmem));
@@ -589,7 +590,7 @@ cudaError_t launch_mt(const GemvArgs& g, cudaStream_t st) {
   }
   if (b_vec) {
     const size_t asmem = gv_async_smem_bytes<T, MT>();
-    static bool async_attr[64] = {};
+    static std::atomic<bool> async_attr[64];  // per device; racing first calls both set the attribute
     if (dev >= 0 && dev < 64 && !async_attr[dev]) {
       cudaError_t e = cudaFuncSetAttribute(gemv_gather_async_kernel<T, MT>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, int(asmem));
@@ -795,7 +796,7 @@ unsigned wave_cluster(int64_t blocks, int64_t k_keep, int sms) {
 template <int MT>
 cudaError_t launch_w8_mt(const GemvArgs& g, const float* scale, int64_t s_stride, cudaStream_t st) {
   const size_t smem = gv_async_smem_bytes<int8_t, MT>();
-  static bool attr_done[64] = {};
+  static std::atomic<bool> attr_done[64];  // per device; racing first calls both set the attribute
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
@@ -822,7 +823,7 @@ cudaError_t launch_gemv_gather_w8(const GemvArgs& g, const float* scale, int64_t
   if (g.M > kGemvMaxRows) return cudaErrorInvalidValue;
   if ((reinterpret_cast<uintptr_t>(g.b) % 16 == 0) && g.ldb % 16 == 0 && (g.batch == 1 || g.strideB % 16 == 0)) {
     const size_t smem = gv_mma_w8_smem_bytes();
-    static bool attr_done[64] = {};
+    static std::atomic<bool> attr_done[64];  // per device; racing first calls both set the attribute
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {

@@ -15,6 +15,7 @@
 //    reads this operand N-major.
 // Pure bit copies. Rows that are not 16-byte aligned take plain-load paths.
 #include <algorithm>
+#include <atomic>
 
 #include "int8_convert.cuh"
 #include "rmm_device.cuh"
@@ -363,7 +364,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 template <typename K>
 void set_smem_attr_once(K kernel) {
-  static bool done[64] = {};
+  static std::atomic<bool> done[64];  // per device; racing first calls both set the attribute
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !done[dev]) {

@@ -18,6 +18,7 @@
 // that the GEMM's split-K round reduce-adds into, while one SM per batch item
 // selects.
 #include <algorithm>
+#include <atomic>
 
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
@@ -304,7 +305,7 @@ cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_ke
   }
   const int keys_in_smem = K <= kSelSmemKeys;
   const size_t smem = keys_in_smem ? size_t(K) * 4 : 0;
-  static bool attr_done[64] = {};
+  static std::atomic<bool> attr_done[64];  // per device; racing first calls both set the attribute
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
