@@ -125,3 +125,65 @@ def test_mlp_70b_projections(which):
                       A_sub, B_sub, idx.cpu().numpy(), 1e-2)
     del X, W, ws
     torch.cuda.empty_cache()
+
+
+def _block_scores(X: torch.Tensor, W64_rows, K: int, rows: int = 1024) -> np.ndarray:
+    """fp64 slice scores of x · W, 1024 slices at a time (slice k needs only
+    column k of x and row k of W); W64_rows(r0, r1) gives W[r0:r1] in fp64."""
+    return np.concatenate([O.slice_scores(f64(X[:, r0:r0 + rows]), W64_rows(r0, min(K, r0 + rows)))
+                           for r0 in range(0, K, rows)])
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_decode_mlp_up_full_size(M):
+    """Decode on the full MLP-up weight, x[M×8192] · W[8192×28672] with W's
+    norms cached, through the fused call the benchmark times: every score
+    against fp64, the selection bit-exact on the library's scores and within
+    the near-tie rule against fp64, the product on 1024 sampled columns."""
+    X, W = inputs.mlp_up(seed=0, device=DEV)
+    X = X[:M].contiguous()
+    K, N = W.shape
+    bn = rmm.b_norms(W)
+    s = rmm.score_b_norms(X, bn)
+    s_ref = _block_scores(X, lambda r0, r1: f64(W[r0:r1]), K)
+    check_scores(s.cpu().numpy(), s_ref)
+    for rho in (0.5, 0.3):
+        k = rmm.keep_count(rho, K)
+        idx = torch.empty(k, dtype=torch.int32, device=DEV)
+        C, ws = rmm.matmul_reduced_b_norms(X, W, bn, rho, idx_out=idx)
+        rmm.check(ws)
+        _check_selection_exact(s, idx, k)
+        check_selection(idx.cpu().numpy(), s_ref, k)
+        _, cols = _rows_cols(M, N, M, 1024, k)
+        cc = torch.as_tensor(cols, device=DEV)
+        check_product(f64(C[:, cc]), f64(X), f64(W[:, cc]), idx.cpu().numpy(), 1e-2)
+    del X, W, ws
+    torch.cuda.empty_cache()
+
+
+def test_w8_decode_mlp_up_full_size():
+    """The INT8-weight decode workload at full size, x[1×8192] · (Wq · diag(scale))
+    with Wq int8 [8192×28672] and W's norms cached: scores against the
+    dequantized weight in fp64, the selection bit-exact on the library's
+    scores, the product on 1024 sampled columns."""
+    X, _ = inputs.mlp_up(seed=0, device=DEV)
+    X = X[:1].contiguous()
+    Wq, sc = inputs.int8_weight(8192, 28672, std=0.01, seed=1, device=DEV)
+    K, N = Wq.shape
+    sc64 = sc.double().cpu().numpy()
+    bn = rmm.b_norms_w8(Wq, sc)
+    s = rmm.score_b_norms(X, bn)
+    s_ref = _block_scores(X, lambda r0, r1: O.dequantize_w8(Wq[r0:r1].cpu().numpy(), sc64), K)
+    check_scores(s.cpu().numpy(), s_ref)
+    k = rmm.keep_count(0.5, K)
+    idx = torch.empty(k, dtype=torch.int32, device=DEV)
+    C, ws = rmm.matmul_reduced_w8(X, Wq, sc, 0.5, b_norm=bn, idx_out=idx)
+    rmm.check(ws)
+    _check_selection_exact(s, idx, k)
+    check_selection(idx.cpu().numpy(), s_ref, k)
+    _, cols = _rows_cols(1, N, 1, 1024, 7)
+    cc = torch.as_tensor(cols, device=DEV)
+    W_sub = O.dequantize_w8(Wq[:, cc].cpu().numpy(), sc64[cols])
+    check_product(f64(C[:, cc]), f64(X), W_sub, idx.cpu().numpy(), 1e-2)
+    del X, Wq, sc, ws
+    torch.cuda.empty_cache()
