@@ -187,3 +187,51 @@ def test_w8_decode_mlp_up_full_size():
     check_product(f64(C[:, cc]), f64(X), W_sub, idx.cpu().numpy(), 1e-2)
     del X, Wq, sc, ws
     torch.cuda.empty_cache()
+
+
+def test_decode_4096_full_size():
+    """x[1×4096] · W[4096×4096] (1 % outlier channels, W's norms cached) through
+    the fused call: all scores, the selection bit-exact on the library's
+    scores, the whole product."""
+    X, W = inputs.linear_projection(M=16, seed=0, device=DEV)
+    X = X[:1].contiguous()
+    K, N = W.shape
+    bn = rmm.b_norms(W)
+    s = rmm.score_b_norms(X, bn)
+    s_ref = O.slice_scores(f64(X), f64(W))
+    check_scores(s.cpu().numpy(), s_ref)
+    k = rmm.keep_count(0.5, K)
+    idx = torch.empty(k, dtype=torch.int32, device=DEV)
+    C, ws = rmm.matmul_reduced_b_norms(X, W, bn, 0.5, idx_out=idx)
+    rmm.check(ws)
+    _check_selection_exact(s, idx, k)
+    check_selection(idx.cpu().numpy(), s_ref, k)
+    check_product(f64(C), f64(X), f64(W), idx.cpu().numpy(), 1e-2)
+
+
+def test_w8_linear_4096_full_size():
+    """X[4096×4096] · (Wq · diag(scale)), Wq int8 [4096×4096], W's norms cached:
+    the pack + tensor-core GEMM route at full size — all scores against the
+    dequantized weight, the selection bit-exact on the library's scores, the
+    product on 128 sampled rows × 512 sampled columns."""
+    X, _ = inputs.linear_projection(seed=0, device=DEV)
+    Wq, sc = inputs.int8_weight(4096, 4096, std=0.02, seed=1, device=DEV)
+    M, K = X.shape
+    N = Wq.shape[1]
+    sc64 = sc.double().cpu().numpy()
+    bn = rmm.b_norms_w8(Wq, sc)
+    s = rmm.score_b_norms(X, bn)
+    W64 = O.dequantize_w8(Wq.cpu().numpy(), sc64)
+    s_ref = O.slice_scores(f64(X), W64)
+    check_scores(s.cpu().numpy(), s_ref)
+    k = rmm.keep_count(0.5, K)
+    idx = torch.empty(k, dtype=torch.int32, device=DEV)
+    C, ws = rmm.matmul_reduced_w8(X, Wq, sc, 0.5, b_norm=bn, idx_out=idx)
+    rmm.check(ws)
+    _check_selection_exact(s, idx, k)
+    check_selection(idx.cpu().numpy(), s_ref, k)
+    rows, cols = _rows_cols(M, N, 128, 512, 11)
+    rr, cc = torch.as_tensor(rows, device=DEV), torch.as_tensor(cols, device=DEV)
+    check_product(f64(C[rr][:, cc]), f64(X[rr]), W64[:, cols], idx.cpu().numpy(), 1e-2)
+    del X, Wq, sc, ws
+    torch.cuda.empty_cache()
