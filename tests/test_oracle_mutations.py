@@ -1,6 +1,7 @@
 """The oracle's pins catch plausible mistakes: each case plants one mistake in
 a temporary copy of the oracle (a dropped square root, a transposed operand, a
-floor for the ceiling, the wrong tie rule, an unscaled INT8 weight, ...) and
+floor for the ceiling, the wrong tie rule, an unscaled INT8 weight, one
+selection for every batch item, ...) and
 runs the pin suite against that copy, which must fail. The oracle itself is
 never modified."""
 from __future__ import annotations
@@ -44,6 +45,18 @@ MUTATIONS = {
     "near_tie_window_absolute": ("ok = all(abs(s[k] - t) <= rel_window * t for k in diff)",
                                  "ok = all(abs(s[k] - t) <= rel_window for k in diff)"),
     "relative_error_unnormalised": ("return float(num / den)", "return float(num)"),
+    "keeps_one_too_many": ("return np.sort(order[:k_keep]).astype(np.int64)",
+                           "return np.sort(order[:min(len(order), k_keep + 1)]).astype(np.int64)"),
+    "batch_items_share_one_selection": ("        C, idx, s = matmul_reduced(A[b], B[b], rho, mode)\n",
+                                        "        C, idx, s = matmul_reduced(A[b], B[b], rho, mode)\n"
+                                        "        if b > 0:\n"
+                                        "            idx = idxs[0]\n"
+                                        "            C = reduced_product(A[b], B[b], idx)\n"),
+    "product_over_dropped_slices": ("    return A_S @ B_S\n",
+                                    "    keep = np.setdiff1d(np.arange(np.asarray(A).shape[1]), idx)\n"
+                                    "    return np.asarray(A, dtype=np.float64)[:, keep] @ "
+                                    "np.asarray(B, dtype=np.float64)[keep, :]\n"),
+    "near_tie_threshold_is_the_largest_kept": ("t = float(np.min(s[list(o)]))", "t = float(np.max(s[list(o)]))"),
 }
 
 
