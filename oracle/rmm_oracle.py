@@ -101,7 +101,14 @@ def select_top(s: np.ndarray, k_keep: int) -> np.ndarray:
 
 
 def pack(A: np.ndarray, B: np.ndarray, idx: np.ndarray):
-    """A_S = A[:, I] (M×k) and B_S = B[I, :] (k×N) ("Mecanismo Central")."""
+    """A_S = A[:, I] (M×k) and B_S = B[I, :] (k×N) ("Mecanismo Central").
+
+    I is a subset of the contraction indices {0, …, K−1}: an index outside
+    that range is an error here (NumPy would wrap a negative one around)."""
+    idx = np.asarray(idx)
+    K = A.shape[1]
+    if idx.size and (idx.min() < 0 or idx.max() >= K):
+        raise IndexError(f"kept index outside [0, {K})")
     return A[:, idx], B[idx, :]
 
 
@@ -184,15 +191,20 @@ def selection_matches(gpu_idx: np.ndarray, oracle_idx: np.ndarray, s: np.ndarray
     Returns (ok, n_boundary): ok is True when every index in the symmetric
     difference of the two sets has an oracle score within rel_window·t of t, the
     oracle's k-th largest score (a near-tie at the selection boundary, where
-    either choice is correct); n_boundary counts those indices."""
-    g = set(int(i) for i in np.asarray(gpu_idx).ravel())
+    either choice is correct); n_boundary counts those indices. A computed set
+    with an index outside [0, K) or a repeated index never matches."""
+    s = np.asarray(s, dtype=np.float64)
+    g_list = [int(i) for i in np.asarray(gpu_idx).ravel()]
+    # I is a set of contraction indices: each in [0, K), none repeated
+    if any(i < 0 or i >= s.shape[0] for i in g_list) or len(set(g_list)) != len(g_list):
+        return False, 0
+    g = set(g_list)
     o = set(int(i) for i in np.asarray(oracle_idx).ravel())
     if len(g) != len(o):
         return False, 0
     diff = g ^ o
     if not diff:
         return True, 0
-    s = np.asarray(s, dtype=np.float64)
     t = float(np.min(s[list(o)]))
     ok = all(abs(s[k] - t) <= rel_window * t for k in diff)
     return ok, len(diff)

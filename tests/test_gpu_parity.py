@@ -78,9 +78,9 @@ def test_stages_match_oracle(shape, dtype, gemm_cta_group):
             for out_dtype in (torch.float32, torch.bfloat16):
                 tol = product_tol(dtype, out_dtype)
                 C = rmm.gemm(A_S, B_S, k, out_dtype, N=N)
-                check_product(f64(C), A64, B64, idx.cpu().numpy(), tol)
+                check_product(C, A64, B64, idx.cpu().numpy(), tol)
                 C2 = rmm.gemm(A_S2, B_St, k, out_dtype, b_kmajor=True)
-                check_product(f64(C2), A64, B64, idx.cpu().numpy(), tol)
+                check_product(C2, A64, B64, idx.cpu().numpy(), tol)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
@@ -114,7 +114,7 @@ def test_batched_qk_small(gemm_cta_group):
         check_single(Q[h], Km[h], 0.5, "product", S[h], idx[h], b_kmajor=True)
     S16, _ = rmm.qk_reduced(Q, Km, 0.5, out_dtype=torch.bfloat16, workspace=ws)
     for h in range(3):
-        check_product(f64(S16[h]), f64(Q[h]), f64(Km[h]).T, idx[h].cpu().numpy(), 1e-2)
+        check_product(S16[h], f64(Q[h]), f64(Km[h]).T, idx[h].cpu().numpy(), 1e-2)
 
 
 def test_batched_pv_small(gemm_cta_group):
@@ -233,7 +233,7 @@ def test_split_k_tiles_zeroed_inside_the_select_launch(batch, gemm_cta_group):
     rmm.check(ws)
     assert rmm.launch_count() - n0 == 4  # score, select (+ zeroing), pack (A and B), gemm
     for b in range(batch):
-        check_product(f64(C[b]), f64(A[b]), f64(B[b]), idx[b].cpu().numpy(), product_tol(torch.bfloat16, torch.float32))
+        check_product(C[b], f64(A[b]), f64(B[b]), idx[b].cpu().numpy(), product_tol(torch.bfloat16, torch.float32))
     # the stage-by-stage GEMM zeroes them with a kernel of its own
     A_S, B_S = rmm.pack(A, B, idx)
     out2 = torch.full((batch, M, N), float("nan"), device=DEV)
@@ -346,7 +346,7 @@ def test_gemv_gather_matches_oracle(shape, dtype):
         idx = rmm.select(rmm.score(A, B), k)
         for out_dtype in (torch.float32, torch.bfloat16):
             C = rmm.gemv_gather(A, B, idx, out_dtype)
-            check_product(f64(C), A64, B64, idx.cpu().numpy(), product_tol(dtype, out_dtype))
+            check_product(C, A64, B64, idx.cpu().numpy(), product_tol(dtype, out_dtype))
         C1 = rmm.gemv_gather(A, B, idx)
         C2 = rmm.gemv_gather(A, B, idx)
         assert torch.equal(C1, C2)  # fixed summation order
@@ -360,7 +360,7 @@ def test_gemv_gather_unaligned_rows():
     B = Bfull[:, 1:N + 1]  # ld N + 3, base off by 2 bytes
     idx = rmm.select(rmm.score(A, B.contiguous()), rmm.keep_count(0.5, K))
     C = rmm.gemv_gather(A, B, idx)
-    check_product(f64(C), f64(A), f64(B), idx.cpu().numpy(), 1e-2)
+    check_product(C, f64(A), f64(B), idx.cpu().numpy(), 1e-2)
 
 
 @pytest.mark.parametrize("M", [1, 16])
@@ -378,7 +378,7 @@ def test_gemv_gather_tensor_core_route(M, N, ld):
         idx = rmm.select(s, k)
         for out_dtype in (torch.float32, torch.bfloat16):
             C = rmm.gemv_gather(A, B, idx, out_dtype)
-            check_product(f64(C), A64, B64, idx.cpu().numpy(), product_tol(torch.bfloat16, out_dtype))
+            check_product(C, A64, B64, idx.cpu().numpy(), product_tol(torch.bfloat16, out_dtype))
         assert torch.equal(rmm.gemv_gather(A, B, idx), rmm.gemv_gather(A, B, idx))
 
 
@@ -425,7 +425,7 @@ def test_fused_call_bit_identical_to_stage_calls(shape, gemm_cta_group):
         A_S, B_S = rmm.pack(A, B, idx)
         C_ref = rmm.gemm(A_S, B_S, k, out_dtype, N=N)
         assert torch.equal(C, C_ref)
-        check_product(f64(C), f64(A), f64(B), idx.cpu().numpy(), product_tol(torch.bfloat16, out_dtype))
+        check_product(C, f64(A), f64(B), idx.cpu().numpy(), product_tol(torch.bfloat16, out_dtype))
 
 
 @pytest.mark.parametrize("K", [4096, 4097, 8192, 50000])

@@ -40,4 +40,4 @@ def test_stalled_producer_times_out_and_context_survives():
 
     C = rmm.gemm(A_S, B_S, k, status=status)
     rmm.check(status)
-    check_product(f64(C), f64(A), f64(B), idx.cpu().numpy(), 1e-2)
+    check_product(C, f64(A), f64(B), idx.cpu().numpy(), 1e-2)

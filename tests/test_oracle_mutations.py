@@ -56,6 +56,9 @@ MUTATIONS = {
                                     "    keep = np.setdiff1d(np.arange(np.asarray(A).shape[1]), idx)\n"
                                     "    return np.asarray(A, dtype=np.float64)[:, keep] @ "
                                     "np.asarray(B, dtype=np.float64)[keep, :]\n"),
+    "selection_range_unchecked": ("    if any(i < 0 or i >= s.shape[0] for i in g_list) or len(set(g_list)) != len(g_list):\n"
+                                  "        return False, 0\n", ""),
+    "pack_range_unchecked": ("        raise IndexError(f\"kept index outside [0, {K})\")\n", "        pass\n"),
     "near_tie_threshold_is_the_largest_kept": ("t = float(np.min(s[list(o)]))", "t = float(np.max(s[list(o)]))"),
 }
 

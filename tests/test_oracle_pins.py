@@ -342,6 +342,25 @@ def test_selection_matches_window_rule():
     assert not ok
 
 
+def test_kept_indices_must_lie_in_the_contraction_range():
+    """I is a subset of {0, ..., K-1} ("Mecanismo Central"): an index of -1
+    (which NumPy indexing would wrap to K-1), an index K or a repeated index
+    is never a valid selection, even when the scores there are near-ties."""
+    s = np.array([1.0, 1.0, 1.0, 1.0])  # every index a near-tie of every other
+    o = O.select_top(s, 2)
+    assert O.selection_matches(np.array([0, 1]), o, s) == (True, 0)
+    for bad in ([-1, 0], [0, 4], [1, 1]):
+        ok, _ = O.selection_matches(np.array(bad), o, s)
+        assert not ok, bad
+    A = np.arange(8.0).reshape(2, 4)
+    B = np.ones((4, 3))
+    with pytest.raises(IndexError):
+        O.reduced_product(A, B, np.array([-1, 2]))
+    with pytest.raises(IndexError):
+        O.reduced_product(A, B, np.array([0, 4]))
+    assert np.array_equal(O.reduced_product(A, B, np.array([1, 3])), np.array([[4.0] * 3, [12.0] * 3]))
+
+
 def test_frobenius_rel_error():
     a = np.array([[3.0, 4.0]])
     assert O.frobenius_rel_error(a, a) == 0.0
