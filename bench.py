@@ -82,6 +82,9 @@ class Problem:
         self.N = B3.shape[1] if b_kmajor else B3.shape[2]
         self.b_norm = None  # B's cached norms: the step uses them (decode: B is a resident weight)
         self.scale = None   # INT8 weight: B holds the int8 codes, W = B · diag(scale)
+        # k = ceil(rho·K): the library's rmm_keep_count on the GPU arm; the CPU
+        # reference arm substitutes the oracle's, so that it never loads librmm
+        self.keep_count = rmm.keep_count
 
     @property
     def gemv(self):
@@ -89,7 +92,7 @@ class Problem:
         return self.M <= 16 and not self.b_kmajor
 
     def k_keep(self, rho):
-        return rmm.keep_count(rho, self.K)
+        return self.keep_count(rho, self.K)
 
     def kept_flops(self, rho):
         return 2.0 * self.batch * self.M * self.N * self.k_keep(rho)
@@ -481,11 +484,12 @@ def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
+    from oracle import rmm_oracle as O
     name = args.workload
     p = make_problem(name, "cpu", 0, args.rho)
+    p.keep_count = O.keep_count
     p.mode = args.score_mode
     rho = p.rho
-    from oracle import rmm_oracle as O  # noqa: F401
     budget = 150.0
     res = oracle_cpu_timing(p, rho, budget_s=budget, max_steps=max(1, args.steps))
     line = {"impl": "reference", "metric": METRIC,

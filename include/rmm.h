@@ -26,6 +26,8 @@
  *   - bf16 data is passed as raw 16-bit words (the bits of __nv_bfloat16).
  *   - All work is enqueued on `stream` in order; no call synchronises the
  *     host except rmm_check.
+ *   - A call makes the stream's device current while it runs and restores the
+ *     caller's current device before it returns.
  *   - Argument errors are detected on the host, before any launch, and
  *     returned as RMM_ERR_INVALID / RMM_ERR_UNSUPPORTED. A failed CUDA
  *     runtime call returns RMM_ERR_CUDA. rmm_last_error_string() describes
@@ -140,9 +142,11 @@ rmm_status rmm_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, 
  *        if b_kmajor == 1: [batch][N][k_pad], B_S[b][j][t] = Kmat[b][j][idx[b][t]].
  *   k_pad = rmm_padded_keep(k_keep); slices t >= k_keep (and columns j >= N of
  *   the row-major form) are written as zero. Copies bits exactly (no
- *   arithmetic). Indices outside [0, K) are a caller error the kernels do not
- *   check. status_word (nullable) receives RMM_STATUS_BIT_TIMEOUT if a bounded
- *   wait for a bulk copy gave up. */
+ *   arithmetic). Indices outside [0, K) are a caller error that the kernels
+ *   do not check; with debug checks on (rmm_set_debug) the call validates idx
+ *   on the device first and returns RMM_ERR_INVALID, launching nothing that
+ *   reads through it. status_word (nullable) receives RMM_STATUS_BIT_TIMEOUT
+ *   if a bounded wait for a bulk copy gave up. */
 rmm_status rmm_pack(const void* A, int64_t lda, int64_t strideA,
                     const void* B, int64_t ldb, int64_t strideB, int b_kmajor,
                     int64_t batch, int64_t M, int64_t K, int64_t N,
@@ -329,7 +333,8 @@ rmm_status rmm_pv_reduced(const void* P, const void* V, int64_t bh, int64_t S_q,
  *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture. A lookup that fails is not remembered: the
+ *     call returns RMM_ERR_CUDA and the next call on that device tries again.
  *   - All calls share the one array and it keeps the last call's contents;
  *     the status word in it is cleared at the start of each call. Calls whose
  *     work overlaps on the GPU (different streams, or other threads) race on
@@ -372,6 +377,20 @@ int rmm_set_gemm_cta_group(int cta_group);
 
 /* Number of kernels this library has launched in this process. */
 uint64_t rmm_launch_count(void);
+
+/* Debug checks, process-wide; returns the previous setting. Off by default,
+ * or on when the environment variable RMM_DEBUG is set to anything but "0"
+ * at the first call. When on:
+ *   - rmm_pack, rmm_pack_w8, rmm_gemv_gather and rmm_gemv_gather_w8 first
+ *     check on the device that every kept index lies in [0, K), synchronise
+ *     the stream, and return RMM_ERR_INVALID (naming the first bad entry)
+ *     without launching the kernels that would read through a bad index;
+ *   - the fused calls synchronise the stream after their kernels and return
+ *     RMM_ERR_NONFINITE / RMM_ERR_TIMEOUT from the status word directly (the
+ *     word is left set for rmm_check).
+ * Calls with debug checks on share one device word for the index check and
+ * must not run concurrently. Not for timed or captured work. */
+int rmm_set_debug(int on);
 
 /* Timing hook (diagnostics; no counterpart in the method). While set, every
  * GEMM launch of this process records `start` on its stream immediately

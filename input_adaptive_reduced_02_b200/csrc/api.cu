@@ -4,16 +4,30 @@
 // Matrix-Product Reduction for LLM Inference", Resumo Técnico › Metodologia).
 // Everything is enqueued on the caller's stream; nothing here allocates or
 // synchronises, except rmm_check.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/rmm.h"
 #include "rmm_internal.h"
 
 namespace rmm {
+
+// A named NVTX range around one stage of a call, so that a profiler's
+// timeline (or an ncu --nvtx filter) shows score, select, pack and the product
+// by name; header-only NVTX costs a branch when no tool is attached.
+struct StageRange {
+  explicit StageRange(const char* name) { nvtxRangePushA(name); }
+  ~StageRange() { nvtxRangePop(); }
+  StageRange(const StageRange&) = delete;
+  StageRange& operator=(const StageRange&) = delete;
+};
 
 static std::atomic<uint64_t> g_launches{0};
 static std::atomic<uint64_t> g_wait_limit_ns{0};
@@ -40,18 +54,81 @@ static rmm_status cuda_fail(cudaError_t e, const char* what, const char* why = n
   return fail(RMM_ERR_CUDA, "%s: %s%s%s", what, cudaGetErrorString(e), why ? " — " : "", why ? why : "");
 }
 
-// Bind the calling thread to the stream's device (the caller's framework may
-// have made another device current).
-static rmm_status bind_device(cudaStream_t st) {
-  int dev = -1;
-  cudaError_t e = cudaStreamGetDevice(st, &dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamGetDevice");
-  int cur = -1;
-  cudaGetDevice(&cur);
-  if (cur != dev) {
-    e = cudaSetDevice(dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+// ---------------------------------------------------------------- debug checks
+// Off by default. On (rmm_set_debug(1), or RMM_DEBUG set to anything but "0"
+// in the environment when the first call is made), the stage calls that take
+// a caller's index list validate it on the device before anything reads
+// through it, and the fused calls wait for their kernels and report the
+// device status word; both synchronise the stream.
+static std::atomic<int> g_debug{-1};  // -1: not yet read from the environment
+
+static bool debug_on() {
+  int d = g_debug.load();
+  if (d < 0) {
+    const char* e = std::getenv("RMM_DEBUG");
+    int want = (e && *e && std::strcmp(e, "0") != 0) ? 1 : 0;
+    g_debug.compare_exchange_strong(d, want);
+    d = g_debug.load();
   }
+  return d == 1;
+}
+
+// [0]: number of indices outside [0, K); [1]: the first such position.
+__device__ uint32_t g_idx_check[2];
+
+__global__ void check_indices_kernel(const int32_t* __restrict__ idx, int64_t n, int64_t K, uint32_t* out) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int32_t v = idx[i];
+    if (v < 0 || int64_t(v) >= K) {
+      atomicAdd(&out[0], 1u);
+      atomicMin(&out[1], uint32_t(i < 0xFFFFFFFFll ? i : 0xFFFFFFFFll));
+    }
+  }
+}
+
+// idx [batch][k_keep]: every entry must lie in [0, K). Synchronises `st`.
+static rmm_status debug_check_indices(const int32_t* idx, int64_t batch, int64_t k_keep, int64_t K, const char* who,
+                                      cudaStream_t st) {
+  uint32_t* out = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&out), g_idx_check);
+  const uint32_t init[2] = {0u, 0xFFFFFFFFu};
+  if (e == cudaSuccess) e = cudaMemcpyAsync(out, init, sizeof(init), cudaMemcpyHostToDevice, st);
+  const int64_t n = batch * k_keep;
+  if (e == cudaSuccess) {
+    const unsigned blocks = unsigned(std::min<int64_t>((n + 255) / 256, 148 * 4));
+    count_launch();
+    check_indices_kernel<<<blocks, 256, 0, st>>>(idx, n, K, out);
+    e = cudaGetLastError();
+  }
+  uint32_t got[2] = {0u, 0u};
+  if (e == cudaSuccess) e = cudaMemcpyAsync(got, out, sizeof(got), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "index check (debug)");
+  if (got[0] == 0) return RMM_OK;
+  int32_t v = 0;
+  e = cudaMemcpy(&v, idx + got[1], sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "index check (debug)");
+  return fail(RMM_ERR_INVALID, "%s: %u kept indices outside [0, %lld); first idx[%lld][%lld] = %d", who, got[0],
+              (long long)K, (long long)(got[1] / k_keep), (long long)(got[1] % k_keep), v);
+}
+
+// Debug mode, after a fused call: wait for it and return its device status.
+static rmm_status debug_call_status(uint32_t* status, cudaStream_t st) {
+  uint32_t w = 0;
+  cudaError_t e = cudaMemcpyAsync(&w, status, sizeof(w), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word (debug)");
+  if (w & RMM_STATUS_BIT_TIMEOUT) return fail(RMM_ERR_TIMEOUT, "a pipeline wait in the GEMM ran out");
+  if (w & RMM_STATUS_BIT_NONFINITE) return fail(RMM_ERR_NONFINITE, "a slice score was NaN or Inf");
+  return RMM_OK;
+}
+
+// Make the stream's device current for the rest of the call (the caller's
+// framework may have made another device current); `g` puts the caller's
+// device back when the entry point returns.
+static rmm_status bind_device(cudaStream_t st, DeviceGuard& g) {
+  const cudaError_t e = g.bind(st);
+  if (e != cudaSuccess) return cuda_fail(e, "selecting the stream's device");
   return RMM_OK;
 }
 
@@ -127,6 +204,7 @@ static rmm_status do_score(const void* A, int64_t lda, int64_t sA, const void* B
                            int b_kmajor, int64_t batch, int64_t M, int64_t K, int64_t N, rmm_dtype in,
                            rmm_score_mode mode, float* s, uint32_t* status, cudaStream_t st,
                            const float* bn = nullptr, int64_t bn_stride = 0, int clear_status = 0) {
+  StageRange range("rmm score");
   const MatView a{A, lda, sA, M, K};
   const int bmode = bn ? 3 : (mode == RMM_SCORE_A_ONLY ? 0 : (b_kmajor ? 2 : 1));
   const MatView b = b_kmajor ? MatView{B, ldb, sB, N, K} : MatView{B, ldb, sB, K, N};
@@ -138,6 +216,7 @@ static rmm_status do_score(const void* A, int64_t lda, int64_t sA, const void* B
 static rmm_status do_pack(const void* A, int64_t lda, int64_t sA, const void* B, int64_t ldb, int64_t sB, int b_kmajor,
                           int64_t batch, int64_t M, int64_t K, int64_t N, const int32_t* idx, int64_t k_keep,
                           rmm_dtype in, void* A_S, void* B_S, uint32_t* status, cudaStream_t st) {
+  StageRange range("rmm pack");
   const ElemKind e = kind(in);
   const int64_t kp = round_up(k_keep, 64);
   const uint64_t lim = wait_limit();
@@ -186,6 +265,7 @@ static GemmArgs gemm_args(const void* A_S, const void* B_S, int b_kmajor, int64_
 static rmm_status do_gemv(const void* A, int64_t lda, int64_t sA, const void* B, int64_t ldb, int64_t sB,
                           int64_t batch, int64_t M, int64_t N, const int32_t* idx, int64_t k_keep, rmm_dtype in,
                           void* C, int64_t ldc, int64_t sC, rmm_dtype out, cudaStream_t st) {
+  StageRange range("rmm gather-gemv");
   GemvArgs g;
   g.a = A;
   g.b = B;
@@ -209,6 +289,7 @@ static rmm_status do_gemv(const void* A, int64_t lda, int64_t sA, const void* B,
 }
 
 static rmm_status do_gemm(const GemmArgs& g, rmm_dtype in, cudaStream_t st) {
+  StageRange range("rmm gemm");
   cudaError_t ce;
   const char* why = nullptr;
   if (in == RMM_BF16)
@@ -279,7 +360,8 @@ rmm_status rmm_score(const void* A, int64_t lda, int64_t strideA, const void* B,
   if (r) return r;
   if (batch > 0 && !s) return fail(RMM_ERR_INVALID, "s is NULL");
   if (batch == 0) return RMM_OK;
-  if ((r = bind_device(stream))) return r;
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
   return do_score(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, in, mode, s, status_word, stream);
 }
 
@@ -291,8 +373,10 @@ rmm_status rmm_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, 
   if (batch > kMaxGridBatch) return fail(RMM_ERR_UNSUPPORTED, "batch > %lld", (long long)kMaxGridBatch);
   if (batch == 0) return RMM_OK;
   if (!s || !idx) return fail(RMM_ERR_INVALID, "s or idx is NULL");
-  rmm_status r = bind_device(stream);
+  DeviceGuard dg;
+  rmm_status r = bind_device(stream, dg);
   if (r) return r;
+  StageRange range("rmm select");
   cudaError_t ce = launch_select(s, batch, K, k_keep, idx, status_word, stream);
   if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
   return RMM_OK;
@@ -313,7 +397,9 @@ rmm_status rmm_pack(const void* A, int64_t lda, int64_t strideA, const void* B, 
   if ((M > 0 && !A_S) || !B_S) return fail(RMM_ERR_INVALID, "A_S or B_S is NULL");
   if ((reinterpret_cast<uintptr_t>(A_S) | reinterpret_cast<uintptr_t>(B_S)) & 15u)
     return fail(RMM_ERR_INVALID, "A_S and B_S must be 16-byte aligned");
-  if ((r = bind_device(stream))) return r;
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
+  if (debug_on() && (r = debug_check_indices(idx, batch, k_keep, K, "rmm_pack", stream))) return r;
   return do_pack(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, idx, k_keep, in, A_S, B_S, status_word,
                  stream);
 }
@@ -328,7 +414,8 @@ rmm_status rmm_gemm(const void* A_S, const void* B_S, int b_kmajor, int64_t batc
   if (!layout_ok(batch, M, N, ldc, strideC)) return fail(RMM_ERR_INVALID, "C layout (ldc/strideC) is too small");
   if (batch == 0 || M == 0 || N == 0) return RMM_OK;
   if (!A_S || !B_S || !C) return fail(RMM_ERR_INVALID, "A_S, B_S or C is NULL");
-  rmm_status r = bind_device(stream);
+  DeviceGuard dg;
+  rmm_status r = bind_device(stream, dg);
   if (r) return r;
   return do_gemm(gemm_args(A_S, B_S, b_kmajor, batch, M, N, k_keep, C, ldc, strideC, out, status_word), in, stream);
 }
@@ -354,7 +441,8 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
   const size_t need = decode_route(M, b_kmajor) ? w.bytes_no_pack : w.bytes;
   if (workspace_bytes < need)
     return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
-  if ((r = bind_device(stream))) return r;
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
   cudaError_t ce = cudaSuccess;
   if (batch == 0) {  // no kernel runs: clear the status word here
     ce = cudaMemsetAsync(w.status, 0, 4, stream);
@@ -374,15 +462,23 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
   const bool gemv = decode_route(M, b_kmajor);
   SplitZero z;
   const bool zero = !gemv && in == RMM_BF16 && gemm_tc_split_zero(g, &z);
-  ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr, gemv);
+  {
+    StageRange range("rmm select");
+    ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr, gemv);
+  }
   if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
   g.c_zeroed = zero ? 1 : 0;
-  if (M == 0 || N == 0) return RMM_OK;
-  if (gemv) return do_gemv(A, lda, strideA, B, ldb, strideB, batch, M, N, idx, k_keep, in, C, ldc, strideC, out, stream);
+  if (M == 0 || N == 0) return debug_on() ? debug_call_status(w.status, stream) : RMM_OK;
+  if (gemv) {
+    if ((r = do_gemv(A, lda, strideA, B, ldb, strideB, batch, M, N, idx, k_keep, in, C, ldc, strideC, out, stream)))
+      return r;
+    return debug_on() ? debug_call_status(w.status, stream) : RMM_OK;
+  }
   if ((r = do_pack(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, idx, k_keep, in, w.a_s, w.b_st,
                    w.status, stream)))
     return r;
-  return do_gemm(g, in, stream);
+  if ((r = do_gemm(g, in, stream))) return r;
+  return debug_on() ? debug_call_status(w.status, stream) : RMM_OK;
 }
 
 static rmm_status check_bn(const float* bn, int64_t bn_stride, int64_t batch, int64_t K) {
@@ -417,7 +513,8 @@ rmm_status rmm_pv_reduced(const void* P, const void* V, int64_t bh, int64_t S_q,
 
 rmm_status rmm_check(void* status_word, cudaStream_t stream) {
   if (!status_word) return fail(RMM_ERR_INVALID, "status_word is NULL");
-  rmm_status r = bind_device(stream);
+  DeviceGuard dg;
+  rmm_status r = bind_device(stream, dg);
   if (r) return r;
   uint32_t w = 0;
   cudaError_t ce = cudaMemcpyAsync(&w, status_word, 4, cudaMemcpyDeviceToHost, stream);
@@ -442,6 +539,12 @@ int rmm_set_gemm_cta_group(int cta_group) {
 }
 
 uint64_t rmm_launch_count(void) { return g_launches.load(); }
+
+int rmm_set_debug(int on) {
+  const int prev = debug_on() ? 1 : 0;
+  g_debug.store(on ? 1 : 0);
+  return prev;
+}
 
 }  // extern "C"
 
@@ -469,13 +572,15 @@ rmm_status rmm_b_norms(const void* B, int64_t ldb, int64_t strideB, int b_kmajor
     return fail(RMM_ERR_INVALID, "B layout (ldb/strideB) is too small");
   if (batch == 0 || N == 0) {
     if (batch > 0 && N == 0 && b_norm) {
-      if ((r = bind_device(stream))) return r;
+      DeviceGuard dg;
+      if ((r = bind_device(stream, dg))) return r;
       cudaError_t ce = cudaMemsetAsync(b_norm, 0, size_t(batch * K) * 4, stream);
       if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemsetAsync(b_norm)");
     }
     return RMM_OK;
   }
-  if ((r = bind_device(stream))) return r;
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
   const cudaError_t ce = launch_b_norms(MatView{B, ldb, strideB, rows, cols}, b_kmajor, kind(in), batch, b_norm,
                                         status_word, stream);
   if (ce != cudaSuccess) return cuda_fail(ce, "b_norms kernel");
@@ -493,7 +598,8 @@ rmm_status rmm_score_b_norms(const void* A, int64_t lda, int64_t strideA, const 
     return fail(RMM_ERR_INVALID, "A layout (lda/strideA) is too small");
   if (batch > 0 && !s) return fail(RMM_ERR_INVALID, "s is NULL");
   if (batch == 0) return RMM_OK;
-  if ((r = bind_device(stream))) return r;
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
   return do_score(A, lda, strideA, nullptr, 0, 0, 0, batch, M, K, 0, in, RMM_SCORE_PRODUCT, s, status_word, stream,
                   b_norm, b_norm_stride);
 }
@@ -523,7 +629,9 @@ rmm_status rmm_gemv_gather(const void* A, int64_t lda, int64_t strideA, const vo
   if (!layout_ok(batch, M, N, ldc, strideC)) return fail(RMM_ERR_INVALID, "C layout (ldc/strideC) is too small");
   if (batch == 0 || M == 0 || N == 0) return RMM_OK;
   if (!idx || !C) return fail(RMM_ERR_INVALID, "idx or C is NULL");
-  if ((r = bind_device(stream))) return r;
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
+  if (debug_on() && (r = debug_check_indices(idx, batch, k_keep, K, "rmm_gemv_gather", stream))) return r;
   return do_gemv(A, lda, strideA, B, ldb, strideB, batch, M, N, idx, k_keep, in, C, ldc, strideC, out, stream);
 }
 
@@ -549,7 +657,8 @@ rmm_status rmm_b_norms_w8(const int8_t* Wq, int64_t ldw, int64_t strideW, const 
   if ((r = check_w8(Wq, ldw, strideW, scale, scale_stride, batch, K, N, false))) return r;
   if (batch > 0 && !b_norm) return fail(RMM_ERR_INVALID, "b_norm is NULL");
   if (batch == 0) return RMM_OK;
-  if ((r = bind_device(stream))) return r;
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
   cudaError_t ce = N == 0 ? cudaMemsetAsync(b_norm, 0, size_t(batch * K) * 4, stream)
                           : launch_b_norms_w8(Wq, ldw, strideW, scale, scale_stride, batch, K, N, b_norm,
                                               status_word, stream);
@@ -561,6 +670,7 @@ static rmm_status do_pack_w8(const void* A, int64_t lda, int64_t sA, const int8_
                              const float* scale, int64_t s_stride, int64_t batch, int64_t M, int64_t K, int64_t N,
                              const int32_t* idx, int64_t k_keep, void* A_S, void* B_S, uint32_t* status,
                              cudaStream_t st) {
+  StageRange range("rmm pack");
   const int64_t kp = round_up(k_keep, 64);
   cudaError_t ce = launch_pack_cols(MatView{A, lda, sA, M, K}, kBF16, batch, idx, k_keep, kp, A_S, status,
                                     wait_limit(), st);
@@ -582,7 +692,9 @@ rmm_status rmm_pack_w8(const void* A, int64_t lda, int64_t strideA, const int8_t
   if ((r = check_w8(Wq, ldw, strideW, scale, scale_stride, batch, K, N, false))) return r;
   if (batch == 0) return RMM_OK;
   if (!idx || (M > 0 && !A_S) || !B_S) return fail(RMM_ERR_INVALID, "idx, A_S or B_S is NULL");
-  if ((r = bind_device(stream))) return r;
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
+  if (debug_on() && (r = debug_check_indices(idx, batch, k_keep, K, "rmm_pack_w8", stream))) return r;
   return do_pack_w8(A, lda, strideA, Wq, ldw, strideW, scale, scale_stride, batch, M, K, N, idx, k_keep, A_S, B_S,
                     status_word, stream);
 }
@@ -617,7 +729,8 @@ rmm_status rmm_matmul_reduced_w8(const void* A, int64_t lda, int64_t strideA, co
   const size_t need = decode_route(M, 0) ? w.bytes_no_pack : w.bytes;
   if (workspace_bytes < need)
     return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
-  if ((r = bind_device(stream))) return r;
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
   cudaError_t ce = cudaSuccess;
   if (batch == 0) {
     ce = cudaMemsetAsync(w.status, 0, 4, stream);
@@ -631,22 +744,31 @@ rmm_status rmm_matmul_reduced_w8(const void* A, int64_t lda, int64_t strideA, co
   const bool gemv = decode_route(M, 0);
   SplitZero z;
   const bool zero = !gemv && gemm_tc_split_zero(g, &z);
-  ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr, gemv);
+  {
+    StageRange range("rmm select");
+    ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr, gemv);
+  }
   if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
   g.c_zeroed = zero ? 1 : 0;
-  if (M == 0 || N == 0) return RMM_OK;
-  if (gemv) return do_gemv_w8(A, lda, strideA, Wq, ldw, strideW, scale, scale_stride, batch, M, N, idx, k_keep, C,
-                              ldc, strideC, out, stream);
-  if ((r = do_pack_w8(A, lda, strideA, Wq, ldw, strideW, scale, scale_stride, batch, M, K, N, idx, k_keep, w.a_s,
-                      w.b_st, w.status, stream)))
-    return r;
-  return do_gemm(g, in, stream);
+  if (M == 0 || N == 0) return debug_on() ? debug_call_status(w.status, stream) : RMM_OK;
+  if (gemv) {
+    if ((r = do_gemv_w8(A, lda, strideA, Wq, ldw, strideW, scale, scale_stride, batch, M, N, idx, k_keep, C, ldc,
+                        strideC, out, stream)))
+      return r;
+  } else {
+    if ((r = do_pack_w8(A, lda, strideA, Wq, ldw, strideW, scale, scale_stride, batch, M, K, N, idx, k_keep, w.a_s,
+                        w.b_st, w.status, stream)))
+      return r;
+    if ((r = do_gemm(g, in, stream))) return r;
+  }
+  return debug_on() ? debug_call_status(w.status, stream) : RMM_OK;
 }
 
 static rmm_status do_gemv_w8(const void* A, int64_t lda, int64_t strideA, const int8_t* Wq, int64_t ldw,
                              int64_t strideW, const float* scale, int64_t scale_stride, int64_t batch, int64_t M,
                              int64_t N, const int32_t* idx, int64_t k_keep, void* C, int64_t ldc, int64_t strideC,
                              rmm_dtype out, cudaStream_t stream) {
+  StageRange range("rmm gather-gemv");
   GemvArgs v;
   v.a = A;
   v.b = Wq;
@@ -683,7 +805,9 @@ rmm_status rmm_gemv_gather_w8(const void* A, int64_t lda, int64_t strideA, const
   if (!layout_ok(batch, M, N, ldc, strideC)) return fail(RMM_ERR_INVALID, "C layout (ldc/strideC) is too small");
   if (batch == 0 || M == 0 || N == 0) return RMM_OK;
   if (!idx || !C) return fail(RMM_ERR_INVALID, "idx or C is NULL");
-  if ((r = bind_device(stream))) return r;
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
+  if (debug_on() && (r = debug_check_indices(idx, batch, k_keep, K, "rmm_gemv_gather_w8", stream))) return r;
   return do_gemv_w8(A, lda, strideA, Wq, ldw, strideW, scale, scale_stride, batch, M, N, idx, k_keep, C, ldc,
                     strideC, out, stream);
 }

@@ -8,6 +8,7 @@
 // workspace. The caller still passes A, B, C (and optionally idx_out and a
 // status word); this file calls no cudaMalloc, cudaFree or any allocating
 // routine.
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 
@@ -23,12 +24,27 @@ constexpr size_t kScratchBytes = size_t(32) << 20;
 // aligned window of kScratchBytes always fit.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes + 1024];
 
-struct DeviceScratch {
-  std::once_flag once;
-  void* base = nullptr;  // device address of g_noalloc_scratch on this device
-  cudaError_t err = cudaSuccess;
-};
-DeviceScratch g_scratch[64];
+constexpr int kMaxDevices = 64;
+// Device address of g_noalloc_scratch per device, once a lookup succeeded.
+// A failed lookup is not cached: the next call on that device tries again.
+std::atomic<void*> g_scratch_base[kMaxDevices];
+std::mutex g_scratch_mu;
+
+// The scratch array's device address on the current device `dev`.
+cudaError_t scratch_base(int dev, void** base) {
+  void* p = g_scratch_base[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    p = g_scratch_base[dev].load(std::memory_order_relaxed);
+    if (p == nullptr) {
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess || p == nullptr) return e != cudaSuccess ? e : cudaErrorInvalidSymbol;
+      g_scratch_base[dev].store(p, std::memory_order_release);
+    }
+  }
+  *base = p;
+  return cudaSuccess;
+}
 
 }  // namespace
 
@@ -49,26 +65,27 @@ extern "C" rmm_status rmm_matmul_reduced_noalloc(const void* A, int64_t lda, con
       return RMM_ERR_INVALID;
     }
   }
-  // Set up this device's scratch address once, with the stream's device current.
+  // Look up this device's scratch address with the stream's device current;
+  // the caller's current device is restored when the call returns.
+  rmm::DeviceGuard guard;
+  cudaError_t e = guard.bind(stream);
   int dev = -1;
-  cudaError_t e = cudaStreamGetDevice(stream, &dev);
-  if (e == cudaSuccess && (dev < 0 || dev >= 64)) e = cudaErrorInvalidDevice;
-  if (e == cudaSuccess) e = cudaSetDevice(dev);
+  if (e == cudaSuccess) e = cudaGetDevice(&dev);
+  if (e == cudaSuccess && (dev < 0 || dev >= kMaxDevices)) e = cudaErrorInvalidDevice;
   if (e != cudaSuccess) {
     snprintf(msg, sizeof(msg), "rmm_matmul_reduced_noalloc: selecting the stream's device: %s",
              cudaGetErrorString(e));
     rmm::set_last_error(msg);
     return RMM_ERR_CUDA;
   }
-  DeviceScratch& ds = g_scratch[dev];
-  std::call_once(ds.once, [&ds] { ds.err = cudaGetSymbolAddress(&ds.base, g_noalloc_scratch); });
-  if (ds.err != cudaSuccess || ds.base == nullptr) {
-    snprintf(msg, sizeof(msg), "rmm_matmul_reduced_noalloc: cudaGetSymbolAddress: %s",
-             cudaGetErrorString(ds.err));
+  void* base = nullptr;
+  e = scratch_base(dev, &base);
+  if (e != cudaSuccess) {
+    snprintf(msg, sizeof(msg), "rmm_matmul_reduced_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
     rmm::set_last_error(msg);
     return RMM_ERR_CUDA;
   }
-  void* ws = reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ds.base) + 1023) & ~uintptr_t(1023));
+  void* ws = reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(base) + 1023) & ~uintptr_t(1023));
   // The fused call clears the status word at the head of the scratch, then
   // validates every argument before it launches anything.
   rmm_status st = rmm_matmul_reduced(A, lda, B, ldb, M, K, N, rho, in, mode, C, ldc, out, idx_out, ws,

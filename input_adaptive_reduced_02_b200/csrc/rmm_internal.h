@@ -22,6 +22,33 @@ struct MatView {
 
 void count_launch();
 
+// Makes the stream's device current for the life of the guard and restores
+// the caller's current device when it goes out of scope (only if it changed).
+struct DeviceGuard {
+  int prev = -1;
+  DeviceGuard() = default;
+  DeviceGuard(const DeviceGuard&) = delete;
+  DeviceGuard& operator=(const DeviceGuard&) = delete;
+  // Returns the CUDA error of the lookup or switch (cudaSuccess on success).
+  cudaError_t bind(cudaStream_t st) {
+    int dev = -1;
+    cudaError_t e = cudaStreamGetDevice(st, &dev);
+    if (e != cudaSuccess) return e;
+    int cur = -1;
+    e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return e;
+    if (cur != dev) {
+      e = cudaSetDevice(dev);
+      if (e != cudaSuccess) return e;
+      if (prev < 0) prev = cur;
+    }
+    return cudaSuccess;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
 // Launch `kernel` on `st` with programmatic stream serialisation (the kernel
 // calls pdl_wait before touching global memory) and, if cluster.x > 0, that
 // thread-block cluster shape.

@@ -78,6 +78,7 @@ _SIGS = {
     "rmm_set_stall_producer_for_test": (None, [_i32]),
     "rmm_set_gemm_cta_group": (_i32, [_i32]),
     "rmm_launch_count": (_u64, []),
+    "rmm_set_debug": (_i32, [_i32]),
     "rmm_set_gemm_events": (None, [ctypes.c_void_p, ctypes.c_void_p]),
 }
 
@@ -521,6 +522,13 @@ def set_gemm_cta_group(cta_group: int) -> int:
 
 def launch_count() -> int:
     return int(lib().rmm_launch_count())
+
+
+def set_debug(on: bool) -> bool:
+    """Debug checks (kept indices validated on the device before a stage call
+    reads through them; fused calls report their device status directly).
+    Returns the previous setting."""
+    return bool(lib().rmm_set_debug(int(bool(on))))
 
 
 def set_gemm_events(start: torch.cuda.Event | None, stop: torch.cuda.Event | None):

@@ -70,6 +70,19 @@ def test_reference_arm_times_the_oracle_on_the_host():
     assert line["config"]["workload"] == "f32_64x256x64" and line["config"]["k_keep"] == 128
 
 
+def test_reference_arm_never_loads_the_library():
+    """The reference arm runs the oracle alone: its process maps no librmm.so
+    (k comes from the oracle's keep_count, not the library's)."""
+    code = ("import sys, json; sys.argv = ['bench.py']; import bench; "
+            "bench.main(['--impl', 'reference', '--steps', '1', '--warmup', '0', '--workload', 'f32_64x256x64']); "
+            "print(json.dumps({'maps_librmm': 'librmm.so' in open('/proc/self/maps').read()}))")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=600,
+                       env={**os.environ, "CUDA_VISIBLE_DEVICES": "", "PYTHONPATH": ROOT})
+    assert r.returncode == 0, r.stderr[-2000:]
+    last = json.loads(r.stdout.strip().splitlines()[-1])
+    assert last == {"maps_librmm": False}
+
+
 def test_reference_arm_follows_the_score_mode():
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0",
                         "--workload", "f32_64x256x64", "--score-mode", "a_only"], cwd=ROOT, capture_output=True,

@@ -3,17 +3,19 @@ that must not allocate device memory (for example code running under another
 framework's allocator, or a plugin handed only its input and output buffers).
 Its scratch is the library's static 32 MiB device array. Called here through
 the C ABI and compared with rmm_matmul_reduced (workspace form) on two calls
-in a row, so the second call runs on scratch the first one left behind."""
+in a row, so the second call runs on scratch the first one left behind:
+bit-identical output and indices, and the fp64 oracle's selection and
+product."""
 from __future__ import annotations
 
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
-from oracle import rmm_oracle as O
 from input_adaptive_reduced_02_b200 import rmm
+
+from _parity import check_single
 
 pytestmark = pytest.mark.gpu
 
@@ -52,9 +54,11 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(first, second):
         assert _call_noalloc(A, B, rho, C, idx, status) == rmm.RMM_OK, rmm.lib().rmm_last_error_string()
         rmm.check(status)
         torch.cuda.synchronize()
+        # same route, same kernels: identical bits, whatever the first call left in the scratch
         assert torch.equal(idx, idx_ref)
-        err = O.frobenius_rel_error(C.cpu().numpy().astype(np.float64), C_ref.cpu().numpy().astype(np.float64))
-        assert err <= 1e-2, err
+        assert torch.equal(C, C_ref)
+        # and the fp64 oracle's selection and product over the kept slices
+        check_single(A, B, rho, "product", C, idx)
 
 
 def test_noalloc_rejects_products_beyond_its_scratch():
