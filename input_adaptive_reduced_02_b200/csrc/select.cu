@@ -3,22 +3,31 @@
 // Reduction for LLM Inference": keep the k = ceil(rho·d) highest-scoring
 // indices). Ties go to the lower index; the kept indices come out ascending.
 //
-// One 1024-thread CTA per batch item. Scores become order-preserving 32-bit
-// keys in shared memory (up to 32768 of them; larger K re-reads the scores
-// from global memory, which stays in L2). The block's smallest and largest
-// keys share every bit above the highest bit where they differ, so an
-// MSB-first radix select starts there: 11-bit digits counted into one shared
-// histogram with shared-memory atomics, a block scan to find the bin of the
-// k-th largest key, and an early stop as soon as that bin is kept whole. Two
-// block-wide scans then compact the kept indices in index order (ties: the
-// lowest indices among keys equal to the threshold). Integer work only: the
-// result depends on the order of the scores, never on rounding.
+// One 512-thread CTA per batch item. Thread t holds the run of keys
+// [t·KPT, (t+1)·KPT) as order-preserving 32-bit keys in registers (K <= 32768,
+// loaded 16 bytes at a time; larger K re-reads the scores from global memory,
+// which stays in L2). The block's smallest and largest keys share every bit
+// above the highest bit where they differ, so an MSB-first radix select
+// starts there, 12 bits per pass:
+//  * histogram: each candidate key adds one to its digit's bin with a shared
+//    atomic (measured: warp-level merging of equal digits before the atomic,
+//    by match.any or by ballots, costs more in vote latency than it saves);
+//  * the bin of the k-th largest key: each thread sums 8 bins (top first), a
+//    warp scan plus a scan of the 16 warp totals locates the crossing thread;
+//  * the two histograms alternate, so clearing the next one needs no barrier
+//    of its own; three barriers per pass, and the passes stop as soon as the
+//    threshold bin is taken whole.
+// Compaction in index order: every thread counts, in its own run, the keys
+// above the threshold and those equal to it; one block scan of the two counts
+// packed in 64 bits gives each thread its first output slot and how many of
+// its equal keys are still kept (equal keys are kept lowest index first), and
+// the thread writes its kept indices in order. Integer work only: the result
+// depends on the order of the scores, never on rounding.
 //
 // Spare blocks of the same launch (in the fused call) zero the f32 C tiles
 // that the GEMM's split-K round reduce-adds into, while one SM per batch item
 // selects.
 #include <algorithm>
-#include <atomic>
 
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
@@ -26,7 +35,14 @@
 namespace rmm {
 namespace {
 
-constexpr int64_t kSelSmemKeys = 32768;
+constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kMaxKeysPerThread = 64;  // keys held in registers: K <= 32768
+constexpr int kDigitBits = 12;
+constexpr int kBins = 1 << kDigitBits;
+constexpr int kBinsPerThread = kBins / kSelThreads;
+static_assert(kBinsPerThread == 8, "the bin scan reads 8 bins per thread as two vectors");
+static_assert(kSelWarps <= 32, "warp totals are scanned by one warp");
 
 // Order-preserving map from f32 to u32 (larger score -> larger key), with
 // -0.0 folded onto +0.0 so that the two compare equal.
@@ -36,55 +52,219 @@ __device__ __forceinline__ uint32_t order_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive scan of one value per thread over the block; *total receives the sum.
-template <int THREADS>
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
-  constexpr int kWarps = THREADS / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t x = v;
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) warp_sums[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t w = lane < kWarps ? warp_sums[lane] : 0u;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    if (lane < kWarps) warp_sums[lane] = w;
-  }
-  __syncthreads();
-  const uint32_t before = (warp ? warp_sums[warp - 1] : 0u) + x - v;
-  *total = warp_sums[kWarps - 1];
-  __syncthreads();
-  return before;
+  return x;
 }
 
-constexpr int kSelThreads = 1024;
-constexpr int kDigitBits = 11;
-constexpr int kBins = 1 << kDigitBits;
+// Exclusive scan over the block of one 64-bit value per thread (used for two
+// packed 32-bit counts); `wtot` holds kSelWarps entries and is free on entry.
+__device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t* wtot, int lane, int warp) {
+  uint64_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wtot[warp] = x;
+  __syncthreads();
+  uint64_t w = lane < kSelWarps ? wtot[lane] : 0ull;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = __shfl_up_sync(0xffffffffu, w, o);
+    if (lane >= o) w += y;
+  }
+  const uint64_t wprev = __shfl_sync(0xffffffffu, w, (warp + 31) & 31);  // warps before this one
+  return (warp ? wprev : 0ull) + x - v;
+}
 
-template <int THREADS>
-__global__ void __launch_bounds__(THREADS, 1)
-select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t* __restrict__ idx,
-              uint32_t* status, int keys_in_smem, int64_t items, const SplitZero zero, int late_launch) {
-  constexpr int kWarps = THREADS / 32;
-  const int K = int(K64);  // K <= 2^21 (checked on the host)
-  extern __shared__ uint32_t keys[];  // K keys when keys_in_smem
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t warp_sums[32];
-  __shared__ uint32_t warp_min[kWarps], warp_max[kWarps];
-  __shared__ uint32_t sh_digit, sh_above, sh_count;
-  __shared__ int sh_nan;
-
+// KPT > 0: thread t holds keys [t·KPT, (t+1)·KPT) in registers (K <= 512·KPT);
+// KPT == 0: thread t owns [t·kpt, (t+1)·kpt), re-read from global memory in
+// every sweep (any K up to 2^21).
+template <int KPT>
+__device__ __forceinline__ void select_item(const float* __restrict__ sb, int K, int64_t k_keep,
+                                            int32_t* __restrict__ ib, uint32_t* status, uint32_t (*hist)[kBins],
+                                            uint32_t* wsum_a, uint32_t* wsum_b, uint64_t* wtot, uint32_t* sh) {
+  constexpr int R = KPT ? KPT : 1;  // register slots
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float* sb = s + int64_t(blockIdx.x) * K;
-  int32_t* ib = idx + int64_t(blockIdx.x) * k_keep;
+  const int kpt = KPT ? KPT : (K + kSelThreads - 1) / kSelThreads;  // keys per thread
+  const int base = tid * kpt;  // this thread's first key
+  uint32_t key[R] = {};
+  // key j of this thread (meaningful only when base + j < K)
+  auto key_of = [&](int j) -> uint32_t {
+    if constexpr (KPT > 0) {
+      return key[j];
+    } else {
+      return order_key(sb[base + j]);
+    }
+  };
+
+  // ---- keys, their min and max, non-finite check; hist[0] cleared meanwhile
+  {
+    uint4* h4 = reinterpret_cast<uint4*>(hist[0]);
+    for (int v = tid; v < kBins / 4; v += kSelThreads) h4[v] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  bool bad = false;
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  auto take_key = [&](int j, float x) {
+    bad |= !isfinite(x);
+    const uint32_t k = order_key(x);
+    if constexpr (KPT > 0) key[j] = k;
+    kmin = min(kmin, k);
+    kmax = max(kmax, k);
+  };
+  bool vec = false;
+  if constexpr (KPT > 0 && KPT % 4 == 0) {
+    // a whole run in range: 16-byte loads (a warp reads 128·KPT contiguous bytes)
+    vec = base + KPT <= K && (reinterpret_cast<uintptr_t>(sb) & 15u) == 0;
+    if (vec) {
+#pragma unroll
+      for (int j = 0; j < KPT; j += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(sb + base + j);
+        take_key(j, x.x);
+        take_key(j + 1, x.y);
+        take_key(j + 2, x.z);
+        take_key(j + 3, x.w);
+      }
+    }
+  }
+  if (!vec) {
+#pragma unroll
+    for (int j = 0; j < kpt; ++j)
+      if (base + j < K) take_key(j, sb[base + j]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  const bool bad_warp = __any_sync(0xffffffffu, bad);
+  if (lane == 0) {
+    wsum_a[warp] = kmin;
+    wsum_b[warp] = kmax;
+    if (bad_warp) status_or(status, RMM_NONFINITE_BIT);
+  }
+  __syncthreads();
+  kmin = lane < kSelWarps ? wsum_a[lane] : 0xFFFFFFFFu;
+  kmax = lane < kSelWarps ? wsum_b[lane] : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (k_keep >= K) {  // everything is kept
+    for (int i = tid; i < K; i += kSelThreads) ib[i] = i;
+    return;
+  }
+
+  // ---- MSB-first radix select over the bits in which the keys differ. After
+  // each pass, `prefix` (under `mask`) is the digit string of the k-th largest
+  // key so far and `remaining` the number of keys still to take among those
+  // matching it.
+  const uint32_t diff = kmin ^ kmax;
+  int hi = diff ? 31 - __clz(diff) : -1;  // highest unresolved bit
+  uint32_t mask = hi >= 0 ? uint32_t(~((uint64_t(2) << hi) - 1)) : 0xFFFFFFFFu;
+  uint32_t prefix = kmin & mask, remaining = uint32_t(k_keep), bin_count = uint32_t(K);
+  int buf = 0;
+  while (hi >= 0) {
+    const int width = min(kDigitBits, hi + 1);
+    const int shift = hi - width + 1;
+    const uint32_t dmask = (1u << width) - 1u;
+    uint32_t* h = hist[buf];
+    {  // the other histogram was last read before the previous pass's final barrier
+      uint4* h4 = reinterpret_cast<uint4*>(hist[buf ^ 1]);
+      for (int v = tid; v < kBins / 4; v += kSelThreads) h4[v] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < kpt; ++j) {
+      if (base + j < K) {
+        const uint32_t k = key_of(j);
+        if ((k & mask) == prefix) atomicAdd(&h[(k >> shift) & dmask], 1u);
+      }
+    }
+    __syncthreads();
+    // thread t holds bins kBins-1-8t .. kBins-8-8t (top first)
+    const uint4 hi4 = reinterpret_cast<const uint4*>(h)[kBins / 4 - 1 - 2 * tid];
+    const uint4 lo4 = reinterpret_cast<const uint4*>(h)[kBins / 4 - 2 - 2 * tid];
+    const uint32_t cnt[8] = {hi4.w, hi4.z, hi4.y, hi4.x, lo4.w, lo4.z, lo4.y, lo4.x};
+    uint32_t c = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) c += cnt[q];
+    const uint32_t incl = warp_incl_scan(c, lane);
+    if (lane == 31) wsum_a[warp] = incl;
+    __syncthreads();
+    uint32_t wv = lane < kSelWarps ? wsum_a[lane] : 0u;
+    wv = warp_incl_scan(wv, lane);
+    const uint32_t wprev = __shfl_sync(0xffffffffu, wv, (warp + 31) & 31);  // warps before this one
+    uint32_t acc = (warp ? wprev : 0u) + incl - c;
+    if (acc < remaining && remaining <= acc + c) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (acc + cnt[q] >= remaining) {
+          sh[0] = uint32_t(kBins - 1 - 8 * tid - q);
+          sh[1] = acc;
+          sh[2] = cnt[q];
+          break;
+        }
+        acc += cnt[q];
+      }
+    }
+    __syncthreads();
+    prefix |= sh[0] << shift;
+    mask |= dmask << shift;
+    remaining -= sh[1];
+    bin_count = sh[2];
+    buf ^= 1;
+    // every key in the chosen bin is kept: no finer threshold is needed
+    if (remaining == bin_count) break;
+    hi = shift - 1;
+  }
+
+  // ---- compaction in index order. Kept: keys whose masked bits exceed
+  // `prefix`, plus the `remaining` lowest-indexed keys whose masked bits equal
+  // it (all of them when the bin is taken whole). Each thread counts both
+  // kinds in its run; one block scan of the packed counts (equal keys in the
+  // upper half) gives every thread its output slot and its share of equal keys.
+  const uint32_t T = prefix, need_eq = remaining;
+  const bool take_all_eq = remaining == bin_count;
+  uint32_t n_gt = 0, n_eq = 0;
+#pragma unroll
+  for (int j = 0; j < kpt; ++j) {
+    if (base + j < K) {
+      const uint32_t k = key_of(j) & mask;
+      n_gt += k > T;
+      n_eq += k == T;
+    }
+  }
+  // wtot is only ever used here (after the passes' barriers, or the first barrier)
+  const uint64_t before = block_excl_scan64((uint64_t(n_eq) << 32) | n_gt, wtot, lane, warp);
+  const uint32_t eq_before = uint32_t(before >> 32), gt_before = uint32_t(before);
+  uint32_t eq_left = take_all_eq ? n_eq : (eq_before >= need_eq ? 0u : min(n_eq, need_eq - eq_before));
+  uint32_t pos = gt_before + (take_all_eq ? eq_before : min(eq_before, need_eq));
+#pragma unroll
+  for (int j = 0; j < kpt; ++j) {
+    if (base + j < K) {
+      const uint32_t k = key_of(j) & mask;
+      const bool tk = k > T || (k == T && eq_left > 0);
+      if (k == T && eq_left > 0) --eq_left;
+      if (tk) ib[pos++] = base + j;
+    }
+  }
+}
+
+template <int KPT>
+__global__ void __launch_bounds__(kSelThreads, 1)
+select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t* __restrict__ idx,
+              uint32_t* status, int64_t items, const SplitZero zero, int late_launch) {
+  const int K = int(K64);  // K <= 2^21 (checked on the host)
+  __shared__ __align__(16) uint32_t hist[2][kBins];
+  __shared__ uint32_t wsum_a[kSelWarps], wsum_b[kSelWarps];
+  __shared__ uint64_t wtot[kSelWarps];
+  __shared__ uint32_t sh[3];
 
   // late_launch: the next kernel (a gather-GEMV in clusters of CTAs with
   // large shared memory) is released only once the previous kernel has
@@ -95,200 +275,11 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
   pdl_wait();
   if (late_launch) pdl_trigger();
   if (blockIdx.x >= items) {  // helper block: zero C tiles for the GEMM later on the stream
-    zero_split_tiles(zero, blockIdx.x - items, gridDim.x - items, tid, THREADS);
+    zero_split_tiles(zero, blockIdx.x - items, gridDim.x - items, threadIdx.x, kSelThreads);
     return;
   }
-  if (tid == 0) sh_nan = 0;
-  __syncthreads();
-  bool nan_seen = false;
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  if (keys_in_smem && (K & 3) == 0 && (reinterpret_cast<uintptr_t>(sb) & 15u) == 0) {
-    const float4* s4 = reinterpret_cast<const float4*>(sb);
-    for (int i = tid; i < K / 4; i += THREADS) {
-      const float4 x = s4[i];
-      nan_seen |= !isfinite(x.x) | !isfinite(x.y) | !isfinite(x.z) | !isfinite(x.w);
-      const uint4 k4 = make_uint4(order_key(x.x), order_key(x.y), order_key(x.z), order_key(x.w));
-      kmin = min(min(kmin, min(k4.x, k4.y)), min(k4.z, k4.w));
-      kmax = max(max(kmax, max(k4.x, k4.y)), max(k4.z, k4.w));
-      reinterpret_cast<uint4*>(keys)[i] = k4;
-    }
-  } else {
-    for (int i = tid; i < K; i += THREADS) {
-      const float x = sb[i];
-      nan_seen |= !isfinite(x);
-      const uint32_t k = order_key(x);
-      kmin = min(kmin, k);
-      kmax = max(kmax, k);
-      if (keys_in_smem) keys[i] = k;
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-  }
-  if (lane == 0) {
-    warp_min[warp] = kmin;
-    warp_max[warp] = kmax;
-  }
-  if (nan_seen) sh_nan = 1;
-  __syncthreads();
-  if (tid == 0 && sh_nan) status_or(status, RMM_NONFINITE_BIT);
-  kmin = warp_min[0];
-  kmax = warp_max[0];
-  for (int w = 1; w < kWarps; ++w) {
-    kmin = min(kmin, warp_min[w]);
-    kmax = max(kmax, warp_max[w]);
-  }
-
-  if (k_keep >= K) {  // everything is kept
-    for (int i = tid; i < K; i += THREADS) ib[i] = i;
-    return;
-  }
-
-  // MSB-first radix select over the bits in which the keys differ: every key
-  // shares the bits of kmin above the highest bit where kmin and kmax differ,
-  // so the first histogram already spreads the keys over many bins. After
-  // each pass, `prefix` (under `mask`) is the digit string of the k-th largest
-  // key so far and `remaining` the number of keys still to take among those
-  // matching it.
-  const uint32_t diff = kmin ^ kmax;
-  int hi = diff ? 31 - __clz(diff) : -1;  // highest unresolved bit
-  uint32_t mask = hi >= 0 ? uint32_t(~((uint64_t(2) << hi) - 1)) : 0xFFFFFFFFu;
-  uint32_t prefix = kmin & mask, remaining = uint32_t(k_keep), bin_count = uint32_t(K);
-  while (hi >= 0) {
-    const int width = min(kDigitBits, hi + 1);
-    const int shift = hi - width + 1;
-    const uint32_t dmask = (1u << width) - 1u;
-    for (int b = tid; b < kBins; b += THREADS) hist[b] = 0u;
-    __syncthreads();
-    for (int i = tid; i < K; i += THREADS) {
-      const uint32_t key = keys_in_smem ? keys[i] : order_key(sb[i]);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
-    }
-    __syncthreads();
-    // descending scan to find the bin of the k-th key: thread t owns bins
-    // kBins-1-2t and kBins-2-2t
-    uint32_t c0 = 0, c1 = 0;
-    if (tid < kBins / 2) {
-      c0 = hist[kBins - 1 - 2 * tid];
-      c1 = hist[kBins - 2 - 2 * tid];
-    }
-    uint32_t all;
-    const uint32_t excl = block_exclusive_scan<THREADS>(c0 + c1, warp_sums, &all);
-    if (tid < kBins / 2 && excl < remaining && remaining <= excl + c0 + c1) {
-      if (excl + c0 >= remaining) {
-        sh_digit = uint32_t(kBins - 1 - 2 * tid);
-        sh_above = excl;
-        sh_count = c0;
-      } else {
-        sh_digit = uint32_t(kBins - 2 - 2 * tid);
-        sh_above = excl + c0;
-        sh_count = c1;
-      }
-    }
-    __syncthreads();
-    prefix |= sh_digit << shift;
-    mask |= dmask << shift;
-    remaining -= sh_above;
-    bin_count = sh_count;
-    // every key in the chosen bin is kept: no finer threshold is needed
-    if (remaining == bin_count) break;
-    hi = shift - 1;
-  }
-  // Kept: keys whose masked bits exceed `prefix`, plus the `remaining`
-  // lowest-indexed keys whose masked bits equal it (all of them when the bin
-  // is taken whole). Larger K: warp w compacts the contiguous chunk w of the
-  // keys, 32 consecutive keys per step (conflict-free shared-memory reads; a
-  // contiguous run per thread would read 32 runs in one bank), in two sweeps:
-  // counts, then writes at offsets from a scan over the warps' counts.
-  const uint32_t T = prefix, need_eq = remaining;
-  const bool take_all_eq = remaining == bin_count;
-  if (K <= 4 * THREADS) {
-    // up to 4 keys per thread: a contiguous run each and two block scans
-    // (measured faster than the warp sweeps below at this size)
-    const int per = (K + THREADS - 1) / THREADS;
-    const int lo = min(K, tid * per), hi_i = min(K, lo + per);
-    uint32_t c_gt = 0, c_eq = 0;
-    for (int i = lo; i < hi_i; ++i) {
-      const uint32_t k = (keys_in_smem ? keys[i] : order_key(sb[i])) & mask;
-      c_gt += (k > T);
-      c_eq += (k == T);
-    }
-    uint32_t total, eq_take = c_eq;
-    if (!take_all_eq) {
-      const uint32_t eq_before = block_exclusive_scan<THREADS>(c_eq, warp_sums, &total);
-      eq_take = eq_before >= need_eq ? 0u : min(c_eq, need_eq - eq_before);
-    }
-    uint32_t pos = block_exclusive_scan<THREADS>(c_gt + eq_take, warp_sums, &total);
-    uint32_t taken_eq = 0;
-    for (int i = lo; i < hi_i; ++i) {
-      const uint32_t k = (keys_in_smem ? keys[i] : order_key(sb[i])) & mask;
-      if (k > T) {
-        ib[pos++] = i;
-      } else if (k == T && taken_eq < eq_take) {
-        ib[pos++] = i;
-        ++taken_eq;
-      }
-    }
-    return;
-  }
-  const int chunk = (K + kWarps - 1) / kWarps;
-  const int w_lo = min(K, warp * chunk), w_hi = min(K, w_lo + chunk);
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  uint32_t n_gt = 0, n_eq = 0;
-  for (int base = w_lo; base < w_hi; base += 32) {
-    const int i = base + lane;
-    const bool valid = i < w_hi;
-    const uint32_t k = valid ? ((keys_in_smem ? keys[i] : order_key(sb[i])) & mask) : 0u;
-    n_gt += __popc(__ballot_sync(0xffffffffu, valid && k > T));
-    n_eq += __popc(__ballot_sync(0xffffffffu, valid && k == T));
-  }
-  // exclusive scans over the warps (in warp order) of the equal counts and of
-  // the kept counts; warp_min/warp_max are free again (the barrier covers the
-  // case without radix passes, where they were last read for kmin/kmax)
-  __syncthreads();
-  if (lane == 0) {
-    warp_min[warp] = n_eq;
-    warp_max[warp] = n_gt;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const uint32_t e = lane < kWarps ? warp_min[lane] : 0u, g = lane < kWarps ? warp_max[lane] : 0u;
-    uint32_t e_incl = e;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, e_incl, o);
-      if (lane >= o) e_incl += y;
-    }
-    const uint32_t e_before = e_incl - e;
-    const uint32_t take = take_all_eq ? e : (e_before >= need_eq ? 0u : min(e, need_eq - e_before));
-    uint32_t k_incl = g + take;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, k_incl, o);
-      if (lane >= o) k_incl += y;
-    }
-    if (lane < kWarps) {
-      warp_min[lane] = take;                  // equal keys this warp keeps
-      warp_max[lane] = k_incl - (g + take);   // first output slot of this warp
-    }
-  }
-  __syncthreads();
-  const uint32_t eq_take = warp_min[warp];
-  uint32_t pos = warp_max[warp], eq_seen = 0;
-  for (int base = w_lo; base < w_hi; base += 32) {
-    const int i = base + lane;
-    const bool valid = i < w_hi;
-    const uint32_t k = valid ? ((keys_in_smem ? keys[i] : order_key(sb[i])) & mask) : 0u;
-    const bool gt = valid && k > T, eq = valid && k == T;
-    const uint32_t eq_mask = __ballot_sync(0xffffffffu, eq);
-    const bool take = gt || (eq && eq_seen + __popc(eq_mask & lt_mask) < eq_take);
-    const uint32_t t_mask = __ballot_sync(0xffffffffu, take);
-    if (take) ib[pos + __popc(t_mask & lt_mask)] = i;
-    pos += __popc(t_mask);
-    eq_seen += __popc(eq_mask);
-  }
+  select_item<KPT>(s + int64_t(blockIdx.x) * K, K, k_keep, idx + int64_t(blockIdx.x) * k_keep, status, hist,
+                   wsum_a, wsum_b, wtot, sh);
 }
 
 }  // namespace
@@ -301,21 +292,23 @@ cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_ke
   if (zero && zero->count > 0) {
     z = *zero;
     const int64_t vecs = z.count * z.tile_rows * (z.tile_cols / 4);
-    helpers = std::min<int64_t>(147, (vecs + 8 * kSelThreads - 1) / (8 * kSelThreads));
+    helpers = std::min<int64_t>(147, (vecs + 16 * kSelThreads - 1) / (16 * kSelThreads));
   }
-  const int keys_in_smem = K <= kSelSmemKeys;
-  const size_t smem = keys_in_smem ? size_t(K) * 4 : 0;
-  static std::atomic<bool> attr_done[64];  // per device; racing first calls both set the attribute
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel<kSelThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(kSelSmemKeys * 4));
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
-  }
-  return launch_pdl(select_kernel<kSelThreads>, dim3(unsigned(batch + helpers)), dim3(kSelThreads), smem, st,
-                    dim3(0, 0, 0), s, K, k_keep, idx, status, keys_in_smem, batch, z, int(late_launch));
+  const dim3 grid(unsigned(batch + helpers)), block(kSelThreads), none(0, 0, 0);
+  const int ll = int(late_launch);
+  const int64_t kpt = (K + kSelThreads - 1) / kSelThreads;
+  if (kpt <= 1) return launch_pdl(select_kernel<1>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
+  if (kpt <= 2) return launch_pdl(select_kernel<2>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
+  if (kpt <= 4) return launch_pdl(select_kernel<4>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
+  if (kpt <= 8) return launch_pdl(select_kernel<8>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
+  if (kpt <= 16)
+    return launch_pdl(select_kernel<16>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
+  if (kpt <= 32)
+    return launch_pdl(select_kernel<32>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
+  if (kpt <= kMaxKeysPerThread)
+    return launch_pdl(select_kernel<kMaxKeysPerThread>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch,
+                      z, ll);
+  return launch_pdl(select_kernel<0>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
 }
 
 }  // namespace rmm
