@@ -21,6 +21,7 @@ Prints one JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import datetime
 import hashlib
 import json
@@ -90,6 +91,22 @@ class Problem:
     def gemv(self):
         """Decode shape: the library streams B's kept rows without packing."""
         return self.M <= 16 and not self.b_kmajor
+
+    @property
+    def stream(self):
+        """Narrow product (N <= 128, bf16): the library zeroes B's dropped rows
+        and streams A whole through the GEMM instead of packing A (the route
+        rule is the library's; a tensor without device memory counts as aligned)."""
+        if self.scale is not None or self.gemv:
+            return False
+        A3 = self.A if self.A.dim() == 3 else self.A.unsqueeze(0)
+        b, M, K = A3.shape
+        lda = A3.stride(1) if M > 1 else K
+        sA = A3.stride(0) if b > 1 else M * lda
+        ptr = self.A.data_ptr() if self.A.is_cuda else 0
+        dt = rmm.RMM_BF16 if self.A.dtype == torch.bfloat16 else rmm.RMM_F32
+        return rmm.lib().rmm_fused_route(b, M, self.N, int(self.b_kmajor), dt, ctypes.c_void_p(ptr), lda,
+                                         sA) == rmm.ROUTE_STREAM
 
     def k_keep(self, rho):
         return self.keep_count(rho, self.K)
@@ -166,14 +183,21 @@ class Pipeline:
         shp = (lambda r, c: (p.batch, r, c)) if p.A.dim() == 3 else (lambda r, c: (r, c))
         self.s = torch.empty((p.batch, p.K) if p.A.dim() == 3 else (p.K,), dtype=torch.float32, device=dev)
         self.idx_store = torch.empty(p.batch * kmax, dtype=torch.int32, device=dev)
-        self.a_store = torch.empty(p.batch * p.M * kp, dtype=p.A.dtype, device=dev)
-        self.b_store = torch.empty(p.batch * kp * max(p.N, rmm.packed_b_ld(p.N)), dtype=p.A.dtype, device=dev)
+        if p.stream:  # B with its dropped rows zeroed; A is read as it is
+            self.a_store = None
+            self.b_mask = torch.empty(shp(p.K, rmm.packed_b_ld(p.N)), dtype=p.A.dtype, device=dev)
+        else:
+            self.a_store = torch.empty(p.batch * p.M * kp, dtype=p.A.dtype, device=dev)
+            self.b_store = torch.empty(p.batch * kp * max(p.N, rmm.packed_b_ld(p.N)), dtype=p.A.dtype, device=dev)
         self.C = torch.empty(shp(p.M, p.N), dtype=p.out_dtype, device=dev)
         self.status = rmm.status_word(dev)
 
     def views(self, rho):
         p = self.p
         k = p.k_keep(rho)
+        if p.stream:
+            idx = self.idx_store[: p.batch * k].view(p.batch, k) if p.A.dim() == 3 else self.idx_store[:k]
+            return k, idx, None, None
         kp = rmm.padded_keep(k)
         bshape = rmm.packed_b_shape(p.A.dim() == 3, p.batch, p.N, kp, p.b_kmajor)
         nb = 1
@@ -220,7 +244,9 @@ class Pipeline:
             if ev:
                 ev[4 if breakdown else 2].record()
             return
-        if p.scale is not None:
+        if p.stream:  # the stream route: B's dropped rows zeroed, then the GEMM over all of A
+            rmm.mask_rows(p.B, idx, out=self.b_mask)
+        elif p.scale is not None:
             rmm.pack_w8(p.A, p.B, p.scale, idx, out=(A_S, B_S), status=self.status)
         else:
             rmm.pack(p.A, p.B, idx, p.b_kmajor, out=(A_S, B_S), status=self.status)
@@ -230,7 +256,10 @@ class Pipeline:
             # the library records these immediately around the GEMM kernel
             # (after the split-K zeroing kernel rmm_gemm may launch first)
             rmm.set_gemm_events(ev[1], ev[2])
-        rmm.gemm(A_S, B_S, k, b_kmajor=p.b_kmajor, N=p.N, out=self.C, status=self.status)
+        if p.stream:
+            rmm.gemm_full(p.A, self.b_mask, p.N, out=self.C, status=self.status)
+        else:
+            rmm.gemm(A_S, B_S, k, b_kmajor=p.b_kmajor, N=p.N, out=self.C, status=self.status)
         if ev and breakdown:
             ev[4].record()
         elif ev:
@@ -290,7 +319,7 @@ def timed_steps(pipe, rho: float, steps: int, flush, breakdown=False):
     Returns (per-step ms, per-stage ms lists). For the staged Pipeline without
     breakdown the stages are {"pre_gemm": score+select+pack, "gemm": gemm};
     for the Fused call {"call": the whole call}."""
-    fused = isinstance(pipe, Fused)
+    fused = isinstance(pipe, (Fused, Dense))
     n_ev = 2 if fused else (5 if breakdown else 3)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)]
     for i in range(steps):
@@ -302,6 +331,26 @@ def timed_steps(pipe, rho: float, steps: int, flush, breakdown=False):
     names = ("call",) if fused else (STAGES if breakdown else ("pre_gemm", "gemm"))
     stage_ms = {s: [e[j].elapsed_time(e[j + 1]) for e in evs] for j, s in enumerate(names)}
     return step_ms, stage_ms
+
+
+class Dense:
+    """The dense product of the same shapes through torch (cuBLAS bf16/f32),
+    timed like the step: context for the reduced call, not part of it."""
+
+    def __init__(self, p: Problem):
+        self.p = p
+        B = p.B
+        if p.scale is not None:
+            B = (B.float() * p.scale[None, :]).to(torch.bfloat16)
+        self.B = B.transpose(-1, -2) if p.b_kmajor else B
+        self.C = None
+
+    def step(self, rho, ev=None, breakdown=False):
+        if ev:
+            ev[0].record()
+        self.C = torch.matmul(self.p.A, self.B)
+        if ev:
+            ev[1].record()
 
 
 # ----------------------------------------------------------------- clocks
@@ -567,6 +616,19 @@ def run_ours(args):
         sweep = {f"{r:g}": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in d.items()}
                  for r, d in sweep.items()}
 
+    # the dense product of the same shapes (cuBLAS through torch), for context
+    dense = None
+    if not args.no_sweep:
+        dn = Dense(p)
+        for _ in range(3):
+            dn.step(1.0)
+        dms, _ = timed_steps(dn, 1.0, max(10, args.steps // 2), flush)
+        d_ms = statistics.median(dms)
+        dense = {"ms": round(d_ms, 5), "impl": "torch.matmul (cuBLAS), dense over all K",
+                 "reduced_call_speedup": {r: round(d_ms / v["ms"], 4) for r, v in sweep.items()}}
+        del dn
+        torch.cuda.empty_cache()
+
     gemm_ms_timed = statistics.mean(stage_ms["gemm"])
     # per-stage breakdown (separate pass: events between stages cost the overlap)
     _, bd = timed_steps(pipe, rho, max(10, args.steps // 2), flush, breakdown=True)
@@ -629,6 +691,8 @@ def run_ours(args):
                                  "comes from a second timed loop of the same step made of the four stage "
                                  "calls, with events before and after the GEMM launch; the stage breakdown "
                                  "from a third pass with events between all stages"},
+            "step_ms_spread": {"min": round(min(step_ms), 5), "median": round(statistics.median(step_ms), 5),
+                               "max": round(max(step_ms), 5)},
             "stages_ms": {s: round(v, 5) for s, v in stage_mean.items()},
             "stages_gbs": stage_gbs(p, rho, stage_mean),
             "cached_b_norm_call": cached,
@@ -640,6 +704,7 @@ def run_ours(args):
             "gemm_ms_max_over_ranks": round(gemm_ms_max, 5),
             "roofline": roof,
             "sweep": sweep,
+            "dense_reference": dense,
             "e2e": e2e,
             "gpu_launches": int(launches),
             "clocks": clk,
@@ -661,6 +726,14 @@ def stage_bytes(p: Problem, rho):
     wb = 1 if p.scale is not None else eb  # bytes per element of B as stored (INT8 codes)
     b_read = 0 if (p.mode == "a_only" or p.b_norm is not None) else p.K * p.N * wb
     ldb = p.N if p.b_kmajor else rmm.packed_b_ld(p.N)
+    if p.stream:  # mask: k rows of B read, K rows written; GEMM: all of A, B_M and C
+        ldm = rmm.packed_b_ld(p.N)
+        return {
+            "score": (p.M * p.K * eb + b_read + 4 * p.K) * p.batch,
+            "select": (4 * p.K + 4 * k) * p.batch,
+            "pack": (k * p.N * eb + p.K * ldm * eb) * p.batch,
+            "gemm": (p.M * p.K * eb + p.K * ldm * eb + p.M * p.N * ob) * p.batch,
+        }
     if p.gemv:  # no pack; the GEMV reads k rows of B, k columns of A, writes C
         return {
             "score": (p.M * p.K * eb + b_read + 4 * p.K) * p.batch,
@@ -748,6 +821,8 @@ def roofline(p: Problem, rho, stage_mean, dominant, peaks, peak_src):
                 "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
                 "algorithmic_bytes_per_launch": gemm_bytes,
+                "bytes_note": ("stream route: all of A (its kept columns reach nearly every 32-byte sector), "
+                               "B with dropped rows zeroed, C" if p.stream else "kept operands and C"),
                 "arithmetic_intensity": round(p.kept_flops(rho) / gemm_bytes, 1), "ridge": round(ridge, 1),
                 "peak_source": f"{peak_src} HBM copy bandwidth"}
     if dominant == "gemm" and p.M >= 128 and p.N >= 128:

@@ -89,13 +89,20 @@ size_t rmm_workspace_size(int64_t batch, int64_t M, int64_t K, int64_t N, int64_
                           rmm_dtype in);
 
 /* The workspace a fused call needs for the route it takes with these sizes
- * and B's layout (b_kmajor as in rmm_score; 0 for the INT8-weight call): with
- * M <= 16 and B row-major the call streams B's kept rows through the
- * gather-GEMV and packs nothing, so the status word, scores and indices are
- * all it uses (for x[1][8192] · W[8192][28672] at rho = 0.5: 49 KiB instead
- * of 224 MiB); otherwise it equals rmm_workspace_size. The fused calls accept
- * any workspace of at least this size; the layout of what they use does not
- * change. */
+ * and B's layout (b_kmajor as in rmm_score; 0 for the INT8-weight call; see
+ * rmm_fused_route):
+ *   - gather-GEMV (M <= 16, B row-major): the status word, scores and indices
+ *     only (for x[1][8192] · W[8192][28672] at rho = 0.5: 49 KiB instead of
+ *     224 MiB);
+ *   - stream (bf16, B row-major, N <= 128, M > 16): those plus B with its
+ *     dropped rows zeroed, [batch][K][rmm_packed_b_ld(N)] (P·V at S = 32768,
+ *     32 heads, rho = 0.5: 256 MiB instead of 34 GiB of packed operands). This
+ *     assumes A can be streamed (16-byte aligned base, row pitch and batch
+ *     stride multiples of 8 elements); an A that cannot takes the pack route,
+ *     which needs rmm_workspace_size;
+ *   - pack: the packed operands A_S and B_S as well.
+ * The fused calls accept any workspace of at least this size; the layout of
+ * what they use does not change. */
 size_t rmm_workspace_size_for(int64_t batch, int64_t M, int64_t K, int64_t N, int64_t k_keep,
                               rmm_dtype in, int b_kmajor);
 
@@ -167,10 +174,47 @@ rmm_status rmm_gemm(const void* A_S, const void* B_S, int b_kmajor, int64_t batc
                     int64_t N, int64_t k_keep, rmm_dtype in, void* C, int64_t ldc, int64_t strideC,
                     rmm_dtype out, uint32_t* status_word, cudaStream_t stream);
 
+/* B_M = B with the rows outside the kept set zeroed ("Mecanismo Central":
+ * A[:, I]·B[I, :] = A·B_M, since a dropped slice then contributes zero):
+ *   B: [batch][K][N] row-major (ldb, strideB; strideB = 0 shares one B);
+ *   idx: [batch][k_keep] ascending kept indices in [0, K) (as rmm_select
+ *   writes them); B_M: [batch][K][rmm_packed_b_ld(N)] output, 16-byte aligned,
+ *   B_M[b][r][j] = B[b][r][j] if r is in idx[b], else 0; columns N <= j <
+ *   rmm_packed_b_ld(N) are 0. Copies bits exactly. With debug checks on,
+ *   idx is validated first (see rmm_set_debug). */
+rmm_status rmm_mask_rows(const void* B, int64_t ldb, int64_t strideB, int64_t batch, int64_t K, int64_t N,
+                         const int32_t* idx, int64_t k_keep, rmm_dtype in, void* B_M, cudaStream_t stream);
+
+/* C[b] = A[b] · B_M[b] over all K slices on the bf16 tensor cores (f32
+ * accumulation): with B_M from rmm_mask_rows this is the reduced product
+ * A[:, I]·B[I, :] computed by streaming A whole, the fused calls' route for
+ * narrow products (rmm_fused_route).
+ *   A: [batch][M][K] row-major, bf16, 16-byte aligned, lda and (batch > 1)
+ *   strideA multiples of 8 and strideA nonzero (RMM_ERR_INVALID otherwise);
+ *   B_M: [batch][K][rmm_packed_b_ld(N)], 16-byte aligned; C as in rmm_gemm.
+ *   in must be RMM_BF16 (RMM_ERR_UNSUPPORTED otherwise). */
+rmm_status rmm_gemm_full(const void* A, int64_t lda, int64_t strideA, const void* B_M, int64_t batch, int64_t M,
+                         int64_t K, int64_t N, rmm_dtype in, void* C, int64_t ldc, int64_t strideC, rmm_dtype out,
+                         uint32_t* status_word, cudaStream_t stream);
+
+/* Which route a fused call (rmm_matmul_reduced, _batched, _b_norms,
+ * rmm_qk_reduced, rmm_pv_reduced) takes for these sizes and this A:
+ *   2 = gather-GEMV (M <= 16 and B row-major: score, select, rmm_gemv_gather);
+ *   1 = stream (bf16, B row-major, N <= 128, M > 16, A streamable as in
+ *       rmm_gemm_full: score, select, rmm_mask_rows, rmm_gemm_full). A
+ *       narrow product is bound by reading A, and A's kept columns reach into
+ *       nearly every 32-byte sector of A, so streaming A once beats packing
+ *       it (read A, write and re-read A_S);
+ *   0 = pack (score, select, rmm_pack, rmm_gemm);
+ *  -1 for invalid sizes or dtype. Host only; never launches anything. */
+int rmm_fused_route(int64_t batch, int64_t M, int64_t N, int b_kmajor, rmm_dtype in, const void* A, int64_t lda,
+                    int64_t strideA);
+
 /* ---------------------------------------------------------------- fused calls */
 
 /* Y ≈ A·B with the top ceil(rho·K) contraction slices kept: score → select →
- * pack → gemm, all enqueued on `stream`.
+ * the product over the kept slices (pack + gemm, or the stream or
+ * gather-GEMV route, see rmm_fused_route), all enqueued on `stream`.
  *   A [M][K] (ld lda), B [K][N] (ld ldb), C [M][N] (ld ldc); dtypes in/out.
  *   idx_out: nullable device [k_keep] i32 that receives the kept indices.
  *   workspace: device buffer of at least rmm_workspace_size_for(1, M, K, N, k,

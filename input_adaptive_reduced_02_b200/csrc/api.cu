@@ -166,15 +166,46 @@ struct Workspace {
   uint32_t* status;
   float* s;
   int32_t* idx;
-  void* a_s;
+  void* a_s;             // pack route: A_S, then B_S
   void* b_st;
+  void* b_m;             // stream route: B with its dropped rows zeroed [batch][K][packed_b_ld(N)]
   size_t bytes;          // every route
+  size_t bytes_pack;     // the pack route: status, scores, indices, A_S, B_S
+  size_t bytes_stream;   // the stream route: status, scores, indices, B_M
   size_t bytes_no_pack;  // the decode route (no packed operands): status, scores, indices
+};
+
+// How a fused call computes the product over the kept slices.
+enum Route {
+  kRoutePack = 0,    // pack A's kept columns and B's kept rows, tensor-core GEMM over k slices
+  kRouteStream = 1,  // zero B's dropped rows, tensor-core GEMM over all K slices of A as given
+  kRouteGemv = 2,    // a few rows of A: gather-GEMV straight from A and B
 };
 
 // The fused calls stream B's kept rows straight into the gather-GEMV, with no
 // packed operands, for a few rows of A and a row-major B.
 static bool decode_route(int64_t M, int b_kmajor) { return M <= kGemvMaxRows && !b_kmajor; }
+
+// Narrow products (N <= 128: one column tile of the GEMM) are bound by reading
+// A, and A's kept columns reach into nearly every 32-byte sector of A, so
+// packing A (read A, write and re-read A_S: (1 + 2·rho)·|A| bytes) costs more
+// than streaming A whole through the GEMM with B's dropped rows zeroed
+// (|A| bytes; the extra multiply-adds by zero stay below the tensor-core
+// time of reading A). The GEMM reads A by TMA, so A must be 16-byte aligned
+// with a row pitch and batch stride that are multiples of 8 elements.
+static bool stream_shape(int64_t M, int64_t N, int b_kmajor, rmm_dtype in) {
+  return in == RMM_BF16 && !b_kmajor && N <= 128 && M > kGemvMaxRows;
+}
+static bool stream_layout_ok(const void* A, int64_t lda, int64_t strideA, int64_t batch) {
+  return (reinterpret_cast<uintptr_t>(A) & 15u) == 0 && lda % 8 == 0 &&
+         (batch == 1 || (strideA % 8 == 0 && strideA != 0));
+}
+static Route choose_route(int64_t batch, int64_t M, int64_t N, int b_kmajor, rmm_dtype in, const void* A,
+                          int64_t lda, int64_t strideA) {
+  if (decode_route(M, b_kmajor)) return kRouteGemv;
+  if (stream_shape(M, N, b_kmajor, in) && stream_layout_ok(A, lda, strideA, batch)) return kRouteStream;
+  return kRoutePack;
+}
 
 static Workspace carve(void* base, int64_t batch, int64_t M, int64_t K, int64_t N, int64_t k_keep, rmm_dtype in) {
   const int64_t kp = round_up(k_keep, 64);
@@ -190,11 +221,16 @@ static Workspace carve(void* base, int64_t batch, int64_t M, int64_t K, int64_t 
   w.idx = reinterpret_cast<int32_t*>(p + off);
   off += al(batch * k_keep * 4);
   w.bytes_no_pack = size_t(off);
+  const int64_t ops = off;
   w.a_s = reinterpret_cast<void*>(p + off);
   off += al(batch * M * kp * eb);
   w.b_st = reinterpret_cast<void*>(p + off);
   off += al(batch * packed_b_ld(N) * kp * eb);
-  w.bytes = size_t(off);
+  w.bytes_pack = size_t(off);
+  w.b_m = reinterpret_cast<void*>(p + ops);
+  w.bytes_stream = size_t(ops + al(batch * K * packed_b_ld(N) * eb));
+  // every route these sizes can take (the stream route needs bf16, N <= 128, M > 16)
+  w.bytes = in == RMM_BF16 && N <= 128 && M > kGemvMaxRows ? std::max(w.bytes_pack, w.bytes_stream) : w.bytes_pack;
   return w;
 }
 
@@ -237,6 +273,16 @@ static rmm_status do_pack(const void* A, int64_t lda, int64_t sA, const void* B,
   return RMM_OK;
 }
 
+// B_M = B with the rows outside idx zeroed, [batch][K][packed_b_ld(N)].
+static rmm_status do_mask(const void* B, int64_t ldb, int64_t sB, int64_t batch, int64_t K, int64_t N,
+                          const int32_t* idx, int64_t k_keep, rmm_dtype in, void* B_M, cudaStream_t st) {
+  StageRange range("rmm mask");
+  const cudaError_t ce = launch_mask_rows(MatView{B, ldb, sB, K, N}, kind(in), batch, idx, k_keep, B_M, packed_b_ld(N),
+                                          st);
+  if (ce != cudaSuccess) return cuda_fail(ce, "mask kernel");
+  return RMM_OK;
+}
+
 static GemmArgs gemm_args(const void* A_S, const void* B_S, int b_kmajor, int64_t batch, int64_t M, int64_t N,
                           int64_t k_keep, void* C, int64_t ldc, int64_t sC, rmm_dtype out, uint32_t* status) {
   GemmArgs g;
@@ -249,6 +295,8 @@ static GemmArgs gemm_args(const void* A_S, const void* B_S, int b_kmajor, int64_
   g.M = M;
   g.N = N;
   g.k_pad = round_up(k_keep, 64);
+  g.lda = g.k_pad;
+  g.strideA = g.k_pad * M;
   g.ldc = ldc;
   g.strideC = sC;
   g.out = kind(out);
@@ -347,7 +395,14 @@ size_t rmm_workspace_size_for(int64_t batch, int64_t M, int64_t K, int64_t N, in
                               int b_kmajor) {
   if (batch < 0 || M < 0 || K < 0 || N < 0 || k_keep < 0 || !dtype_ok(in)) return 0;
   const Workspace w = carve(nullptr, batch, M, K, N, k_keep, in);
-  return decode_route(M, b_kmajor) ? w.bytes_no_pack : w.bytes;
+  if (decode_route(M, b_kmajor)) return w.bytes_no_pack;
+  return stream_shape(M, N, b_kmajor, in) ? w.bytes_stream : w.bytes_pack;
+}
+
+int rmm_fused_route(int64_t batch, int64_t M, int64_t N, int b_kmajor, rmm_dtype in, const void* A, int64_t lda,
+                    int64_t strideA) {
+  if (batch < 0 || M < 0 || N < 0 || !dtype_ok(in)) return -1;
+  return int(choose_route(batch, M, N, b_kmajor, in, A, lda, strideA));
 }
 
 rmm_status rmm_score(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb, int64_t strideB,
@@ -420,6 +475,45 @@ rmm_status rmm_gemm(const void* A_S, const void* B_S, int b_kmajor, int64_t batc
   return do_gemm(gemm_args(A_S, B_S, b_kmajor, batch, M, N, k_keep, C, ldc, strideC, out, status_word), in, stream);
 }
 
+rmm_status rmm_mask_rows(const void* B, int64_t ldb, int64_t strideB, int64_t batch, int64_t K, int64_t N,
+                         const int32_t* idx, int64_t k_keep, rmm_dtype in, void* B_M, cudaStream_t stream) {
+  rmm_status r = check_common(batch, 1, K, N, in);
+  if (r) return r;
+  if (k_keep < 1 || k_keep > K) return fail(RMM_ERR_INVALID, "k_keep must be in [1, K]");
+  if (batch > 0 && N > 0 && !B) return fail(RMM_ERR_INVALID, "B is NULL");
+  if (!layout_ok(batch, K, N, ldb, strideB, true)) return fail(RMM_ERR_INVALID, "B layout (ldb/strideB) is too small");
+  if (batch == 0) return RMM_OK;
+  if (!idx || !B_M) return fail(RMM_ERR_INVALID, "idx or B_M is NULL");
+  if (reinterpret_cast<uintptr_t>(B_M) & 15u) return fail(RMM_ERR_INVALID, "B_M must be 16-byte aligned");
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
+  if (debug_on() && (r = debug_check_indices(idx, batch, k_keep, K, "rmm_mask_rows", stream))) return r;
+  return do_mask(B, ldb, strideB, batch, K, N, idx, k_keep, in, B_M, stream);
+}
+
+rmm_status rmm_gemm_full(const void* A, int64_t lda, int64_t strideA, const void* B_M, int64_t batch, int64_t M,
+                         int64_t K, int64_t N, rmm_dtype in, void* C, int64_t ldc, int64_t strideC, rmm_dtype out,
+                         uint32_t* status_word, cudaStream_t stream) {
+  if (!dtype_ok(in) || !dtype_ok(out)) return fail(RMM_ERR_INVALID, "unknown dtype");
+  if (in != RMM_BF16) return fail(RMM_ERR_UNSUPPORTED, "rmm_gemm_full runs on the bf16 tensor cores only");
+  if (batch < 0 || M < 0 || N < 0 || K < 1) return fail(RMM_ERR_INVALID, "need batch, M, N >= 0 and K >= 1");
+  if (batch > kMaxGridBatch) return fail(RMM_ERR_UNSUPPORTED, "batch > %lld", (long long)kMaxGridBatch);
+  if (!layout_ok(batch, M, K, lda, strideA)) return fail(RMM_ERR_INVALID, "A layout (lda/strideA) is too small");
+  if (!layout_ok(batch, M, N, ldc, strideC)) return fail(RMM_ERR_INVALID, "C layout (ldc/strideC) is too small");
+  if (batch == 0 || M == 0 || N == 0) return RMM_OK;
+  if (!A || !B_M || !C) return fail(RMM_ERR_INVALID, "A, B_M or C is NULL");
+  if (!stream_layout_ok(A, lda, strideA, batch))
+    return fail(RMM_ERR_INVALID, "A must be 16-byte aligned with a row pitch and batch stride that are multiples of 8");
+  DeviceGuard dg;
+  rmm_status r = bind_device(stream, dg);
+  if (r) return r;
+  GemmArgs g = gemm_args(A, B_M, 0, batch, M, N, K, C, ldc, strideC, out, status_word);
+  g.lda = lda;
+  g.strideA = strideA;
+  g.k_pad = K;
+  return do_gemm(g, in, stream);
+}
+
 static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb,
                              int64_t strideB, int b_kmajor, const float* bn, int64_t bn_stride, int64_t batch,
                              int64_t M, int64_t K, int64_t N, double rho, rmm_dtype in, rmm_score_mode mode, void* C,
@@ -438,9 +532,14 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
   if (!workspace) return fail(RMM_ERR_INVALID, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(workspace) & 1023u) return fail(RMM_ERR_INVALID, "workspace must be 1 KiB aligned");
   const Workspace w = carve(workspace, batch, M, K, N, k_keep, in);
-  const size_t need = decode_route(M, b_kmajor) ? w.bytes_no_pack : w.bytes;
+  const Route route = choose_route(batch, M, N, b_kmajor, in, A, lda, strideA);
+  const size_t need = route == kRouteGemv ? w.bytes_no_pack : route == kRouteStream ? w.bytes_stream : w.bytes_pack;
   if (workspace_bytes < need)
-    return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes%s", workspace_bytes, need,
+                route == kRoutePack && stream_shape(M, N, b_kmajor, in)
+                    ? " (A's layout does not allow streaming it: 16-byte aligned base, row pitch and batch stride "
+                      "multiples of 8 elements)"
+                    : "");
   DeviceGuard dg;
   if ((r = bind_device(stream, dg))) return r;
   cudaError_t ce = cudaSuccess;
@@ -457,9 +556,16 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
   // split-K round adds into are zeroed meanwhile by helper blocks of the same
   // launch instead of by a launch of their own.
   GemmArgs g = gemm_args(w.a_s, w.b_st, b_kmajor, batch, M, N, k_keep, C, ldc, strideC, out, w.status);
+  if (route == kRouteStream) {  // the GEMM contracts over all of A with B's dropped rows zeroed
+    g.a = A;
+    g.lda = lda;
+    g.strideA = strideA;
+    g.k_pad = K;
+    g.b = w.b_m;
+  }
   // A few rows of A (decode): the product streams B's kept rows straight
   // through idx, with no packed copy.
-  const bool gemv = decode_route(M, b_kmajor);
+  const bool gemv = route == kRouteGemv;
   SplitZero z;
   const bool zero = !gemv && in == RMM_BF16 && gemm_tc_split_zero(g, &z);
   {
@@ -474,9 +580,12 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
       return r;
     return debug_on() ? debug_call_status(w.status, stream) : RMM_OK;
   }
-  if ((r = do_pack(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, idx, k_keep, in, w.a_s, w.b_st,
-                   w.status, stream)))
+  if (route == kRouteStream) {
+    if ((r = do_mask(B, ldb, strideB, batch, K, N, idx, k_keep, in, w.b_m, stream))) return r;
+  } else if ((r = do_pack(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, idx, k_keep, in, w.a_s,
+                          w.b_st, w.status, stream))) {
     return r;
+  }
   if ((r = do_gemm(g, in, stream))) return r;
   return debug_on() ? debug_call_status(w.status, stream) : RMM_OK;
 }

@@ -507,7 +507,7 @@ Plan make_plan(const GemmArgs& g, int sms, bool c_tma) {
   q.bm = BM * cg;
   q.tiles_m = int32_t((g.M + q.bm - 1) / q.bm);
   q.tiles_n = int32_t((g.N + q.bn - 1) / q.bn);
-  q.num_kb = int32_t(g.k_pad / BK);
+  q.num_kb = int32_t((g.k_pad + BK - 1) / BK);
   q.total_tiles = int64_t(q.tiles_m) * q.tiles_n * g.batch;
   q.units = std::max<int64_t>(1, (sms > 0 ? sms : 148) / cg);
   q.rem = q.total_tiles % q.units;
@@ -536,8 +536,10 @@ cudaError_t launch_cfg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, co
   using Cfg = TcCfg<BN, CG>;
   const uint64_t kp = uint64_t(g.k_pad);
   CUtensorMap tmA, tmB, tmC;
-  bool ok = encode_3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.a, kp, uint64_t(g.M), uint64_t(g.batch), kp * 2,
-                      kp * 2 * uint64_t(g.M), BK, BM);
+  // a batch of one takes any batch stride (TMA needs a nonzero multiple of 16 bytes)
+  const uint64_t sA = g.batch == 1 ? uint64_t(g.lda) * 2 * uint64_t(g.M) : uint64_t(g.strideA) * 2;
+  bool ok = encode_3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.a, kp, uint64_t(g.M), uint64_t(g.batch),
+                      uint64_t(g.lda) * 2, sA == 0 ? 16 : sA, BK, BM);
   if (BMN) {
     const uint64_t ldb = uint64_t(g.ldb);
     ok = ok && encode_3d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.b, uint64_t(g.N), kp, uint64_t(g.batch), ldb * 2,
@@ -626,7 +628,11 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st, const char** why)
     return cudaErrorNoKernelImageForDevice;
   }
   if ((reinterpret_cast<uintptr_t>(g.a) & 15u) || (reinterpret_cast<uintptr_t>(g.b) & 15u)) {
-    *why = "packed operands must be 16-byte aligned";
+    *why = "the operands must be 16-byte aligned";
+    return cudaErrorInvalidValue;
+  }
+  if ((uint64_t(g.lda) * 2) % 16 != 0 || (g.batch > 1 && (uint64_t(g.strideA) * 2) % 16 != 0)) {
+    *why = "A's row pitch and batch stride must be multiples of 8 elements";
     return cudaErrorInvalidValue;
   }
   if (g.M > INT32_MAX || g.N > INT32_MAX || g.k_pad > INT32_MAX || g.batch > INT32_MAX) {

@@ -573,3 +573,89 @@ cudaError_t launch_pack_rows_w8(const int8_t* Wq, int64_t ldw, int64_t sW, const
 }
 
 }  // namespace rmm
+
+// ------------------------------------------------------------------ masked rows
+// B with its dropped rows zeroed, for the route that streams A whole: A[:, I]
+// · B[I, :] = A · B_M with B_M[r] = B[r] for r in I and 0 otherwise.
+namespace rmm {
+namespace {
+
+constexpr int kMaskSeg = 64;  // kept indices per CTA
+
+// CTA c owns kept positions [c·64, c·64 + 64) of item b and the rows from its
+// first kept index (row 0 for c = 0) up to the next CTA's first kept index
+// (K for the last CTA): kept rows are copied, the rows between them zeroed,
+// columns N <= j < ldo zeroed. A warp per row, 16-byte vectors when the rows
+// of X are 16-byte aligned.
+template <typename T>
+__global__ void __launch_bounds__(kPackThreads)
+mask_rows_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t K, int64_t N,
+                 const int32_t* __restrict__ idx, int64_t k_keep, T* __restrict__ out, int64_t ldo, int vec) {
+  constexpr int V = 16 / sizeof(T);
+  __shared__ int32_t seg[kMaskSeg + 1];
+  const int64_t b = blockIdx.y;
+  const int64_t t0 = int64_t(blockIdx.x) * kMaskSeg;
+  const int64_t t1 = min(k_keep, t0 + kMaskSeg);
+  const int32_t* ib = idx + b * k_keep;
+  pdl_trigger();
+  pdl_wait();
+  if (threadIdx.x <= t1 - t0) seg[threadIdx.x] = threadIdx.x < t1 - t0 ? ib[t0 + threadIdx.x] : 0;
+  __syncthreads();
+  const int64_t r_lo = t0 == 0 ? 0 : seg[0];
+  const int64_t r_hi = t1 == k_keep ? K : int64_t(ib[t1]);
+  const int n = int(t1 - t0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const T* Xb = X + b * bstride;
+  T* Ob = out + b * K * ldo;
+  // kept rows of the segment come in ascending order: walk them with the rows
+  int p = 0;  // first segment entry >= r (all warps walk the same rows in the same order)
+  for (int64_t r0 = r_lo; r0 < r_hi; r0 += kPackThreads / 32) {
+    const int64_t r = r0 + warp;
+    // advance p to the first kept index >= r0 (the same for every warp)
+    while (p < n && seg[p] < r0) ++p;
+    if (r >= r_hi) continue;
+    bool kept = false;
+    for (int q = p; q < n && seg[q] <= r; ++q) kept |= seg[q] == r;
+    T* dst = Ob + r * ldo;
+    if (vec) {
+      const int64_t nv = ldo / V;  // ldo is a multiple of V when vec
+      for (int64_t j = lane; j < nv; j += 32) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (kept && (j + 1) * V <= N) v = *reinterpret_cast<const uint4*>(Xb + r * ld + j * V);
+        else if (kept) {
+          alignas(16) T tmp[V];
+#pragma unroll
+          for (int e = 0; e < V; ++e) tmp[e] = j * V + e < N ? Xb[r * ld + j * V + e] : T(0);
+          v = *reinterpret_cast<const uint4*>(tmp);
+        }
+        *reinterpret_cast<uint4*>(dst + j * V) = v;
+      }
+    } else {
+      for (int64_t j = lane; j < ldo; j += 32) dst[j] = (kept && j < N) ? Xb[r * ld + j] : T(0);
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_mask_rows_t(const MatView& X, int64_t batch, const int32_t* idx, int64_t k_keep, void* out,
+                               int64_t ldo, cudaStream_t st) {
+  constexpr int V = 16 / sizeof(T);
+  const int vec = (reinterpret_cast<uintptr_t>(X.ptr) & 15u) == 0 && (X.ld % V) == 0 &&
+                  (batch == 1 || X.bstride % V == 0) && (reinterpret_cast<uintptr_t>(out) & 15u) == 0 &&
+                  ldo % V == 0;
+  const int64_t ctas = (k_keep + kMaskSeg - 1) / kMaskSeg;
+  return launch_pdl(mask_rows_kernel<T>, dim3(unsigned(ctas), unsigned(batch)), dim3(kPackThreads), 0, st,
+                    dim3(0, 0, 0), static_cast<const T*>(X.ptr), X.ld, X.bstride, X.rows, X.cols, idx, k_keep,
+                    static_cast<T*>(out), ldo, vec);
+}
+
+}  // namespace
+
+cudaError_t launch_mask_rows(const MatView& X, ElemKind e, int64_t batch, const int32_t* idx, int64_t k_keep,
+                             void* out, int64_t ldo, cudaStream_t st) {
+  if (batch == 0 || X.rows == 0) return cudaSuccess;
+  return e == kBF16 ? launch_mask_rows_t<uint16_t>(X, batch, idx, k_keep, out, ldo, st)
+                    : launch_mask_rows_t<uint32_t>(X, batch, idx, k_keep, out, ldo, st);
+}
+
+}  // namespace rmm

@@ -128,6 +128,11 @@ cudaError_t launch_pack_rows(const MatView& X, ElemKind e, int64_t batch, const 
                              int64_t k_keep, int64_t k_pad, void* out, int64_t ldo, uint32_t* status,
                              uint64_t wait_ns, cudaStream_t st);
 
+//  out[b][r][:] = X[b][r][:] for r in idx[b], zero for the other rows r < K
+//  (X.rows = K), row pitch ldo >= cols, columns cols <= j < ldo zero.
+cudaError_t launch_mask_rows(const MatView& X, ElemKind e, int64_t batch, const int32_t* idx, int64_t k_keep,
+                             void* out, int64_t ldo, cudaStream_t st);
+
 //  Both packs (A's columns, B's rows) in one launch when both take the bulk
 //  paths and A's rows are at most 32 KB; *handled reports whether it did.
 cudaError_t launch_pack_both(const MatView& A, const MatView& B, ElemKind e, int64_t batch, const int32_t* idx,
@@ -145,12 +150,18 @@ cudaError_t launch_pack_rows_w8(const int8_t* Wq, int64_t ldw, int64_t sW, const
 
 // gemm_tc.cu (bf16 tensor cores) / gemm_simt.cu (f32 CUDA cores)
 struct GemmArgs {
-  const void* a;  // [batch][M][k_pad]
+  const void* a;  // [batch][M][k_pad] packed, or a caller's A (lda, strideA)
   const void* b;  // b_kmajor: [batch][N][k_pad]; else [batch][k_pad][ldb]
   int b_kmajor;
   int64_t ldb;    // row pitch of the N-major B operand (elements)
   void* c;        // [batch][M][N] (ldc, strideC)
   int64_t batch, M, N, k_pad, ldc, strideC;
+  // A's row pitch and batch stride (elements); the packed operands have
+  // lda = k_pad and strideA = M·k_pad. The tensor-core GEMM contracts over the
+  // first k_pad slices; a caller's A with K not a multiple of 64 passes
+  // k_pad = K (its tensor maps read zeros past K). The CUDA-core GEMM takes
+  // packed operands only.
+  int64_t lda, strideA;
   ElemKind out;
   uint32_t* status;
   uint64_t wait_limit_ns;

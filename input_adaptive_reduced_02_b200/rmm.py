@@ -72,6 +72,9 @@ _SIGS = {
                                      _vp]),
     "rmm_gemv_gather_w8": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _i64,
                                   _vp, _i64, _i64, _i32, _vp]),
+    "rmm_mask_rows": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _vp]),
+    "rmm_gemm_full": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _i32, _vp, _i64, _i64, _i32, _vp, _vp]),
+    "rmm_fused_route": (_i32, [_i64, _i64, _i64, _i32, _i32, _vp, _i64, _i64]),
     "rmm_check": (_i32, [_vp, _vp]),
     "rmm_last_error_string": (ctypes.c_char_p, []),
     "rmm_set_wait_limit_ns": (None, [_u64]),
@@ -344,6 +347,47 @@ def gemv_gather(A: torch.Tensor, B: torch.Tensor, idx: torch.Tensor, out_dtype=t
     return out
 
 
+ROUTE_PACK, ROUTE_STREAM, ROUTE_GEMV = 0, 1, 2
+
+
+def fused_route(A: torch.Tensor, N: int, b_kmajor: bool = False) -> int:
+    """Route a fused call takes for A (2-D or 3-D) and N: ROUTE_PACK,
+    ROUTE_STREAM (B's dropped rows zeroed, A streamed whole) or ROUTE_GEMV."""
+    ba, M, K, lda, sA = _mat(A, "A")
+    return int(lib().rmm_fused_route(ba, M, N, int(b_kmajor), _dtype(A), _ptr(A), lda, sA))
+
+
+def _fused_ws_bytes(A: torch.Tensor, N: int, k: int, b_kmajor: bool) -> int:
+    """Workspace of a fused call on the route it takes for this A."""
+    ba, M, K, _, _ = _mat(A, "A")
+    if fused_route(A, N, b_kmajor) == ROUTE_PACK:
+        return workspace_size(ba, M, K, N, k, A.dtype)
+    return workspace_size_for(ba, M, K, N, k, A.dtype, b_kmajor)
+
+
+def mask_rows(B: torch.Tensor, idx: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """B_M = B with the rows outside idx zeroed: [(b)][K][packed_b_ld(N)]."""
+    bb, K, N, ldb, sB = _mat(B, "B")
+    k = idx.shape[-1]
+    if out is None:
+        shp = (K, packed_b_ld(N))
+        out = torch.empty((bb, *shp) if B.dim() == 3 else shp, dtype=B.dtype, device=B.device)
+    _check(lib().rmm_mask_rows(_ptr(B), ldb, sB, bb, K, N, _ptr(idx), k, _dtype(B), _ptr(out), _stream(B)))
+    return out
+
+
+def gemm_full(A: torch.Tensor, B_M: torch.Tensor, N: int, out_dtype=torch.float32, out: torch.Tensor | None = None,
+              status: torch.Tensor | None = None) -> torch.Tensor:
+    """C = A · B_M over all K slices (bf16 tensor cores), B_M as mask_rows writes it."""
+    ba, M, K, lda, sA = _mat(A, "A")
+    if out is None:
+        out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
+    _, _, _, ldc, sC = _mat(out, "C")
+    _check(lib().rmm_gemm_full(_ptr(A), lda, sA, _ptr(B_M), ba, M, K, N, _dtype(A), _ptr(out), ldc, sC,
+                               _out_code(out.dtype), _ptr(status), _stream(A)))
+    return out
+
+
 # ---------------------------------------------------------------- fused calls
 def matmul_reduced(A: torch.Tensor, B: torch.Tensor, rho: float, mode: str = "product",
                    out_dtype=torch.float32, out: torch.Tensor | None = None, workspace: Workspace | None = None,
@@ -356,7 +400,7 @@ def matmul_reduced(A: torch.Tensor, B: torch.Tensor, rho: float, mode: str = "pr
     bb, r, c, ldb, sB = _mat(B, "B")
     N = r if b_kmajor else c
     k = keep_count(rho, K)
-    ws = _ensure_ws(workspace, workspace_size_for(ba, M, K, N, k, A.dtype, b_kmajor), A.device)
+    ws = _ensure_ws(workspace, _fused_ws_bytes(A, N, k, b_kmajor), A.device)
     if out is None:
         out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
     _, _, _, ldc, sC = _mat(out, "C")
@@ -377,7 +421,7 @@ def matmul_reduced_b_norms(A: torch.Tensor, B: torch.Tensor, b_norm: torch.Tenso
     N = r if b_kmajor else c
     stride = _bn_stride(b_norm, ba, K)
     k = keep_count(rho, K)
-    ws = _ensure_ws(workspace, workspace_size_for(ba, M, K, N, k, A.dtype, b_kmajor), A.device)
+    ws = _ensure_ws(workspace, _fused_ws_bytes(A, N, k, b_kmajor), A.device)
     if out is None:
         out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
     _, _, _, ldc, sC = _mat(out, "C")
@@ -482,7 +526,7 @@ def qk_reduced(Q: torch.Tensor, Kmat: torch.Tensor, rho: float, mode: str = "pro
     bh, S_q, d = Q.shape
     S_k = Kmat.shape[1]
     k = keep_count(rho, d)
-    ws = _ensure_ws(workspace, workspace_size_for(bh, S_q, d, S_k, k, Q.dtype, True), Q.device)
+    ws = _ensure_ws(workspace, _fused_ws_bytes(Q, S_k, k, True), Q.device)
     if out is None:
         out = torch.empty(bh, S_q, S_k, dtype=out_dtype, device=Q.device)
     _check(lib().rmm_qk_reduced(_ptr(Q), _ptr(Kmat), bh, S_q, S_k, d, float(rho), _dtype(Q), SCORE_MODES[mode],
@@ -498,7 +542,7 @@ def pv_reduced(P: torch.Tensor, V: torch.Tensor, rho: float, mode: str = "produc
     bh, S_q, S_k = P.shape
     d = V.shape[2]
     k = keep_count(rho, S_k)
-    ws = _ensure_ws(workspace, workspace_size_for(bh, S_q, S_k, d, k, P.dtype), P.device)
+    ws = _ensure_ws(workspace, _fused_ws_bytes(P, d, k, False), P.device)
     if out is None:
         out = torch.empty(bh, S_q, d, dtype=out_dtype, device=P.device)
     _check(lib().rmm_pv_reduced(_ptr(P), _ptr(V), bh, S_q, S_k, d, float(rho), _dtype(P), SCORE_MODES[mode],

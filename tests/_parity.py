@@ -17,11 +17,13 @@ Element-wise bound. Let y = sum_t a_t b_t over the k kept slices (exact, fp64
 oracle) and S = sum_t |a_t| |b_t| (the entry of |A_S|·|B_S|). The library
 forms every product exactly in f32 (bf16 x bf16, and bf16 x int8, fit in 24
 significant bits; f32 x f32 products are fused into the FMA) and adds the k
-products in f32 along some tree whose height is at most k + 16 (tensor-core
-K-groups, split-K reduce-adds, cluster partial sums). Each addition errs by
-at most 2u relative (u = 2^-24; the factor 2 admits accumulators that
-truncate instead of rounding to nearest), so the f32 result obeys
-    |y_f32 - y| <= E = g·S,   g = 2u·(k + 16) / (1 - 2u·(k + 16)).
+products in f32 along some tree whose height is at most K + 16, K the full
+contraction length (tensor-core K-groups, split-K reduce-adds, cluster
+partial sums; the route that streams A whole adds the dropped slices as
+exact zeros). Each addition errs by at most 2u relative (u = 2^-24; the
+factor 2 admits accumulators that truncate instead of rounding to nearest),
+so the f32 result obeys
+    |y_f32 - y| <= E = g·S,   g = 2u·(K + 16) / (1 - 2u·(K + 16)).
 A final scaling (the INT8 column scale) and the store add at most
 2u·(|y| + E); rounding the result to bf16 adds at most 2^-8·(|y| + E) (bf16
 has 8 significant bits, round to nearest even); weights rounded to bf16
@@ -39,7 +41,7 @@ WINDOW = 1e-5
 U_F32 = 2.0 ** -24   # unit roundoff of f32 (24 significant bits, round to nearest)
 U_BF16 = 2.0 ** -8   # unit roundoff of bf16 (8 significant bits, round to nearest even)
 ACC_FACTOR = 2.0     # per-addition error in units of U_F32 (truncating accumulation allowed)
-TREE_SLACK = 16      # extra levels of the summation tree beyond k
+TREE_SLACK = 16      # extra levels of the summation tree beyond K
 
 
 def f64(t: torch.Tensor) -> np.ndarray:
@@ -82,12 +84,14 @@ def check_selection(idx_gpu: np.ndarray, s_ref: np.ndarray, k_keep: int) -> int:
     return n
 
 
-def element_bound(A_S: np.ndarray, B_S: np.ndarray, ref: np.ndarray, out_bf16: bool, w_rel: float = 0.0):
+def element_bound(A_S: np.ndarray, B_S: np.ndarray, ref: np.ndarray, out_bf16: bool, w_rel: float = 0.0,
+                  K: int | None = None):
     """Largest admissible |C - ref| per entry for the f32-accumulated product
-    of the kept operands A_S (M x k) and B_S (k x N); see the module docstring."""
-    k = A_S.shape[1]
+    of the kept operands A_S (M x k) and B_S (k x N) out of K slices; see the
+    module docstring."""
+    K = A_S.shape[1] if K is None else K
     S = np.abs(A_S) @ np.abs(B_S)
-    h = ACC_FACTOR * U_F32 * (k + TREE_SLACK)
+    h = ACC_FACTOR * U_F32 * (K + TREE_SLACK)
     E = (h / (1.0 - h)) * S
     mag = np.abs(ref) + E
     bound = E + 2.0 * U_F32 * mag + w_rel * S
@@ -120,7 +124,7 @@ def check_product(C_gpu, A64: np.ndarray, B64: np.ndarray, idx: np.ndarray, tol:
     assert np.all(np.isfinite(C_gpu)), "non-finite product entries"
     err = O.frobenius_rel_error(C_gpu, ref)
     assert err <= tol, f"product rel Frobenius error {err:.3e} > {tol}"
-    bound = element_bound(A64[:, I], B64[I, :], ref, out_dtype == torch.bfloat16, w_rel)
+    bound = element_bound(A64[:, I], B64[I, :], ref, out_dtype == torch.bfloat16, w_rel, K=A64.shape[1])
     excess = np.abs(C_gpu - ref) - bound
     if np.any(excess > 0):
         i, j = np.unravel_index(int(np.argmax(excess)), excess.shape)

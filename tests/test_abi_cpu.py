@@ -71,6 +71,47 @@ def test_workspace_size_for_the_decode_route():
     assert rmm.workspace_size_for(3, 16, K, N, k, rmm.torch.float32) == al(4) + al(3 * K * 4) + al(3 * k * 4)
 
 
+def test_workspace_size_for_the_stream_route():
+    """bf16, B row-major, N <= 128, M > 16 (P·V): the fused calls stream A whole
+    and need B with its dropped rows zeroed, [batch][K][packed_b_ld(N)],
+    instead of the packed operands; rmm_workspace_size covers both routes."""
+    al = lambda x: (x + 1023) // 1024 * 1024  # noqa: E731
+    bh, S, d, rho = 32, 32768, 128, 0.5
+    k = rmm.keep_count(rho, S)
+    stream = rmm.workspace_size_for(bh, S, S, d, k, rmm.torch.bfloat16)
+    head = al(4) + al(bh * S * 4) + al(bh * k * 4)
+    assert stream == head + al(bh * S * d * 2)
+    pack = head + al(bh * S * k * 2) + al(bh * k * d * 2)
+    assert rmm.workspace_size(bh, S, S, d, k, rmm.torch.bfloat16) == max(pack, stream) == pack
+    assert stream < pack / 100
+    # f32, a K-major B or N > 128 take the pack route
+    assert rmm.workspace_size_for(bh, S, S, d, k, rmm.torch.bfloat16, b_kmajor=True) == pack
+    assert rmm.workspace_size_for(1, 300, 1000, 129, 500, rmm.torch.bfloat16) == \
+        rmm.workspace_size(1, 300, 1000, 129, 500, rmm.torch.bfloat16)
+    # few rows of A and a wide K: the stream operand is the larger one
+    M, K, N, k = 17, 8192, 128, 4096
+    s2 = rmm.workspace_size_for(1, M, K, N, k, rmm.torch.bfloat16)
+    assert s2 == al(4) + al(K * 4) + al(k * 4) + al(K * N * 2)
+    assert rmm.workspace_size(1, M, K, N, k, rmm.torch.bfloat16) == s2
+
+
+def test_fused_route_rule():
+    """rmm_fused_route: the gather-GEMV for M <= 16 with B row-major, the stream
+    route for narrow bf16 products whose A can be streamed, the pack route
+    otherwise; it only inspects the pointer's alignment."""
+    L = rmm.lib()
+    a = V(1 << 20)
+    assert L.rmm_fused_route(1, 16, 4096, 0, 0, a, 4096, 0) == 2
+    assert L.rmm_fused_route(32, 8192, 128, 0, 0, a, 8192, 8192 * 8192) == 1
+    assert L.rmm_fused_route(32, 8192, 128, 0, 1, a, 8192, 8192 * 8192) == 0   # f32
+    assert L.rmm_fused_route(32, 8192, 128, 1, 0, a, 8192, 8192 * 8192) == 0   # K-major B
+    assert L.rmm_fused_route(32, 8192, 129, 0, 0, a, 8192, 8192 * 8192) == 0   # wider than one tile
+    assert L.rmm_fused_route(1, 700, 128, 0, 0, a, 700, 0) == 0                # row pitch not 16 bytes
+    assert L.rmm_fused_route(1, 700, 128, 0, 0, V((1 << 20) + 2), 704, 0) == 0  # base not 16-byte aligned
+    assert L.rmm_fused_route(2, 700, 128, 0, 0, a, 704, 0) == 0                # one A shared by the batch
+    assert L.rmm_fused_route(-1, 700, 128, 0, 0, a, 704, 0) == -1
+
+
 V = ctypes.c_void_p
 
 

@@ -143,6 +143,9 @@ def test_roofline_bound_follows_arithmetic_intensity():
     p = _meta(bench, "pv_16384", (32, 16384, 16384), (32, 16384, 128), torch.bfloat16)
     r = bench.roofline(p, 0.5, {"gemm": 3.0}, "gemm", PEAKS, "measured")
     assert r["bound"] == "hbm" and r["arithmetic_intensity"] < r["ridge"]
+    # ... on the stream route: all of P, V with its dropped rows zeroed, O in f32
+    assert p.stream and r["bytes_note"].startswith("stream route")
+    assert r["algorithmic_bytes_per_launch"] == 32 * (16384 * 16384 * 2 + 16384 * 128 * 2 + 16384 * 128 * 4)
     # Q·Kᵀ (B = Kᵀ given K-major, bf16 out): the output write keeps it below the ridge
     p = _meta(bench, "qk_32x4096x128", (32, 4096, 128), (32, 4096, 128), torch.bfloat16, b_kmajor=True,
               out=torch.bfloat16)
