@@ -36,7 +36,9 @@ Parity pins (tests/test_oracle_pins.py): hand-worked examples with closed-form
 values (tests/golden/), exact integer arithmetic for ρ = 1 and for the split
 A·B = A_S·B_S + A_D·B_D, the triangle-inequality error bound, brute force over
 every subset on tiny inputs, the B = I closed form, zero slices ranked last,
-and the minimax statement checked by construction.
+and the minimax statement checked by construction. The softmax producer of
+P·V: a hand-worked causal softmax, row sums, shift and scale invariants, and
+the bf16 rounding against hand-picked halfway cases and torch's own cast.
 """
 from __future__ import annotations
 
@@ -208,3 +210,51 @@ def selection_matches(gpu_idx: np.ndarray, oracle_idx: np.ndarray, s: np.ndarray
     t = float(np.min(s[list(o)]))
     ok = all(abs(s[k] - t) <= rel_window * t for k in diff)
     return ok, len(diff)
+
+
+# ---------------------------------------------------------------- P·V with its softmax producer
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (8 significant bits), ties
+    to even: the stored P of the attention workload. Written from the format's
+    definition (value = significand · 2^e with an 8-bit significand), not from
+    any library routine. Finite inputs of normal bf16 range only."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    nz = x != 0
+    e = np.floor(np.log2(np.abs(x[nz])))
+    # exact powers of two can land one off in log2; fix the exponent so that
+    # |x| / 2^e lies in [1, 2)
+    m = np.abs(x[nz]) / np.exp2(e)
+    e = np.where(m >= 2.0, e + 1, np.where(m < 1.0, e - 1, e))
+    q = x[nz] / np.exp2(e - 7)          # significand scaled to an integer grid of 2^7 steps
+    out[nz] = np.rint(q) * np.exp2(e - 7)  # np.rint rounds halves to even
+    return out
+
+
+def causal_softmax(L: np.ndarray, scale: float = 1.0, causal: bool = True) -> np.ndarray:
+    """Row softmax of scale·L in float64 ("Escopo de Aplicação": P is the
+    attention matrix, P = softmax of the scaled logits). With the causal mask,
+    query row q sees key k only when k <= q + (S_k - S_q) (the last query sees
+    every key); masked entries of P are 0. L: [..., S_q, S_k]."""
+    L = np.asarray(L, dtype=np.float64) * scale
+    S_q, S_k = L.shape[-2], L.shape[-1]
+    if causal:
+        q = np.arange(S_q)[:, None]
+        k = np.arange(S_k)[None, :]
+        visible = k <= q + (S_k - S_q)
+        L = np.where(visible, L, -np.inf)
+    m = np.max(L, axis=-1, keepdims=True)
+    E = np.exp(L - m)
+    return E / np.sum(E, axis=-1, keepdims=True)
+
+
+def pv_softmax_reduced(L: np.ndarray, V: np.ndarray, rho: float, mode: str = SCORE_PRODUCT, scale: float = 1.0,
+                       causal: bool = True):
+    """P·V with P produced from the logits, in the pages' order: P = softmax
+    (stored as bf16), the slice scores of P·V, the top-ceil(rho·S_k) keys per
+    head, the reduced product over them ("Escopo de Aplicação": P·V reduced
+    over the keys). L [bh][S_q][S_k], V [bh][S_k][d]. Returns (O, idx, s, P)
+    with P the stored bf16 values as float64."""
+    P = round_bf16(causal_softmax(L, scale, causal))
+    O, idx, s = pv_reduced(P, np.asarray(V, dtype=np.float64), rho, mode)
+    return O, idx, s, P

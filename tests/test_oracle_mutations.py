@@ -59,6 +59,15 @@ MUTATIONS = {
     "selection_range_unchecked": ("    if any(i < 0 or i >= s.shape[0] for i in g_list) or len(set(g_list)) != len(g_list):\n"
                                   "        return False, 0\n", ""),
     "pack_range_unchecked": ("        raise IndexError(f\"kept index outside [0, {K})\")\n", "        pass\n"),
+    "bf16_rounding_truncates": ("    out[nz] = np.rint(q) * np.exp2(e - 7)  # np.rint rounds halves to even\n",
+                                "    out[nz] = np.trunc(q) * np.exp2(e - 7)\n"),
+    "causal_mask_off_by_one": ("        visible = k <= q + (S_k - S_q)\n", "        visible = k < q + (S_k - S_q)\n"),
+    "causal_mask_aligned_to_the_first_query": ("        visible = k <= q + (S_k - S_q)\n", "        visible = k <= q\n"),
+    "softmax_over_queries": ("    m = np.max(L, axis=-1, keepdims=True)\n    E = np.exp(L - m)\n"
+                             "    return E / np.sum(E, axis=-1, keepdims=True)\n",
+                             "    m = np.max(L, axis=-2, keepdims=True)\n    E = np.exp(L - m)\n"
+                             "    return E / np.sum(E, axis=-2, keepdims=True)\n"),
+    "softmax_scale_ignored": ("    L = np.asarray(L, dtype=np.float64) * scale\n", "    L = np.asarray(L, dtype=np.float64)\n"),
     "near_tie_threshold_is_the_largest_kept": ("t = float(np.min(s[list(o)]))", "t = float(np.max(s[list(o)]))"),
 }
 

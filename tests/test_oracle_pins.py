@@ -406,3 +406,59 @@ def test_w8_uniform_scale_keeps_the_selection_and_scales_the_product():
 def test_w8_rejects_non_int8_weights():
     with pytest.raises(TypeError):
         O.dequantize_w8(np.zeros((2, 2), dtype=np.int16), np.ones(2))
+
+
+# ---------------------------------------------------------------- P·V with its softmax producer
+def test_round_bf16_matches_the_format():
+    # halfway cases go to the even significand; exact values stay
+    got = O.round_bf16(np.array([1.0, 1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 + 2 ** -7, 0.75, -(1 + 2 ** -8), 3 * 2 ** -130,
+                                 2.0 ** 100 * (1 + 2 ** -9)]))
+    want = np.array([1.0, 1.0, 1 + 2 ** -6, 1 + 2 ** -7, 0.75, -1.0, 3 * 2 ** -130, 2.0 ** 100])
+    assert np.array_equal(got, want)
+    # and a library routine that implements the same rounding (torch's float64 -> bfloat16 cast)
+    import torch
+    r = np.random.default_rng(3)
+    x = r.standard_normal(20000) * np.exp(4 * r.standard_normal(20000))
+    assert np.array_equal(O.round_bf16(x), torch.tensor(x).to(torch.bfloat16).double().numpy())
+
+
+def test_causal_softmax_hand_example():
+    L = np.array([[0.0, 5.0, 7.0], [np.log(2.0), 0.0, 9.0], [0.0, np.log(3.0), 0.0]])
+    P = O.causal_softmax(L)
+    want = np.array([[1.0, 0.0, 0.0], [2 / 3, 1 / 3, 0.0], [0.2, 0.6, 0.2]])
+    assert np.allclose(P, want, rtol=0, atol=1e-15)
+    assert P[0, 1] == 0.0 and P[0, 2] == 0.0 and P[1, 2] == 0.0  # masked entries exactly zero
+    # without the mask every key counts
+    Pn = O.causal_softmax(L, causal=False)
+    assert np.allclose(Pn[0], np.exp([0.0, 5.0, 7.0]) / np.exp([0.0, 5.0, 7.0]).sum(), rtol=1e-14)
+    # fewer queries than keys: the last query sees every key, the mask is aligned to it
+    P2 = O.causal_softmax(np.zeros((2, 3)))
+    assert np.allclose(P2, [[0.5, 0.5, 0.0], [1 / 3, 1 / 3, 1 / 3]], rtol=0, atol=1e-15)
+
+
+def test_causal_softmax_invariants():
+    r = np.random.default_rng(11)
+    L = 3.0 * r.standard_normal((2, 9, 9))
+    P = O.causal_softmax(L)
+    assert np.allclose(P.sum(axis=-1), 1.0, rtol=0, atol=1e-14)
+    assert np.all(P[:, np.triu_indices(9, 1)[0], np.triu_indices(9, 1)[1]] == 0.0)
+    # a constant added to each row changes nothing; a zero scale gives the uniform distribution
+    assert np.allclose(O.causal_softmax(L + r.standard_normal((2, 9, 1))), P, rtol=1e-12, atol=1e-15)
+    U = O.causal_softmax(L, scale=0.0)
+    assert np.allclose(U[0, 4, :5], 0.2, rtol=0, atol=1e-15)
+    # the scale multiplies the logits
+    assert np.allclose(O.causal_softmax(L, scale=0.5), O.causal_softmax(0.5 * L), rtol=1e-14, atol=0)
+
+
+def test_pv_softmax_pipeline_stores_bf16_and_reduces_over_keys():
+    r = np.random.default_rng(12)
+    L = 3.0 * r.standard_normal((2, 12, 12))
+    V = r.standard_normal((2, 12, 4))
+    O_, idx, s, P = O.pv_softmax_reduced(L, V, 1.0)
+    # P is the bf16 rounding of the softmax, and rho = 1 is the whole product P·V
+    assert np.array_equal(P, O.round_bf16(O.causal_softmax(L)))
+    assert np.allclose(O_, P @ V, rtol=1e-13, atol=1e-15)
+    # the causal mask makes the last key's column the sparsest: only the last query sees it
+    assert np.count_nonzero(P[:, :, -1]) == 2
+    O5, idx5, s5, _ = O.pv_softmax_reduced(L, V, 0.5)
+    assert idx5.shape == (2, 6)
