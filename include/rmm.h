@@ -360,6 +360,55 @@ rmm_status rmm_pv_reduced(const void* P, const void* V, int64_t bh, int64_t S_q,
                           void* O, rmm_dtype out, int32_t* idx_out,
                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------- P·V with its softmax producer
+ * "Escopo de Aplicação": P·V reduced over the keys, P the attention matrix
+ * (the row softmax of the scaled logits). The key score s_k = ||P[:, k]||_2 ·
+ * ||V[k, :]||_2 (product mode; ||P[:, k]||_2 in A-only mode) needs the column
+ * sums of squares of P, which the kernel that writes P has in hand: P is not
+ * read back to be scored.
+ *   L: logits [bh][S_q][S_k] contiguous, dtype ldt (bf16 or f32); P =
+ *   softmax(scale·L) per row. With causal != 0 query q sees key k only when
+ *   k <= q + S_k - S_q (the last query sees every key; S_q <= S_k required)
+ *   and masked entries of P are 0.
+ *   P: [bh][S_q][S_k] bf16 output (round to nearest even), every entry written.
+ *   V: [bh][S_k][d] bf16 contiguous. */
+
+/* Row statistics of the softmax: stats[b][q][0] = max over the visible keys of
+ * x = scale·log2(e)·L[b][q][k], stats[b][q][1] = 1 / sum exp2(x - max).
+ * status_word (nullable) receives RMM_STATUS_BIT_NONFINITE for a row whose
+ * statistics are not finite. */
+rmm_status rmm_softmax_row_stats(const void* L, rmm_dtype ldt, float scale, int causal, int64_t bh, int64_t S_q,
+                                 int64_t S_k, float* stats, uint32_t* status_word, cudaStream_t stream);
+
+/* P from the logits and their row statistics, and (s non-null) the key scores
+ * of P·V over the stored bf16 values: s[b][k] = ||P[b][:, k]||_2 ·
+ * ||V[b][k, :]||_2, or ||P[b][:, k]||_2 when V is NULL (A-only). Column sums
+ * in f32 in a fixed order (bit-reproducible; not the bits rmm_score gives for
+ * the same P, which sums in another order). d: V's columns (ignored without
+ * V). */
+rmm_status rmm_softmax_score(const void* L, rmm_dtype ldt, float scale, int causal, const float* stats, const void* V,
+                             int64_t d, int64_t bh, int64_t S_q, int64_t S_k, void* P, float* s,
+                             uint32_t* status_word, cudaStream_t stream);
+
+/* Workspace of rmm_pv_softmax_reduced, 1 KiB-aligned sections: the status
+ * word, row statistics [bh][S_q][2] f32, scores [bh][S_k] f32, kept indices
+ * [bh][k_keep] i32, and V with its dropped rows zeroed [bh][S_k][rmm_packed_b_ld(d)]. */
+size_t rmm_pv_softmax_workspace_size(int64_t bh, int64_t S_q, int64_t S_k, int64_t d, int64_t k_keep);
+
+/* O ≈ P·V with P = softmax(scale·L) produced by this call: row statistics,
+ * P and the key scores in one pass over P (rmm_softmax_score), the top
+ * ceil(rho·S_k) keys per head (rmm_select), V's dropped rows zeroed
+ * (rmm_mask_rows) and the tensor-core GEMM over P as written (rmm_gemm_full).
+ *   P must be 16-byte aligned and S_k a multiple of 8 (RMM_ERR_UNSUPPORTED
+ *   otherwise): the GEMM reads it by TMA.
+ *   O: [bh][S_q][d] (contiguous, dtype out); idx_out: nullable [bh][k_keep].
+ *   workspace: rmm_pv_softmax_workspace_size bytes, 1 KiB-aligned; its first
+ *   4 bytes are the status word (rmm_check). */
+rmm_status rmm_pv_softmax_reduced(const void* L, rmm_dtype ldt, float scale, int causal, const void* V, int64_t bh,
+                                  int64_t S_q, int64_t S_k, int64_t d, double rho, rmm_score_mode mode, void* P,
+                                  void* O, rmm_dtype out, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream);
+
 /* Allocation-free form of rmm_matmul_reduced (the paper has no counterpart:
  * this is a deployment convenience of this library).
  * For callers that must not allocate device memory — for example code running

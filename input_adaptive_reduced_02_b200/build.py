@@ -19,7 +19,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "librmm.so")
-SOURCES = ["api.cu", "score.cu", "select.cu", "pack.cu", "gemm_tc.cu", "gemm_simt.cu", "gemv.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "score.cu", "select.cu", "pack.cu", "gemm_tc.cu", "gemm_simt.cu", "gemv.cu", "softmax.cu",
+           "noalloc.cu"]
 HEADERS = ["rmm_device.cuh", "rmm_internal.h", "int8_convert.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

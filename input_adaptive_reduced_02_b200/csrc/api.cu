@@ -590,6 +590,105 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
   return debug_on() ? debug_call_status(w.status, stream) : RMM_OK;
 }
 
+// ---------------------------------------------------------------- P·V with its softmax producer
+struct SoftmaxWorkspace {
+  uint32_t* status;
+  float* stats;  // [bh][S_q][2]
+  float* s;      // [bh][S_k]
+  int32_t* idx;  // [bh][k_keep]
+  void* v_m;     // [bh][S_k][packed_b_ld(d)] bf16
+  size_t bytes;
+};
+
+static SoftmaxWorkspace carve_softmax(void* base, int64_t bh, int64_t S_q, int64_t S_k, int64_t d, int64_t k_keep) {
+  auto al = [](int64_t x) { return round_up(x, 1024); };
+  const uintptr_t p = reinterpret_cast<uintptr_t>(base);
+  int64_t off = 0;
+  SoftmaxWorkspace w;
+  w.status = reinterpret_cast<uint32_t*>(p + off);
+  off += al(4);
+  w.stats = reinterpret_cast<float*>(p + off);
+  off += al(bh * S_q * 8);
+  w.s = reinterpret_cast<float*>(p + off);
+  off += al(bh * S_k * 4);
+  w.idx = reinterpret_cast<int32_t*>(p + off);
+  off += al(bh * k_keep * 4);
+  w.v_m = reinterpret_cast<void*>(p + off);
+  off += al(bh * S_k * packed_b_ld(d) * 2);
+  w.bytes = size_t(off);
+  return w;
+}
+
+static rmm_status check_softmax(const void* L, rmm_dtype ldt, int causal, int64_t bh, int64_t S_q, int64_t S_k) {
+  if (!dtype_ok(ldt)) return fail(RMM_ERR_INVALID, "unknown logits dtype");
+  if (bh < 0 || S_q < 0 || S_k < 1) return fail(RMM_ERR_INVALID, "need bh, S_q >= 0 and S_k >= 1");
+  if (causal && S_q > S_k) return fail(RMM_ERR_INVALID, "the causal mask needs S_q <= S_k (every query sees a key)");
+  if (bh > kMaxGridBatch) return fail(RMM_ERR_UNSUPPORTED, "bh > %lld", (long long)kMaxGridBatch);
+  if (S_k > kMaxSelectK) return fail(RMM_ERR_UNSUPPORTED, "S_k > %lld keys per selection", (long long)kMaxSelectK);
+  if (bh > 0 && S_q > 0 && !L) return fail(RMM_ERR_INVALID, "logits are NULL");
+  return RMM_OK;
+}
+
+static rmm_status fused_softmax_call(const void* L, rmm_dtype ldt, float scale, int causal, const void* V,
+                                     int64_t bh, int64_t S_q, int64_t S_k, int64_t d, double rho,
+                                     rmm_score_mode mode, void* P, void* O, rmm_dtype out, int32_t* idx_out,
+                                     void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  rmm_status r = check_softmax(L, ldt, causal, bh, S_q, S_k);
+  if (r) return r;
+  if (!dtype_ok(out)) return fail(RMM_ERR_INVALID, "unknown output dtype");
+  if (mode != RMM_SCORE_PRODUCT && mode != RMM_SCORE_A_ONLY) return fail(RMM_ERR_INVALID, "unknown score mode");
+  if (d < 1) return fail(RMM_ERR_INVALID, "d must be >= 1");
+  const int64_t k_keep = rmm_keep_count(rho, S_k);
+  if (k_keep < 1) return fail(RMM_ERR_INVALID, "rho must lie in (0, 1] (got %g)", rho);
+  if (bh > 0 && (!V || !P || (S_q > 0 && !O))) return fail(RMM_ERR_INVALID, "V, P or O is NULL");
+  // P is the GEMM's A operand, read by TMA
+  if ((reinterpret_cast<uintptr_t>(P) & 15u) || S_k % 8 != 0)
+    return fail(RMM_ERR_UNSUPPORTED, "P must be 16-byte aligned and S_k a multiple of 8");
+  if (!workspace) return fail(RMM_ERR_INVALID, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(workspace) & 1023u) return fail(RMM_ERR_INVALID, "workspace must be 1 KiB aligned");
+  const SoftmaxWorkspace w = carve_softmax(workspace, bh, S_q, S_k, d, k_keep);
+  if (workspace_bytes < w.bytes)
+    return fail(RMM_ERR_INVALID, "workspace too small: %zu < %zu bytes", workspace_bytes, w.bytes);
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
+  cudaError_t ce = cudaMemsetAsync(w.status, 0, 4, stream);  // (the row-stats kernel clears it again)
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemsetAsync(status)");
+  if (bh == 0) return RMM_OK;
+  int32_t* idx = idx_out ? idx_out : w.idx;
+  if (S_q == 0) {  // no query: every score is 0, so the selection keeps the lowest indices
+    ce = cudaMemsetAsync(w.s, 0, size_t(bh * S_k) * 4, stream);
+    if (ce == cudaSuccess) ce = launch_select(w.s, bh, S_k, k_keep, idx, w.status, stream);
+    return ce == cudaSuccess ? RMM_OK : cuda_fail(ce, "select kernel");
+  }
+  const ElemKind lk = kind(ldt);
+  {
+    StageRange range("rmm softmax row stats");
+    ce = launch_softmax_stats(L, lk, bh, S_q, S_k, scale, causal, w.stats, w.status, 1, stream);
+  }
+  if (ce != cudaSuccess) return cuda_fail(ce, "softmax row-stats kernel");
+  {
+    StageRange range("rmm softmax + score");
+    ce = launch_softmax_score(L, lk, bh, S_q, S_k, scale, causal, w.stats, P, mode == RMM_SCORE_PRODUCT ? V : nullptr,
+                              d, w.s, w.status, stream);
+  }
+  if (ce != cudaSuccess) return cuda_fail(ce, "softmax + score kernel");
+  GemmArgs g = gemm_args(P, w.v_m, 0, bh, S_q, d, S_k, O, d, S_q * d, out, w.status);
+  g.lda = S_k;
+  g.strideA = S_q * S_k;
+  g.k_pad = S_k;
+  SplitZero z;
+  const bool zero = gemm_tc_split_zero(g, &z);
+  {
+    StageRange range("rmm select");
+    ce = launch_select(w.s, bh, S_k, k_keep, idx, w.status, stream, zero ? &z : nullptr, false);
+  }
+  if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
+  g.c_zeroed = zero ? 1 : 0;
+  if ((r = do_mask(V, d, S_k * d, bh, S_k, d, idx, k_keep, RMM_BF16, w.v_m, stream))) return r;
+  if ((r = do_gemm(g, RMM_BF16, stream))) return r;
+  return debug_on() ? debug_call_status(w.status, stream) : RMM_OK;
+}
+
 static rmm_status check_bn(const float* bn, int64_t bn_stride, int64_t batch, int64_t K) {
   if (batch > 0 && !bn) return fail(RMM_ERR_INVALID, "b_norm is NULL");
   if (bn_stride < 0 || (batch > 1 && bn_stride != 0 && bn_stride < K))
@@ -648,6 +747,53 @@ int rmm_set_gemm_cta_group(int cta_group) {
 }
 
 uint64_t rmm_launch_count(void) { return g_launches.load(); }
+
+rmm_status rmm_softmax_row_stats(const void* L, rmm_dtype ldt, float scale, int causal, int64_t bh, int64_t S_q,
+                                 int64_t S_k, float* stats, uint32_t* status_word, cudaStream_t stream) {
+  rmm_status r = check_softmax(L, ldt, causal, bh, S_q, S_k);
+  if (r) return r;
+  if (bh == 0 || S_q == 0) return RMM_OK;
+  if (!stats) return fail(RMM_ERR_INVALID, "stats is NULL");
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
+  StageRange range("rmm softmax row stats");
+  const cudaError_t ce = launch_softmax_stats(L, kind(ldt), bh, S_q, S_k, scale, causal, stats, status_word, 0, stream);
+  return ce == cudaSuccess ? RMM_OK : cuda_fail(ce, "softmax row-stats kernel");
+}
+
+rmm_status rmm_softmax_score(const void* L, rmm_dtype ldt, float scale, int causal, const float* stats, const void* V,
+                             int64_t d, int64_t bh, int64_t S_q, int64_t S_k, void* P, float* s,
+                             uint32_t* status_word, cudaStream_t stream) {
+  rmm_status r = check_softmax(L, ldt, causal, bh, S_q, S_k);
+  if (r) return r;
+  if (bh == 0) return RMM_OK;
+  if (S_q > 0 && (!stats || !P)) return fail(RMM_ERR_INVALID, "stats or P is NULL");
+  if (V && d < 1) return fail(RMM_ERR_INVALID, "d must be >= 1 when V is given");
+  DeviceGuard dg;
+  if ((r = bind_device(stream, dg))) return r;
+  if (S_q == 0) {  // no query: every column of P is empty
+    if (!s) return RMM_OK;
+    const cudaError_t ce = cudaMemsetAsync(s, 0, size_t(bh * S_k) * 4, stream);
+    return ce == cudaSuccess ? RMM_OK : cuda_fail(ce, "cudaMemsetAsync(s)");
+  }
+  StageRange range("rmm softmax + score");
+  const cudaError_t ce = launch_softmax_score(L, kind(ldt), bh, S_q, S_k, scale, causal, stats, P, V, d, s,
+                                              status_word, stream);
+  return ce == cudaSuccess ? RMM_OK : cuda_fail(ce, "softmax + score kernel");
+}
+
+size_t rmm_pv_softmax_workspace_size(int64_t bh, int64_t S_q, int64_t S_k, int64_t d, int64_t k_keep) {
+  if (bh < 0 || S_q < 0 || S_k < 0 || d < 0 || k_keep < 0) return 0;
+  return carve_softmax(nullptr, bh, S_q, S_k, d, k_keep).bytes;
+}
+
+rmm_status rmm_pv_softmax_reduced(const void* L, rmm_dtype ldt, float scale, int causal, const void* V, int64_t bh,
+                                  int64_t S_q, int64_t S_k, int64_t d, double rho, rmm_score_mode mode, void* P,
+                                  void* O, rmm_dtype out, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream) {
+  return fused_softmax_call(L, ldt, scale, causal, V, bh, S_q, S_k, d, rho, mode, P, O, out, idx_out, workspace,
+                            workspace_bytes, stream);
+}
 
 int rmm_set_debug(int on) {
   const int prev = debug_on() ? 1 : 0;

@@ -148,6 +148,18 @@ cudaError_t launch_pack_rows_w8(const int8_t* Wq, int64_t ldw, int64_t sW, const
                                 int64_t batch, int64_t N, const int32_t* idx, int64_t k_keep, int64_t k_pad,
                                 void* out, int64_t ldo, cudaStream_t st);
 
+// softmax.cu: P = softmax(scale·L) row by row (causal: key k visible to query q
+// when k <= q + S_k - S_q), stored bf16 [bh][S_q][S_k], L contiguous.
+//  stats[b][q] = (max of scale·log2(e)·L over visible keys, 1 / sum exp2(. - max));
+//  clear_status zeroes *status first (the fused call's first kernel).
+cudaError_t launch_softmax_stats(const void* L, ElemKind e, int64_t bh, int64_t S_q, int64_t S_k, float scale,
+                                 int causal, float* stats, uint32_t* status, int clear_status, cudaStream_t st);
+//  P from L and stats; with s_out, s_out[b][k] = ||P[b][:, k]|| · (V ? ||V[b][k, :]|| : 1)
+//  over the stored bf16 values (V bf16 [bh][S_k][d] contiguous, nullable).
+cudaError_t launch_softmax_score(const void* L, ElemKind e, int64_t bh, int64_t S_q, int64_t S_k, float scale,
+                                 int causal, const float* stats, void* P, const void* V, int64_t d, float* s_out,
+                                 uint32_t* status, cudaStream_t st);
+
 // gemm_tc.cu (bf16 tensor cores) / gemm_simt.cu (f32 CUDA cores)
 struct GemmArgs {
   const void* a;  // [batch][M][k_pad] packed, or a caller's A (lda, strideA)

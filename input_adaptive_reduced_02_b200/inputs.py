@@ -129,6 +129,23 @@ def attention_pv(bh: int = 32, S: int = 8192, d: int = 128, temperature: float =
     return P, V
 
 
+def attention_logits(bh: int = 32, S: int = 8192, d: int = 128, temperature: float = 3.0, seed: int = 0,
+                     device="cpu", dtype=torch.bfloat16, S_q: int | None = None):
+    """Logits L [bh][S_q][S] = temperature·N(0,1) (stored in `dtype`) and V
+    [bh][S][d] bf16 N(0,1): the inputs of P·V when P is produced from its
+    logits (P = causal row softmax of L). Head h draws from seed + h."""
+    S_q = S if S_q is None else S_q
+    L = torch.empty(bh, S_q, S, device=device, dtype=dtype)
+    V = torch.empty(bh, S, d, device=device, dtype=torch.bfloat16)
+    for h in range(bh):
+        g = _gen(seed * 1000003 + h, device)
+        for r0 in range(0, S_q, 1024):
+            r1 = min(S_q, r0 + 1024)
+            L[h, r0:r1].copy_(temperature * torch.randn(r1 - r0, S, generator=g, device=device, dtype=torch.float32))
+        V[h].copy_(torch.randn(S, d, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16))
+    return L, V
+
+
 def mlp_up(M: int = 2048, K: int = 8192, N: int = 28672, seed: int = 0, device="cpu"):
     """Up-projection: X (M×K) bf16 N(0,1) with 0.5% outlier channels ×20; W (K×N) N(0, 0.01²)."""
     X, _ = outlier_activations(M, K, 0.005, 20.0, seed, device)

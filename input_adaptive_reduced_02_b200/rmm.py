@@ -75,6 +75,12 @@ _SIGS = {
     "rmm_mask_rows": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _vp]),
     "rmm_gemm_full": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _i32, _vp, _i64, _i64, _i32, _vp, _vp]),
     "rmm_fused_route": (_i32, [_i64, _i64, _i64, _i32, _i32, _vp, _i64, _i64]),
+    "rmm_softmax_row_stats": (_i32, [_vp, _i32, ctypes.c_float, _i32, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "rmm_softmax_score": (_i32, [_vp, _i32, ctypes.c_float, _i32, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp, _vp,
+                                 _vp]),
+    "rmm_pv_softmax_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64, _i64]),
+    "rmm_pv_softmax_reduced": (_i32, [_vp, _i32, ctypes.c_float, _i32, _vp, _i64, _i64, _i64, _i64, _f64, _i32, _vp,
+                                      _vp, _i32, _vp, _vp, ctypes.c_size_t, _vp]),
     "rmm_check": (_i32, [_vp, _vp]),
     "rmm_last_error_string": (ctypes.c_char_p, []),
     "rmm_set_wait_limit_ns": (None, [_u64]),
@@ -549,6 +555,66 @@ def pv_reduced(P: torch.Tensor, V: torch.Tensor, rho: float, mode: str = "produc
                                 _ptr(out), _out_code(out.dtype), _ptr(idx_out), ctypes.c_void_p(ws.ptr), ws.nbytes,
                                 _stream(P)))
     return out, ws
+
+
+# ---------------------------------------------------------------- P·V with its softmax producer
+def softmax_row_stats(L: torch.Tensor, scale: float = 1.0, causal: bool = True, out: torch.Tensor | None = None,
+                      status: torch.Tensor | None = None) -> torch.Tensor:
+    """[bh][S_q][2] f32: max of scale·log2(e)·L over each row's visible keys, and 1 / sum exp2(. - max)."""
+    bh, S_q, S_k = L.shape
+    if not L.is_contiguous():
+        raise ValueError("L must be contiguous")
+    if out is None:
+        out = torch.empty(bh, S_q, 2, dtype=torch.float32, device=L.device)
+    _check(lib().rmm_softmax_row_stats(_ptr(L), _dtype(L), float(scale), int(causal), bh, S_q, S_k, _ptr(out),
+                                       _ptr(status), _stream(L)))
+    return out
+
+
+def softmax_score(L: torch.Tensor, stats: torch.Tensor, V: torch.Tensor | None = None, scale: float = 1.0,
+                  causal: bool = True, score: bool = True, P: torch.Tensor | None = None,
+                  s: torch.Tensor | None = None, status: torch.Tensor | None = None):
+    """(P, s): P = softmax(scale·L) stored bf16, and (score=True) s[b][k] =
+    ||P[b][:, k]|| · ||V[b][k, :]|| (or ||P[b][:, k]|| without V)."""
+    bh, S_q, S_k = L.shape
+    if not L.is_contiguous():
+        raise ValueError("L must be contiguous")
+    if V is not None and (V.dtype != torch.bfloat16 or not V.is_contiguous() or V.shape[:2] != (bh, S_k)):
+        raise ValueError("V must be a contiguous bf16 [bh][S_k][d] tensor")
+    d = V.shape[2] if V is not None else 0
+    if P is None:
+        P = torch.empty(bh, S_q, S_k, dtype=torch.bfloat16, device=L.device)
+    if score and s is None:
+        s = torch.empty(bh, S_k, dtype=torch.float32, device=L.device)
+    _check(lib().rmm_softmax_score(_ptr(L), _dtype(L), float(scale), int(causal), _ptr(stats), _ptr(V), d, bh, S_q,
+                                   S_k, _ptr(P), _ptr(s if score else None), _ptr(status), _stream(L)))
+    return P, (s if score else None)
+
+
+def pv_softmax_workspace_size(bh: int, S_q: int, S_k: int, d: int, k_keep: int) -> int:
+    return int(lib().rmm_pv_softmax_workspace_size(bh, S_q, S_k, d, k_keep))
+
+
+def pv_softmax_reduced(L: torch.Tensor, V: torch.Tensor, rho: float, scale: float = 1.0, causal: bool = True,
+                       mode: str = "product", out_dtype=torch.float32, P: torch.Tensor | None = None,
+                       out: torch.Tensor | None = None, workspace: Workspace | None = None,
+                       idx_out: torch.Tensor | None = None):
+    """O ≈ P·V with P = softmax(scale·L) written by the call (bf16) and scored
+    as it is written. Returns (O, P, workspace)."""
+    bh, S_q, S_k = L.shape
+    d = V.shape[2]
+    if not L.is_contiguous() or not V.is_contiguous() or V.dtype != torch.bfloat16:
+        raise ValueError("L must be contiguous and V a contiguous bf16 tensor")
+    k = keep_count(rho, S_k)
+    ws = _ensure_ws(workspace, pv_softmax_workspace_size(bh, S_q, S_k, d, k), L.device)
+    if P is None:
+        P = torch.empty(bh, S_q, S_k, dtype=torch.bfloat16, device=L.device)
+    if out is None:
+        out = torch.empty(bh, S_q, d, dtype=out_dtype, device=L.device)
+    _check(lib().rmm_pv_softmax_reduced(_ptr(L), _dtype(L), float(scale), int(causal), _ptr(V), bh, S_q, S_k, d,
+                                        float(rho), SCORE_MODES[mode], _ptr(P), _ptr(out), _out_code(out.dtype),
+                                        _ptr(idx_out), ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(L)))
+    return out, P, ws
 
 
 def set_wait_limit_ns(ns: int):
