@@ -56,6 +56,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="linear_4096",
                     choices=["linear_4096", "f32_64x256x64", "qk_32x4096x128", "pv_8192", "pv_16384", "pv_32768",
+                             "pv_softmax_8192", "pv_softmax_16384", "pv_softmax_32768",
                              "mlp_up", "mlp_down", "decode_4096", "decode_mlp_up", "decode_mlp_up_m1",
                              "w8_linear_4096", "w8_decode_mlp_up_m1"])
     ap.add_argument("--rho", type=float, default=None, help="retention ratio of the headline step")
@@ -83,6 +84,7 @@ class Problem:
         self.N = B3.shape[1] if b_kmajor else B3.shape[2]
         self.b_norm = None  # B's cached norms: the step uses them (decode: B is a resident weight)
         self.scale = None   # INT8 weight: B holds the int8 codes, W = B · diag(scale)
+        self.logits = None  # P·V with its softmax producer: the logits; A is the P the call writes
         # k = ceil(rho·K): the library's rmm_keep_count on the GPU arm; the CPU
         # reference arm substitutes the oracle's, so that it never loads librmm
         self.keep_count = rmm.keep_count
@@ -97,7 +99,7 @@ class Problem:
         """Narrow product (N <= 128, bf16): the library zeroes B's dropped rows
         and streams A whole through the GEMM instead of packing A (the route
         rule is the library's; a tensor without device memory counts as aligned)."""
-        if self.scale is not None or self.gemv:
+        if self.scale is not None or self.gemv or self.logits is not None:
             return False
         A3 = self.A if self.A.dim() == 3 else self.A.unsqueeze(0)
         b, M, K = A3.shape
@@ -128,6 +130,15 @@ def make_problem(name, device, seed, rho):
         Q, Km = inputs.attention_qk(seed=seed, device=device)
         return Problem(name, Q, Km, True, torch.bfloat16, rho or 0.5,
                        "Q,K [32][4096][128] bf16 (4 channels x8), S = Q·K^T reduced over head_dim, bf16 out")
+    if name.startswith("pv_softmax_"):
+        S = int(name.split("_")[2])
+        L, V = inputs.attention_logits(bh=32, S=S, d=128, seed=seed, device=device)
+        P = torch.zeros(32, S, S, dtype=torch.bfloat16, device=device)
+        p = Problem(name, P, V, False, torch.float32, rho or 0.5,
+                    f"L [32][{S}][{S}] bf16 logits 3·N(0,1) -> P = causal softmax (bf16, written by the call) · "
+                    f"V [32][{S}][128] bf16, reduced over keys, scored while P is written")
+        p.logits = L
+        return p
     if name.startswith("pv_"):
         S = int(name.split("_")[1])
         P, V = inputs.attention_pv(bh=32, S=S, d=128, seed=seed, device=device)
@@ -175,15 +186,20 @@ def make_problem(name, device, seed, rho):
 class Pipeline:
     """Device buffers for one problem and the staged C-ABI calls of one step."""
 
-    def __init__(self, p: Problem, rho_max: float):
+    def __init__(self, p: Problem, rho_max: float, force_pack: bool = False):
         self.p = p
+        self.stream = p.stream and not force_pack  # force_pack: the pack route's stage calls, for comparison
         dev = p.A.device
         kmax = p.k_keep(rho_max)
         kp = rmm.padded_keep(kmax)
         shp = (lambda r, c: (p.batch, r, c)) if p.A.dim() == 3 else (lambda r, c: (r, c))
         self.s = torch.empty((p.batch, p.K) if p.A.dim() == 3 else (p.K,), dtype=torch.float32, device=dev)
         self.idx_store = torch.empty(p.batch * kmax, dtype=torch.int32, device=dev)
-        if p.stream:  # B with its dropped rows zeroed; A is read as it is
+        if p.logits is not None:  # softmax producer: row stats, then P and the scores in one pass
+            self.a_store = None
+            self.stats = torch.empty(p.batch, p.M, 2, dtype=torch.float32, device=dev)
+            self.b_mask = torch.empty(shp(p.K, rmm.packed_b_ld(p.N)), dtype=p.A.dtype, device=dev)
+        elif self.stream:  # B with its dropped rows zeroed; A is read as it is
             self.a_store = None
             self.b_mask = torch.empty(shp(p.K, rmm.packed_b_ld(p.N)), dtype=p.A.dtype, device=dev)
         else:
@@ -195,7 +211,7 @@ class Pipeline:
     def views(self, rho):
         p = self.p
         k = p.k_keep(rho)
-        if p.stream:
+        if self.stream or p.logits is not None:
             idx = self.idx_store[: p.batch * k].view(p.batch, k) if p.A.dim() == 3 else self.idx_store[:k]
             return k, idx, None, None
         kp = rmm.padded_keep(k)
@@ -223,7 +239,11 @@ class Pipeline:
         k, idx, A_S, B_S = self.views(rho)
         if ev:
             ev[0].record()
-        if p.b_norm is not None:
+        if p.logits is not None:  # the producer writes P and the key scores
+            rmm.softmax_row_stats(p.logits, out=self.stats, status=self.status)
+            rmm.softmax_score(p.logits, self.stats, p.B if p.mode == "product" else None, P=p.A, s=self.s,
+                              status=self.status)
+        elif p.b_norm is not None:
             rmm.score_b_norms(p.A, p.b_norm, out=self.s, status=self.status)
         else:
             rmm.score(p.A, p.B, p.mode, p.b_kmajor, out=self.s, status=self.status)
@@ -244,7 +264,7 @@ class Pipeline:
             if ev:
                 ev[4 if breakdown else 2].record()
             return
-        if p.stream:  # the stream route: B's dropped rows zeroed, then the GEMM over all of A
+        if self.stream or p.logits is not None:  # B's dropped rows zeroed, then the GEMM over all of A
             rmm.mask_rows(p.B, idx, out=self.b_mask)
         elif p.scale is not None:
             rmm.pack_w8(p.A, p.B, p.scale, idx, out=(A_S, B_S), status=self.status)
@@ -256,7 +276,9 @@ class Pipeline:
             # the library records these immediately around the GEMM kernel
             # (after the split-K zeroing kernel rmm_gemm may launch first)
             rmm.set_gemm_events(ev[1], ev[2])
-        if p.stream:
+        if p.logits is not None:  # P is causal: tiles stop at their last row's keys
+            rmm.gemm_full(p.A, self.b_mask, p.N, out=self.C, status=self.status, causal_off=p.K - p.M)
+        elif self.stream:
             rmm.gemm_full(p.A, self.b_mask, p.N, out=self.C, status=self.status)
         else:
             rmm.gemm(A_S, B_S, k, b_kmajor=p.b_kmajor, N=p.N, out=self.C, status=self.status)
@@ -279,15 +301,20 @@ class Fused:
         self.p = p
         dev = p.A.device
         self.C = torch.empty((p.batch, p.M, p.N) if p.A.dim() == 3 else (p.M, p.N), dtype=p.out_dtype, device=dev)
-        self.ws = rmm.Workspace(rmm.workspace_size_for(p.batch, p.M, p.K, p.N, p.k_keep(rho_max), p.A.dtype,
-                                                       p.b_kmajor), dev)
+        if p.logits is not None:
+            nb = rmm.pv_softmax_workspace_size(p.batch, p.M, p.K, p.N, p.k_keep(rho_max))
+        else:
+            nb = rmm.workspace_size_for(p.batch, p.M, p.K, p.N, p.k_keep(rho_max), p.A.dtype, p.b_kmajor)
+        self.ws = rmm.Workspace(nb, dev)
         self.b_norm = b_norm if b_norm is not None else p.b_norm
 
     def step(self, rho, ev=None, breakdown=False):
         p = self.p
         if ev:
             ev[0].record()
-        if p.scale is not None:
+        if p.logits is not None:
+            rmm.pv_softmax_reduced(p.logits, p.B, rho, mode=p.mode, P=p.A, out=self.C, workspace=self.ws)
+        elif p.scale is not None:
             rmm.matmul_reduced_w8(p.A, p.B, p.scale, rho, b_norm=p.b_norm, mode=p.mode, out=self.C,
                                   workspace=self.ws)
         elif self.b_norm is not None:
@@ -295,6 +322,29 @@ class Fused:
                                        b_kmajor=p.b_kmajor)
         else:
             rmm.matmul_reduced(p.A, p.B, rho, p.mode, out=self.C, workspace=self.ws, b_kmajor=p.b_kmajor)
+        if ev:
+            ev[1].record()
+
+
+class Unfused:
+    """P·V with its softmax producer done in two library calls: the producer
+    writes P alone, then rmm_pv_reduced scores P by reading it back, selects,
+    and multiplies (what the fused call saves is that read of P)."""
+
+    def __init__(self, p: Problem, rho: float):
+        self.p = p
+        dev = p.A.device
+        self.stats = torch.empty(p.batch, p.M, 2, dtype=torch.float32, device=dev)
+        self.C = torch.empty(p.batch, p.M, p.N, dtype=p.out_dtype, device=dev)
+        self.ws = None
+
+    def step(self, rho, ev=None, breakdown=False):
+        p = self.p
+        if ev:
+            ev[0].record()
+        rmm.softmax_row_stats(p.logits, out=self.stats)
+        rmm.softmax_score(p.logits, self.stats, score=False, P=p.A)
+        _, self.ws = rmm.pv_reduced(p.A, p.B, rho, p.mode, out=self.C, workspace=self.ws)
         if ev:
             ev[1].record()
 
@@ -319,7 +369,7 @@ def timed_steps(pipe, rho: float, steps: int, flush, breakdown=False):
     Returns (per-step ms, per-stage ms lists). For the staged Pipeline without
     breakdown the stages are {"pre_gemm": score+select+pack, "gemm": gemm};
     for the Fused call {"call": the whole call}."""
-    fused = isinstance(pipe, (Fused, Dense))
+    fused = isinstance(pipe, (Fused, Dense, Unfused))
     n_ev = 2 if fused else (5 if breakdown else 3)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)]
     for i in range(steps):
@@ -451,40 +501,61 @@ def recorded_traffic():
 
 # ----------------------------------------------------------------- CPU oracle timing
 def oracle_cpu_timing(p: Problem, rho: float, budget_s: float, max_steps: int):
-    """Time the fp64 oracle on the whole workload (rank 0 host cores)."""
+    """Time the fp64 oracle on the workload (rank 0 host cores): whole steps
+    while they fit the budget, else the batch items (heads) it completes,
+    scaled to the step (said in `sample`)."""
     from oracle import rmm_oracle as O
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
         cores = os.cpu_count()
-    A64 = p.A.to("cpu", torch.float32).numpy().astype(np.float64)
-    if p.scale is not None:
-        B64 = O.dequantize_w8(p.B.to("cpu").numpy(), p.scale.to("cpu").numpy())
-    else:
-        B64 = p.B.to("cpu", torch.float32).numpy().astype(np.float64)
-    if p.A.dim() == 2:
-        A64, B64 = A64[None], B64[None]
-    if p.b_kmajor:
-        B64 = np.swapaxes(B64, 1, 2)
-    times = []
-    t_start = time.perf_counter()
-    while len(times) < max_steps and (not times or time.perf_counter() - t_start < budget_s):
-        t0 = time.perf_counter()
-        for b in range(A64.shape[0]):
-            O.matmul_reduced(A64[b], B64[b], rho, O.SCORE_A_ONLY if p.mode == "a_only" else O.SCORE_PRODUCT)
-            if time.perf_counter() - t_start > 4 * budget_s:
-                break
+    mode = O.SCORE_A_ONLY if p.mode == "a_only" else O.SCORE_PRODUCT
+
+    def f64(t):
+        return t.to("cpu", torch.float32).numpy().astype(np.float64)
+
+    def item(b):
+        """The oracle's inputs for batch item b, converted when needed."""
+        A = p.A[b] if p.A.dim() == 3 else p.A
+        B = p.B[b] if p.B.dim() == 3 else p.B
+        if p.logits is not None:
+            return f64(p.logits[b][None]), f64(B[None])
+        B64 = O.dequantize_w8(B.to("cpu").numpy(), p.scale.to("cpu").numpy()) if p.scale is not None else f64(B)
+        return f64(A), (B64.T if p.b_kmajor else B64)
+
+    def run(a, b):
+        if p.logits is not None:
+            O.pv_softmax_reduced(a, b, rho, mode)
         else:
-            times.append(time.perf_counter() - t0)
-            continue
-        break
-    if not times:
+            O.matmul_reduced(a, b, rho, mode)
+
+    steps, items, t_items = 0, 0, 0.0
+    t_start = time.perf_counter()
+    while steps < max_steps:
+        done = 0
+        for b in range(p.batch):
+            a, bb = item(b)
+            t0 = time.perf_counter()
+            run(a, bb)
+            t_items += time.perf_counter() - t0
+            done += 1
+            items += 1
+            if time.perf_counter() - t_start > budget_s:
+                break
+        if done == p.batch:
+            steps += 1
+        if time.perf_counter() - t_start > budget_s:
+            break
+    if items == 0:
         return None
-    t = statistics.mean(times)
+    t = t_items / items * p.batch  # seconds per whole step
+    sample = (f"{steps} full step(s)" if items % p.batch == 0 and steps else
+              f"{items} of {p.batch} batch items timed, scaled to the step (extrapolated)")
     return {"value": p.kept_flops(rho) / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{len(times)} full step(s) of {p.name} at rho={rho} (fp64 NumPy oracle: score, top-k, "
-                      f"reduced product), mean {t * 1e3:.1f} ms/step"}
+            "sample": f"{sample} of {p.name} at rho={rho} (fp64 NumPy oracle: "
+                      f"{'softmax, ' if p.logits is not None else ''}score, top-k, reduced product), "
+                      f"{t * 1e3:.1f} ms per step"}
 
 
 # ----------------------------------------------------------------- arms
@@ -616,6 +687,35 @@ def run_ours(args):
         sweep = {f"{r:g}": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in d.items()}
                  for r, d in sweep.items()}
 
+    # P·V with its softmax producer: the same work in two calls (P written, then
+    # read back by rmm_pv_reduced to be scored), timed the same way
+    unfused = None
+    if p.logits is not None:
+        uf = Unfused(p, rho)
+        for _ in range(3):
+            uf.step(rho)
+        ums, _ = timed_steps(uf, rho, max(5, args.steps), flush)
+        u_ms = statistics.median(ums)
+        unfused = {"ms": round(u_ms, 5), "fused_speedup": round(u_ms / statistics.median(step_ms), 4),
+                   "calls": "rmm_softmax_row_stats + rmm_softmax_score (P only) + rmm_pv_reduced (reads P to score)"}
+        del uf
+        torch.cuda.empty_cache()
+
+    # the stream route against the pack route it replaces (stage calls score,
+    # select, pack, GEMM), same inputs, same timing
+    pack_ref = None
+    if p.stream and not args.no_sweep:
+        pk = Pipeline(p, rho, force_pack=True)
+        for _ in range(3):
+            pk.step(rho)
+        pms, _ = timed_steps(pk, rho, max(5, args.steps), flush)
+        rmm.check(pk.status)
+        p_ms = statistics.median(pms)
+        pack_ref = {"ms": round(p_ms, 5), "stream_route_speedup": round(p_ms / statistics.median(step_ms), 4),
+                    "calls": "rmm_score + rmm_select + rmm_pack + rmm_gemm (A packed)"}
+        del pk
+        torch.cuda.empty_cache()
+
     # the dense product of the same shapes (cuBLAS through torch), for context
     dense = None
     if not args.no_sweep:
@@ -639,7 +739,7 @@ def run_ours(args):
 
     # the same call with B's norms cached (a weight's norms are computed once)
     cached = None
-    if p.mode == "product" and p.b_norm is None:
+    if p.mode == "product" and p.b_norm is None and p.logits is None:
         bn = rmm.b_norms(p.B, p.b_kmajor)
         ccall = Fused(p, rho, b_norm=bn)
         for _ in range(3):
@@ -705,6 +805,8 @@ def run_ours(args):
             "roofline": roof,
             "sweep": sweep,
             "dense_reference": dense,
+            "unfused_reference": unfused,
+            "pack_route_reference": pack_ref,
             "e2e": e2e,
             "gpu_launches": int(launches),
             "clocks": clk,
@@ -726,6 +828,20 @@ def stage_bytes(p: Problem, rho):
     wb = 1 if p.scale is not None else eb  # bytes per element of B as stored (INT8 codes)
     b_read = 0 if (p.mode == "a_only" or p.b_norm is not None) else p.K * p.N * wb
     ldb = p.N if p.b_kmajor else rmm.packed_b_ld(p.N)
+    if p.logits is not None:
+        # producer: the visible logits twice (row statistics, then P), P written
+        # whole, V read; GEMM: P's key blocks up to each 256-row tile's last row
+        ldm = rmm.packed_b_ld(p.N)
+        off = p.K - p.M
+        vis = sum(min(p.K, q + 1 + off) for q in range(p.M))
+        tiles = sum(min(256, p.M - m0) * min(p.K, -(-(min(p.M, m0 + 256) + off) // 64) * 64)
+                    for m0 in range(0, p.M, 256))
+        return {
+            "score": (2 * vis * eb + p.M * p.K * 2 + p.K * p.N * eb + 8 * p.M + 4 * p.K) * p.batch,
+            "select": (4 * p.K + 4 * k) * p.batch,
+            "pack": (k * p.N * eb + p.K * ldm * eb) * p.batch,
+            "gemm": (tiles * 2 + p.K * ldm * eb + p.M * p.N * ob) * p.batch,
+        }
     if p.stream:  # mask: k rows of B read, K rows written; GEMM: all of A, B_M and C
         ldm = rmm.packed_b_ld(p.N)
         return {

@@ -192,10 +192,14 @@ rmm_status rmm_mask_rows(const void* B, int64_t ldb, int64_t strideB, int64_t ba
  *   A: [batch][M][K] row-major, bf16, 16-byte aligned, lda and (batch > 1)
  *   strideA multiples of 8 and strideA nonzero (RMM_ERR_INVALID otherwise);
  *   B_M: [batch][K][rmm_packed_b_ld(N)], 16-byte aligned; C as in rmm_gemm.
+ *   causal_off: -1 for a dense A; >= 0 declares A[i][k] = 0 for k > i +
+ *   causal_off (a causal attention matrix, causal_off = S_k - S_q), and each
+ *   tile of rows stops at the last key its rows see (the blocks above hold
+ *   zeros and are not read).
  *   in must be RMM_BF16 (RMM_ERR_UNSUPPORTED otherwise). */
 rmm_status rmm_gemm_full(const void* A, int64_t lda, int64_t strideA, const void* B_M, int64_t batch, int64_t M,
-                         int64_t K, int64_t N, rmm_dtype in, void* C, int64_t ldc, int64_t strideC, rmm_dtype out,
-                         uint32_t* status_word, cudaStream_t stream);
+                         int64_t K, int64_t N, int64_t causal_off, rmm_dtype in, void* C, int64_t ldc, int64_t strideC,
+                         rmm_dtype out, uint32_t* status_word, cudaStream_t stream);
 
 /* Which route a fused call (rmm_matmul_reduced, _batched, _b_norms,
  * rmm_qk_reduced, rmm_pv_reduced) takes for these sizes and this A:
@@ -398,7 +402,8 @@ size_t rmm_pv_softmax_workspace_size(int64_t bh, int64_t S_q, int64_t S_k, int64
 /* O ≈ P·V with P = softmax(scale·L) produced by this call: row statistics,
  * P and the key scores in one pass over P (rmm_softmax_score), the top
  * ceil(rho·S_k) keys per head (rmm_select), V's dropped rows zeroed
- * (rmm_mask_rows) and the tensor-core GEMM over P as written (rmm_gemm_full).
+ * (rmm_mask_rows) and the tensor-core GEMM over P as written (rmm_gemm_full;
+ * with the causal mask it skips the key blocks above each tile's last row).
  *   P must be 16-byte aligned and S_k a multiple of 8 (RMM_ERR_UNSUPPORTED
  *   otherwise): the GEMM reads it by TMA.
  *   O: [bh][S_q][d] (contiguous, dtype out); idx_out: nullable [bh][k_keep].

@@ -297,6 +297,7 @@ static GemmArgs gemm_args(const void* A_S, const void* B_S, int b_kmajor, int64_
   g.k_pad = round_up(k_keep, 64);
   g.lda = g.k_pad;
   g.strideA = g.k_pad * M;
+  g.causal_off = -1;
   g.ldc = ldc;
   g.strideC = sC;
   g.out = kind(out);
@@ -492,8 +493,8 @@ rmm_status rmm_mask_rows(const void* B, int64_t ldb, int64_t strideB, int64_t ba
 }
 
 rmm_status rmm_gemm_full(const void* A, int64_t lda, int64_t strideA, const void* B_M, int64_t batch, int64_t M,
-                         int64_t K, int64_t N, rmm_dtype in, void* C, int64_t ldc, int64_t strideC, rmm_dtype out,
-                         uint32_t* status_word, cudaStream_t stream) {
+                         int64_t K, int64_t N, int64_t causal_off, rmm_dtype in, void* C, int64_t ldc, int64_t strideC,
+                         rmm_dtype out, uint32_t* status_word, cudaStream_t stream) {
   if (!dtype_ok(in) || !dtype_ok(out)) return fail(RMM_ERR_INVALID, "unknown dtype");
   if (in != RMM_BF16) return fail(RMM_ERR_UNSUPPORTED, "rmm_gemm_full runs on the bf16 tensor cores only");
   if (batch < 0 || M < 0 || N < 0 || K < 1) return fail(RMM_ERR_INVALID, "need batch, M, N >= 0 and K >= 1");
@@ -507,10 +508,12 @@ rmm_status rmm_gemm_full(const void* A, int64_t lda, int64_t strideA, const void
   DeviceGuard dg;
   rmm_status r = bind_device(stream, dg);
   if (r) return r;
+  if (causal_off < -1) return fail(RMM_ERR_INVALID, "causal_off must be -1 (dense A) or >= 0");
   GemmArgs g = gemm_args(A, B_M, 0, batch, M, N, K, C, ldc, strideC, out, status_word);
   g.lda = lda;
   g.strideA = strideA;
   g.k_pad = K;
+  g.causal_off = causal_off;
   return do_gemm(g, in, stream);
 }
 
@@ -676,6 +679,7 @@ static rmm_status fused_softmax_call(const void* L, rmm_dtype ldt, float scale, 
   g.lda = S_k;
   g.strideA = S_q * S_k;
   g.k_pad = S_k;
+  if (causal) g.causal_off = S_k - S_q;  // P is zero above the mask: tiles skip those key blocks
   SplitZero z;
   const bool zero = gemm_tc_split_zero(g, &z);
   {

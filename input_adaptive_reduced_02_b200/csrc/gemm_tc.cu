@@ -74,6 +74,8 @@ struct TcParams {
   // units each (same tile, two halves of K) that add into a zeroed C.
   int64_t full_units, total_units;
   int32_t kb_mid;
+  int64_t causal_off;  // >= 0: A[i][k] = 0 for k > i + causal_off; -1: dense
+  int32_t cg2;         // 1: 2-SM tiles (BM·2 rows)
   uint32_t* status;
   uint64_t wait_limit_ns;
   int stall_producer;
@@ -105,6 +107,13 @@ __device__ __forceinline__ Unit unit_info(int64_t u, const TcParams& p) {
     w.kb0 = 0;
     w.kb1 = p.num_kb;
     w.split = false;
+    if (p.causal_off >= 0) {  // the tile's last row sees keys up to that row + causal_off
+      int32_t b, mb, nb;
+      decode_tile(u, p, b, mb, nb);
+      const int64_t last_row = min(int64_t(p.M), int64_t(mb + 1) * BM * (p.cg2 ? 2 : 1)) - 1;
+      const int64_t kb_end = (last_row + p.causal_off) / BK + 1;
+      if (kb_end < w.kb1) w.kb1 = int32_t(kb_end);
+    }
   } else {
     const int64_t j = u - p.full_units;
     w.tile = p.full_units + (j >> 1);
@@ -511,7 +520,7 @@ Plan make_plan(const GemmArgs& g, int sms, bool c_tma) {
   q.total_tiles = int64_t(q.tiles_m) * q.tiles_n * g.batch;
   q.units = std::max<int64_t>(1, (sms > 0 ? sms : 148) / cg);
   q.rem = q.total_tiles % q.units;
-  q.split = g.out == kF32 && c_tma && q.num_kb >= 2 && q.rem > 0 && 2 * q.rem <= q.units;
+  q.split = g.out == kF32 && c_tma && q.num_kb >= 2 && q.rem > 0 && 2 * q.rem <= q.units && g.causal_off < 0;
   return q;
 }
 
@@ -579,6 +588,8 @@ cudaError_t launch_cfg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, co
   p.full_units = q.split ? p.total_tiles - q.rem : p.total_tiles;
   p.total_units = q.split ? p.full_units + 2 * q.rem : p.total_tiles;
   p.kb_mid = p.num_kb / 2;
+  p.causal_off = g.causal_off;
+  p.cg2 = CG == 2 ? 1 : 0;
   if (q.split && !g.c_zeroed) {
     const SplitZero z = split_zero(g, q);
     cudaError_t e = launch_pdl(zero_split_tiles_kernel, dim3(unsigned(std::min<int64_t>(z.count * 8, 1184))),

@@ -174,6 +174,10 @@ struct GemmArgs {
   // k_pad = K (its tensor maps read zeros past K). The CUDA-core GEMM takes
   // packed operands only.
   int64_t lda, strideA;
+  // >= 0: A is causal, A[i][k] = 0 for k > i + causal_off (P of a causal
+  // softmax, causal_off = S_k - S_q), so a tile of rows stops at the last key
+  // its rows see; -1: dense A. Tensor-core GEMM only.
+  int64_t causal_off;
   ElemKind out;
   uint32_t* status;
   uint64_t wait_limit_ns;

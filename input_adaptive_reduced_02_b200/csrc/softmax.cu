@@ -12,27 +12,39 @@
 //    logits once (16-byte loads, several in flight) and keeps a running
 //    maximum and rescaled sum of exp2: stats[q] = (max of x, 1 / sum exp2(x -
 //    max)) with x = scale·log2(e)·L, the row's normalisation.
-//  * softmax_score_kernel: one CTA per (64-key strip, head) walks every query
-//    row of its strip: p = exp2(x - max)·(1/sum) for visible keys, 0 for
-//    masked ones, rounded to bf16 (nearest even) and stored (16-byte stores),
-//    and the squares of the stored values summed per key column in a fixed
-//    order (each thread in row order, then the 32 row lanes in order). Rows
-//    whose keys in the strip are all masked are written as zeros without
-//    reading their logits. The strip's ||V[k, :]||^2 come from a warp per key;
-//    the kernel writes s_k (or P alone when no score is asked for).
+//  * softmax_score_kernel: a cluster of up to 8 CTAs per (64-key strip, head)
+//    splits the strip's query rows: p = exp2(x - max)·(1/sum) for visible
+//    keys, 0 for masked ones, rounded to bf16 (nearest even) and stored
+//    (16-byte stores), and the squares of the stored values summed per key
+//    column in a fixed order (each thread in row order, the 32 row lanes in
+//    order, then the cluster's CTAs in rank order through distributed shared
+//    memory). Rows whose keys in the strip are all masked are written as
+//    zeros without reading their logits. The strip's ||V[k, :]||^2 come from a
+//    warp per key; the kernel writes s_k (or P alone when no score is asked
+//    for). Splitting the rows keeps the strips near the first key (which
+//    every query sees) from running far longer than the others.
 // With the causal mask query q sees key k when k <= q + S_k - S_q (the last
 // query sees every key), so about half of the logits are never read.
 #include <algorithm>
+#include <atomic>
+#include <cooperative_groups.h>
 
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace rmm {
 namespace {
 
 constexpr int kSmThreads = 256;
+constexpr unsigned kSmMaxCluster = 8;  // CTAs splitting one strip's rows
 constexpr int kStrip = 64;      // keys per CTA of the score kernel
-constexpr int kRowUnroll = 8;   // rows in flight per thread
+constexpr int kRowUnroll = 8;   // rows per ring stage per thread
+constexpr int kRing = 3;        // ring stages (two in flight while one is used)
+// ring of 16-byte logits slots per thread, then the rows' statistics (float2
+// per row lane; 32 row lanes at most)
+constexpr size_t kScoreSmem = size_t(kRing) * kRowUnroll * kSmThreads * 16 + size_t(kRing) * kRowUnroll * 32 * 8;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ uint4 ld_nc16(const void* p) {
@@ -59,6 +71,24 @@ __device__ __forceinline__ void unpack16(uint4 u, float (&x)[4]) {
   x[3] = __uint_as_float(u.w);
 }
 
+// 2^x by the SFU instruction (PTX ex2.approx.ftz.f32: relative error below
+// 2^-22, subnormal results flushed to zero, 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void cp_async_zfill16(uint32_t smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_dst), "l"(gsrc), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_zfill8(uint32_t smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_dst), "l"(gsrc), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 __device__ __forceinline__ int64_t visible_keys(int64_t q, int64_t S_q, int64_t S_k, int causal) {
   return causal ? min(S_k, q + 1 + (S_k - S_q)) : S_k;
 }
@@ -66,20 +96,20 @@ __device__ __forceinline__ int64_t visible_keys(int64_t q, int64_t S_q, int64_t 
 // Fold x into a running (max m, sum of exp2(. - m)) pair.
 __device__ __forceinline__ void online_add(float& m, float& s, float x) {
   if (x > m) {
-    s = s * exp2f(m - x) + 1.f;
+    s = s * ex2(m - x) + 1.f;
     m = x;
   } else {
-    s += exp2f(x - m);
+    s += ex2(x - m);
   }
 }
 
 // Merge two running pairs.
 __device__ __forceinline__ void online_merge(float& m, float& s, float m2, float s2) {
   if (m2 > m) {
-    s = s * exp2f(m - m2) + s2;
+    s = s * ex2(m - m2) + s2;
     m = m2;
   } else if (m2 > -INFINITY) {
-    s += s2 * exp2f(m2 - m);
+    s += s2 * ex2(m2 - m);
   }
 }
 
@@ -117,11 +147,11 @@ softmax_stats_kernel(const T* __restrict__ L, int64_t bh, int64_t S_q, int64_t S
 #pragma unroll
           for (int e = 1; e < V; ++e) mv = fmaxf(mv, x[e] * xscale);
           if (mv > m) {
-            s *= exp2f(m - mv);
+            s *= ex2(m - mv);
             m = mv;
           }
 #pragma unroll
-          for (int e = 0; e < V; ++e) s += exp2f(x[e] * xscale - m);
+          for (int e = 0; e < V; ++e) s += ex2(x[e] * xscale - m);
         }
       }
       for (; j < nv; j += 32) {
@@ -153,7 +183,7 @@ __device__ __forceinline__ void p_group(const float (&x)[VT], int64_t c, int64_t
                                         float (&acc)[VT], uint32_t (&pk)[VT / 2]) {
   float p[VT];
 #pragma unroll
-  for (int e = 0; e < VT; ++e) p[e] = c + e < n ? exp2f(fmaf(x[e], xscale, -m)) * rz : 0.f;
+  for (int e = 0; e < VT; ++e) p[e] = c + e < n ? ex2(fmaf(x[e], xscale, -m)) * rz : 0.f;
 #pragma unroll
   for (int e = 0; e < VT / 2; ++e) {
     pk[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
@@ -164,9 +194,12 @@ __device__ __forceinline__ void p_group(const float (&x)[VT], int64_t c, int64_t
 }
 
 // T: logits element. Threads: CL column lanes of VT keys (64 keys = one strip)
-// x RL row lanes. P is bf16 [bh][S_q][S_k]; s_out[b][k] (nullable: P only).
+// x RL row lanes; the CTAs of a cluster split the strip's rows, and with
+// s_out their partial column sums are added in rank order through
+// distributed shared memory. P is bf16 [bh][S_q][S_k]; s_out[b][k] (nullable:
+// P only).
 template <typename T>
-__global__ void __launch_bounds__(kSmThreads)
+__global__ void __launch_bounds__(kSmThreads, 2)
 softmax_score_kernel(const T* __restrict__ L, int64_t S_q, int64_t S_k, float xscale, int causal, int vec,
                      const float2* __restrict__ stats, uint16_t* __restrict__ P, const uint16_t* __restrict__ Vm,
                      int64_t d, int v_vec, float* __restrict__ s_out, uint32_t* status) {
@@ -174,8 +207,12 @@ softmax_score_kernel(const T* __restrict__ L, int64_t S_q, int64_t S_k, float xs
   constexpr int CL = kStrip / VT;          // column lanes
   constexpr int RL = kSmThreads / CL;      // row lanes
   __shared__ float red[RL][kStrip + 1];
+  __shared__ float part[kStrip];
   __shared__ float vsq[kStrip];
-  const int64_t b = blockIdx.y;
+  cg::cluster_group cluster = cg::this_cluster();
+  const unsigned cs = cluster.num_blocks();
+  const unsigned crank = cluster.block_rank();
+  const int64_t b = blockIdx.z;
   const int64_t k0 = int64_t(blockIdx.x) * kStrip;
   const int tid = threadIdx.x, rl = tid / CL, cl = tid % CL;
   const int64_t c0 = k0 + int64_t(cl) * VT;  // this thread's first key
@@ -189,70 +226,11 @@ softmax_score_kernel(const T* __restrict__ L, int64_t S_q, int64_t S_k, float xs
   const float2* st = stats + b * S_q;
   const bool full16 = vec && c0 + VT <= S_k;  // whole 16-byte logits group inside the row
 
-  // zero rows: P = 0 without reading logits
-  for (int64_t q = rl; q < q_first; q += RL) {
-    uint16_t* pr = Pb + q * S_k;
-    if (full16) {
-      if constexpr (VT == 8) {
-        *reinterpret_cast<uint4*>(pr + c0) = make_uint4(0u, 0u, 0u, 0u);
-      } else {
-        *reinterpret_cast<uint2*>(pr + c0) = make_uint2(0u, 0u);
-      }
-    } else {
-      for (int e = 0; e < VT; ++e)
-        if (c0 + e < S_k) pr[c0 + e] = 0;
-    }
-  }
-
-  float acc[VT];
-#pragma unroll
-  for (int e = 0; e < VT; ++e) acc[e] = 0.f;
-  int64_t q = q_first + rl;
-  if (full16) {
-    for (; q + int64_t(RL) * (kRowUnroll - 1) < S_q; q += int64_t(RL) * kRowUnroll) {
-      uint4 u[kRowUnroll];
-      float2 sv[kRowUnroll];
-#pragma unroll
-      for (int t = 0; t < kRowUnroll; ++t) {
-        const int64_t qq = q + int64_t(RL) * t;
-        u[t] = ld_nc16(Lb + qq * S_k + c0);
-        sv[t] = st[qq];
-      }
-#pragma unroll
-      for (int t = 0; t < kRowUnroll; ++t) {
-        const int64_t qq = q + int64_t(RL) * t;
-        float x[VT];
-        unpack16(u[t], x);
-        uint32_t pk[VT / 2];
-        p_group<VT>(x, c0, visible_keys(qq, S_q, S_k, causal), xscale, sv[t].x, sv[t].y, acc, pk);
-        if constexpr (VT == 8) {
-          *reinterpret_cast<uint4*>(Pb + qq * S_k + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        } else {
-          *reinterpret_cast<uint2*>(Pb + qq * S_k + c0) = make_uint2(pk[0], pk[1]);
-        }
-      }
-    }
-  }
-  for (; q < S_q; q += RL) {
-    const float2 sv = st[q];
-    const int64_t n = visible_keys(q, S_q, S_k, causal);
-    float x[VT];
-#pragma unroll
-    for (int e = 0; e < VT; ++e) x[e] = c0 + e < S_k ? elem_to_f32(Lb[q * S_k + c0 + e]) : 0.f;
-    uint32_t pk[VT / 2];
-    p_group<VT>(x, c0, n, xscale, sv.x, sv.y, acc, pk);
-    for (int e = 0; e < VT; ++e)
-      if (c0 + e < S_k) Pb[q * S_k + c0 + e] = uint16_t(pk[e >> 1] >> ((e & 1) * 16));
-  }
-  if (!s_out) return;
-
-  // column sums of squares: row lanes in order
-#pragma unroll
-  for (int e = 0; e < VT; ++e) red[rl][cl * VT + e] = acc[e];
-  // ||V[k, :]||^2 of the strip's keys, a warp per key
+  // ||V[k, :]||^2 of the strip's keys: CTA r of the cluster takes keys r, r + cs,
+  // ..., a warp per key, before its main loop so that the loads overlap it
   const int warp = tid >> 5, lane = tid & 31;
-  if (Vm) {
-    for (int j = warp; j < kStrip; j += kSmThreads / 32) {
+  if (s_out && Vm) {
+    for (int j = int(crank) + warp * int(cs); j < kStrip; j += int(cs) * (kSmThreads / 32)) {
       const int64_t k = k0 + j;
       float a = 0.f;
       if (k < S_k) {
@@ -276,14 +254,126 @@ softmax_score_kernel(const T* __restrict__ L, int64_t S_q, int64_t S_k, float xs
       if (lane == 0) vsq[j] = a;
     }
   }
+
+  // zero rows: P = 0 without reading logits (this CTA's share)
+  {
+    const int64_t zper = (q_first + cs - 1) / cs;
+    const int64_t z0 = min(q_first, int64_t(crank) * zper), z1 = min(q_first, z0 + zper);
+    for (int64_t q = z0 + rl; q < z1; q += RL) {
+      uint16_t* pr = Pb + q * S_k;
+      if (full16) {
+        if constexpr (VT == 8) {
+          *reinterpret_cast<uint4*>(pr + c0) = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+          *reinterpret_cast<uint2*>(pr + c0) = make_uint2(0u, 0u);
+        }
+      } else {
+        for (int e = 0; e < VT; ++e)
+          if (c0 + e < S_k) pr[c0 + e] = 0;
+      }
+    }
+  }
+
+  // computed rows: this CTA's share of [q_first, S_q), in row order per thread
+  const int64_t per = (S_q - q_first + cs - 1) / cs;
+  const int64_t r0 = min(S_q, q_first + int64_t(crank) * per), r1 = min(S_q, r0 + per);
+  float acc[VT];
+#pragma unroll
+  for (int e = 0; e < VT; ++e) acc[e] = 0.f;
+  if (full16) {
+    // The logits of this thread's rows reach shared memory by cp.async into
+    // its own ring slots (kRing stages of kRowUnroll rows, two stages in
+    // flight): no registers are held while the loads are in flight. The
+    // first column lane of each row also copies the row's statistics into a
+    // slot the row's 8 lanes read after a warp barrier.
+    extern __shared__ __align__(16) unsigned char sm_ring[];
+    const uint32_t ring = smem_addr(sm_ring);
+    const uint32_t srow = ring + uint32_t(kRing * kRowUnroll * kSmThreads * 16);  // [kRing][kRowUnroll][RL] float2
+    const int64_t nrows = r1 - r0 > rl ? (r1 - r0 - rl + RL - 1) / RL : 0;  // rows of this thread
+    const int64_t nbat = (nrows + kRowUnroll - 1) / kRowUnroll;
+    const int64_t nbat_cta = ((r1 - r0 + RL - 1) / RL + kRowUnroll - 1) / kRowUnroll;  // the same in every thread
+    const T* Lt = Lb + c0;
+    uint16_t* Pt = Pb + c0;
+    auto issue = [&](int64_t j) {
+      if (j < nbat_cta) {
+        const uint32_t st0 = uint32_t(j % kRing) * kRowUnroll;
+#pragma unroll
+        for (int t = 0; t < kRowUnroll; ++t) {
+          const int64_t i = j * kRowUnroll + t;
+          const int64_t qq = r0 + rl + int64_t(RL) * i;
+          const bool live = i < nrows;
+          cp_async_zfill16(ring + ((st0 + t) * kSmThreads + tid) * 16, live ? Lt + qq * S_k : Lt, live ? 16u : 0u);
+          if (cl == 0)
+            cp_async_zfill8(srow + ((st0 + t) * RL + rl) * 8, live ? st + qq : st, live ? 8u : 0u);
+        }
+      }
+      cp_async_commit_group();  // one group per stage in every thread, empty or not
+    };
+    issue(0);
+    issue(1);
+    for (int64_t j = 0; j < nbat_cta; ++j) {
+      issue(j + 2);
+      cp_async_wait_group<2>();  // this thread's copies of stage j have landed
+      __syncwarp();              // and the statistics its row's first lane copied
+      const uint32_t st0 = uint32_t(j % kRing) * kRowUnroll;
+#pragma unroll
+      for (int t = 0; t < kRowUnroll; ++t) {
+        const int64_t i = j * kRowUnroll + t;
+        if (i < nrows) {
+          const int64_t qq = r0 + rl + int64_t(RL) * i;
+          uint4 u;
+          float2 sv;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
+                       : "r"(ring + ((st0 + t) * kSmThreads + tid) * 16));
+          asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(sv.x), "=f"(sv.y) : "r"(srow + ((st0 + t) * RL + rl) * 8));
+          float x[VT];
+          unpack16(u, x);
+          uint32_t pk[VT / 2];
+          p_group<VT>(x, c0, visible_keys(qq, S_q, S_k, causal), xscale, sv.x, sv.y, acc, pk);
+          if constexpr (VT == 8) {
+            *reinterpret_cast<uint4*>(Pt + qq * S_k) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          } else {
+            *reinterpret_cast<uint2*>(Pt + qq * S_k) = make_uint2(pk[0], pk[1]);
+          }
+        }
+      }
+      __syncwarp();  // the stage's slots are read before the next issue overwrites them
+    }
+    cp_async_wait_group<0>();
+  } else {
+    for (int64_t q = r0 + rl; q < r1; q += RL) {
+      const float2 sv = st[q];
+      const int64_t n = visible_keys(q, S_q, S_k, causal);
+      float x[VT];
+#pragma unroll
+      for (int e = 0; e < VT; ++e) x[e] = c0 + e < S_k ? elem_to_f32(Lb[q * S_k + c0 + e]) : 0.f;
+      uint32_t pk[VT / 2];
+      p_group<VT>(x, c0, n, xscale, sv.x, sv.y, acc, pk);
+      for (int e = 0; e < VT; ++e)
+        if (c0 + e < S_k) Pb[q * S_k + c0 + e] = uint16_t(pk[e >> 1] >> ((e & 1) * 16));
+    }
+  }
+  if (!s_out) return;  // (the same in every CTA of the cluster)
+
+  // this CTA's column sums of squares: row lanes in order
+#pragma unroll
+  for (int e = 0; e < VT; ++e) red[rl][cl * VT + e] = acc[e];
   __syncthreads();
-  if (tid < kStrip && k0 + tid < S_k) {
+  if (tid < kStrip) {
     float t = 0.f;
     for (int r = 0; r < RL; ++r) t += red[r][tid];
+    part[tid] = t;
+  }
+  cluster.sync();  // every CTA's partial sums are written and visible cluster-wide
+  if (crank == 0 && tid < kStrip && k0 + tid < S_k) {
+    float t = 0.f;
+    for (unsigned r = 0; r < cs; ++r) t += cluster.map_shared_rank(part, r)[tid];
     float sc = sqrtf(t);
-    if (Vm) sc *= sqrtf(vsq[tid]);
+    if (Vm) sc *= sqrtf(cluster.map_shared_rank(vsq, tid % cs)[tid]);
     s_out[b * S_k + k0 + tid] = sc;
   }
+  cluster.sync();  // keep shared memory alive until rank 0 has read it
 }
 
 template <typename T>
@@ -301,8 +391,20 @@ cudaError_t launch_softmax_t(const void* L, int64_t bh, int64_t S_q, int64_t S_k
                       static_cast<const T*>(L), bh, S_q, S_k, xscale, causal, vec, stats, status, clear_status);
   }
   const int v_vec = V && (reinterpret_cast<uintptr_t>(V) & 15u) == 0 && d % 8 == 0;
-  return launch_pdl(softmax_score_kernel<T>, dim3(unsigned((S_k + kStrip - 1) / kStrip), unsigned(bh)),
-                    dim3(kSmThreads), 0, st, dim3(0, 0, 0), static_cast<const T*>(L), S_q, S_k, xscale, causal, vec,
+  // CTAs per strip: split the rows until a CTA has about 512 of them
+  unsigned cs = 1;
+  while (cs < kSmMaxCluster && S_q >= int64_t(cs) * 2 * 512) cs *= 2;
+  static std::atomic<bool> attr_done[64];  // per device; racing first calls both set the attribute
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(softmax_score_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(kScoreSmem));
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  return launch_pdl(softmax_score_kernel<T>, dim3(unsigned((S_k + kStrip - 1) / kStrip), cs, unsigned(bh)),
+                    dim3(kSmThreads), kScoreSmem, st, dim3(1, cs, 1), static_cast<const T*>(L), S_q, S_k, xscale, causal, vec,
                     static_cast<const float2*>(stats), P, V, d, v_vec, s_out, status);
 }
 

@@ -73,7 +73,8 @@ _SIGS = {
     "rmm_gemv_gather_w8": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _i64,
                                   _vp, _i64, _i64, _i32, _vp]),
     "rmm_mask_rows": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _vp, _i64, _i32, _vp, _vp]),
-    "rmm_gemm_full": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _i32, _vp, _i64, _i64, _i32, _vp, _vp]),
+    "rmm_gemm_full": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _vp, _i64, _i64, _i32, _vp,
+                             _vp]),
     "rmm_fused_route": (_i32, [_i64, _i64, _i64, _i32, _i32, _vp, _i64, _i64]),
     "rmm_softmax_row_stats": (_i32, [_vp, _i32, ctypes.c_float, _i32, _i64, _i64, _i64, _vp, _vp, _vp]),
     "rmm_softmax_score": (_i32, [_vp, _i32, ctypes.c_float, _i32, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp, _vp,
@@ -383,14 +384,15 @@ def mask_rows(B: torch.Tensor, idx: torch.Tensor, out: torch.Tensor | None = Non
 
 
 def gemm_full(A: torch.Tensor, B_M: torch.Tensor, N: int, out_dtype=torch.float32, out: torch.Tensor | None = None,
-              status: torch.Tensor | None = None) -> torch.Tensor:
-    """C = A · B_M over all K slices (bf16 tensor cores), B_M as mask_rows writes it."""
+              status: torch.Tensor | None = None, causal_off: int = -1) -> torch.Tensor:
+    """C = A · B_M over all K slices (bf16 tensor cores), B_M as mask_rows writes it.
+    causal_off >= 0 declares A[i][k] = 0 for k > i + causal_off (blocks above are skipped)."""
     ba, M, K, lda, sA = _mat(A, "A")
     if out is None:
         out = torch.empty((ba, M, N) if A.dim() == 3 else (M, N), dtype=out_dtype, device=A.device)
     _, _, _, ldc, sC = _mat(out, "C")
-    _check(lib().rmm_gemm_full(_ptr(A), lda, sA, _ptr(B_M), ba, M, K, N, _dtype(A), _ptr(out), ldc, sC,
-                               _out_code(out.dtype), _ptr(status), _stream(A)))
+    _check(lib().rmm_gemm_full(_ptr(A), lda, sA, _ptr(B_M), ba, M, K, N, int(causal_off), _dtype(A), _ptr(out), ldc,
+                               sC, _out_code(out.dtype), _ptr(status), _stream(A)))
     return out
 
 

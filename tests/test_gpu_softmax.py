@@ -82,8 +82,12 @@ def test_fused_softmax_pv_matches_the_oracle(case, rho):
     stats = rmm.softmax_row_stats(L, scale, causal)
     P2, s2 = rmm.softmax_score(L, stats, V, scale, causal)
     idx2 = rmm.select(s2, k)
-    O2 = rmm.gemm_full(P2, rmm.mask_rows(V, idx2), d)
+    O2 = rmm.gemm_full(P2, rmm.mask_rows(V, idx2), d, causal_off=(S_k - S_q) if causal else -1)
     assert torch.equal(P2, P) and torch.equal(idx2, idx) and torch.equal(O2, Oo)
+    if causal:  # the dense GEMM over the same P (zeros above the mask included) gives the same product
+        O3 = rmm.gemm_full(P2, rmm.mask_rows(V, idx2), d)
+        for h in range(bh):
+            check_product(O3[h], f64(P[h]), f64(V[h]), idx[h].cpu().numpy(), 1e-2)
 
 
 def test_oracle_pipeline_end_to_end_small():
