@@ -234,3 +234,45 @@ def test_w8_linear_4096_full_size():
     check_product(C[rr][:, cc], f64(X[rr]), W64[:, cols], idx.cpu().numpy(), 1e-2, w_rel=U_BF16)
     del X, Wq, sc, ws
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("S", [8192, 32768])
+def test_pv_softmax_long_context(S):
+    """P·V with its softmax producer at full size (32 heads, d 128, logits
+    3·N(0,1) stored bf16, causal): the stored P on sampled rows against the
+    fp64 causal softmax, the producer's scores on sampled keys against the
+    oracle's scores of that P, every head's selection bit-exact on the
+    producer's scores, and 256 whole output rows of two heads against the
+    oracle's product over the kept keys."""
+    L, V = inputs.attention_logits(bh=32, S=S, d=128, seed=0, device=DEV)
+    k = rmm.keep_count(0.5, S)
+    idx = torch.empty(32, k, dtype=torch.int32, device=DEV)
+    Oo, P, ws = rmm.pv_softmax_reduced(L, V, 0.5, idx_out=idx)
+    rmm.check(ws)
+    # the producer's own scores (its stage call rewrites the same P, bit for bit)
+    P_before = P[5, S - 3].clone()
+    stats = rmm.softmax_row_stats(L)
+    _, s = rmm.softmax_score(L, stats, V, score=True, P=P)
+    assert torch.equal(P[5, S - 3], P_before)
+    for h in range(32):
+        _check_selection_exact(s[h], idx[h], k)
+    p_rel = 2.0 ** -8 + 2e-4 + 2.0 ** -8 * 2e-4
+    for h in (0, 21):
+        rows, cols = _rows_cols(S, S, 256, 1024, h + S)
+        rr, cc = torch.as_tensor(rows, device=DEV), torch.as_tensor(cols, device=DEV)
+        # P on sampled rows: softmax of the whole row (its visible part), masked entries zero
+        L_rows = f64(L[h][rr])
+        visible = np.arange(S)[None, :] <= rows[:, None]
+        Lm = np.where(visible, L_rows, -np.inf)
+        P_ref = np.exp(Lm - Lm.max(axis=1, keepdims=True))
+        P_ref /= P_ref.sum(axis=1, keepdims=True)
+        got = f64(P[h][rr])
+        assert np.all(got[~visible] == 0)
+        assert np.all(np.abs(got - P_ref) <= p_rel * P_ref + 1e-38)
+        # scores of sampled keys from the whole stored columns of P
+        s_ref = O.slice_scores(f64(P[h][:, cc]), f64(V[h][cc]))
+        check_scores(s[h][cc].cpu().numpy(), s_ref)
+        # whole output rows: O[r, :] = P[r, I] · V[I, :]
+        check_product(Oo[h][rr], f64(P[h][rr]), f64(V[h]), idx[h].cpu().numpy(), 1e-2)
+    del L, V, P, Oo, ws
+    torch.cuda.empty_cache()
