@@ -60,6 +60,8 @@ def parse_args(argv=None):
                              "mlp_up", "mlp_down", "decode_4096", "decode_mlp_up", "decode_mlp_up_m1",
                              "w8_linear_4096", "w8_decode_mlp_up_m1"])
     ap.add_argument("--rho", type=float, default=None, help="retention ratio of the headline step")
+    ap.add_argument("--heads", type=int, default=32,
+                    help="heads of the attention workloads (32 is the workload; fewer for small profiling runs)")
     ap.add_argument("--no-sweep", action="store_true", help="skip the rho sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -117,7 +119,7 @@ class Problem:
         return 2.0 * self.batch * self.M * self.N * self.k_keep(rho)
 
 
-def make_problem(name, device, seed, rho):
+def make_problem(name, device, seed, rho, heads=32):
     if name == "linear_4096":
         X, W = inputs.linear_projection(seed=seed, device=device)
         return Problem(name, X, W, False, torch.float32, rho or 0.5,
@@ -132,18 +134,18 @@ def make_problem(name, device, seed, rho):
                        "Q,K [32][4096][128] bf16 (4 channels x8), S = Q·K^T reduced over head_dim, bf16 out")
     if name.startswith("pv_softmax_"):
         S = int(name.split("_")[2])
-        L, V = inputs.attention_logits(bh=32, S=S, d=128, seed=seed, device=device)
-        P = torch.zeros(32, S, S, dtype=torch.bfloat16, device=device)
+        L, V = inputs.attention_logits(bh=heads, S=S, d=128, seed=seed, device=device)
+        P = torch.zeros(heads, S, S, dtype=torch.bfloat16, device=device)
         p = Problem(name, P, V, False, torch.float32, rho or 0.5,
-                    f"L [32][{S}][{S}] bf16 logits 3·N(0,1) -> P = causal softmax (bf16, written by the call) · "
-                    f"V [32][{S}][128] bf16, reduced over keys, scored while P is written")
+                    f"L [{heads}][{S}][{S}] bf16 logits 3·N(0,1) -> P = causal softmax (bf16, written by the call) · "
+                    f"V [{heads}][{S}][128] bf16, reduced over keys, scored while P is written")
         p.logits = L
         return p
     if name.startswith("pv_"):
         S = int(name.split("_")[1])
-        P, V = inputs.attention_pv(bh=32, S=S, d=128, seed=seed, device=device)
+        P, V = inputs.attention_pv(bh=heads, S=S, d=128, seed=seed, device=device)
         return Problem(name, P, V, False, torch.float32, rho or 0.5,
-                       f"P [32][{S}][{S}] causal softmax bf16 · V [32][{S}][128] bf16, reduced over keys")
+                       f"P [{heads}][{S}][{S}] causal softmax bf16 · V [{heads}][{S}][128] bf16, reduced over keys")
     if name == "mlp_up":
         X, W = inputs.mlp_up(seed=seed, device=device)
         return Problem(name, X, W, False, torch.float32, rho or 0.5,
@@ -606,7 +608,7 @@ def run_reference(args):
         return 0
     from oracle import rmm_oracle as O
     name = args.workload
-    p = make_problem(name, "cpu", 0, args.rho)
+    p = make_problem(name, "cpu", 0, args.rho, heads=args.heads)
     p.keep_count = O.keep_count
     p.mode = args.score_mode
     rho = p.rho
@@ -630,7 +632,7 @@ def run_ours(args):
     rank, world, local = dist_setup(args)
     torch.cuda.set_device(local)
     dev = torch.device(f"cuda:{local}")
-    p = make_problem(args.workload, dev, seed=rank, rho=args.rho)
+    p = make_problem(args.workload, dev, seed=rank, rho=args.rho, heads=args.heads)
     p.mode = args.score_mode
     rho = p.rho
     rho_max = rho if args.no_sweep else 1.0

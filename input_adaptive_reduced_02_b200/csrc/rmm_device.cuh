@@ -307,28 +307,33 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Zero the tiles of `z` with the threads of blocks [0, nblocks) (this thread
-// is thread `tid` of `nthreads` in block `block`): 16-byte stores, consecutive
-// threads on consecutive 16 bytes of a tile row. Tile rows start 16-byte
-// aligned (C, ldc, strideC and tile_cols are multiples of 4 floats).
+// is thread `tid` of `nthreads` in block `block`): a warp per tile row, lanes
+// on consecutive 16 bytes of it (the row's tile, batch item and position are
+// decoded once per row, not per store). Tile rows start 16-byte aligned (C,
+// ldc, strideC and tile_cols are multiples of 4 floats).
 __device__ __forceinline__ void zero_split_tiles(const SplitZero& z, int64_t block, int64_t nblocks, int tid,
                                                  int nthreads) {
-  const int64_t vec_per_row = z.tile_cols / 4;
-  const int64_t per_tile = int64_t(z.tile_rows) * vec_per_row;
-  const int64_t total = z.count * per_tile;
+  const int lane = tid & 31;
+  const int64_t warps = int64_t(nthreads) / 32;
+  const int64_t rows_total = z.count * z.tile_rows;
   const int64_t per_item = int64_t(z.tiles_m) * z.tiles_n;
-  for (int64_t v = block * nthreads + tid; v < total; v += nblocks * nthreads) {
-    const int64_t t = z.first_tile + v / per_tile;
-    const int64_t w = v % per_tile;
-    const int64_t b = t / per_item, r = t % per_item;
-    const int64_t nb = r / z.tiles_m, mb = r % z.tiles_m;
-    const int64_t row = mb * z.tile_rows + w / vec_per_row;
-    const int64_t col = nb * z.tile_cols + (w % vec_per_row) * 4;
-    if (row >= z.M || col >= z.N) continue;
-    float* dst = z.c + b * z.strideC + row * z.ldc + col;
-    if (col + 4 <= z.N) {
-      *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
-    } else {
-      for (int64_t j = 0; j < z.N - col; ++j) dst[j] = 0.f;
+  for (int64_t rr = block * warps + (tid >> 5); rr < rows_total; rr += nblocks * warps) {
+    const int64_t i = rr / z.tile_rows;
+    const int64_t r_in = rr - i * z.tile_rows;
+    const int64_t t = z.first_tile + i;
+    const int64_t b = t / per_item, r = t - b * per_item;
+    const int64_t nb = r / z.tiles_m, mb = r - nb * z.tiles_m;
+    const int64_t row = mb * z.tile_rows + r_in;
+    if (row >= z.M) continue;
+    const int64_t col0 = nb * z.tile_cols;
+    const int64_t ncols = min(int64_t(z.tile_cols), z.N - col0);
+    float* dst = z.c + b * z.strideC + row * z.ldc + col0;
+    for (int64_t j = int64_t(lane) * 4; j < ncols; j += 128) {
+      if (j + 4 <= ncols) {
+        *reinterpret_cast<float4*>(dst + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        for (int64_t e = j; e < ncols; ++e) dst[e] = 0.f;
+      }
     }
   }
 }

@@ -292,7 +292,7 @@ cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_ke
   if (zero && zero->count > 0) {
     z = *zero;
     const int64_t vecs = z.count * z.tile_rows * (z.tile_cols / 4);
-    helpers = std::min<int64_t>(147, (vecs + 16 * kSelThreads - 1) / (16 * kSelThreads));
+    helpers = std::min<int64_t>(147, (vecs + 4 * kSelThreads - 1) / (4 * kSelThreads));
   }
   const dim3 grid(unsigned(batch + helpers)), block(kSelThreads), none(0, 0, 0);
   const int ll = int(late_launch);
