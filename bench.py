@@ -293,6 +293,26 @@ class Pipeline:
 STAGES = ("score", "select", "pack", "gemm")
 
 
+def step_descr(p) -> str:
+    """What one timed step launches, by route (the stage names of stages_ms
+    follow STAGES whatever the route: 'pack' is the masking of B's dropped
+    rows on the stream route, 'score' the softmax producer when P is written)."""
+    if p.logits is not None:
+        return ("one rmm_pv_softmax_reduced call (row statistics, P written with the key scores, select, "
+                "V's dropped rows zeroed, causal GEMM over P: 5 kernels)")
+    if p.scale is not None:
+        if p.gemv:
+            return "one rmm_matmul_reduced_w8 call with W's norms cached (score, select, INT8 gather-GEMV: 3 kernels)"
+        return "one rmm_matmul_reduced_w8 call with W's norms cached (score, select, INT8 pack, gemm: 4 kernels)"
+    if p.gemv:
+        return "one rmm_matmul_reduced_b_norms call (score of x, select, gather-GEMV: 3 kernels)"
+    if p.stream:
+        return "one rmm_matmul_reduced call, stream route (score, select, B's dropped rows zeroed, gemm over A: 4 kernels)"
+    if p.b_kmajor:
+        return "one rmm_matmul_reduced call (score, select, pack of A's columns, pack of Kmat's columns, gemm: 5 kernels)"
+    return "one rmm_matmul_reduced call (score, select, pack, gemm: 4 kernels)"
+
+
 class Fused:
     """The one-call public path: rmm_matmul_reduced into a preallocated C with a
     reusable workspace (sized for rho_max). With b_norm, the call with B's
@@ -787,7 +807,7 @@ def run_ours(args):
                        "out_dtype": str(p.out_dtype).replace("torch.", ""),
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed before every timed step (256 MiB written, then another 256 MiB read)",
-                       "step": "one rmm_matmul_reduced call (score, select, pack, gemm: 4 kernels)",
+                       "step": step_descr(p),
                        "timing": "CUDA events on the launching stream around each call; a device sleep before "
                                  "each step hides host launch overhead. The GEMM's duration for the roofline "
                                  "comes from a second timed loop of the same step made of the four stage "
