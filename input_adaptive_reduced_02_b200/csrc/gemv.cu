@@ -13,8 +13,9 @@
 //  * bf16, rows 16-byte aligned: gemv_gather_mma_kernel (tensor-core path,
 //    below) — cp.async ring of 32-slice passes, mma.sync m16n8k16;
 //  * INT8 with per-column scales, rows 16-byte aligned:
-//    gemv_gather_mma_w8_kernel — the same, after an exact int8 -> bf16
-//    conversion of each pass;
+//    gemv_gather_mma_w8_kernel — mma.sync m16n8k16 too, each warp streaming
+//    its own column strip through a private cp.async ring and converting the
+//    int8 bytes exactly, straight into the MMA's bf16 B fragments;
 //  * f32 with rows 16-byte aligned, or INT8 with rows only 4-byte aligned:
 //    gemv_gather_async_kernel (FFMA, cp.async of 4 columns into per-lane
 //    slots);
@@ -617,25 +618,38 @@ cudaError_t launch_t(const GemvArgs& g, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- INT8 weight, tensor cores
-// The mma path for an INT8 weight: each pass's int8 rows (512 columns = 512
-// bytes per slice, one 16-byte cp.async per 16 weights, so a pass moves as
-// many bytes as the bf16 kernel's) are converted exactly to bf16 into a
-// swizzled staging buffer, which an ldmatrix + mma.sync loop reads (64 columns
-// per warp); column j of the sums is scaled by scale[j] at the end.
-constexpr int kW8Cols = 512;                  // columns of C per CTA
-constexpr int kW8Bufs = 3;                    // int8 ring buffers (kW8Bufs - 1 in flight)
-constexpr int kW8Chunk = 512;                 // slices whose indices and A values are staged at once
-constexpr int kW8Row = kW8Cols * 2;           // bytes of one staged bf16 slice
+// The mma path for an INT8 weight. A CTA owns 512 columns of C, 64 per warp,
+// and each warp streams its own 64-byte column strip of the kept rows through
+// a private cp.async ring of 32-slice passes, so the main loop synchronises
+// only within a warp; the whole block waits only while the indices and A's
+// values of the next 512 slices are staged. Each thread converts its own
+// bytes straight into the MMA's B fragments — no bf16 staging, no ldmatrix of
+// B. A warp's 64 columns are two halves of four n8 tiles; within a half,
+// fragment column g of tile j is weight column 4g + j, so one 32-bit shared
+// load of a slice row gives a thread its byte for all four tiles. For a
+// 16-slice step a thread loads rows 2t, 2t+1, 2t+8 and 2t+9 (t = lane % 4) —
+// the rows of its b0/b1 fragment registers — converts them exactly
+// (s8x4_to_f32) and packs byte j of rows 2t and 2t+1 (and of 2t+8, 2t+9) into
+// tile j's b0 (b1); the 80-byte pitch of a warp's ring puts rows 2t of
+// t = 0..3 eight banks apart, so these loads are free of bank conflicts.
+// Column j of the sums is scaled by scale[j] at the end.
+constexpr int kW8Cols = 512;                      // columns of C per CTA
+constexpr int kW8WarpCols = kW8Cols / kGvWarps;   // one warp's column strip
+constexpr int kW8Bufs = 4;                        // passes per warp ring (kW8Bufs - 1 in flight)
+constexpr int kW8Chunk = 512;                     // slices whose indices and A values are staged at once
+constexpr int kW8Pitch = kW8WarpCols + 16;        // bytes per slice row in a warp's ring
+constexpr uint32_t kW8Stage = uint32_t(kMmaPass) * kW8Pitch;  // one pass of one warp
 
 constexpr size_t gv_mma_w8_smem_bytes() {
-  return size_t(kW8Bufs) * kMmaPass * kW8Cols  // int8 ring (then the CTA's partial)
-         + size_t(kMmaPass) * kW8Row           // bf16 staging of one pass
-         + size_t(16) * kW8Chunk * 2           // A
-         + size_t(kW8Chunk) * 4;               // row numbers
+  return size_t(kGvWarps) * kW8Bufs * kW8Stage  // warp rings (then the CTA's partial)
+         + size_t(16) * kW8Chunk * 2            // A
+         + size_t(kW8Chunk) * 4;                // row numbers
 }
-static_assert(size_t(16) * kW8Cols * 4 <= size_t(kW8Bufs) * kMmaPass * kW8Cols, "the partial fits in the ring");
-static_assert(kMmaPass * (kW8Cols / 16) == 4 * kGvThreads, "four 16-byte copies per thread per pass");
-static_assert(kW8Cols == kGvWarps * 64, "64 columns per warp");
+static_assert(size_t(16) * kW8Cols * 4 <= size_t(kGvWarps) * kW8Bufs * kW8Stage, "the partial fits in the rings");
+static_assert(kW8WarpCols == 64, "two halves of four n8 tiles per warp");
+static_assert(kMmaPass * (kW8WarpCols / 16) == 4 * 32, "four 16-byte copies per lane per pass");
+static_assert((2 * (kW8Pitch / 4)) % 32 == 8 && kW8Pitch % 16 == 0, "rows 2t of t = 0..3 fall 8 banks apart");
+static_assert(kW8Chunk % kMmaPass == 0, "whole passes per chunk");
 
 // Requires Wq's rows (and its base) 16-byte aligned.
 __global__ void __launch_bounds__(kGvThreads)
@@ -644,13 +658,11 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
                           int64_t k_keep, void* __restrict__ C, int64_t ldc, int64_t sC, int out_bf16,
                           const float* __restrict__ scale, int64_t s_stride) {
   constexpr int AROW = kW8Chunk * 2;
-  constexpr int R8 = kW8Cols;  // bytes per slice in the int8 ring
   extern __shared__ __align__(128) unsigned char gvw_smem[];
-  unsigned char* ring = gvw_smem;                                    // [kW8Bufs][kMmaPass][R8]
-  unsigned char* cvt = ring + size_t(kW8Bufs) * kMmaPass * R8;        // [kMmaPass][kW8Row], swizzled bf16
-  unsigned char* as = cvt + size_t(kMmaPass) * kW8Row;                // [16][AROW]
-  int32_t* rows = reinterpret_cast<int32_t*>(as + 16 * AROW);        // [kW8Chunk]
-  float* cta = reinterpret_cast<float*>(ring);                       // [16][kW8Cols], once the ring is drained
+  unsigned char* rings = gvw_smem;                                     // [warp][kW8Bufs][kMmaPass][kW8Pitch]
+  unsigned char* as = rings + size_t(kGvWarps) * kW8Bufs * kW8Stage;   // [16][AROW]
+  int32_t* rows = reinterpret_cast<int32_t*>(as + 16 * AROW);          // [kW8Chunk]
+  float* cta = reinterpret_cast<float*>(rings);                        // [16][kW8Cols], once the rings are drained
 
   cg::cluster_group cluster = cg::this_cluster();
   const unsigned cs = cluster.num_blocks();
@@ -658,23 +670,27 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
   const int64_t b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n0 = int64_t(blockIdx.x) * kW8Cols;
-  const int cchunk = tid & 31;                   // this thread's 16 columns in the copies
-  const int64_t c = n0 + 16 * cchunk;
+  // this lane's copies: slices lane/4 + 8j of a pass, 16 bytes at 16·(lane % 4) of the warp's strip
+  const int64_t c = n0 + int64_t(warp) * kW8WarpCols + 16 * (lane & 3);
   const uint32_t src_bytes = c >= N ? 0u : uint32_t(min(int64_t(16), N - c));
   const uint16_t* Ab = A + b * sA;
   const int8_t* Bc = B + b * sB + (src_bytes ? c : 0);
   const int32_t* ib = idx + b * k_keep;
   const int64_t per = (k_keep + cs - 1) / cs;
   const int64_t t_begin = min(k_keep, int64_t(crank) * per), t_end = min(k_keep, t_begin + per);
-  const uint32_t ring_s = smem_addr(ring), cvt_s = smem_addr(cvt), as_s = smem_addr(as);
+  const unsigned char* ring = rings + size_t(warp) * kW8Bufs * kW8Stage;
+  const uint32_t ring_s = smem_addr(ring), as_s = smem_addr(as);
+  const uint32_t cp_off = uint32_t(lane >> 2) * kW8Pitch + uint32_t(lane & 3) * 16u;
   const int a_m = (lane & 7) + ((lane >> 3) & 1) * 8, a_kc = lane >> 4;
-  const int b_k = (lane & 7) + ((lane >> 3) & 1) * 8, b_nt = lane >> 4;
+  const int g = lane >> 2, t = lane & 3;  // fragment group and thread-in-group
+  // this thread's fragment bytes: row 2t of a step, columns 4g .. 4g + 3 of each half
+  const uint32_t frag_off = uint32_t(2 * t) * kW8Pitch + uint32_t(4 * g);
 
   for (int e = tid; e < 16 * AROW / 16; e += kGvThreads) reinterpret_cast<uint4*>(as)[e] = make_uint4(0u, 0u, 0u, 0u);
 
   float d[8][4];
 #pragma unroll
-  for (int t = 0; t < 8; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+  for (int j = 0; j < 8; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0.f;
 
   pdl_trigger();
   pdl_wait();
@@ -682,19 +698,20 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
   for (int64_t c0 = t_begin; c0 < t_end; c0 += kW8Chunk) {
     const int nc = int(min(int64_t(kW8Chunk), t_end - c0));
     const int np = (nc + kMmaPass - 1) / kMmaPass;
-    __syncthreads();
+    __syncthreads();  // every warp is done with the previous chunk's rows and A (and the zero fill is done)
     for (int i = tid; i < np * kMmaPass; i += kGvThreads) rows[i] = i < nc ? ib[c0 + i] : 0;
     __syncthreads();
+    // this lane's copies of pass p (zeros past the chunk end); one commit group
+    // per call in every lane, so that group counts stay uniform
     auto issue = [&](int p) {
       if (p < np) {
-        const uint32_t boff = uint32_t(p % kW8Bufs) * kMmaPass * R8;
+        const uint32_t dst = ring_s + uint32_t(p % kW8Bufs) * kW8Stage + cp_off;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int il = (tid >> 5) + 8 * j;  // slice within the pass
-          const int i = p * kMmaPass + il;
+          const int i = p * kMmaPass + (lane >> 2) + 8 * j;
           const bool live = i < nc && src_bytes != 0;
-          cp_async16_zfill(ring_s + boff + uint32_t(il) * R8 + uint32_t(cchunk) * 16u,
-                           live ? Bc + int64_t(rows[i]) * ldb : Bc, live ? src_bytes : 0u);
+          cp_async16_zfill(dst + uint32_t(8 * j) * kW8Pitch, live ? Bc + int64_t(rows[i]) * ldb : Bc,
+                           live ? src_bytes : 0u);
         }
       }
       cp_async_commit();
@@ -711,51 +728,53 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
       for (int m = 0; m < 16; ++m)
         if (m < M) *reinterpret_cast<uint16_t*>(as + swz(m, AROW, i >> 3) + (i & 7) * 2) = v[m];
     }
+    __syncthreads();  // A's values of this chunk are visible to every warp
 #pragma unroll 1
     for (int p = 0; p < np; ++p) {
       cp_async_wait<kW8Bufs - 2>();
-      __syncthreads();  // pass p's int8 rows are visible; the previous pass is done with the staging
-      {
-        const unsigned char* src = ring + size_t(p % kW8Bufs) * kMmaPass * R8;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int il = (tid >> 5) + 8 * j;
-          const uint4 q = *reinterpret_cast<const uint4*>(src + il * R8 + cchunk * 16);
-          const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-          uint32_t o[8];
-#pragma unroll
-          for (int h = 0; h < 4; ++h) s8x4_to_bf16x4(w[h], o[2 * h], o[2 * h + 1]);
-          *reinterpret_cast<uint4*>(cvt + swz(il, kW8Row, 2 * cchunk)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(cvt + swz(il, kW8Row, 2 * cchunk + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
-        }
-      }
-      __syncthreads();  // the bf16 staging of pass p is complete
+      __syncwarp();  // the warp's copies of pass p are visible to all its lanes
+      const unsigned char* rb = ring + size_t(p % kW8Bufs) * kW8Stage + frag_off;
 #pragma unroll
       for (int kc = 0; kc < kMmaPass / 16; ++kc) {
         uint32_t a0, a1, a2, a3;
         ldsm_x4(as_s + swz(a_m, AROW, (p * kMmaPass + kc * 16) / 8 + a_kc), a0, a1, a2, a3);
+        const unsigned char* r0 = rb + kc * 16 * kW8Pitch;
 #pragma unroll
-        for (int t2 = 0; t2 < 4; ++t2) {  // this warp's 8 tiles of 8 columns, two per ldmatrix
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(cvt_s + swz(kc * 16 + b_k, kW8Row, warp * 8 + 2 * t2 + b_nt), b0, b1, b2, b3);
-          mma_bf16_16816(d[2 * t2], a0, a1, a2, a3, b0, b1);
-          mma_bf16_16816(d[2 * t2 + 1], a0, a1, a2, a3, b2, b3);
+        for (int h = 0; h < 2; ++h) {
+          // rows 2t, 2t+1, 2t+8, 2t+9 of the step; byte j of each is column 4g + j of tile j
+          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(r0 + 32 * h);
+          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(r0 + kW8Pitch + 32 * h);
+          const uint32_t w2 = *reinterpret_cast<const uint32_t*>(r0 + 8 * kW8Pitch + 32 * h);
+          const uint32_t w3 = *reinterpret_cast<const uint32_t*>(r0 + 9 * kW8Pitch + 32 * h);
+          float f0[4], f1[4], f2[4], f3[4];
+          s8x4_to_f32(w0, f0[0], f0[1], f0[2], f0[3]);
+          s8x4_to_f32(w1, f1[0], f1[1], f1[2], f1[3]);
+          s8x4_to_f32(w2, f2[0], f2[1], f2[2], f2[3]);
+          s8x4_to_f32(w3, f3[0], f3[1], f3[2], f3[3]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            mma_bf16_16816(d[4 * h + j], a0, a1, a2, a3, pack_bf16x2_exact(f0[j], f1[j]),
+                           pack_bf16x2_exact(f2[j], f3[j]));
         }
       }
-      __syncthreads();  // every warp is done with the staging and with ring buffer p
+      __syncwarp();  // every lane is done reading buffer p before it is refilled
       issue(p + kW8Bufs - 1);
     }
     cp_async_wait<0>();
   }
-  __syncthreads();
+  __syncthreads();  // every warp is done with its ring: the partial reuses them
+  // accumulator fragment of tile 4h + j: rows g and g + 8, fragment columns 2t and
+  // 2t + 1, i.e. strip columns 32h + 4·(2t) + j and 32h + 4·(2t + 1) + j
 #pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    const int col = warp * 64 + t * 8 + (lane & 3) * 2;
-    const int m = lane >> 2;
-    cta[m * kW8Cols + col] = d[t][0];
-    cta[m * kW8Cols + col + 1] = d[t][1];
-    cta[(m + 8) * kW8Cols + col] = d[t][2];
-    cta[(m + 8) * kW8Cols + col + 1] = d[t][3];
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int col0 = warp * kW8WarpCols + 32 * h + 8 * t + j, col1 = col0 + 4;
+      cta[g * kW8Cols + col0] = d[4 * h + j][0];
+      cta[g * kW8Cols + col1] = d[4 * h + j][1];
+      cta[(g + 8) * kW8Cols + col0] = d[4 * h + j][2];
+      cta[(g + 8) * kW8Cols + col1] = d[4 * h + j][3];
+    }
   }
   cluster.sync();
   if (crank == 0) {
@@ -763,14 +782,14 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
       const int m = e / kW8Cols;
       const int64_t col = n0 + (e % kW8Cols);
       if (m >= M || col >= N) continue;
-      float t = 0.f;
-      for (unsigned q = 0; q < cs; ++q) t += cluster.map_shared_rank(cta, q)[e];
-      t *= scale[b * s_stride + col];
+      float acc = 0.f;
+      for (unsigned q = 0; q < cs; ++q) acc += cluster.map_shared_rank(cta, q)[e];
+      acc *= scale[b * s_stride + col];
       const int64_t off = b * sC + int64_t(m) * ldc + col;
       if (out_bf16)
-        static_cast<uint16_t*>(C)[off] = uint16_t(pack_bf16x2(t, 0.f) & 0xFFFFu);
+        static_cast<uint16_t*>(C)[off] = uint16_t(pack_bf16x2(acc, 0.f) & 0xFFFFu);
       else
-        static_cast<float*>(C)[off] = t;
+        static_cast<float*>(C)[off] = acc;
     }
   }
   cluster.sync();
