@@ -433,7 +433,7 @@ rmm_status rmm_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, 
   rmm_status r = bind_device(stream, dg);
   if (r) return r;
   StageRange range("rmm select");
-  cudaError_t ce = launch_select(s, batch, K, k_keep, idx, status_word, stream);
+  cudaError_t ce = launch_select(const_cast<float*>(s), batch, K, k_keep, idx, status_word, stream);
   if (ce != cudaSuccess) return cuda_fail(ce, "select kernel");
   return RMM_OK;
 }
@@ -517,6 +517,41 @@ rmm_status rmm_gemm_full(const void* A, int64_t lda, int64_t strideA, const void
   return do_gemm(g, in, stream);
 }
 
+// On the decode route a score that needs only A (B's row norms given, or the
+// A-only score) is computed by the selection kernel itself when A has at
+// most kRowScoreMaxM rows and K <= kRowScoreMaxK: the call then launches the
+// selection and the gather-GEMV only. The selection's only block
+// clears the status word when there is one batch item; with several, a memset
+// does it first.
+static bool select_scores(bool gemv, const float* bn, rmm_score_mode mode, int64_t M, int64_t K) {
+  return gemv && (bn || mode == RMM_SCORE_A_ONLY) && M <= kRowScoreMaxM && K <= kRowScoreMaxK;
+}
+
+static RowScore row_score(const void* A, int64_t lda, int64_t strideA, int64_t batch, int64_t M, rmm_dtype in,
+                          const float* bn, int64_t bn_stride) {
+  const int64_t e = in == RMM_BF16 ? 2 : 4;
+  RowScore rs;
+  rs.A = A;
+  rs.lda = lda;
+  rs.sA = strideA;
+  rs.M = int32_t(M);
+  rs.bf16 = in == RMM_BF16 ? 1 : 0;
+  rs.a_vec = (reinterpret_cast<uintptr_t>(A) & 15u) == 0 && (lda * e) % 16 == 0 && (batch == 1 || (strideA * e) % 16 == 0) ? 1 : 0;
+  rs.bn = bn;
+  rs.bn_stride = bn_stride;
+  return rs;
+}
+
+static cudaError_t select_with_scores(const RowScore& rs, float* s, int64_t batch, int64_t K, int64_t k_keep,
+                                      int32_t* idx, uint32_t* status, cudaStream_t stream) {
+  StageRange range("rmm score + select");
+  if (batch > 1) {
+    const cudaError_t ce = cudaMemsetAsync(status, 0, 4, stream);
+    if (ce != cudaSuccess) return ce;
+  }
+  return launch_select(s, batch, K, k_keep, idx, status, stream, nullptr, true, &rs, batch == 1);
+}
+
 static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const void* B, int64_t ldb,
                              int64_t strideB, int b_kmajor, const float* bn, int64_t bn_stride, int64_t batch,
                              int64_t M, int64_t K, int64_t N, double rho, rmm_dtype in, rmm_score_mode mode, void* C,
@@ -551,9 +586,11 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
     return ce == cudaSuccess ? RMM_OK : cuda_fail(ce, "cudaMemsetAsync(status)");
   }
   int32_t* idx = idx_out ? idx_out : w.idx;
+  const bool gemv = route == kRouteGemv;
+  const bool fold = select_scores(gemv, bn, mode, M, K);
   // the score kernel clears the status word (it is the call's first kernel)
-  if ((r = do_score(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, in, mode, w.s, w.status, stream,
-                    bn, bn_stride, 1)))
+  if (!fold && (r = do_score(A, lda, strideA, B, ldb, strideB, b_kmajor, batch, M, K, N, in, mode, w.s, w.status,
+                             stream, bn, bn_stride, 1)))
     return r;
   // The select runs on one SM per batch item; the C tiles that the GEMM's
   // split-K round adds into are zeroed meanwhile by helper blocks of the same
@@ -568,10 +605,12 @@ static rmm_status fused_call(const void* A, int64_t lda, int64_t strideA, const 
   }
   // A few rows of A (decode): the product streams B's kept rows straight
   // through idx, with no packed copy.
-  const bool gemv = route == kRouteGemv;
   SplitZero z;
   const bool zero = !gemv && in == RMM_BF16 && gemm_tc_split_zero(g, &z);
-  {
+  if (fold) {
+    ce = select_with_scores(row_score(A, lda, strideA, batch, M, in, bn, bn_stride), w.s, batch, K, k_keep, idx,
+                            w.status, stream);
+  } else {
     StageRange range("rmm select");
     ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr, gemv);
   }
@@ -996,14 +1035,19 @@ rmm_status rmm_matmul_reduced_w8(const void* A, int64_t lda, int64_t strideA, co
     return ce == cudaSuccess ? RMM_OK : cuda_fail(ce, "cudaMemsetAsync(status)");
   }
   int32_t* idx = idx_out ? idx_out : w.idx;
-  if ((r = do_score(A, lda, strideA, nullptr, 0, 0, 0, batch, M, K, N, in, mode, w.s, w.status, stream,
-                    mode == RMM_SCORE_PRODUCT ? b_norm : nullptr, b_norm_stride, 1)))
+  const float* bn = mode == RMM_SCORE_PRODUCT ? b_norm : nullptr;
+  const bool gemv = decode_route(M, 0);
+  const bool fold = select_scores(gemv, bn, mode, M, K);
+  if (!fold && (r = do_score(A, lda, strideA, nullptr, 0, 0, 0, batch, M, K, N, in, mode, w.s, w.status, stream, bn,
+                             b_norm_stride, 1)))
     return r;
   GemmArgs g = gemm_args(w.a_s, w.b_st, 0, batch, M, N, k_keep, C, ldc, strideC, out, w.status);
-  const bool gemv = decode_route(M, 0);
   SplitZero z;
   const bool zero = !gemv && gemm_tc_split_zero(g, &z);
-  {
+  if (fold) {
+    ce = select_with_scores(row_score(A, lda, strideA, batch, M, in, bn, b_norm_stride), w.s, batch, K, k_keep, idx,
+                            w.status, stream);
+  } else {
     StageRange range("rmm select");
     ce = launch_select(w.s, batch, K, k_keep, idx, w.status, stream, zero ? &z : nullptr, gemv);
   }

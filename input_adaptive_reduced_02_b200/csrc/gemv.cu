@@ -11,7 +11,8 @@
 // adds the CTAs' partials in rank order through distributed shared memory
 // (fixed order throughout: bit-reproducible, no atomics). By B:
 //  * bf16, rows 16-byte aligned: gemv_gather_mma_kernel (tensor-core path,
-//    below) — cp.async ring of 32-slice passes, mma.sync m16n8k16;
+//    below) — each warp streams its own column strip through a private
+//    cp.async ring of 32-slice passes, mma.sync m16n8k16;
 //  * INT8 with per-column scales, rows 16-byte aligned:
 //    gemv_gather_mma_w8_kernel — mma.sync m16n8k16 too, each warp streaming
 //    its own column strip through a private cp.async ring and converting the
@@ -354,26 +355,53 @@ static_assert(size_t(kGvWarps) * 16 * kGvCols * 4 <= size_t(2) * kGvPass * 32 * 
 
 // ---------------------------------------------------------------- bf16 tensor-core path
 // Same data movement idea as the async path, but the products run on the
-// tensor cores as warp-level mma.sync m16n8k16 (bf16 x bf16 -> f32): A is x_S
-// padded to 16 rows; each warp owns 16 of the CTA's 128 columns (two n8 tiles)
-// and walks every kept slice, so warps never share an output and no warp
-// reduction is needed.
-//  * The CTA's slices are taken in chunks of up to kMmaChunk: one step loads
-//    the chunk's row numbers and A values (bf16) into shared memory, so the
-//    copies of B never wait on a global load inside the loop.
-//  * B's rows stream by cp.async through a ring of kMmaBufs passes of
-//    kMmaPass rows; kMmaBufs - 1 passes are in flight while one is summed.
-//  * Ring rows (256 bytes) and A rows are XOR-swizzled in 16-byte chunks so
-//    that ldmatrix reads are free of bank conflicts; slices past the end are
-//    zero in both.
-constexpr int kMmaPass = 32;                  // kept slices per ring buffer
-constexpr int kMmaBufs = 4;                   // ring buffers (kMmaBufs - 1 in flight)
-constexpr int kMmaChunk = 1024;               // slices whose indices and A values are staged at once
-constexpr int kMmaCols = 256;                 // columns of C per CTA: 8 per lane, 16-byte copies
-constexpr int kMmaRow = kMmaCols * 2;         // bytes of one slice of B in the ring
+// tensor cores as warp-level mma.sync m16n8k16 (bf16 x bf16 -> f32), A being
+// x_S padded to 16 rows. A CTA owns 8·WC columns of C, WC per warp, and each
+// warp streams its own column strip (2·WC bytes of a row) of the kept rows
+// through a private cp.async ring of 32-slice passes, so the main loop
+// synchronises only within a warp; the whole block waits only while the
+// indices and A's values of the next kMmaChunk slices are staged. WC = 64
+// (512 columns per CTA) puts the grid of a large layer in one wave of two CTAs
+// per SM; WC = 32 keeps more CTAs busy on a small one.
+//  * B's rows stream through MmaCfg<WC>::BUFS passes per warp; BUFS - 1 are
+//    in flight while one is summed.
+//  * Ring rows and A rows are XOR-swizzled in 16-byte chunks so that
+//    ldmatrix reads are free of bank conflicts; slices past the end are zero
+//    in both.
+constexpr int kMmaPass = 32;    // kept slices per ring buffer
+constexpr int kMmaChunk = 256;  // slices whose indices and A values are staged at once
 
+template <int WC>
+struct MmaCfg {
+  static constexpr int COLS = kGvWarps * WC;       // columns of C per CTA
+  static constexpr int ROW = WC * 2;               // bytes of one slice of a warp's strip
+  static constexpr int CPR = ROW / 16;             // 16-byte chunks per strip row
+  static constexpr int BUFS = WC == 64 ? 3 : 4;    // passes per warp ring
+  static constexpr uint32_t STAGE = uint32_t(kMmaPass) * ROW;  // one pass of one warp
+  static constexpr int COPIES = kMmaPass * CPR / 32;          // 16-byte copies per lane per pass
+  static constexpr size_t SMEM = size_t(kGvWarps) * BUFS * STAGE  // warp rings (then the CTA's partial)
+                                 + size_t(16) * kMmaChunk * 2      // A: 16 rows of kMmaChunk bf16
+                                 + size_t(kMmaChunk) * 4;          // row numbers
+  static_assert(WC == 32 || WC == 64, "four or eight n8 tiles per warp");
+  static_assert(size_t(16) * COLS * 4 <= size_t(kGvWarps) * BUFS * STAGE, "the partial fits in the rings");
+  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+};
+static_assert(kMmaChunk % kMmaPass == 0 && kMmaPass % 16 == 0, "pass shape");
+
+// 16-byte chunk `chunk` of row `row` of a swizzled array of rows of row_bytes
+// (a multiple of 128): chunk ^ (row % 8), so the same chunk of 8 consecutive
+// rows falls in 8 different bank groups.
 __device__ __forceinline__ uint32_t swz(int row, int row_bytes, int chunk) {
   return uint32_t(row) * uint32_t(row_bytes) + (uint32_t(chunk ^ (row & 7)) << 4);
+}
+// The same for rows of CPR = 4 or 8 chunks: with 4 chunks (64-byte rows) two
+// rows share a 128-byte bank line, so the XOR pattern advances every 2 rows.
+template <int CPR>
+__device__ __forceinline__ uint32_t swz_strip(int row, int chunk) {
+  if constexpr (CPR == 8)
+    return uint32_t(row) * 128u + (uint32_t(chunk ^ (row & 7)) << 4);
+  else
+    return uint32_t(row) * 64u + (uint32_t(chunk ^ ((row >> 1) & 3)) << 4);
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -399,48 +427,40 @@ __device__ __forceinline__ void cp_async16_zfill(uint32_t smem_dst, const void* 
                : "memory");
 }
 
-constexpr size_t gv_mma_smem_bytes() {
-  return size_t(kMmaBufs) * kMmaPass * kMmaRow  // ring (then the CTA's partial)
-         + size_t(16) * kMmaChunk * 2           // A: 16 rows of kMmaChunk bf16
-         + size_t(kMmaChunk) * 4;               // row numbers
-}
-static_assert(size_t(16) * kMmaCols * 4 <= size_t(kMmaBufs) * kMmaPass * kMmaRow, "the partial fits in the ring");
-static_assert(kMmaPass % kGvWarps == 0 && kMmaPass % 16 == 0 && kMmaChunk % kMmaPass == 0, "pass shape");
-static_assert(kMmaCols == 32 * 8 && kMmaCols == kGvWarps * 32, "8 columns per lane, 32 per warp");
-
 // Requires B's rows (and its base) 16-byte aligned.
+template <int WC>
 __global__ void __launch_bounds__(kGvThreads)
 gemv_gather_mma_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t sA, const uint16_t* __restrict__ B,
                        int64_t ldb, int64_t sB, int64_t M, int64_t N, const int32_t* __restrict__ idx, int64_t k_keep,
                        void* __restrict__ C, int64_t ldc, int64_t sC, int out_bf16) {
-  constexpr int RPW = kMmaPass / kGvWarps;  // slices each warp copies per pass
-  constexpr int AROW = kMmaChunk * 2;       // bytes per row of A in shared memory
+  using Cfg = MmaCfg<WC>;
+  constexpr int AROW = kMmaChunk * 2;  // bytes per row of A in shared memory
+  constexpr int NT = WC / 8;           // n8 tiles per warp
+  constexpr int LPR = 32 / Cfg::CPR;   // slice rows one copy step of the warp covers
   extern __shared__ __align__(128) unsigned char gvm_smem[];
-  unsigned char* ring = gvm_smem;                                   // [kMmaBufs][kMmaPass][kMmaRow]
-  unsigned char* as = ring + size_t(kMmaBufs) * kMmaPass * kMmaRow;  // [16][AROW]
-  int32_t* rows = reinterpret_cast<int32_t*>(as + 16 * AROW);       // [kMmaChunk]
-  float* cta = reinterpret_cast<float*>(ring);                      // [16][kMmaCols], once the ring is drained
+  unsigned char* rings = gvm_smem;                                      // [warp][BUFS][kMmaPass][ROW]
+  unsigned char* as = rings + size_t(kGvWarps) * Cfg::BUFS * Cfg::STAGE;  // [16][AROW]
+  int32_t* rows = reinterpret_cast<int32_t*>(as + 16 * AROW);           // [kMmaChunk]
+  float* cta = reinterpret_cast<float*>(rings);                         // [16][COLS], once the rings are drained
 
   cg::cluster_group cluster = cg::this_cluster();
   const unsigned cs = cluster.num_blocks();
   const unsigned crank = cluster.block_rank();
   const int64_t b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t n0 = int64_t(blockIdx.x) * kMmaCols;
-  const int64_t c = n0 + 8 * lane;  // this lane's 8 columns in the copies
+  const int64_t n0 = int64_t(blockIdx.x) * Cfg::COLS;
+  // this lane's copies: slices lane / CPR + LPR·j of a pass, 8 columns at chunk lane % CPR of the warp's strip
+  const int cchunk = lane % Cfg::CPR;
+  const int64_t c = n0 + int64_t(warp) * WC + 8 * cchunk;
   const uint32_t src_bytes = c >= N ? 0u : uint32_t(min(int64_t(8), N - c) * 2);
   const uint16_t* Ab = A + b * sA;
   const uint16_t* Bc = B + b * sB + (src_bytes ? c : 0);  // this lane's column start in row 0
   const int32_t* ib = idx + b * k_keep;
   const int64_t per = (k_keep + cs - 1) / cs;
   const int64_t t_begin = min(k_keep, int64_t(crank) * per), t_end = min(k_keep, t_begin + per);
-  const uint32_t ring_s = smem_addr(ring), as_s = smem_addr(as);
-  // this lane's copy destinations within a ring buffer (slice warp + 8j, 16-byte chunk `lane`)
-  uint32_t dst[RPW];
-#pragma unroll
-  for (int j = 0; j < RPW; ++j) dst[j] = ring_s + swz(warp + kGvWarps * j, kMmaRow, lane);
+  const uint32_t ring_s = smem_addr(rings) + uint32_t(warp) * Cfg::BUFS * Cfg::STAGE, as_s = smem_addr(as);
   // ldmatrix lane roles: A x4 = (m 0-7 | 8-15) x (k 0-7 | 8-15) of a 16-slice step;
-  // B x4.trans = (k 0-7 | 8-15) x (two of this warp's four 8-column tiles)
+  // B x4.trans = (k 0-7 | 8-15) x (two of this warp's NT 8-column tiles)
   const int a_m = (lane & 7) + ((lane >> 3) & 1) * 8, a_kc = lane >> 4;
   const int b_k = (lane & 7) + ((lane >> 3) & 1) * 8, b_nt = lane >> 4;
 
@@ -448,9 +468,9 @@ gemv_gather_mma_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t sA, 
   for (int e = tid; e < 16 * AROW / 16; e += kGvThreads)
     reinterpret_cast<uint4*>(as)[e] = make_uint4(0u, 0u, 0u, 0u);
 
-  float d[4][4];
+  float d[NT][4];
 #pragma unroll
-  for (int t = 0; t < 4; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+  for (int t = 0; t < NT; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
 
   pdl_trigger();
   pdl_wait();
@@ -458,25 +478,27 @@ gemv_gather_mma_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t sA, 
   for (int64_t c0 = t_begin; c0 < t_end; c0 += kMmaChunk) {
     const int nc = int(min(int64_t(kMmaChunk), t_end - c0));
     const int np = (nc + kMmaPass - 1) / kMmaPass;
-    __syncthreads();  // the previous chunk is done with rows and A (and the zero fill is done)
+    __syncthreads();  // every warp is done with the previous chunk's rows and A (and the zero fill is done)
     for (int i = tid; i < np * kMmaPass; i += kGvThreads) rows[i] = i < nc ? ib[c0 + i] : 0;
     __syncthreads();
-    // copies of pass p's slices of B (zeros past the chunk end); one commit
-    // group per call in every thread, so that group counts stay uniform
+    // this lane's copies of pass p (zeros past the chunk end); one commit group
+    // per call in every lane, so that group counts stay uniform
     auto issue = [&](int p) {
       if (p < np) {
-        const uint32_t boff = uint32_t(p % kMmaBufs) * kMmaPass * kMmaRow;
+        const uint32_t boff = uint32_t(p % Cfg::BUFS) * Cfg::STAGE;
 #pragma unroll
-        for (int j = 0; j < RPW; ++j) {
-          const int i = p * kMmaPass + warp + kGvWarps * j;
+        for (int j = 0; j < Cfg::COPIES; ++j) {
+          const int sl = lane / Cfg::CPR + LPR * j;  // slice within the pass
+          const int i = p * kMmaPass + sl;
           const bool live = i < nc && src_bytes != 0;
-          cp_async16_zfill(dst[j] + boff, live ? Bc + int64_t(rows[i]) * ldb : Bc, live ? src_bytes : 0u);
+          cp_async16_zfill(ring_s + boff + swz_strip<Cfg::CPR>(sl, cchunk), live ? Bc + int64_t(rows[i]) * ldb : Bc,
+                           live ? src_bytes : 0u);
         }
       }
       cp_async_commit();
     };
 #pragma unroll 1
-    for (int q = 0; q < kMmaBufs - 1; ++q) issue(q);
+    for (int q = 0; q < Cfg::BUFS - 1; ++q) issue(q);
     // A[m][idx] as bf16 bits for m < M (zero past the chunk end), loaded while
     // the first passes of B are in flight; all loads before the stores
     for (int i = tid; i < np * kMmaPass; i += kGvThreads) {
@@ -488,43 +510,45 @@ gemv_gather_mma_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t sA, 
       for (int m = 0; m < 16; ++m)
         if (m < M) *reinterpret_cast<uint16_t*>(as + swz(m, AROW, i >> 3) + (i & 7) * 2) = v[m];
     }
+    __syncthreads();  // A's values of this chunk are visible to every warp
 #pragma unroll 1
     for (int p = 0; p < np; ++p) {
-      cp_async_wait<kMmaBufs - 2>();  // this thread's copies of pass p have landed
-      __syncthreads();                // and everyone's (and A's values) are visible to all warps
-      const uint32_t rb = ring_s + uint32_t(p % kMmaBufs) * kMmaPass * kMmaRow;
+      cp_async_wait<Cfg::BUFS - 2>();  // this lane's copies of pass p have landed
+      __syncwarp();                    // and the whole warp's are visible to all its lanes
+      const uint32_t rb = ring_s + uint32_t(p % Cfg::BUFS) * Cfg::STAGE;
 #pragma unroll
       for (int kc = 0; kc < kMmaPass / 16; ++kc) {
-        uint32_t a0, a1, a2, a3, b0, b1, b2, b3, b4, b5, b6, b7;
+        uint32_t a0, a1, a2, a3;
         ldsm_x4(as_s + swz(a_m, AROW, (p * kMmaPass + kc * 16) / 8 + a_kc), a0, a1, a2, a3);
-        ldsm_x4_t(rb + swz(kc * 16 + b_k, kMmaRow, warp * 4 + b_nt), b0, b1, b2, b3);
-        ldsm_x4_t(rb + swz(kc * 16 + b_k, kMmaRow, warp * 4 + 2 + b_nt), b4, b5, b6, b7);
-        mma_bf16_16816(d[0], a0, a1, a2, a3, b0, b1);
-        mma_bf16_16816(d[1], a0, a1, a2, a3, b2, b3);
-        mma_bf16_16816(d[2], a0, a1, a2, a3, b4, b5);
-        mma_bf16_16816(d[3], a0, a1, a2, a3, b6, b7);
+#pragma unroll
+        for (int t2 = 0; t2 < NT / 2; ++t2) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(rb + swz_strip<Cfg::CPR>(kc * 16 + b_k, 2 * t2 + b_nt), b0, b1, b2, b3);
+          mma_bf16_16816(d[2 * t2], a0, a1, a2, a3, b0, b1);
+          mma_bf16_16816(d[2 * t2 + 1], a0, a1, a2, a3, b2, b3);
+        }
       }
-      __syncthreads();  // every warp is done with this buffer
-      issue(p + kMmaBufs - 1);
+      __syncwarp();  // every lane is done reading this buffer before it is refilled
+      issue(p + Cfg::BUFS - 1);
     }
     cp_async_wait<0>();
   }
-  __syncthreads();  // every warp is done with the ring: the partial takes its place
-  // accumulator fragment: rows lane/4 and lane/4 + 8, columns 2·(lane%4) + {0, 1} of each tile
+  __syncthreads();  // every warp is done with its ring: the partial takes their place
+  // accumulator fragment of tile t: rows lane/4 and lane/4 + 8, columns 2·(lane%4) + {0, 1}
 #pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const int col = warp * 32 + t * 8 + (lane & 3) * 2;
+  for (int t = 0; t < NT; ++t) {
+    const int col = warp * WC + t * 8 + (lane & 3) * 2;
     const int m = lane >> 2;
-    cta[m * kMmaCols + col] = d[t][0];
-    cta[m * kMmaCols + col + 1] = d[t][1];
-    cta[(m + 8) * kMmaCols + col] = d[t][2];
-    cta[(m + 8) * kMmaCols + col + 1] = d[t][3];
+    cta[m * Cfg::COLS + col] = d[t][0];
+    cta[m * Cfg::COLS + col + 1] = d[t][1];
+    cta[(m + 8) * Cfg::COLS + col] = d[t][2];
+    cta[(m + 8) * Cfg::COLS + col + 1] = d[t][3];
   }
   cluster.sync();
   if (crank == 0) {
-    for (int e = tid; e < 16 * kMmaCols; e += kGvThreads) {
-      const int m = e / kMmaCols;
-      const int64_t col = n0 + (e % kMmaCols);
+    for (int e = tid; e < 16 * Cfg::COLS; e += kGvThreads) {
+      const int m = e / Cfg::COLS;
+      const int64_t col = n0 + (e % Cfg::COLS);
       if (m >= M || col >= N) continue;
       float t = 0.f;
       for (unsigned q = 0; q < cs; ++q) t += cluster.map_shared_rank(cta, q)[e];
@@ -536,6 +560,41 @@ gemv_gather_mma_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t sA, 
     }
   }
   cluster.sync();
+}
+
+// cluster size (slices split over 1..8 CTAs): the one whose grid fills whole
+// waves of two CTAs per SM best, each CTA keeping >= 64 slices
+unsigned mma_cluster(int64_t blocks, int64_t k_keep, int sms) {
+  unsigned best_q = 1;
+  double best = -1.0;
+  for (unsigned q = 1; q <= kGvMaxCluster; ++q) {
+    if (q > 1 && k_keep < int64_t(q) * 64) break;
+    const double waves = double(blocks * q) / double(2 * sms);
+    const double eff = waves / std::max(1.0, std::ceil(waves));
+    if (eff > best + 1e-9) {
+      best = eff;
+      best_q = q;
+    }
+  }
+  return best_q;
+}
+
+template <int WC>
+cudaError_t launch_mma(const GemvArgs& g, int sms, int dev, cudaStream_t st) {
+  using Cfg = MmaCfg<WC>;
+  static std::atomic<bool> attr_done[64];  // per device; racing first calls both set the attribute
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_gather_mma_kernel<WC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(Cfg::SMEM));
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  const int64_t mblk = (g.N + Cfg::COLS - 1) / Cfg::COLS;
+  const unsigned mcs = mma_cluster(mblk * g.batch, g.k_keep, sms);
+  return launch_pdl(gemv_gather_mma_kernel<WC>, dim3(unsigned(mblk), mcs, unsigned(g.batch)), dim3(kGvThreads),
+                    Cfg::SMEM, st, dim3(1, mcs, 1), static_cast<const uint16_t*>(g.a), g.lda, g.strideA,
+                    static_cast<const uint16_t*>(g.b), g.ldb, g.strideB, g.M, g.N, g.idx, g.k_keep, g.c, g.ldc,
+                    g.strideC, int(g.out == kBF16));
 }
 
 template <typename T, int MT>
@@ -562,32 +621,12 @@ cudaError_t launch_mt(const GemvArgs& g, cudaStream_t st) {
   const int b_vec = (reinterpret_cast<uintptr_t>(g.b) % 16 == 0) && (g.ldb * int64_t(sizeof(T))) % 16 == 0 &&
                     (g.batch == 1 || (g.strideB * int64_t(sizeof(T))) % 16 == 0);
   if (b_vec && sizeof(T) == 2) {
-    const size_t msmem = gv_mma_smem_bytes();
-    const int64_t mblk = (g.N + kMmaCols - 1) / kMmaCols;
-    // cluster size (slices split over 1..8 CTAs): the one whose grid fills
-    // whole waves of two CTAs per SM best, each CTA keeping >= 64 slices
-    unsigned mcs = 1;
-    double best = -1.0;
-    for (unsigned q = 1; q <= kGvMaxCluster; ++q) {
-      if (q > 1 && g.k_keep < int64_t(q) * 64) break;
-      const double waves = double(mblk * g.batch * q) / double(2 * sms);
-      const double eff = waves / std::max(1.0, std::ceil(waves));
-      if (eff > best + 1e-9) {
-        best = eff;
-        mcs = q;
-      }
-    }
-    static std::atomic<bool> mma_attr[64];  // per device; racing first calls both set the attribute
-    if (dev >= 0 && dev < 64 && !mma_attr[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(gemv_gather_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           int(msmem));
-      if (e != cudaSuccess) return e;
-      mma_attr[dev] = true;
-    }
-    return launch_pdl(gemv_gather_mma_kernel, dim3(unsigned(mblk), mcs, unsigned(g.batch)), dim3(kGvThreads), msmem,
-                      st, dim3(1, mcs, 1), static_cast<const uint16_t*>(g.a), g.lda, g.strideA,
-                      static_cast<const uint16_t*>(g.b), g.ldb, g.strideB, g.M, g.N, g.idx, g.k_keep, g.c, g.ldc,
-                      g.strideC, int(g.out == kBF16));
+    // 512 columns per CTA when that grid, with clusters of up to 8 CTAs, can
+    // fill a wave of two CTAs per SM; 256 otherwise (small layers)
+    const int64_t wide = (g.N + MmaCfg<64>::COLS - 1) / MmaCfg<64>::COLS;
+    if (wide * g.batch * int64_t(kGvMaxCluster) >= 2 * int64_t(sms))
+      return launch_mma<64>(g, sms, dev, st);
+    return launch_mma<32>(g, sms, dev, st);
   }
   if (b_vec) {
     const size_t asmem = gv_async_smem_bytes<T, MT>();
@@ -795,23 +834,6 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
   cluster.sync();
 }
 
-// cluster size (1..8) whose grid fills whole waves of two CTAs per SM best,
-// each CTA keeping >= 64 slices
-unsigned wave_cluster(int64_t blocks, int64_t k_keep, int sms) {
-  unsigned best_q = 1;
-  double best = -1.0;
-  for (unsigned q = 1; q <= kGvMaxCluster; ++q) {
-    if (q > 1 && k_keep < int64_t(q) * 64) break;
-    const double waves = double(blocks * q) / double(2 * sms);
-    const double eff = waves / std::max(1.0, std::ceil(waves));
-    if (eff > best + 1e-9) {
-      best = eff;
-      best_q = q;
-    }
-  }
-  return best_q;
-}
-
 template <int MT>
 cudaError_t launch_w8_mt(const GemvArgs& g, const float* scale, int64_t s_stride, cudaStream_t st) {
   const size_t smem = gv_async_smem_bytes<int8_t, MT>();
@@ -853,7 +875,7 @@ cudaError_t launch_gemv_gather_w8(const GemvArgs& g, const float* scale, int64_t
     }
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t mblk = (g.N + kW8Cols - 1) / kW8Cols;
-    const unsigned mcs = wave_cluster(mblk * g.batch, g.k_keep, sms);
+    const unsigned mcs = mma_cluster(mblk * g.batch, g.k_keep, sms);
     return launch_pdl(gemv_gather_mma_w8_kernel, dim3(unsigned(mblk), mcs, unsigned(g.batch)), dim3(kGvThreads),
                       smem, st, dim3(1, mcs, 1), static_cast<const uint16_t*>(g.a), g.lda, g.strideA,
                       static_cast<const int8_t*>(g.b), g.ldb, g.strideB, g.M, g.N, g.idx, g.k_keep, g.c, g.ldc,

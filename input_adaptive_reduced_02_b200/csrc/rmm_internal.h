@@ -107,15 +107,38 @@ struct SplitZero {
   int32_t tiles_m, tiles_n, tile_rows, tile_cols;
 };
 
+// Scores of a few rows of A (the decode shapes) that the selection computes
+// itself instead of reading them: s_k = sqrt(sum_m A[m][k]^2), times bn[k]
+// when B's row norms are given (bn null: the A-only score). The sums follow
+// the score kernel's order for these shapes, so the scores are the same bits.
+struct RowScore {
+  const void* A;  // [batch][M][K] at lda / sA elements
+  int64_t lda, sA;
+  int32_t M;      // <= kRowScoreMaxM
+  int32_t bf16;   // 1: bf16 elements, 0: f32
+  int32_t a_vec;  // A's base, lda and sA allow 16-byte loads
+  const float* bn;  // [batch][K] at bn_stride, or null
+  int64_t bn_stride;
+};
+// Largest K whose selection keeps its keys in registers, and the sizes up to
+// which the selection scores A's rows itself (RowScore): at most 16 keys per
+// thread and 4 rows, so that all of a thread's loads fit in flight at once.
+constexpr int64_t kSelectRegisterK = 512 * 64;
+constexpr int64_t kRowScoreMaxK = 512 * 16;
+constexpr int32_t kRowScoreMaxM = 4;
+
 // select.cu
 //  Blocks [batch, batch + zero_blocks) of the launch zero `zero`'s tiles
 //  meanwhile (zero may be null); the select itself uses one block per item.
 //  late_launch: release the next kernel only once the kernel before the
 //  selection has completed (the fused calls' decode route, whose GEMV needs
 //  whole free SMs for its clusters).
-cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,
+//  rows: non-null (K <= kRowScoreMaxK): compute the scores from A's rows
+//  (and write them to s) instead of reading s. clear_status: the selection is
+//  the call's first kernel and its only block clears the status word first.
+cudaError_t launch_select(float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,
                           uint32_t* status, cudaStream_t st, const SplitZero* zero = nullptr,
-                          bool late_launch = false);
+                          bool late_launch = false, const RowScore* rows = nullptr, bool clear_status = false);
 
 // pack.cu
 //  out[b][r][t] = X[b][r][idx[b][t]] for t < k_keep, 0 for k_keep <= t < k_pad.

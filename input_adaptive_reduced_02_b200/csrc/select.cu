@@ -38,6 +38,9 @@ namespace {
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kMaxKeysPerThread = 64;  // keys held in registers: K <= 32768
+static_assert(int64_t(kSelThreads) * kMaxKeysPerThread == kSelectRegisterK, "register-key limit");
+constexpr int kRowScoreKeys = 16;  // keys per thread up to which the selection can score A's rows
+static_assert(int64_t(kSelThreads) * kRowScoreKeys == kRowScoreMaxK, "row-score limit");
 constexpr int kDigitBits = 12;
 constexpr int kBins = 1 << kDigitBits;
 constexpr int kBinsPerThread = kBins / kSelThreads;
@@ -86,9 +89,10 @@ __device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t* wtot
 // KPT == 0: thread t owns [t·kpt, (t+1)·kpt), re-read from global memory in
 // every sweep (any K up to 2^21).
 template <int KPT>
-__device__ __forceinline__ void select_item(const float* __restrict__ sb, int K, int64_t k_keep,
+__device__ __forceinline__ void select_item(float* __restrict__ sb, int K, int64_t k_keep,
                                             int32_t* __restrict__ ib, uint32_t* status, uint32_t (*hist)[kBins],
-                                            uint32_t* wsum_a, uint32_t* wsum_b, uint64_t* wtot, uint32_t* sh) {
+                                            uint32_t* wsum_a, uint32_t* wsum_b, uint64_t* wtot, uint32_t* sh,
+                                            const RowScore& rs, int64_t item) {
   constexpr int R = KPT ? KPT : 1;  // register slots
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kpt = KPT ? KPT : (K + kSelThreads - 1) / kSelThreads;  // keys per thread
@@ -117,10 +121,114 @@ __device__ __forceinline__ void select_item(const float* __restrict__ sb, int K,
     kmin = min(kmin, k);
     kmax = max(kmax, k);
   };
+  bool taken = false;  // keys computed from A's rows
+  if constexpr (KPT > 0 && KPT <= kRowScoreKeys) {
+    if (rs.A) {
+      // Scores of this thread's run from A's rows (and B's row norms): per
+      // key the rounded squares added in row order from 0, as the score
+      // kernel's single CTA per strip adds its row lanes (one row each for
+      // these M); then sqrt, then the product with ||B[k,:]||. Every operation
+      // rounds on its own (no fused multiply-add), so the bits match. All
+      // loads of a pair of rows (and the norms) are issued before any use:
+      // one memory round trip per pair of rows.
+      const bool full = base + KPT <= K;
+      const float* bnb = rs.bn ? rs.bn + item * rs.bn_stride : nullptr;
+      float nb[KPT];
+      if (bnb) {
+        if (KPT % 4 == 0 && full && (reinterpret_cast<uintptr_t>(bnb + base) & 15u) == 0) {
+#pragma unroll
+          for (int q = 0; q < KPT / 4; ++q) {
+            const float4 v = reinterpret_cast<const float4*>(bnb + base)[q];
+            nb[4 * q] = v.x;
+            nb[4 * q + 1] = v.y;
+            nb[4 * q + 2] = v.z;
+            nb[4 * q + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < KPT; ++q) nb[q] = base + q < K ? bnb[base + q] : 0.f;
+        }
+      }
+      float ss[KPT];
+#pragma unroll
+      for (int q = 0; q < KPT; ++q) ss[q] = 0.f;
+      const int64_t e = rs.bf16 ? 2 : 4;
+      const bool avec = rs.a_vec && full && (KPT * e) % 16 == 0;
+      const unsigned char* a_run = static_cast<const unsigned char*>(rs.A) + (item * rs.sA + base) * e;
+      for (int m0 = 0; m0 < rs.M; m0 += 2) {
+        float x[2][KPT];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int m = m0 + r;
+#pragma unroll
+          for (int q = 0; q < KPT; ++q) x[r][q] = 0.f;
+          if (m >= rs.M) continue;
+          const unsigned char* row = a_run + int64_t(m) * rs.lda * e;
+          if (rs.bf16) {
+            if (avec) {
+#pragma unroll
+              for (int q = 0; q < KPT / 8; ++q) {
+                const uint4 u = reinterpret_cast<const uint4*>(row)[q];
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  x[r][8 * q + 2 * h] = __uint_as_float(w[h] << 16);
+                  x[r][8 * q + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int q = 0; q < KPT; ++q)
+                if (base + q < K) x[r][q] = bf16_to_f32(reinterpret_cast<const uint16_t*>(row)[q]);
+            }
+          } else {
+            if (avec) {
+#pragma unroll
+              for (int q = 0; q < KPT / 4; ++q) {
+                const float4 v = reinterpret_cast<const float4*>(row)[q];
+                x[r][4 * q] = v.x;
+                x[r][4 * q + 1] = v.y;
+                x[r][4 * q + 2] = v.z;
+                x[r][4 * q + 3] = v.w;
+              }
+            } else {
+#pragma unroll
+              for (int q = 0; q < KPT; ++q)
+                if (base + q < K) x[r][q] = reinterpret_cast<const float*>(row)[q];
+            }
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          if (m0 + r >= rs.M) break;
+#pragma unroll
+          for (int q = 0; q < KPT; ++q) ss[q] = __fadd_rn(ss[q], __fmul_rn(x[r][q], x[r][q]));
+        }
+      }
+      float sc[KPT];
+#pragma unroll
+      for (int q = 0; q < KPT; ++q) {
+        sc[q] = sqrtf(ss[q]);
+        if (bnb) sc[q] = __fmul_rn(sc[q], nb[q]);
+        if (base + q < K) take_key(q, sc[q]);
+      }
+      // the scores, for the caller's workspace
+      if (KPT % 4 == 0 && full && (reinterpret_cast<uintptr_t>(sb + base) & 15u) == 0) {
+#pragma unroll
+        for (int q = 0; q < KPT / 4; ++q)
+          reinterpret_cast<float4*>(sb + base)[q] = make_float4(sc[4 * q], sc[4 * q + 1], sc[4 * q + 2], sc[4 * q + 3]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < KPT; ++q)
+          if (base + q < K) sb[base + q] = sc[q];
+      }
+      taken = true;
+    }
+  }
   bool vec = false;
   if constexpr (KPT > 0 && KPT % 4 == 0) {
     // a whole run in range: 16-byte loads (a warp reads 128·KPT contiguous bytes)
-    vec = base + KPT <= K && (reinterpret_cast<uintptr_t>(sb) & 15u) == 0;
+    vec = !taken && base + KPT <= K && (reinterpret_cast<uintptr_t>(sb) & 15u) == 0;
     if (vec) {
 #pragma unroll
       for (int j = 0; j < KPT; j += 4) {
@@ -132,7 +240,7 @@ __device__ __forceinline__ void select_item(const float* __restrict__ sb, int K,
       }
     }
   }
-  if (!vec) {
+  if (!vec && !taken) {
 #pragma unroll
     for (int j = 0; j < kpt; ++j)
       if (base + j < K) take_key(j, sb[base + j]);
@@ -258,8 +366,9 @@ __device__ __forceinline__ void select_item(const float* __restrict__ sb, int K,
 
 template <int KPT>
 __global__ void __launch_bounds__(kSelThreads, 1)
-select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t* __restrict__ idx,
-              uint32_t* status, int64_t items, const SplitZero zero, int late_launch) {
+select_kernel(float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t* __restrict__ idx,
+              uint32_t* status, int64_t items, const SplitZero zero, int late_launch, const RowScore rs,
+              int clear_status) {
   const int K = int(K64);  // K <= 2^21 (checked on the host)
   __shared__ __align__(16) uint32_t hist[2][kBins];
   __shared__ uint32_t wsum_a[kSelWarps], wsum_b[kSelWarps];
@@ -274,18 +383,23 @@ select_kernel(const float* __restrict__ s, int64_t K64, int64_t k_keep, int32_t*
   if (!late_launch) pdl_trigger();
   pdl_wait();
   if (late_launch) pdl_trigger();
+  if (clear_status) {  // a launch of one block, the call's first kernel
+    if (threadIdx.x == 0) *status = 0u;
+    __syncthreads();
+  }
   if (blockIdx.x >= items) {  // helper block: zero C tiles for the GEMM later on the stream
     zero_split_tiles(zero, blockIdx.x - items, gridDim.x - items, threadIdx.x, kSelThreads);
     return;
   }
   select_item<KPT>(s + int64_t(blockIdx.x) * K, K, k_keep, idx + int64_t(blockIdx.x) * k_keep, status, hist,
-                   wsum_a, wsum_b, wtot, sh);
+                   wsum_a, wsum_b, wtot, sh, rs, int64_t(blockIdx.x));
 }
 
 }  // namespace
 
-cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,
-                          uint32_t* status, cudaStream_t st, const SplitZero* zero, bool late_launch) {
+cudaError_t launch_select(float* s, int64_t batch, int64_t K, int64_t k_keep, int32_t* idx,
+                          uint32_t* status, cudaStream_t st, const SplitZero* zero, bool late_launch,
+                          const RowScore* rows, bool clear_status) {
   if (batch == 0) return cudaSuccess;
   SplitZero z = {};
   int64_t helpers = 0;
@@ -294,21 +408,26 @@ cudaError_t launch_select(const float* s, int64_t batch, int64_t K, int64_t k_ke
     const int64_t vecs = z.count * z.tile_rows * (z.tile_cols / 4);
     helpers = std::min<int64_t>(147, (vecs + 4 * kSelThreads - 1) / (4 * kSelThreads));
   }
+  RowScore rs = {};
+  if (rows) {
+    if (K > kRowScoreMaxK || rows->M > kRowScoreMaxM) return cudaErrorInvalidValue;
+    rs = *rows;
+  }
+  if (clear_status && batch + helpers != 1) return cudaErrorInvalidValue;
   const dim3 grid(unsigned(batch + helpers)), block(kSelThreads), none(0, 0, 0);
-  const int ll = int(late_launch);
+  const int ll = int(late_launch), cl = int(clear_status);
   const int64_t kpt = (K + kSelThreads - 1) / kSelThreads;
-  if (kpt <= 1) return launch_pdl(select_kernel<1>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
-  if (kpt <= 2) return launch_pdl(select_kernel<2>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
-  if (kpt <= 4) return launch_pdl(select_kernel<4>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
-  if (kpt <= 8) return launch_pdl(select_kernel<8>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
-  if (kpt <= 16)
-    return launch_pdl(select_kernel<16>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
-  if (kpt <= 32)
-    return launch_pdl(select_kernel<32>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
-  if (kpt <= kMaxKeysPerThread)
-    return launch_pdl(select_kernel<kMaxKeysPerThread>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch,
-                      z, ll);
-  return launch_pdl(select_kernel<0>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll);
+#define RMM_SELECT(KPT_) \
+  launch_pdl(select_kernel<KPT_>, grid, block, 0, st, none, s, K, k_keep, idx, status, batch, z, ll, rs, cl)
+  if (kpt <= 1) return RMM_SELECT(1);
+  if (kpt <= 2) return RMM_SELECT(2);
+  if (kpt <= 4) return RMM_SELECT(4);
+  if (kpt <= 8) return RMM_SELECT(8);
+  if (kpt <= 16) return RMM_SELECT(16);
+  if (kpt <= 32) return RMM_SELECT(32);
+  if (kpt <= kMaxKeysPerThread) return RMM_SELECT(kMaxKeysPerThread);
+  return RMM_SELECT(0);
+#undef RMM_SELECT
 }
 
 }  // namespace rmm

@@ -290,7 +290,6 @@ softmax_score_kernel(const T* __restrict__ L, int64_t S_q, int64_t S_k, float xs
     const uint32_t ring = smem_addr(sm_ring);
     const uint32_t srow = ring + uint32_t(kRing * kRowUnroll * kSmThreads * 16);  // [kRing][kRowUnroll][RL] float2
     const int64_t nrows = r1 - r0 > rl ? (r1 - r0 - rl + RL - 1) / RL : 0;  // rows of this thread
-    const int64_t nbat = (nrows + kRowUnroll - 1) / kRowUnroll;
     const int64_t nbat_cta = ((r1 - r0 + RL - 1) / RL + kRowUnroll - 1) / kRowUnroll;  // the same in every thread
     const T* Lt = Lb + c0;
     uint16_t* Pt = Pb + c0;
