@@ -203,7 +203,11 @@ rmm_status rmm_gemm_full(const void* A, int64_t lda, int64_t strideA, const void
 
 /* Which route a fused call (rmm_matmul_reduced, _batched, _b_norms,
  * rmm_qk_reduced, rmm_pv_reduced) takes for these sizes and this A:
- *   2 = gather-GEMV (M <= 16 and B row-major: score, select, rmm_gemv_gather);
+ *   2 = gather-GEMV (M <= 16 and B row-major: score, select, rmm_gemv_gather;
+ *       when the score needs only A — B's row norms given, or the A-only
+ *       score — and M <= 4, K <= 8192, the selection kernel computes the
+ *       scores itself, bit-identical to rmm_score_b_norms / rmm_score, so the
+ *       call launches two kernels);
  *   1 = stream (bf16, B row-major, N <= 128, M > 16, A streamable as in
  *       rmm_gemm_full: score, select, rmm_mask_rows, rmm_gemm_full). A
  *       narrow product is bound by reading A, and A's kept columns reach into
