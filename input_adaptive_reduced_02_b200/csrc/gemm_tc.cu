@@ -16,7 +16,10 @@
 //   warp 1      allocates tensor memory; in the leader one lane issues
 //               tcgen05.mma (kind::f16, bf16 x bf16 -> f32, K = 16) into one of
 //               two TMEM accumulators and commits ring stages back to both CTAs
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, optional bf16
+//   warps 2..    epilogue (4 warps, one per TMEM lane quadrant; or 8, two per
+//               quadrant each taking half the columns, when a tile has at most
+//               two k-blocks and the product is bound by writing C):
+//               tcgen05.ld 32 lanes x 32 columns, optional bf16
 //               rounding, swizzled staging in shared memory, TMA tile store
 // Two accumulators let the epilogue of tile i overlap the mainloop of tile
 // i+1. Tiles are visited m-fastest so a column block of B is shared through
@@ -46,24 +49,26 @@ namespace {
 constexpr int BM = 128;  // rows of A per CTA
 constexpr int BK = 64;   // 64 bf16 = one 128-byte swizzle row
 constexpr int kUmmaK = 16;
-constexpr int kEpiWarps = 4;
-constexpr int kTcThreads = 64 + 32 * kEpiWarps;
-
-template <int BN, int CG>
+// Epilogue warps EW: 4, one per TMEM lane quadrant; or 8 (two per quadrant,
+// each taking half of the tile's columns) for write-bound products with few
+// k-blocks per tile, at the cost of one ring stage.
+template <int BN, int CG, int EW = 4>
 struct TcCfg {
+  static constexpr int THREADS = 64 + 32 * EW;
   static constexpr int BN_CTA = BN / CG;  // columns of B held by one CTA
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN_CTA * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = int((192u * 1024u) / STAGE_BYTES);
+  static constexpr int STAGES = int(((EW == 8 ? 160u : 192u) * 1024u) / STAGE_BYTES);
   static constexpr uint32_t EPI_BUF = 32 * 128;  // 32 rows x 128 bytes
-  static constexpr uint32_t EPI_BYTES = kEpiWarps * 2 * EPI_BUF;
+  static constexpr uint32_t EPI_BYTES = EW * 2 * EPI_BUF;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
   static constexpr uint32_t BAR_BYTES = 256;
   static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
 };
 static_assert(TcCfg<256, 1>::SMEM <= 232448 && TcCfg<128, 1>::SMEM <= 232448, "shared memory budget");
 static_assert(TcCfg<256, 2>::SMEM <= 232448 && TcCfg<128, 2>::SMEM <= 232448, "shared memory budget");
+static_assert(TcCfg<256, 2, 8>::SMEM <= 232448 && TcCfg<128, 2, 8>::SMEM <= 232448, "shared memory budget");
 static_assert(TcCfg<128, 2>::STAGES * 2 + 6 <= 32, "barrier area");
 
 struct TcParams {
@@ -130,11 +135,11 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t* 
   status_or(status, RMM_TIMEOUT_BIT);
 }
 
-template <int BN, bool BMN, int CG>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <int BN, bool BMN, int CG, int EW>
+__global__ void __launch_bounds__(TcCfg<BN, CG, EW>::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, const TcParams p) {
-  using Cfg = TcCfg<BN, CG>;
+  using Cfg = TcCfg<BN, CG, EW>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int BN_CTA = Cfg::BN_CTA;
   extern __shared__ uint8_t tc_smem_raw[];
@@ -164,7 +169,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], kEpiWarps * CG);
+      mbar_init(&tempty[a], EW * CG);
     }
     mbar_init(drain, 1);
     *abort_sh = 0;
@@ -317,6 +322,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     bool ok = true;
     const int cols_per_chunk = p.out_bf16 ? 64 : 32;
     const int chunks = BN / cols_per_chunk;
+    // this warp's chunks: all of them, or one half with two warps per quadrant
+    const int c_begin = EW == 8 ? ((warp - 2) >> 2) * (chunks / 2) : 0;
+    const int c_end = EW == 8 ? c_begin + chunks / 2 : chunks;
     for (int64_t u = pair; ok && u < p.total_units; u += npairs) {
       const Unit unit = unit_info(u, p);
       int32_t b, mb, nb;
@@ -331,7 +339,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       tc_fence_after();
       const uint32_t t_row = tmem_base + (uint32_t(q * 32) << 16) + acc * BN;
       const int32_t row0 = mb * BM * CG + int32_t(rank) * BM + q * 32;
-      for (int c = 0; c < chunks; ++c) {
+      for (int c = c_begin; c < c_end; ++c) {
         uint32_t packed[32];
         if (p.out_bf16) {
           uint32_t r0[32], r1[32];
@@ -347,8 +355,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           tmem_ld_32x32b_x32(t_row + c * 32, packed);
           tmem_ld_wait();
         }
-        if (c == chunks - 1) {
-          // whole accumulator read: hand it back to the leader's MMA lane
+        if (c == c_end - 1) {
+          // this warp's part of the accumulator read: hand it back to the leader's MMA lane
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
@@ -456,10 +464,10 @@ struct DevInfo {
   bool attr_done = false;
 };
 
-template <int BN, bool BMN, int CG>
+template <int BN, bool BMN, int CG, int EW = 4>
 void set_attr() {
-  cudaFuncSetAttribute(gemm_tc_kernel<BN, BMN, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       int(TcCfg<BN, CG>::SMEM));
+  cudaFuncSetAttribute(gemm_tc_kernel<BN, BMN, CG, EW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       int(TcCfg<BN, CG, EW>::SMEM));
 }
 
 DevInfo& dev_info(int dev) {
@@ -480,6 +488,10 @@ DevInfo& dev_info(int dev) {
       set_attr<128, false, 2>();
       set_attr<256, true, 2>();
       set_attr<128, true, 2>();
+      set_attr<256, false, 2, 8>();
+      set_attr<128, false, 2, 8>();
+      set_attr<256, true, 2, 8>();
+      set_attr<128, true, 2, 8>();
     }
     d.attr_done = true;
   }
@@ -540,9 +552,9 @@ SplitZero split_zero(const GemmArgs& g, const Plan& q) {
   return z;
 }
 
-template <int BN, bool BMN, int CG>
+template <int BN, bool BMN, int CG, int EW>
 cudaError_t launch_cfg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, const char** why) {
-  using Cfg = TcCfg<BN, CG>;
+  using Cfg = TcCfg<BN, CG, EW>;
   const uint64_t kp = uint64_t(g.k_pad);
   CUtensorMap tmA, tmB, tmC;
   // a batch of one takes any batch stride (TMA needs a nonzero multiple of 16 bytes)
@@ -601,17 +613,27 @@ cudaError_t launch_cfg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, co
     cudaError_t e = cudaEventRecord(g.ev_start, st);
     if (e != cudaSuccess) return e;
   }
-  cudaError_t e = launch_pdl(gemm_tc_kernel<BN, BMN, CG>, dim3(unsigned(grid)), dim3(kTcThreads), Cfg::SMEM, st,
+  cudaError_t e = launch_pdl(gemm_tc_kernel<BN, BMN, CG, EW>, dim3(unsigned(grid)), dim3(Cfg::THREADS), Cfg::SMEM, st,
                              CG == 2 ? dim3(2, 1, 1) : dim3(0, 0, 0), tmA, tmB, tmC, p);
   if (e == cudaSuccess && g.ev_stop) e = cudaEventRecord(g.ev_stop, st);
   return e;
 }
 
+template <int CG, int EW>
+cudaError_t launch_cg_ew(const GemmArgs& g, const DevInfo& di, cudaStream_t st, const char** why) {
+  if (g.b_kmajor)
+    return g.N <= 128 ? launch_cfg<128, false, CG, EW>(g, di, st, why) : launch_cfg<256, false, CG, EW>(g, di, st, why);
+  return g.N <= 128 ? launch_cfg<128, true, CG, EW>(g, di, st, why) : launch_cfg<256, true, CG, EW>(g, di, st, why);
+}
+
+// With at most two k-blocks per tile the product is bound by writing C: the
+// 2-SM kernels then run 8 epilogue warps.
 template <int CG>
 cudaError_t launch_cg(const GemmArgs& g, const DevInfo& di, cudaStream_t st, const char** why) {
-  if (g.b_kmajor)
-    return g.N <= 128 ? launch_cfg<128, false, CG>(g, di, st, why) : launch_cfg<256, false, CG>(g, di, st, why);
-  return g.N <= 128 ? launch_cfg<128, true, CG>(g, di, st, why) : launch_cfg<256, true, CG>(g, di, st, why);
+  if constexpr (CG == 2) {
+    if (g.k_pad <= 2 * BK) return launch_cg_ew<2, 8>(g, di, st, why);
+  }
+  return launch_cg_ew<CG, 4>(g, di, st, why);
 }
 
 }  // namespace
