@@ -61,16 +61,21 @@ __device__ __forceinline__ bool wait_loads(uint64_t* bar, uint64_t limit_ns, uin
 
 // Gather kept columns of nr staged rows; ib points at the kept indices (in
 // shared memory or global memory; read as 16-byte vectors when ib_vec, i.e.
-// ib is 16-byte aligned, else one by one).
+// ib is 16-byte aligned, else one by one). The threads take the nr x (k_pad / V)
+// output vectors in order, so that short output rows (few kept columns, e.g.
+// a head dimension of 128) still keep every thread busy and the stores stay
+// contiguous.
 template <typename T>
 __device__ __forceinline__ void gather_rows(const T* srow, int nr, int64_t C, const int32_t* ib, bool ib_vec,
                                             int64_t k_keep, int64_t k_pad, T* dst) {
   constexpr int V = 16 / sizeof(T);
-  const int64_t ng = k_pad / V;
-  for (int rr = 0; rr < nr; ++rr) {
+  const int ng = int(k_pad / V);  // k_pad <= 2^21 and nr <= 64: nr · ng fits an int
+  const int total = nr * ng;
+  for (int e = threadIdx.x; e < total; e += kPackThreads) {
+    const int rr = e / ng, g = e - rr * ng;
     const T* row = srow + rr * C;
-    for (int64_t g = threadIdx.x; g < ng; g += kPackThreads) {
-      const int64_t t0 = g * V;
+    {
+      const int64_t t0 = int64_t(g) * V;
       Vec16<T> v;
       if (ib_vec && t0 + V <= k_keep) {
         const int4 i0 = *reinterpret_cast<const int4*>(ib + t0);
@@ -154,7 +159,6 @@ __global__ void __launch_bounds__(kPackThreads)
 pack_cols_plain_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int64_t R, int64_t C,
                        const int32_t* __restrict__ idx, int64_t k_keep, int64_t k_pad, T* __restrict__ out,
                        int rows_per_cta) {
-  constexpr int V = 16 / sizeof(T);
   extern __shared__ __align__(128) unsigned char pack_smem[];
   T* srow = reinterpret_cast<T*>(pack_smem);
   const int64_t b = blockIdx.y;
@@ -180,19 +184,7 @@ pack_cols_plain_kernel(const T* __restrict__ X, int64_t ld, int64_t bstride, int
   }
   __syncthreads();
   const int32_t* ib = idx + b * k_keep;
-  T* dst = out + (b * R + r0) * k_pad;
-  for (int rr = 0; rr < nr; ++rr) {
-    const T* row = srow + rr * C;
-    for (int64_t g = threadIdx.x; g < k_pad / V; g += kPackThreads) {
-      Vec16<T> v;
-#pragma unroll
-      for (int j = 0; j < V; ++j) {
-        const int64_t t = g * V + j;
-        v.e[j] = t < k_keep ? row[ib[t]] : T(0);
-      }
-      reinterpret_cast<uint4*>(dst + rr * k_pad)[g] = v.u;
-    }
-  }
+  gather_rows(srow, nr, C, ib, (reinterpret_cast<uintptr_t>(ib) & 15u) == 0, k_keep, k_pad, out + (b * R + r0) * k_pad);
 }
 
 // Rows too long for shared memory: gather straight from global memory.
