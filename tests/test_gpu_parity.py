@@ -468,3 +468,37 @@ def test_select_matches_definition_across_shapes(K, batch):
                 want = O.select_top(s[b].double().cpu().numpy(), k).tolist()
                 assert idx[b].cpu().numpy().tolist() == want, (name, k, b)
 
+
+
+@pytest.mark.parametrize("M,K,N,out_dtype", [(4096, 200, 4096, torch.float32), (4096, 200, 4096, torch.bfloat16),
+                                              (2048, 256, 100, torch.float32), (1000, 60, 777, torch.float32)],
+                         ids=["4096x200x4096-f32-split", "4096x200x4096-bf16", "2048x256x100-f32-split",
+                              "1000x60x777-f32"])
+def test_write_bound_gemm_epilogue(M, K, N, out_dtype):
+    """Packed products with at most two k-blocks per tile (k_pad <= 128) run
+    the 2-SM GEMM with 8 epilogue warps, two per TMEM lane quadrant, each
+    storing half of a tile's columns; with f32 C and a partial last round
+    that round is also split along K (both halves reduce-add into zeroed
+    tiles; N <= 128 puts every tile there). The stage-call GEMM must match the
+    oracle on rows sampled from every 256-row band (both CTAs of a pair, all
+    four lane quadrants), ragged edges included, and the fused call must equal
+    the stage calls of its own route bit for bit (N <= 128 streams A through
+    the GEMM with B's dropped rows zeroed, a different summation order)."""
+    A, B = _ab(M, K, N, torch.bfloat16, seed=M + K + N)
+    k = rmm.keep_count(0.5, K)
+    assert rmm.padded_keep(k) <= 128
+    idx = torch.empty(k, dtype=torch.int32, device=DEV)
+    C, ws = rmm.matmul_reduced(A, B, 0.5, out_dtype=out_dtype, idx_out=idx)
+    torch.cuda.synchronize()
+    rmm.check(ws)
+    A_S, B_S = rmm.pack(A, B, idx)
+    C_packed = rmm.gemm(A_S, B_S, k, out_dtype, N=N)
+    if rmm.fused_route(A, N) == rmm.ROUTE_STREAM:
+        assert torch.equal(C, rmm.gemm_full(A, rmm.mask_rows(B, idx), N, out_dtype))
+    else:
+        assert torch.equal(C, C_packed)
+    rows = sorted(set(range(0, M, 37)) | {M - 1})
+    A64, B64, ii = f64(A), f64(B), idx.cpu().numpy()
+    tol = product_tol(torch.bfloat16, out_dtype)
+    check_product(C_packed[rows], A64[rows], B64, ii, tol)
+    check_product(C[rows], A64[rows], B64, ii, tol)
