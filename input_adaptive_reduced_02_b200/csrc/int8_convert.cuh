@@ -29,12 +29,4 @@ __device__ __forceinline__ uint32_t pack_bf16x2_exact(float lo, float hi) {
   return __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x7632);
 }
 
-// Four signed bytes -> two bf16x2 words (bytes 0,1 in lo; 2,3 in hi), exactly.
-__device__ __forceinline__ void s8x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  float f0, f1, f2, f3;
-  s8x4_to_f32(w, f0, f1, f2, f3);
-  lo = pack_bf16x2_exact(f0, f1);
-  hi = pack_bf16x2_exact(f2, f3);
-}
-
 }  // namespace rmm
