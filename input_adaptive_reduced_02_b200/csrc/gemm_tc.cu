@@ -339,33 +339,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       tc_fence_after();
       const uint32_t t_row = tmem_base + (uint32_t(q * 32) << 16) + acc * BN;
       const int32_t row0 = mb * BM * CG + int32_t(rank) * BM + q * 32;
-      for (int c = c_begin; c < c_end; ++c) {
-        uint32_t packed[32];
-        if (p.out_bf16) {
-          uint32_t r0[32], r1[32];
-          tmem_ld_32x32b_x32(t_row + c * 64, r0);
-          tmem_ld_32x32b_x32(t_row + c * 64 + 32, r1);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            packed[j] = pack_bf16x2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
-            packed[16 + j] = pack_bf16x2(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
-          }
-        } else {
-          tmem_ld_32x32b_x32(t_row + c * 32, packed);
-          tmem_ld_wait();
-        }
-        if (c == c_end - 1) {
-          // this warp's part of the accumulator read: hand it back to the leader's MMA lane
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            if (CG == 1 || rank == 0)
-              mbar_arrive(&tempty[acc]);
-            else
-              mbar_arrive_cluster(mapa_shared(smem_addr(&tempty[acc]), 0));
-          }
-        }
+      // Store chunk c (32 rows x cols_per_chunk columns, `packed` holding its 32
+      // words per lane) through the staging buffers, or directly.
+      auto store_chunk = [&](int c, const uint32_t (&packed)[32]) {
         const int32_t col0 = nb * BN + c * cols_per_chunk;
         if (p.tma_store) {
           uint8_t* buf = bufs + nbuf * Cfg::EPI_BUF;
@@ -405,6 +381,71 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               }
             }
           }
+        }
+      };
+      if constexpr (EW == 8) {
+        // This warp's whole share of the tile (BN / 2 columns) is read from
+        // TMEM at once, and the accumulator is handed back before any store:
+        // one TMEM round trip per tile instead of one per chunk.
+        constexpr int NLD = BN / 64;  // 32-column loads
+        uint32_t r[NLD][32];
+        const uint32_t col_base = uint32_t(c_begin * cols_per_chunk);
+#pragma unroll
+        for (int l = 0; l < NLD; ++l) tmem_ld_32x32b_x32(t_row + col_base + 32 * l, r[l]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (CG == 1 || rank == 0)
+            mbar_arrive(&tempty[acc]);
+          else
+            mbar_arrive_cluster(mapa_shared(smem_addr(&tempty[acc]), 0));
+        }
+        if (p.out_bf16) {
+#pragma unroll
+          for (int i = 0; i < NLD / 2; ++i) {
+            uint32_t packed[32];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              packed[j] = pack_bf16x2(__uint_as_float(r[2 * i][2 * j]), __uint_as_float(r[2 * i][2 * j + 1]));
+              packed[16 + j] =
+                  pack_bf16x2(__uint_as_float(r[2 * i + 1][2 * j]), __uint_as_float(r[2 * i + 1][2 * j + 1]));
+            }
+            store_chunk(c_begin + i, packed);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < NLD; ++i) store_chunk(c_begin + i, r[i]);
+        }
+      } else {
+        for (int c = c_begin; c < c_end; ++c) {
+          uint32_t packed[32];
+          if (p.out_bf16) {
+            uint32_t r0[32], r1[32];
+            tmem_ld_32x32b_x32(t_row + c * 64, r0);
+            tmem_ld_32x32b_x32(t_row + c * 64 + 32, r1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              packed[j] = pack_bf16x2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
+              packed[16 + j] = pack_bf16x2(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
+            }
+          } else {
+            tmem_ld_32x32b_x32(t_row + c * 32, packed);
+            tmem_ld_wait();
+          }
+          if (c == c_end - 1) {
+            // this warp's part of the accumulator read: hand it back to the leader's MMA lane
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if (CG == 1 || rank == 0)
+                mbar_arrive(&tempty[acc]);
+              else
+                mbar_arrive_cluster(mapa_shared(smem_addr(&tempty[acc]), 0));
+            }
+          }
+          store_chunk(c, packed);
         }
       }
       acc ^= 1u;
