@@ -7,9 +7,10 @@
 // With a handful of rows the product is a matrix-vector product that streams
 // the kept rows of B once; skipping a row of B saves its bytes outright, so
 // every kernel here is built around HBM reads of B, and in all of them the
-// CTAs of a thread-block cluster (up to 8) split the kept slices and rank 0
-// adds the CTAs' partials in rank order through distributed shared memory
-// (fixed order throughout: bit-reproducible, no atomics). By B:
+// CTAs of a thread-block cluster (up to 8) split the kept slices, and the
+// cluster's CTAs then share out the output elements, each adding the CTAs'
+// partials in rank order through distributed shared memory (fixed order
+// throughout: bit-reproducible, no atomics). By B:
 //  * bf16, rows 16-byte aligned: gemv_gather_mma_kernel (tensor-core path,
 //    below) — each warp streams its own column strip through a private
 //    cp.async ring of 32-slice passes, mma.sync m16n8k16;
@@ -95,6 +96,44 @@ __device__ __forceinline__ void fma_row(float (&acc)[MT][4], const float* xrow, 
   }
 }
 
+// C[m][n0 + j] (m < M, j < cols, clipped to N) = the sum of the cluster's
+// CTA partials part[m·cols + j], added in rank order from 0 (the same bits
+// whichever thread adds them), times scale[n0 + j] when a column scale is
+// given. The elements are shared out over all of the cluster's CTAs, and each
+// thread keeps the remote loads of four elements in flight.
+__device__ __forceinline__ void cluster_sum_store(cg::cluster_group& cluster, float* part, int cols, int64_t M,
+                                                  int64_t n0, int64_t N, int64_t b, int64_t sC, int64_t ldc, void* C,
+                                                  int out_bf16, const float* scale, int nthreads) {
+  const int cs = int(cluster.num_blocks()), crank = int(cluster.block_rank());
+  const int total = int(M) * cols;
+  const int per = (total + cs - 1) / cs;
+  const int e0 = crank * per, e1 = min(total, e0 + per);
+  for (int e = e0 + int(threadIdx.x); e < e1; e += 4 * nthreads) {
+    float t[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int q = 0; q < cs; ++q) {
+      const float* src = cluster.map_shared_rank(part, q);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (e + u * nthreads < e1) t[u] += src[e + u * nthreads];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int eu = e + u * nthreads;
+      if (eu >= e1) break;
+      const int m = eu / cols;
+      const int64_t col = n0 + (eu - m * cols);
+      if (col >= N) continue;
+      float v = t[u];
+      if (scale) v *= scale[col];
+      const int64_t off = b * sC + int64_t(m) * ldc + col;
+      if (out_bf16)
+        static_cast<uint16_t*>(C)[off] = uint16_t(pack_bf16x2(v, 0.f) & 0xFFFFu);
+      else
+        static_cast<float*>(C)[off] = v;
+    }
+  }
+}
+
 // T: uint16_t (bf16 bits) or uint32_t (f32 bits). MT >= M rows of A.
 template <typename T, int MT>
 __global__ void __launch_bounds__(kGvThreads)
@@ -160,21 +199,8 @@ gemv_gather_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, const T* __
     cta[e] = t;
   }
   cluster.sync();  // every CTA's partial is written and visible cluster-wide
-  if (crank == 0) {
-    for (int e = tid; e < MT * kGvCols; e += kGvThreads) {
-      const int m = e / kGvCols;
-      const int64_t col = n0 + (e % kGvCols);
-      if (m >= M || col >= N) continue;
-      float t = 0.f;
-      for (unsigned q = 0; q < cs; ++q) t += cluster.map_shared_rank(cta, q)[e];
-      const int64_t off = b * sC + int64_t(m) * ldc + col;
-      if (out_bf16)
-        static_cast<uint16_t*>(C)[off] = uint16_t(pack_bf16x2(t, 0.f) & 0xFFFFu);
-      else
-        static_cast<float*>(C)[off] = t;
-    }
-  }
-  cluster.sync();  // keep shared memory alive until rank 0 has read it
+  cluster_sum_store(cluster, cta, kGvCols, M, n0, N, b, sC, ldc, C, out_bf16, nullptr, kGvThreads);
+  cluster.sync();  // keep shared memory alive until every rank has read it
 }
 
 // ---------------------------------------------------------------- async path
@@ -334,21 +360,8 @@ gemv_gather_async_kernel(const T* __restrict__ A, int64_t lda, int64_t sA, const
     cta[e] = t;
   }
   cluster.sync();
-  if (crank == 0) {
-    for (int e = tid; e < MT * kGvCols; e += kGvThreads) {
-      const int m = e / kGvCols;
-      const int64_t col = n0 + (e % kGvCols);
-      if (m >= M || col >= N) continue;
-      float t = 0.f;
-      for (unsigned q = 0; q < cs; ++q) t += cluster.map_shared_rank(cta, q)[e];
-      if (col_scale) t *= col_scale[b * s_stride + col];
-      const int64_t off = b * sC + int64_t(m) * ldc + col;
-      if (out_bf16)
-        static_cast<uint16_t*>(C)[off] = uint16_t(pack_bf16x2(t, 0.f) & 0xFFFFu);
-      else
-        static_cast<float*>(C)[off] = t;
-    }
-  }
+  cluster_sum_store(cluster, cta, kGvCols, M, n0, N, b, sC, ldc, C, out_bf16,
+                    col_scale ? col_scale + b * s_stride : nullptr, kGvThreads);
   cluster.sync();
 }
 static_assert(size_t(kGvWarps) * 16 * kGvCols * 4 <= size_t(2) * kGvPass * 32 * 8, "warp partials fit in the ring");
@@ -545,20 +558,7 @@ gemv_gather_mma_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t sA, 
     cta[(m + 8) * Cfg::COLS + col + 1] = d[t][3];
   }
   cluster.sync();
-  if (crank == 0) {
-    for (int e = tid; e < 16 * Cfg::COLS; e += kGvThreads) {
-      const int m = e / Cfg::COLS;
-      const int64_t col = n0 + (e % Cfg::COLS);
-      if (m >= M || col >= N) continue;
-      float t = 0.f;
-      for (unsigned q = 0; q < cs; ++q) t += cluster.map_shared_rank(cta, q)[e];
-      const int64_t off = b * sC + int64_t(m) * ldc + col;
-      if (out_bf16)
-        static_cast<uint16_t*>(C)[off] = uint16_t(pack_bf16x2(t, 0.f) & 0xFFFFu);
-      else
-        static_cast<float*>(C)[off] = t;
-    }
-  }
+  cluster_sum_store(cluster, cta, Cfg::COLS, M, n0, N, b, sC, ldc, C, out_bf16, nullptr, kGvThreads);
   cluster.sync();
 }
 
@@ -816,21 +816,7 @@ gemv_gather_mma_w8_kernel(const uint16_t* __restrict__ A, int64_t lda, int64_t s
     }
   }
   cluster.sync();
-  if (crank == 0) {
-    for (int e = tid; e < 16 * kW8Cols; e += kGvThreads) {
-      const int m = e / kW8Cols;
-      const int64_t col = n0 + (e % kW8Cols);
-      if (m >= M || col >= N) continue;
-      float acc = 0.f;
-      for (unsigned q = 0; q < cs; ++q) acc += cluster.map_shared_rank(cta, q)[e];
-      acc *= scale[b * s_stride + col];
-      const int64_t off = b * sC + int64_t(m) * ldc + col;
-      if (out_bf16)
-        static_cast<uint16_t*>(C)[off] = uint16_t(pack_bf16x2(acc, 0.f) & 0xFFFFu);
-      else
-        static_cast<float*>(C)[off] = acc;
-    }
-  }
+  cluster_sum_store(cluster, cta, kW8Cols, M, n0, N, b, sC, ldc, C, out_bf16, scale + b * s_stride, kGvThreads);
   cluster.sync();
 }
 
