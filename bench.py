@@ -300,12 +300,18 @@ def step_descr(p) -> str:
     if p.logits is not None:
         return ("one rmm_pv_softmax_reduced call (row statistics, P written with the key scores, select, "
                 "V's dropped rows zeroed, causal GEMM over P: 5 kernels)")
+    # decode shapes whose score needs only x: the selection scores x itself
+    folded = p.gemv and p.M <= 4 and p.K <= 8192
     if p.scale is not None:
         if p.gemv:
-            return "one rmm_matmul_reduced_w8 call with W's norms cached (score, select, INT8 gather-GEMV: 3 kernels)"
+            return ("one rmm_matmul_reduced_w8 call with W's norms cached ("
+                    + ("select scoring x itself, INT8 gather-GEMV: 2 kernels)" if folded
+                       else "score, select, INT8 gather-GEMV: 3 kernels)"))
         return "one rmm_matmul_reduced_w8 call with W's norms cached (score, select, INT8 pack, gemm: 4 kernels)"
     if p.gemv:
-        return "one rmm_matmul_reduced_b_norms call (score of x, select, gather-GEMV: 3 kernels)"
+        return ("one rmm_matmul_reduced_b_norms call ("
+                + ("select scoring x itself, gather-GEMV: 2 kernels)" if folded
+                   else "score of x, select, gather-GEMV: 3 kernels)"))
     if p.stream:
         return "one rmm_matmul_reduced call, stream route (score, select, B's dropped rows zeroed, gemm over A: 4 kernels)"
     if p.b_kmajor:

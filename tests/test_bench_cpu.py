@@ -155,3 +155,21 @@ def test_roofline_bound_follows_arithmetic_intensity():
     p = _meta(bench, "linear_4096", (4096, 4096), (4096, 4096), torch.bfloat16)
     r = bench.roofline(p, 0.5, {"pack": 0.02}, "pack", PEAKS, "measured")
     assert r["bound"] == "hbm" and r["algorithmic_bytes_per_launch"] == 83886080
+
+
+def test_step_description_follows_the_route():
+    """The bench line's config.step names the kernels a step launches on each
+    route (shape-only problems: no device memory needed)."""
+    import torch
+    bench = _bench()
+    p = _meta(bench, "linear_4096", (4096, 4096), (4096, 4096), torch.bfloat16)
+    assert "4 kernels" in bench.step_descr(p) and "pack" in bench.step_descr(p)
+    p = _meta(bench, "decode_mlp_up_m1", (1, 8192), (8192, 28672), torch.bfloat16)
+    assert "gather-GEMV: 2 kernels" in bench.step_descr(p)
+    p = _meta(bench, "decode_mlp_up", (16, 8192), (8192, 28672), torch.bfloat16)
+    assert "gather-GEMV: 3 kernels" in bench.step_descr(p)
+    p = _meta(bench, "pv_16384", (32, 16384, 16384), (32, 16384, 128), torch.bfloat16)
+    assert p.stream and "stream route" in bench.step_descr(p)
+    p = _meta(bench, "qk_32x4096x128", (32, 4096, 128), (32, 4096, 128), torch.bfloat16, b_kmajor=True,
+              out=torch.bfloat16)
+    assert "5 kernels" in bench.step_descr(p)
