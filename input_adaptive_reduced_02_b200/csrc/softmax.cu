@@ -12,7 +12,7 @@
 //    logits once (16-byte loads, several in flight) and keeps a running
 //    maximum and rescaled sum of exp2: stats[q] = (max of x, 1 / sum exp2(x -
 //    max)) with x = scale·log2(e)·L, the row's normalisation.
-//  * softmax_score_kernel: a cluster of up to 8 CTAs per (64-key strip, head)
+//  * softmax_score_kernel: a cluster of up to 8 CTAs per (128-key strip, head)
 //    splits the strip's query rows: p = exp2(x - max)·(1/sum) for visible
 //    keys, 0 for masked ones, rounded to bf16 (nearest even) and stored
 //    (16-byte stores), and the squares of the stored values summed per key
@@ -39,7 +39,7 @@ namespace {
 
 constexpr int kSmThreads = 256;
 constexpr unsigned kSmMaxCluster = 8;  // CTAs splitting one strip's rows
-constexpr int kStrip = 64;      // keys per CTA of the score kernel
+constexpr int kStrip = 128;     // keys per CTA of the score kernel (256-byte row segments for bf16)
 constexpr int kRowUnroll = 8;   // rows per ring stage per thread
 constexpr int kRing = 3;        // ring stages (two in flight while one is used)
 // ring of 16-byte logits slots per thread, then the rows' statistics (float2
@@ -193,7 +193,7 @@ __device__ __forceinline__ void p_group(const float (&x)[VT], int64_t c, int64_t
   }
 }
 
-// T: logits element. Threads: CL column lanes of VT keys (64 keys = one strip)
+// T: logits element. Threads: CL column lanes of VT keys (kStrip keys = one strip)
 // x RL row lanes; the CTAs of a cluster split the strip's rows, and with
 // s_out their partial column sums are added in rank order through
 // distributed shared memory. P is bf16 [bh][S_q][S_k]; s_out[b][k] (nullable:
@@ -285,7 +285,7 @@ softmax_score_kernel(const T* __restrict__ L, int64_t S_q, int64_t S_k, float xs
     // its own ring slots (kRing stages of kRowUnroll rows, two stages in
     // flight): no registers are held while the loads are in flight. The
     // first column lane of each row also copies the row's statistics into a
-    // slot the row's 8 lanes read after a warp barrier.
+    // slot the row's CL lanes (all in one warp) read after a warp barrier.
     extern __shared__ __align__(16) unsigned char sm_ring[];
     const uint32_t ring = smem_addr(sm_ring);
     const uint32_t srow = ring + uint32_t(kRing * kRowUnroll * kSmThreads * 16);  // [kRing][kRowUnroll][RL] float2
