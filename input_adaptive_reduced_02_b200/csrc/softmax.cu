@@ -225,6 +225,10 @@ softmax_score_kernel(const T* __restrict__ L, int64_t S_q, int64_t S_k, float xs
   uint16_t* Pb = P + b * S_q * S_k;
   const float2* st = stats + b * S_q;
   const bool full16 = vec && c0 + VT <= S_k;  // whole 16-byte logits group inside the row
+  // The ring path (with its warp barriers) only when every thread of the CTA
+  // has a whole 16-byte group: the choice must be the same for all lanes of a
+  // warp. A partial last strip takes the scalar path in every thread.
+  const bool ring_path = vec && k0 + kStrip <= S_k;
 
   // ||V[k, :]||^2 of the strip's keys: CTA r of the cluster takes keys r, r + cs,
   // ..., a warp per key, before its main loop so that the loads overlap it
@@ -280,7 +284,7 @@ softmax_score_kernel(const T* __restrict__ L, int64_t S_q, int64_t S_k, float xs
   float acc[VT];
 #pragma unroll
   for (int e = 0; e < VT; ++e) acc[e] = 0.f;
-  if (full16) {
+  if (ring_path) {
     // The logits of this thread's rows reach shared memory by cp.async into
     // its own ring slots (kRing stages of kRowUnroll rows, two stages in
     // flight): no registers are held while the loads are in flight. The

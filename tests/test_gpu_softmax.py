@@ -40,6 +40,9 @@ CASES = [  # bh, S_q, S_k, d, logits dtype, scale, causal
     (2, 200, 512, 128, torch.bfloat16, 0.125, True),  # fewer queries than keys, a scale
     (2, 256, 384, 72, torch.bfloat16, 1.0, False),    # no mask; d not a multiple of 8 for V
     (2, 512, 512, 128, torch.float32, 1.0, True),     # f32 logits
+    (2, 200, 200, 64, torch.bfloat16, 1.0, True),     # 16-byte rows, a partial last strip (200 % 128)
+    (1, 136, 392, 128, torch.bfloat16, 1.0, True),    # the same with fewer queries than keys
+    (2, 96, 200, 64, torch.float32, 1.0, False),      # f32 logits, a partial last strip, no mask
 ]
 
 
